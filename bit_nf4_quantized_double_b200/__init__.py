@@ -1,0 +1,226 @@
+"""Python binding of libqlora_nf4.so (the QLoRA NF4 + double-quant layer, sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/qlora_nf4.h. PyTorch supplies
+device memory and streams. There is no fallback: if the shared library is
+missing, importing the binding's entry points raises.
+
+Entry points (same names as the C ABI):
+    qlora_nf4_quantize(W)                    -> NF4Tensor
+    qlora_nf4_dequant(q)                     -> bf16 [rows, cols]
+    qlora_linear_fwd(X, q, A, B, s)          -> (Y, XA)
+    qlora_linear_bwd(X, dY, q, A, B, s, XA)  -> (dX, dA, dB)
+    qlora_get_device_status()                -> status code (0 = ok)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
+
+QLORA_OK = 0
+QLORA_ERR_INVALID_ARG = 1
+QLORA_ERR_UNSUPPORTED_SHAPE = 2
+QLORA_ERR_WORKSPACE = 3
+QLORA_ERR_NONFINITE = 4
+QLORA_ERR_TIMEOUT = 5
+QLORA_ERR_CUDA = 6
+QLORA_F32 = 0
+QLORA_BF16 = 1
+
+
+class QloraError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: status {status} ({status_string(status)})")
+
+
+class _Tensor(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("codes", ctypes.c_void_p),
+                ("scale8", ctypes.c_void_p), ("scale2", ctypes.c_void_p), ("offset", ctypes.c_void_p)]
+
+
+_lib = None
+
+_SIGS = {
+    "qlora_nf4_storage_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
+    "qlora_nf4_quantize_workspace": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
+    "qlora_nf4_quantize": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(_Tensor), ctypes.c_void_p,
+                                          ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_nf4_dequant": (ctypes.c_int, [ctypes.POINTER(_Tensor), ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_linear_fwd_workspace": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int]),
+    "qlora_linear_fwd": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(_Tensor), ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_linear_bwd_workspace": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int]),
+    "qlora_linear_bwd": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(_Tensor),
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_get_device_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "qlora_nf4_codebook": (None, [ctypes.c_void_p]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} not found: build it with bit_nf4_quantized_double_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().qlora_status_string(int(s)).decode()
+
+
+def _check(status: int, what: str):
+    if status != QLORA_OK:
+        raise QloraError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+@dataclass
+class NF4Tensor:
+    """The stored format: four device buffers owned by torch."""
+    rows: int
+    cols: int
+    codes: torch.Tensor    # uint8 [ceil(n/2)]
+    scale8: torch.Tensor   # int8 [ceil(n/64)]
+    scale2: torch.Tensor   # float32 [ceil(nb/256)]
+    offset: torch.Tensor   # float32 [1]
+
+    def ctype(self) -> _Tensor:
+        return _Tensor(self.rows, self.cols, self.codes.data_ptr(), self.scale8.data_ptr(),
+                       self.scale2.data_ptr(), self.offset.data_ptr())
+
+    @property
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.codes, self.scale8, self.scale2, self.offset))
+
+
+def nf4_sizes(rows: int, cols: int):
+    n = rows * cols
+    nb = -(-n // 64)
+    return n, -(-n // 2), nb, -(-nb // 256)
+
+
+def nf4_empty(rows: int, cols: int, device="cuda") -> NF4Tensor:
+    n, ncode, nb, nb2 = nf4_sizes(rows, cols)
+    return NF4Tensor(rows, cols, torch.empty(ncode, dtype=torch.uint8, device=device),
+                     torch.empty(nb, dtype=torch.int8, device=device),
+                     torch.empty(nb2, dtype=torch.float32, device=device),
+                     torch.empty(1, dtype=torch.float32, device=device))
+
+
+def _workspace(nbytes: int, device, ws=None):
+    if nbytes == 0:
+        return None, 0
+    if ws is not None and ws.numel() * ws.element_size() >= nbytes:
+        return ws, ws.numel() * ws.element_size()
+    t = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return t, nbytes
+
+
+def qlora_nf4_storage_bytes(rows: int, cols: int) -> int:
+    return int(lib().qlora_nf4_storage_bytes(rows, cols))
+
+
+def qlora_nf4_codebook():
+    buf = (ctypes.c_float * 16)()
+    lib().qlora_nf4_codebook(ctypes.cast(buf, ctypes.c_void_p))
+    return [float(v) for v in buf]
+
+
+def qlora_nf4_quantize(W: torch.Tensor, out: NF4Tensor | None = None, ws: torch.Tensor | None = None,
+                       stream=None) -> NF4Tensor:
+    """Quantise a [rows, cols] fp32 or bf16 CUDA tensor (contiguous)."""
+    if W.dim() == 1:
+        W = W.view(1, -1)
+    rows, cols = W.shape
+    dt = {torch.float32: QLORA_F32, torch.bfloat16: QLORA_BF16}[W.dtype]
+    if out is None:
+        out = nf4_empty(rows, cols, W.device)
+    L = lib()
+    need = int(L.qlora_nf4_quantize_workspace(rows, cols))
+    wsb, wsn = _workspace(need, W.device, ws)
+    t = out.ctype()
+    _check(L.qlora_nf4_quantize(_ptr(W.contiguous()), dt, ctypes.byref(t), _ptr(wsb), wsn, _stream(stream)),
+           "qlora_nf4_quantize")
+    return out
+
+
+def qlora_nf4_dequant(q: NF4Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(q.rows, q.cols, dtype=torch.bfloat16, device=q.codes.device)
+    t = q.ctype()
+    _check(lib().qlora_nf4_dequant(ctypes.byref(t), _ptr(out), _stream(stream)), "qlora_nf4_dequant")
+    return out
+
+
+def qlora_linear_fwd(X: torch.Tensor, W: NF4Tensor, A: torch.Tensor | None, B: torch.Tensor | None, s: float,
+                     Y: torch.Tensor | None = None, XA_save: torch.Tensor | bool | None = True,
+                     ws: torch.Tensor | None = None, stream=None):
+    """Y = X W^ + s (X A) B. Returns (Y, XA) where XA is bf16 [M, r] (or None)."""
+    M = X.shape[0]
+    r = 0 if A is None else A.shape[1]
+    if Y is None:
+        Y = torch.empty(M, W.rows, dtype=torch.bfloat16, device=X.device)
+    if XA_save is True:
+        XA_save = torch.empty(M, r, dtype=torch.bfloat16, device=X.device) if r else None
+    elif XA_save is False:
+        XA_save = None
+    L = lib()
+    wsb, wsn = _workspace(int(L.qlora_linear_fwd_workspace(M, W.rows, W.cols, r)), X.device, ws)
+    t = W.ctype()
+    _check(L.qlora_linear_fwd(_ptr(X), M, ctypes.byref(t), _ptr(A), _ptr(B), r, float(s), _ptr(Y),
+                              _ptr(XA_save), _ptr(wsb), wsn, _stream(stream)), "qlora_linear_fwd")
+    return Y, XA_save
+
+
+def qlora_linear_bwd(X: torch.Tensor, dY: torch.Tensor, W: NF4Tensor, A: torch.Tensor | None,
+                     B: torch.Tensor | None, s: float, XA: torch.Tensor | None = None,
+                     dX: torch.Tensor | None = None, dA: torch.Tensor | None = None, dB: torch.Tensor | None = None,
+                     ws: torch.Tensor | None = None, stream=None):
+    """dX = dY W^T + s (dY B^T) A^T, dA = s X^T (dY B^T), dB = s (XA)^T dY. Returns (dX, dA, dB)."""
+    M = dY.shape[0]
+    r = 0 if A is None else A.shape[1]
+    dev = dY.device
+    if dX is None:
+        dX = torch.empty(M, W.cols, dtype=torch.bfloat16, device=dev)
+    if r and dA is None:
+        dA = torch.empty(W.cols, r, dtype=torch.float32, device=dev)
+    if r and dB is None:
+        dB = torch.empty(r, W.rows, dtype=torch.float32, device=dev)
+    L = lib()
+    wsb, wsn = _workspace(int(L.qlora_linear_bwd_workspace(M, W.rows, W.cols, r)), dev, ws)
+    t = W.ctype()
+    _check(L.qlora_linear_bwd(_ptr(X), _ptr(dY), M, ctypes.byref(t), _ptr(A), _ptr(B), r, float(s), _ptr(XA),
+                              _ptr(dX), _ptr(dA), _ptr(dB), _ptr(wsb), wsn, _stream(stream)), "qlora_linear_bwd")
+    return dX, dA, dB
+
+
+def qlora_get_device_status(stream=None) -> int:
+    return int(lib().qlora_get_device_status(_stream(stream)))

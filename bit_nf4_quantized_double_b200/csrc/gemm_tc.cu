@@ -1,0 +1,953 @@
+// tcgen05 / TMEM kernels of the QLoRA linear layer (sm_100a).
+//
+// Layer (page "QLoRA: put the large model in memory, then change it with a
+// small adapter", wq-win.github.io/llm/074-qlora, section 1 equation):
+//   Y  = X W^ + s X A B                 (forward)
+//   dX = dY W^T + s (dY B^T) A^T        (backward; W^ gets no gradient)
+//   dA = s X^T (dY B^T),  dB = s (X A)^T dY
+// with W^ = Dequant(W4, scales) = (stored [d_out, d_in] matrix)^T, dequantised
+// to bf16 on the fly (section 3).
+//
+// Kernels
+//   k_fused_fwd   persistent; tile = 128 weight rows x 256 tokens. Dequant warps
+//                 turn each 64-weight block of a weight row into bf16 through a
+//                 16-entry per-block table (prmt lookups) and store it straight
+//                 into TMEM with tcgen05.st; tcgen05.mma takes that as its A
+//                 operand and the TMA-staged X tile (128-byte swizzle) as B, so
+//                 the dequantised weight never touches shared memory. One extra
+//                 K block multiplies B_lora^T (TMEM) by s*XA (TMA), which adds
+//                 the adapter term inside the same accumulator.
+//   k_fused_dgrad the transposed twin: the dequant warps write W^ tiles into
+//                 shared memory in the MN-major 128-byte-swizzled layout
+//                 tcgen05.mma reads directly, dY streams through TMA; the extra
+//                 K block multiplies A_lora (TMA) by s*G (TMA).
+//   k_skinny      TMA-fed tcgen05 GEMM for the rank-r products X*A, dY*B^T,
+//                 X^T*(sG), dY^T*XA with split-K partials; k_reduce_* sum the
+//                 partials in a fixed order and apply scale/layout.
+// Both fused kernels keep the accumulator tile D[row, token] in TMEM and store
+// it transposed (out[token, row]) through a shared-memory staging tile and a
+// TMA store.
+#include <mutex>
+
+#include "launch.h"
+#include "tc.cuh"
+
+namespace qnf4 {
+using namespace tc;
+
+// ------------------------------------------------------------------ dequant
+// Per-block bf16 table T[c] = bf16(fl(Q[c] * c^)) split into byte planes:
+// L[i] holds the low bytes of T[4i..4i+3], H[i] the high bytes.
+__device__ __forceinline__ void make_table(const Codebook &cb, float chat, uint32_t (&L)[4], uint32_t (&H)[4]) {
+    uint32_t tw[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) tw[j] = pack_bf16x2(__fmul_rn(cb.q[2 * j], chat), __fmul_rn(cb.q[2 * j + 1], chat));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        L[i] = prmt(tw[2 * i], tw[2 * i + 1], 0x6420u);
+        H[i] = prmt(tw[2 * i], tw[2 * i + 1], 0x7531u);
+    }
+}
+
+// One 32-bit word of packed codes (8 elements e0..e7 in memory order, byte k =
+// e[2k] << 4 | e[2k+1]) -> four bf16x2 words (e0|e1<<16, e2|e3<<16, ...).
+// prmt selects bytes by 3-bit index; bit 3 of each code picks the table half.
+__device__ __forceinline__ void lookup8(uint32_t w, const uint32_t (&L)[4], const uint32_t (&H)[4], uint32_t *out) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t v = h ? (w >> 16) : w;
+        const uint32_t sel = v & 0x7777u;
+        const uint32_t sel2 = ((v >> 1) & 0x4444u) | 0x3210u;
+        const uint32_t lo = prmt(prmt(L[0], L[1], sel), prmt(L[2], L[3], sel), sel2);
+        const uint32_t hi = prmt(prmt(H[0], H[1], sel), prmt(H[2], H[3], sel), sel2);
+        // nibble order inside the half-word is e1, e0, e3, e2
+        out[2 * h] = prmt(lo, hi, 0x4051u);
+        out[2 * h + 1] = prmt(lo, hi, 0x6273u);
+    }
+}
+
+// 64 codes (32 bytes) of one block -> 32 bf16x2 words in element order.
+__device__ __forceinline__ void dequant_block(const uint4 &c0, const uint4 &c1, const Codebook &cb, float chat,
+                                              uint32_t (&o)[32]) {
+    uint32_t L[4], H[4];
+    make_table(cb, chat, L, H);
+    lookup8(c0.x, L, H, o + 0);
+    lookup8(c0.y, L, H, o + 4);
+    lookup8(c0.z, L, H, o + 8);
+    lookup8(c0.w, L, H, o + 12);
+    lookup8(c1.x, L, H, o + 16);
+    lookup8(c1.y, L, H, o + 20);
+    lookup8(c1.z, L, H, o + 24);
+    lookup8(c1.w, L, H, o + 28);
+}
+
+// Bounded wait without the abort short-cut, for draining in-flight copies.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            raise_status(QLORA_ERR_TIMEOUT);
+            return;
+        }
+    }
+}
+
+struct FusedParams {
+    NF4View w;        // stored weight [rows, cols]
+    int M;            // tokens
+    int rows, cols;   // d_out, d_in
+    int r;            // adapter rank (0: none)
+    int tiles_tok;    // token tiles (256 each)
+    int tiles_row;    // output-row tiles (128 each): weight rows (fwd) or d_in columns (dgrad)
+    const __nv_bfloat16 *lora_t;  // fwd: B_lora [r, rows] (read transposed by the dequant warps)
+};
+
+constexpr int kTileRows = 128;   // TMEM lanes / MMA M
+constexpr int kTileTok = 256;    // MMA N
+constexpr int kTokStage = kTileTok * 128;          // 32 KB: 256 tokens x 64 bf16
+constexpr int kStaging = kTileTok * kTileRows * 2; // 64 KB output staging [256 tokens][128 rows]
+
+// Epilogue shared by both fused kernels: TMEM D[row, token] -> bf16 staging
+// [token][row] -> TMA store at (x = row0, y = tok0). Returns false on abort.
+__device__ __forceinline__ void fused_epilogue_tile(uint32_t tmem_d, int q, int lane, int et, uint8_t *staging,
+                                                    const CUtensorMap *tm_out, int row0, int tok0) {
+    uint16_t *st16 = reinterpret_cast<uint16_t *>(staging);
+    const int row_local = q * 32 + lane;
+    if (et == 0) bulk_wait_read0();      // previous store has finished reading the staging tile
+    named_bar_sync(1, 128);
+#pragma unroll 1
+    for (int c = 0; c < kTileTok / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)(32 * c), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[i]));
+            st16[(32 * c + i) * kTileRows + row_local] = *reinterpret_cast<const uint16_t *>(&h);
+        }
+    }
+}
+
+__device__ __forceinline__ void fused_epilogue_finish(int et, uint8_t *staging, const CUtensorMap *tm_out,
+                                                      int row0, int tok0) {
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    if (et == 0) {
+        tma_store_2d(tm_out, smem_addr(staging), row0, tok0);
+        bulk_commit();
+    }
+}
+
+// ================================================================ forward
+namespace fwd {
+constexpr int S = 4;                         // pipeline stages (even: stage parity = dequant group)
+constexpr int kCodeStage = kTileRows * 32;   // 4 KB: 128 rows x 32 code bytes
+constexpr int kStage = kTokStage + kCodeStage;
+constexpr int kSmem = 1024 + S * kStage + kStaging;
+constexpr int kThreads = 448;                // 14 warps
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemD = 0, kTmemA = 256;
+}  // namespace fwd
+
+__global__ void __launch_bounds__(fwd::kThreads, 1)
+k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
+            const __grid_constant__ CUtensorMap tm_xa, const __grid_constant__ CUtensorMap tm_y,
+            FusedParams p, Codebook cb) {
+    using namespace fwd;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[3 * S + 3];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *xs = smem;
+    uint8_t *cs = smem + S * kTokStage;
+    uint8_t *staging = cs + S * kCodeStage;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t bar0 = smem_addr(bars);
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto afull = [&](int s) { return bar0 + 8u * (S + s); };
+    auto empty = [&](int s) { return bar0 + 8u * (2 * S + s); };
+    const uint32_t tfull = bar0 + 8u * (3 * S), tempty = tfull + 8u, fin = tfull + 16u;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(afull(s), 4);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(tfull, 1);
+        mbar_init(tempty, 4);
+        mbar_init(fin, 1);
+        s_abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_codes);
+        tma_prefetch_desc(&tm_xa);
+        tma_prefetch_desc(&tm_y);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(&s_tmem), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    volatile int *abort = &s_abort;
+
+    const int KB = p.cols / 64;
+    const int LKB = (p.r + 63) / 64;
+    const int KBT = KB + LKB;
+    const int ntiles = p.tiles_tok * p.tiles_row;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const int tok0 = (tile % p.tiles_tok) * kTileTok, row0 = (tile / p.tiles_tok) * kTileRows;
+                for (int kb = 0; kb < KBT; ++kb, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait(empty(s), ph ^ 1u, abort)) { ok = false; break; }
+                    if (kb < KB) {
+                        mbar_arrive_expect_tx(full(s), kStage);
+                        tma_load_2d(smem_addr(xs + s * kTokStage), &tm_x, full(s), kb * 64, tok0);
+                        tma_load_2d(smem_addr(cs + s * kCodeStage), &tm_codes, full(s), kb * 32, row0);
+                    } else {
+                        mbar_arrive_expect_tx(full(s), kTokStage);
+                        tma_load_2d(smem_addr(xs + s * kTokStage), &tm_xa, full(s), (kb - KB) * 64, tok0);
+                    }
+                }
+            }
+            // every issued copy must land before the CTA can exit
+            const uint32_t first = it > (uint32_t)S ? it - S : 0;
+            for (uint32_t i = first; i < it; ++i) drain_wait(full(i % S), (i / S) & 1u);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(kTileRows, kTileTok, false, false);
+            uint32_t it = 0, lt = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++lt) {
+                if (!mbar_wait(tempty, (lt & 1u) ^ 1u, abort)) break;
+                tc_fence_after();
+                for (int kb = 0; kb < KBT; ++kb, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait(full(s), ph, abort) || !mbar_wait(afull(s), ph, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a = tmem + kTmemA + 32u * s;
+                    const uint32_t xb = smem_addr(xs + s * kTokStage);
+                    const int nk = kb < KB ? 4 : min(4, (p.r - (kb - KB) * 64 + 15) / 16);
+                    for (int k = 0; k < nk; ++k)
+                        mma_ts(tmem + kTmemD, a + 8u * k, sw128_desc(xb + 32u * k, 16, 1024), idesc,
+                               (kb | k) != 0 ? 1u : 0u);
+                    mma_commit(empty(s));
+                }
+                if (ok) mma_commit(tfull);
+            }
+            mma_commit(fin);          // all MMAs of this CTA complete before TMEM is released
+            drain_wait(fin, 0);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------ epilogue (warps 2..5)
+        const int q = warp & 3, et = threadIdx.x - 64;
+        uint32_t lt = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
+            const int tok0 = (tile % p.tiles_tok) * kTileTok, row0 = (tile / p.tiles_tok) * kTileRows;
+            if (!mbar_wait(tfull, lt & 1u, abort)) break;
+            tc_fence_after();
+            fused_epilogue_tile(tmem + kTmemD, q, lane, et, staging, &tm_y, row0, tok0);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty);
+            fused_epilogue_finish(et, staging, &tm_y, row0, tok0);
+        }
+        if (et == 0) bulk_wait0();
+    } else {
+        // ------------------------------------------------ dequant (warps 6..13)
+        const int g = (warp - 6) >> 2;          // handles iterations with it % 2 == g
+        const int q = warp & 3;                 // TMEM lane quarter
+        const int row_local = q * 32 + lane;
+        const float mu = *p.w.offset;
+        const int64_t kbs = p.cols / 64;        // 64-blocks per weight row
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+            const int row0 = (tile / p.tiles_tok) * kTileRows;
+            const int n = row0 + row_local;
+            const bool valid = n < p.rows;
+            for (int kb = 0; kb < KBT; ++kb, ++it) {
+                if ((int)(it & 1u) != g) continue;
+                const int s = it % S;
+                const uint32_t ph = (it / S) & 1u;
+                int8_t q8 = 0;
+                float s2 = 0.0f;
+                if (kb < KB && valid) {
+                    const int64_t b = (int64_t)n * kbs + kb;
+                    q8 = p.w.scale8[b];
+                    s2 = p.w.scale2[b >> 8];
+                }
+                if (!mbar_wait(full(s), ph, abort)) { ok = false; break; }
+                uint32_t v[32];
+                if (kb < KB) {
+                    if (valid) {
+                        const uint8_t *src = cs + s * kCodeStage + row_local * 32;
+                        const uint4 c0 = *reinterpret_cast<const uint4 *>(src);
+                        const uint4 c1 = *reinterpret_cast<const uint4 *>(src + 16);
+                        dequant_block(c0, c1, cb, dq_constant(q8, s2, mu), v);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = 0u;
+                    }
+                } else {
+                    // adapter block: A operand row n = B_lora[:, n] (rank index along K)
+                    const int j0 = (kb - KB) * 64;
+                    const uint16_t *bl = reinterpret_cast<const uint16_t *>(p.lora_t);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int k = j0 + 2 * i;
+                        const uint32_t lo = (valid && k < p.r) ? bl[(int64_t)k * p.rows + n] : 0u;
+                        const uint32_t hi = (valid && k + 1 < p.r) ? bl[(int64_t)(k + 1) * p.rows + n] : 0u;
+                        v[i] = lo | (hi << 16);
+                    }
+                }
+                tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + kTmemA + 32u * s, v);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(afull(s));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ================================================================ dgrad
+namespace dg {
+constexpr int S = 3;
+constexpr int kAStage = kTileRows * 128;     // 16 KB: 2 MN-chunks (64 d_in) x 64 K rows (d_out) x 128 B
+constexpr int kCodeStage = 64 * 64;          // 4 KB: 64 weight rows x 64 code bytes (128 d_in)
+constexpr int kStage = kAStage + kTokStage + kCodeStage;
+constexpr int kSmem = 1024 + S * kStage + kStaging;
+constexpr int kThreads = 448;
+constexpr uint32_t kTmemCols = 256;
+}  // namespace dg
+
+__global__ void __launch_bounds__(dg::kThreads, 1)
+k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_codes,
+              const __grid_constant__ CUtensorMap tm_alora, const __grid_constant__ CUtensorMap tm_gs,
+              const __grid_constant__ CUtensorMap tm_dx, FusedParams p, Codebook cb) {
+    using namespace dg;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[3 * S + 3];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *as = smem;
+    uint8_t *bs = smem + S * kAStage;
+    uint8_t *cs = bs + S * kTokStage;
+    uint8_t *staging = cs + S * kCodeStage;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t bar0 = smem_addr(bars);
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto afull = [&](int s) { return bar0 + 8u * (S + s); };
+    auto empty = [&](int s) { return bar0 + 8u * (2 * S + s); };
+    const uint32_t tfull = bar0 + 8u * (3 * S), tempty = tfull + 8u, fin = tfull + 16u;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(afull(s), 4);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(tfull, 1);
+        mbar_init(tempty, 4);
+        mbar_init(fin, 1);
+        s_abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tm_dy);
+        tma_prefetch_desc(&tm_codes);
+        tma_prefetch_desc(&tm_alora);
+        tma_prefetch_desc(&tm_gs);
+        tma_prefetch_desc(&tm_dx);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(&s_tmem), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    volatile int *abort = &s_abort;
+
+    const int KB = (p.rows + 63) / 64;           // contraction over d_out in blocks of 64 rows
+    const int LKB = (p.r + 63) / 64;
+    const int KBT = KB + LKB;
+    const int ntiles = p.tiles_tok * p.tiles_row;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const int tok0 = (tile % p.tiles_tok) * kTileTok, col0 = (tile / p.tiles_tok) * kTileRows;
+                for (int kb = 0; kb < KBT; ++kb, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait(empty(s), ph ^ 1u, abort)) { ok = false; break; }
+                    if (kb < KB) {
+                        mbar_arrive_expect_tx(full(s), kTokStage + kCodeStage);
+                        tma_load_2d(smem_addr(bs + s * kTokStage), &tm_dy, full(s), kb * 64, tok0);
+                        tma_load_2d(smem_addr(cs + s * kCodeStage), &tm_codes, full(s), col0 / 2, kb * 64);
+                    } else {
+                        mbar_arrive_expect_tx(full(s), kAStage + kTokStage);
+                        tma_load_2d(smem_addr(as + s * kAStage), &tm_alora, full(s), (kb - KB) * 64, col0);
+                        tma_load_2d(smem_addr(bs + s * kTokStage), &tm_gs, full(s), (kb - KB) * 64, tok0);
+                    }
+                }
+            }
+            const uint32_t first = it > (uint32_t)S ? it - S : 0;
+            for (uint32_t i = first; i < it; ++i) drain_wait(full(i % S), (i / S) & 1u);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc_main = idesc_bf16(kTileRows, kTileTok, true, false);
+            const uint32_t idesc_lora = idesc_bf16(kTileRows, kTileTok, false, false);
+            uint32_t it = 0, lt = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++lt) {
+                if (!mbar_wait(tempty, (lt & 1u) ^ 1u, abort)) break;
+                tc_fence_after();
+                for (int kb = 0; kb < KBT; ++kb, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait(full(s), ph, abort) || !mbar_wait(afull(s), ph, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t ab = smem_addr(as + s * kAStage);
+                    const uint32_t bb = smem_addr(bs + s * kTokStage);
+                    if (kb < KB) {
+                        for (int k = 0; k < 4; ++k)
+                            mma_ss(tmem, sw128_desc(ab + 2048u * k, 8192, 1024), sw128_desc(bb + 32u * k, 16, 1024),
+                                   idesc_main, (kb | k) != 0 ? 1u : 0u);
+                    } else {
+                        const int nk = min(4, (p.r - (kb - KB) * 64 + 15) / 16);
+                        for (int k = 0; k < nk; ++k)
+                            mma_ss(tmem, sw128_desc(ab + 32u * k, 16, 1024), sw128_desc(bb + 32u * k, 16, 1024),
+                                   idesc_lora, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(empty(s));
+                }
+                if (ok) mma_commit(tfull);
+            }
+            mma_commit(fin);
+            drain_wait(fin, 0);
+        }
+    } else if (warp < 6) {
+        const int q = warp & 3, et = threadIdx.x - 64;
+        uint32_t lt = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
+            const int tok0 = (tile % p.tiles_tok) * kTileTok, col0 = (tile / p.tiles_tok) * kTileRows;
+            if (!mbar_wait(tfull, lt & 1u, abort)) break;
+            tc_fence_after();
+            fused_epilogue_tile(tmem, q, lane, et, staging, &tm_dx, col0, tok0);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty);
+            fused_epilogue_finish(et, staging, &tm_dx, col0, tok0);
+        }
+        if (et == 0) bulk_wait0();
+    } else {
+        // dequant: thread tg = (warp % 4) * 32 + lane -> weight row kb*64 + (tg % 64), d_in chunk tg / 64
+        const int g = (warp - 6) >> 2;
+        const int tg = (warp & 3) * 32 + lane;
+        const int n_local = tg & 63, chunk = tg >> 6;
+        const float mu = *p.w.offset;
+        const int64_t kbs = p.cols / 64;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+            const int col0 = (tile / p.tiles_tok) * kTileRows;
+            const int kcol = col0 + 64 * chunk;
+            for (int kb = 0; kb < KBT; ++kb, ++it) {
+                if ((int)(it & 1u) != g) continue;
+                const int s = it % S;
+                const uint32_t ph = (it / S) & 1u;
+                const int n = kb * 64 + n_local;
+                const bool valid = kb < KB && n < p.rows && kcol < p.cols;
+                int8_t q8 = 0;
+                float s2 = 0.0f;
+                if (valid) {
+                    const int64_t b = (int64_t)n * kbs + kcol / 64;
+                    q8 = p.w.scale8[b];
+                    s2 = p.w.scale2[b >> 8];
+                }
+                if (!mbar_wait(full(s), ph, abort)) { ok = false; break; }
+                if (kb < KB) {
+                    uint32_t v[32];
+                    if (valid) {
+                        const uint8_t *src = cs + s * kCodeStage + n_local * 64 + chunk * 32;
+                        const uint4 c0 = *reinterpret_cast<const uint4 *>(src);
+                        const uint4 c1 = *reinterpret_cast<const uint4 *>(src + 16);
+                        dequant_block(c0, c1, cb, dq_constant(q8, s2, mu), v);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = 0u;
+                    }
+                    uint8_t *dst = as + s * kAStage + chunk * 8192;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4 *>(dst + sw128_offset(n_local, j)) =
+                            make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(afull(s));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ================================================================ skinny
+// D[128 x BN] = sum over K of A[128 x K] * B[BN x K]^T, operands by TMA in
+// 128-byte-swizzled tiles of 64 K; A and B each K-major or MN-major. One CTA
+// per (M tile, K split); fp32 partials [split][Mp][Np].
+struct SkinnyParams {
+    int Mp, Np, BN;        // output rows, columns (r), MMA N (Np rounded up to 16)
+    int kb_total, kb_per_split;
+    int stages;
+    float *partial;
+};
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(128, 1)
+k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, SkinnyParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[2 * 8 + 2];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int S = p.stages;
+    const int a_bytes = 128 * 128;
+    const int b_chunks = B_MN ? (p.BN + 63) / 64 : 1;
+    const int b_bytes = B_MN ? b_chunks * 8192 : p.BN * 128;
+    const int b_alloc = (b_bytes + 1023) & ~1023;
+    uint8_t *as = smem;
+    uint8_t *bs = smem + S * a_bytes;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t bar0 = smem_addr(bars);
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (8 + s); };
+    const uint32_t done = bar0 + 8u * 16, fin = done + 8u;
+    uint32_t ncols = 32;
+    while ((int)ncols < p.BN) ncols <<= 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(done, 1);
+        mbar_init(fin, 1);
+        s_abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tm_a);
+        tma_prefetch_desc(&tm_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(&s_tmem), ncols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    volatile int *abort = &s_abort;
+
+    const int m0 = blockIdx.x * 128;
+    const int split = blockIdx.y;
+    const int kb0 = split * p.kb_per_split;
+    const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+
+    if (warp == 0 && lane == 0) {
+        uint32_t it = 0;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            const int s = it % S;
+            const uint32_t ph = (it / S) & 1u;
+            if (!mbar_wait(empty(s), ph ^ 1u, abort)) break;
+            mbar_arrive_expect_tx(full(s), a_bytes + b_bytes);
+            const uint32_t a = smem_addr(as + s * a_bytes), b = smem_addr(bs + s * b_alloc);
+            if (A_MN) {
+                tma_load_2d(a, &tm_a, full(s), m0, kb * 64);
+                tma_load_2d(a + 8192, &tm_a, full(s), m0 + 64, kb * 64);
+            } else {
+                tma_load_2d(a, &tm_a, full(s), kb * 64, m0);
+            }
+            if (B_MN) {
+                for (int c = 0; c < b_chunks; ++c) tma_load_2d(b + 8192u * c, &tm_b, full(s), 64 * c, kb * 64);
+            } else {
+                tma_load_2d(b, &tm_b, full(s), kb * 64, 0);
+            }
+        }
+        const uint32_t first = it > (uint32_t)S ? it - S : 0;
+        for (uint32_t i = first; i < it; ++i) drain_wait(full(i % S), (i / S) & 1u);
+    } else if (warp == 1 && lane == 0) {
+        const uint32_t idesc = idesc_bf16(128, p.BN, A_MN, B_MN);
+        uint32_t it = 0;
+        bool ok = true;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            const int s = it % S;
+            const uint32_t ph = (it / S) & 1u;
+            if (!mbar_wait(full(s), ph, abort)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a = smem_addr(as + s * a_bytes), b = smem_addr(bs + s * b_alloc);
+            for (int k = 0; k < 4; ++k) {
+                const uint64_t ad = A_MN ? sw128_desc(a + 2048u * k, 8192, 1024) : sw128_desc(a + 32u * k, 16, 1024);
+                const uint64_t bd = B_MN ? sw128_desc(b + 2048u * k, 8192, 1024) : sw128_desc(b + 32u * k, 16, 1024);
+                mma_ss(tmem, ad, bd, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
+            }
+            mma_commit(empty(s));
+        }
+        if (ok) mma_commit(done);
+        mma_commit(fin);
+        drain_wait(fin, 0);
+    }
+    __syncwarp();
+    // epilogue: all 4 warps (warp w reads TMEM lanes 32w..32w+31)
+    if (mbar_wait(done, 0, abort)) {
+        tc_fence_after();
+        const int row = m0 + warp * 32 + lane;
+        float *dst = p.partial + ((int64_t)split * p.Mp + row) * p.Np;
+        for (int c = 0; c < p.BN; c += 16) {
+            uint32_t v[16];
+            tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+            tmem_wait_ld();
+            if (row < p.Mp) {
+                if (c + 16 <= p.Np) {
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4)
+                        *reinterpret_cast<float4 *>(dst + c + i) =
+                            make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                                        __uint_as_float(v[i + 3]));
+                } else {
+                    for (int i = 0; i < 16 && c + i < p.Np; ++i) dst[c + i] = __uint_as_float(v[i]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, ncols);
+    }
+}
+
+// ------------------------------------------------------------------ reduce
+// Sums of split-K partials in split order (deterministic), then scale/convert.
+__global__ void k_reduce_xa(const float *__restrict__ part, int splits, int64_t count, float s,
+                            __nv_bfloat16 *__restrict__ xa, __nv_bfloat16 *__restrict__ xas) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
+        float v = 0.0f;
+        for (int sp = 0; sp < splits; ++sp) v += part[sp * count + i];
+        if (xa) xa[i] = __float2bfloat16_rn(v);
+        if (xas) xas[i] = __float2bfloat16_rn(s * v);
+    }
+}
+__global__ void k_reduce_f32(const float *__restrict__ part, int splits, int64_t count, float s,
+                             float *__restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
+        float v = 0.0f;
+        for (int sp = 0; sp < splits; ++sp) v += part[sp * count + i];
+        out[i] = s * v;
+    }
+}
+// part [split][rows][r] -> out [r][rows] (transposed), times s
+__global__ void k_reduce_f32_t(const float *__restrict__ part, int splits, int64_t rows, int r, float s,
+                               float *__restrict__ out) {
+    const int64_t count = rows * r;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t j = i / rows, n = i % rows;   // output index [j][n], coalesced over n
+        float v = 0.0f;
+        for (int sp = 0; sp < splits; ++sp) v += part[sp * count + n * r + j];
+        out[i] = s * v;
+    }
+}
+
+// ================================================================ host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2D tensor map: dim0 = inner (contiguous) extent, dim1 = outer extent,
+// row stride in bytes; box {box0, box1}; out-of-range elements read as zero.
+static bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+                     uint64_t stride_bytes, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {stride_bytes};
+    cuuint32_t box[2] = {box0, box1};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+static bool map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box0, uint32_t box1,
+                     CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
+    return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, inner, outer, inner * 2, box0, box1, sw);
+}
+
+template <typename K>
+static cudaError_t set_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+constexpr int kTargetCtas = 296;   // split-K sizing target (two waves of 148 SMs)
+
+struct SplitPlan { int kb_total, kb_per_split, splits; };
+static SplitPlan plan_splits(int64_t Mp, int64_t Kp) {
+    SplitPlan sp;
+    sp.kb_total = (int)ceil_div(Kp, 64);
+    const int mt = (int)ceil_div(Mp, 128);
+    int want = (int)ceil_div(kTargetCtas, mt);
+    if (want < 1) want = 1;
+    if (want > sp.kb_total) want = sp.kb_total;
+    sp.kb_per_split = (int)ceil_div(sp.kb_total, want);
+    sp.splits = (int)ceil_div(sp.kb_total, sp.kb_per_split);
+    return sp;
+}
+static size_t partial_bytes(int64_t Mp, int64_t Kp, int r) {
+    return align256((size_t)plan_splits(Mp, Kp).splits * (size_t)Mp * (size_t)r * 4);
+}
+
+// Launch one skinny product. A operand: K-major [Mp rows, Kp] or MN-major
+// [Kp rows, Mp]; B operand: K-major [r rows, Kp] or MN-major [Kp rows, r].
+static cudaError_t run_skinny(bool a_mn, const void *a, int64_t a_ld_rows, bool b_mn, const void *b, int64_t Mp,
+                              int64_t Kp, int r, float *partial, int *splits_out, cudaStream_t st) {
+    CUtensorMap ta, tb;
+    const int BN = (int)ceil_div(r, 16) * 16;
+    bool ok;
+    if (a_mn) ok = map_bf16(&ta, a, (uint64_t)Mp, (uint64_t)Kp, 64, 64);
+    else ok = map_bf16(&ta, a, (uint64_t)Kp, (uint64_t)Mp, 64, 128);
+    (void)a_ld_rows;
+    if (b_mn) ok = ok && map_bf16(&tb, b, (uint64_t)r, (uint64_t)Kp, 64, 64);
+    else ok = ok && map_bf16(&tb, b, (uint64_t)Kp, (uint64_t)r, 64, (uint32_t)BN);
+    if (!ok) return cudaErrorInvalidValue;
+    const SplitPlan sp = plan_splits(Mp, Kp);
+    SkinnyParams p;
+    p.Mp = (int)Mp;
+    p.Np = r;
+    p.BN = BN;
+    p.kb_total = sp.kb_total;
+    p.kb_per_split = sp.kb_per_split;
+    p.partial = partial;
+    const int b_bytes = b_mn ? (int)ceil_div(BN, 64) * 8192 : BN * 128;
+    const int stage = 128 * 128 + ((b_bytes + 1023) & ~1023);
+    int stages = (200 * 1024) / stage;
+    if (stages > 8) stages = 8;
+    if (stages > sp.kb_per_split) stages = sp.kb_per_split < 2 ? 2 : sp.kb_per_split;
+    p.stages = stages;
+    const int smem = 1024 + stages * stage;
+    dim3 grid((unsigned)ceil_div(Mp, 128), (unsigned)sp.splits);
+    cudaError_t e;
+#define QNF4_SK(AM, BM)                                                      \
+    e = set_smem(k_skinny<AM, BM>, smem);                                    \
+    if (e != cudaSuccess) return e;                                          \
+    k_skinny<AM, BM><<<grid, 128, smem, st>>>(ta, tb, p);
+    if (a_mn && b_mn) { QNF4_SK(true, true) }
+    else if (a_mn) { QNF4_SK(true, false) }
+    else if (b_mn) { QNF4_SK(false, true) }
+    else { QNF4_SK(false, false) }
+#undef QNF4_SK
+    *splits_out = sp.splits;
+    return cudaGetLastError();
+}
+
+static unsigned reduce_grid(int64_t count) {
+    int64_t g = ceil_div(count, 256);
+    const int64_t cap = (int64_t)num_sms() * 8;
+    return (unsigned)(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+static size_t mr_bytes(int64_t M, int r) { return align256((size_t)M * (size_t)r * 2); }
+
+size_t fwd_workspace_bytes_large(int64_t M, int64_t rows, int64_t cols, int r) {
+    (void)rows;
+    if (r == 0) return 0;
+    return mr_bytes(M, r) + partial_bytes(M, cols, r);
+}
+
+size_t xa_small_workspace(int64_t M, int64_t cols, int r) { return mr_bytes(M, r) + partial_bytes(M, cols, r); }
+
+// XA = X A for the small-M path: XA_save = bf16(XA) (optional), XAs = bf16(s XA).
+cudaError_t launch_xa_small(const __nv_bfloat16 *X, int64_t M, int64_t cols, const __nv_bfloat16 *A, int r, float s,
+                            __nv_bfloat16 *XA_save, __nv_bfloat16 *XAs, void *part_ws, cudaStream_t st) {
+    int splits = 0;
+    float *part = static_cast<float *>(part_ws);
+    cudaError_t e = run_skinny(false, X, M, true, A, M, cols, r, part, &splits, st);
+    if (e != cudaSuccess) return e;
+    k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, XA_save, XAs);
+    return cudaGetLastError();
+}
+
+size_t bwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
+    if (r == 0) return 0;
+    size_t part = partial_bytes(M, cols, r);                 // X*A
+    size_t p2 = partial_bytes(M, rows, r);                   // dY*B^T
+    size_t p3 = partial_bytes(cols, M, r);                   // X^T*(sG)
+    size_t p4 = partial_bytes(rows, M, r);                   // dY^T*XA
+    if (p2 > part) part = p2;
+    if (p3 > part) part = p3;
+    if (p4 > part) part = p4;
+    return 2 * mr_bytes(M, r) + part;
+}
+
+static cudaError_t run_fused_fwd(const __nv_bfloat16 *X, int64_t M, const NF4View &W, const __nv_bfloat16 *XAs,
+                                 const __nv_bfloat16 *Blora, int r, __nv_bfloat16 *Y, cudaStream_t st) {
+    CUtensorMap tx, tc_, txa, ty;
+    bool ok = map_bf16(&tx, X, (uint64_t)W.cols, (uint64_t)M, 64, kTileTok);
+    ok = ok && make_map(&tc_, W.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)(W.cols / 2), (uint64_t)W.rows,
+                        (uint64_t)(W.cols / 2), 32, kTileRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (r > 0) ok = ok && map_bf16(&txa, XAs, (uint64_t)r, (uint64_t)M, 64, kTileTok);
+    else txa = tx;
+    ok = ok && map_bf16(&ty, Y, (uint64_t)W.rows, (uint64_t)M, kTileRows, kTileTok, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return cudaErrorInvalidValue;
+    FusedParams p;
+    p.w = W;
+    p.M = (int)M;
+    p.rows = (int)W.rows;
+    p.cols = (int)W.cols;
+    p.r = r;
+    p.tiles_tok = (int)ceil_div(M, kTileTok);
+    p.tiles_row = (int)ceil_div(W.rows, kTileRows);
+    p.lora_t = Blora;
+    const int ntiles = p.tiles_tok * p.tiles_row;
+    const int grid = ntiles < num_sms() ? ntiles : num_sms();
+    cudaError_t e = set_smem(k_fused_fwd, fwd::kSmem);
+    if (e != cudaSuccess) return e;
+    k_fused_fwd<<<grid, fwd::kThreads, fwd::kSmem, st>>>(tx, tc_, txa, ty, p, host_codebook());
+    return cudaGetLastError();
+}
+
+static cudaError_t run_fused_dgrad(const __nv_bfloat16 *dY, int64_t M, const NF4View &W, const __nv_bfloat16 *Alora,
+                                   const __nv_bfloat16 *Gs, int r, __nv_bfloat16 *dX, cudaStream_t st) {
+    CUtensorMap tdy, tc_, ta, tg, tdx;
+    bool ok = map_bf16(&tdy, dY, (uint64_t)W.rows, (uint64_t)M, 64, kTileTok);
+    ok = ok && make_map(&tc_, W.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)(W.cols / 2), (uint64_t)W.rows,
+                        (uint64_t)(W.cols / 2), 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (r > 0) {
+        ok = ok && map_bf16(&ta, Alora, (uint64_t)r, (uint64_t)W.cols, 64, kTileRows);
+        ok = ok && map_bf16(&tg, Gs, (uint64_t)r, (uint64_t)M, 64, kTileTok);
+    } else {
+        ta = tdy;
+        tg = tdy;
+    }
+    ok = ok && map_bf16(&tdx, dX, (uint64_t)W.cols, (uint64_t)M, kTileRows, kTileTok, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return cudaErrorInvalidValue;
+    FusedParams p;
+    p.w = W;
+    p.M = (int)M;
+    p.rows = (int)W.rows;
+    p.cols = (int)W.cols;
+    p.r = r;
+    p.tiles_tok = (int)ceil_div(M, kTileTok);
+    p.tiles_row = (int)ceil_div(W.cols, kTileRows);
+    p.lora_t = nullptr;
+    const int ntiles = p.tiles_tok * p.tiles_row;
+    const int grid = ntiles < num_sms() ? ntiles : num_sms();
+    cudaError_t e = set_smem(k_fused_dgrad, dg::kSmem);
+    if (e != cudaSuccess) return e;
+    k_fused_dgrad<<<grid, dg::kThreads, dg::kSmem, st>>>(tdy, tc_, ta, tg, tdx, p, host_codebook());
+    return cudaGetLastError();
+}
+
+cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4View &W, const __nv_bfloat16 *A,
+                                    const __nv_bfloat16 *B, int r, float s, __nv_bfloat16 *Y,
+                                    __nv_bfloat16 *XA_save, void *ws, cudaStream_t st) {
+    __nv_bfloat16 *XAs = nullptr;
+    if (r > 0) {
+        XAs = static_cast<__nv_bfloat16 *>(ws);
+        float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + mr_bytes(M, r));
+        int splits = 0;
+        cudaError_t e = run_skinny(false, X, M, true, A, M, W.cols, r, part, &splits, st);
+        if (e != cudaSuccess) return e;
+        k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, XA_save, XAs);
+    }
+    return run_fused_fwd(X, M, W, XAs, B, r, Y, st);
+}
+
+cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, int64_t M, const NF4View &W,
+                              const __nv_bfloat16 *A, const __nv_bfloat16 *B, int r, float s,
+                              const __nv_bfloat16 *XA, __nv_bfloat16 *dX, float *dA, float *dB, void *ws,
+                              cudaStream_t st) {
+    __nv_bfloat16 *Gs = nullptr;
+    cudaError_t e;
+    if (r > 0) {
+        Gs = static_cast<__nv_bfloat16 *>(ws);
+        __nv_bfloat16 *XAbuf = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + mr_bytes(M, r));
+        float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + 2 * mr_bytes(M, r));
+        int splits = 0;
+        if (!XA) {
+            e = run_skinny(false, X, M, true, A, M, W.cols, r, part, &splits, st);
+            if (e != cudaSuccess) return e;
+            k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, 1.0f, XAbuf, nullptr);
+            XA = XAbuf;
+        }
+        // G = dY B^T -> sG (bf16)
+        e = run_skinny(false, dY, M, false, B, M, W.rows, r, part, &splits, st);
+        if (e != cudaSuccess) return e;
+        k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, nullptr, Gs);
+    }
+    e = run_fused_dgrad(dY, M, W, A, Gs, r, dX, st);
+    if (e != cudaSuccess) return e;
+    if (r > 0) {
+        float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + 2 * mr_bytes(M, r));
+        int splits = 0;
+        // dA = X^T (sG)
+        e = run_skinny(true, X, M, true, Gs, W.cols, M, r, part, &splits, st);
+        if (e != cudaSuccess) return e;
+        k_reduce_f32<<<reduce_grid(W.cols * r), 256, 0, st>>>(part, splits, W.cols * r, 1.0f, dA);
+        // dB = s (XA)^T dY, computed as (dY^T XA)^T
+        e = run_skinny(true, dY, M, true, XA, W.rows, M, r, part, &splits, st);
+        if (e != cudaSuccess) return e;
+        k_reduce_f32_t<<<reduce_grid(W.rows * r), 256, 0, st>>>(part, splits, W.rows, r, s, dB);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace qnf4

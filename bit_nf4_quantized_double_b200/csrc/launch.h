@@ -1,0 +1,24 @@
+// Internal launch interface between the C-ABI layer and the kernel files.
+#pragma once
+
+#include "common.cuh"
+
+namespace qnf4 {
+
+cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlora_nf4_tensor &out,
+                            float *c1, double *part, cudaStream_t st);
+cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st);
+
+size_t fwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r);
+size_t bwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r);
+
+cudaError_t launch_linear_fwd(const __nv_bfloat16 *X, int64_t M, const NF4View &W,
+                              const __nv_bfloat16 *A, const __nv_bfloat16 *B, int r, float s,
+                              __nv_bfloat16 *Y, __nv_bfloat16 *XA_save, void *ws, cudaStream_t st);
+
+cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, int64_t M, const NF4View &W,
+                              const __nv_bfloat16 *A, const __nv_bfloat16 *B, int r, float s,
+                              const __nv_bfloat16 *XA, __nv_bfloat16 *dX, float *dA, float *dB,
+                              void *ws, cudaStream_t st);
+
+}  // namespace qnf4

@@ -1,0 +1,285 @@
+// NF4 quantisation, double quantisation and dequantisation kernels (sm_100a).
+//
+// Method: "QLoRA: put the large model in memory, then change it with a small
+// adapter" (wq-win.github.io/llm/074-qlora), section 2 (64-weight absmax
+// blocks, 16-value normal-quantile codebook, 8-bit constants with an offset and
+// one fp32 constant per 256 constants) and section 3 (quantise W, then the
+// constants; dequantise to BF16 on demand).
+//
+// Launch sequence of a quantisation (all HBM-bound):
+//   k_quantize_codes  one CTA per second-level group (256 blocks = 16384 weights):
+//                     absmax per 64-block by warp shuffles, IEEE division, 4-step
+//                     threshold search, nibble packing; writes the exact fp32
+//                     absmax and the group's fp64 pairwise partial sum;
+//   k_offset          one CTA: the upper levels of the fp64 pairwise tree -> mean;
+//   k_double_quant    one warp per group: s2 = max |c1 - mu|, int8 constants.
+
+#include "common.cuh"
+
+namespace qnf4 {
+
+__device__ unsigned int g_status_bits = 0;
+
+// Number of thresholds strictly below x (t ascending, 15 entries in shared
+// memory): a 4-step binary search that returns the same count as comparing
+// against all 15. A value equal to a threshold stays on the lower code.
+__device__ __forceinline__ int nf4_code(float x, const float *t) {
+    int c = (x > t[7]) ? 8 : 0;
+    c += (x > t[c + 3]) ? 4 : 0;
+    c += (x > t[c + 1]) ? 2 : 0;
+    c += (x > t[c]) ? 1 : 0;
+    return c;
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T, int VEC>
+__device__ __forceinline__ void load_vec(const T *p, float (&v)[VEC]) {
+    const uint4 raw = *reinterpret_cast<const uint4 *>(p);
+    if constexpr (sizeof(T) == 4) {
+        v[0] = __uint_as_float(raw.x); v[1] = __uint_as_float(raw.y);
+        v[2] = __uint_as_float(raw.z); v[3] = __uint_as_float(raw.w);
+    } else {
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) { v[2 * k] = bf16_lo(w[k]); v[2 * k + 1] = bf16_hi(w[k]); }
+    }
+}
+
+// One CTA of 256 threads per second-level group j (blocks 256j .. 256j+255).
+// Warp w handles blocks 256j + 32w .. +31; a 64-block is spread over
+// LPB = 64 / VEC lanes that each load 16 bytes.
+template <typename T>
+__global__ void __launch_bounds__(256)
+k_quantize_codes(const T *__restrict__ W, int64_t n, int64_t nb, Codebook cb,
+                 float *__restrict__ c1_out, double *__restrict__ part_out,
+                 uint8_t *__restrict__ codes) {
+    constexpr int VEC = 16 / sizeof(T);   // elements per 16-byte lane load
+    constexpr int LPB = kBlock1 / VEC;    // lanes per block
+    constexpr int BPI = 32 / LPB;         // blocks per warp iteration
+    constexpr int ITERS = 32 / BPI;       // iterations per warp (32 blocks)
+    constexpr int NBYTES = VEC / 2;       // code bytes per lane per iteration
+
+    __shared__ float s_t[16];
+    __shared__ float s_c1[kBlock2];
+    __shared__ double s_part[8];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x < 15) s_t[threadIdx.x] = cb.t[threadIdx.x];
+    __syncthreads();
+
+    const int64_t group = blockIdx.x;
+    const int sub = lane / LPB, li = lane % LPB;
+    const int64_t ncode = (n + 1) / 2;
+    bool nonfinite = false;
+
+#pragma unroll 4
+    for (int it = 0; it < ITERS; ++it) {
+        const int local = warp * 32 + it * BPI + sub;          // block index within the group
+        const int64_t b = group * kBlock2 + local;
+        const int64_t e0 = b * kBlock1 + (int64_t)li * VEC;     // first element of this lane
+        float v[VEC];
+        if (e0 + VEC <= n) {
+            load_vec<T, VEC>(W + e0, v);
+        } else {
+#pragma unroll
+            for (int k = 0; k < VEC; ++k) v[k] = (e0 + k < n) ? to_f32<T>(W[e0 + k]) : 0.0f;
+        }
+        float m = 0.0f;
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) {
+            nonfinite |= !isfinite(v[k]);
+            m = fmaxf(m, fabsf(v[k]));
+        }
+#pragma unroll
+        for (int o = LPB / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (li == 0) {
+            s_c1[local] = m;
+            if (b < nb) c1_out[b] = m;
+        }
+        // codes of the lane's VEC elements: NBYTES bytes, byte k = hi << 4 | lo
+        uint32_t packed = 0;
+#pragma unroll
+        for (int k = 0; k < VEC; k += 2) {
+            const float x0 = (m == 0.0f) ? 0.0f : __fdiv_rn(v[k], m);
+            const float x1 = (m == 0.0f) ? 0.0f : __fdiv_rn(v[k + 1], m);
+            const uint32_t byte = ((uint32_t)nf4_code(x0, s_t) << 4) | (uint32_t)nf4_code(x1, s_t);
+            packed |= byte << (8 * (k / 2));
+        }
+        const int64_t c0 = e0 / 2;
+        if (c0 + NBYTES <= ncode) {
+            if constexpr (NBYTES == 4) *reinterpret_cast<uint32_t *>(codes + c0) = packed;
+            else *reinterpret_cast<uint16_t *>(codes + c0) = (uint16_t)packed;
+        } else {
+#pragma unroll
+            for (int k = 0; k < NBYTES; ++k)
+                if (c0 + k < ncode) codes[c0 + k] = (uint8_t)(packed >> (8 * k));
+        }
+    }
+    if (__any_sync(0xffffffffu, nonfinite) && lane == 0) raise_status(QLORA_ERR_NONFINITE);
+    __syncthreads();
+
+    // fp64 pairwise tree over the group's 256 leaves (blocks past nb are 0):
+    // node i of level l+1 = node 2i + node 2i+1 of level l.
+    double v = (double)s_c1[threadIdx.x];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double u = __shfl_down_sync(0xffffffffu, v, o);
+        if ((lane & (2 * o - 1)) == 0) v = v + u;
+    }
+    if (lane == 0) s_part[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        v = (lane < 8) ? s_part[lane] : 0.0;
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+            const double u = __shfl_down_sync(0xffffffffu, v, o);
+            if ((lane & (2 * o - 1)) == 0) v = v + u;
+        }
+        if (lane == 0) part_out[group] = v;
+    }
+}
+
+// Upper levels of the pairwise tree over the nb2 group partials, zero-padded
+// to a power of two (>= 1024): thread t first reduces leaves [tC, tC+C) with
+// a binary-counter stack (which forms exactly the subtree of those leaves),
+// then the 1024 subtree sums are combined level by level. mu = fl(S / nb).
+__global__ void __launch_bounds__(1024)
+k_offset(const double *__restrict__ part, int64_t nb2, int64_t nb, float *__restrict__ offset_out) {
+    __shared__ double s_w[32];
+    int64_t L = 1024;
+    while (L < nb2) L <<= 1;
+    const int64_t C = L / 1024;
+    const int64_t i0 = (int64_t)threadIdx.x * C;
+    double v = 0.0;
+    if (i0 < nb2) {
+        double stack[48];
+        int level[48];
+        int sp = 0;
+        for (int64_t i = 0; i < C; ++i) {
+            double x = (i0 + i < nb2) ? part[i0 + i] : 0.0;
+            int l = 0;
+            while (sp > 0 && level[sp - 1] == l) { x = stack[--sp] + x; ++l; }
+            stack[sp] = x;
+            level[sp] = l;
+            ++sp;
+        }
+        v = stack[0];
+    }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double u = __shfl_down_sync(0xffffffffu, v, o);
+        if ((lane & (2 * o - 1)) == 0) v = v + u;
+    }
+    if (lane == 0) s_w[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        v = s_w[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double u = __shfl_down_sync(0xffffffffu, v, o);
+            if ((lane & (2 * o - 1)) == 0) v = v + u;
+        }
+        if (lane == 0) *offset_out = __double2float_rn(__ddiv_rn(v, (double)nb));
+    }
+}
+
+// One warp per second-level group: d_b = fl(c1_b - mu), s2 = max |d_b|,
+// q8_b = rint(fl(fl(d_b / s2) * 127)) (0 when s2 == 0).
+__global__ void __launch_bounds__(256)
+k_double_quant(const float *__restrict__ c1, int64_t nb, int64_t nb2, const float *__restrict__ offset,
+               int8_t *__restrict__ q8, float *__restrict__ s2) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t j = (int64_t)blockIdx.x * 8 + warp;
+    if (j >= nb2) return;
+    const float mu = *offset;
+    float d[8];
+    float m = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int64_t b = j * kBlock2 + k * 32 + lane;
+        d[k] = (b < nb) ? __fsub_rn(c1[b], mu) : 0.0f;
+        m = fmaxf(m, fabsf(d[k]));
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) s2[j] = m;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int64_t b = j * kBlock2 + k * 32 + lane;
+        if (b < nb) {
+            int q = 0;
+            if (m != 0.0f) q = __float2int_rn(__fmul_rn(__fdiv_rn(d[k], m), 127.0f));
+            q8[b] = (int8_t)q;
+        }
+    }
+}
+
+// Dequantisation: each thread expands 16 code bytes (32 weights, half a
+// block) into 64 bytes of bf16. Codebook in shared memory (16 distinct words,
+// so lookups from a warp never conflict).
+__global__ void __launch_bounds__(256)
+k_dequant(NF4View q, int64_t n, Codebook cb, __nv_bfloat16 *__restrict__ out) {
+    __shared__ float s_q[16];
+    if (threadIdx.x < 16) s_q[threadIdx.x] = cb.q[threadIdx.x];
+    __syncthreads();
+    const float mu = *q.offset;
+    const int64_t nchunk = (n + 31) / 32;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < nchunk; c += stride) {
+        const int64_t e0 = c * 32;
+        const int64_t b = e0 / kBlock1;
+        const float ch = dq_constant(q.scale8[b], q.scale2[b / kBlock2], mu);
+        if (e0 + 32 <= n) {
+            const uint4 raw = ldg_nc_v4(q.codes + e0 / 2);
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+            uint32_t o[16];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t byte = (w[i] >> (8 * k)) & 0xffu;
+                    o[4 * i + k] = pack_bf16x2(__fmul_rn(s_q[byte >> 4], ch), __fmul_rn(s_q[byte & 15u], ch));
+                }
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(out + e0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        } else {
+            for (int64_t e = e0; e < n; ++e) {
+                const uint8_t byte = q.codes[e / 2];
+                const uint32_t code = (e % 2 == 0) ? (byte >> 4) : (byte & 15u);
+                out[e] = __float2bfloat16_rn(__fmul_rn(s_q[code], ch));
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- launchers
+cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlora_nf4_tensor &out,
+                            float *c1, double *part, cudaStream_t st) {
+    const int64_t nb = ceil_div(n, kBlock1), nb2 = ceil_div(nb, kBlock2);
+    const Codebook &cb = host_codebook();
+    if (dt == QLORA_F32)
+        k_quantize_codes<float><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const float *>(W), n, nb, cb, c1, part, out.codes);
+    else
+        k_quantize_codes<__nv_bfloat16><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W), n, nb, cb, c1, part, out.codes);
+    k_offset<<<1, 1024, 0, st>>>(part, nb2, nb, out.offset);
+    k_double_quant<<<(unsigned)ceil_div(nb2, 8), 256, 0, st>>>(c1, nb, nb2, out.offset, out.scale8, out.scale2);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st) {
+    const int64_t n = q.rows * q.cols;
+    const int64_t nchunk = ceil_div(n, 32);
+    int64_t grid = ceil_div(nchunk, 256);
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (grid > cap) grid = cap;
+    k_dequant<<<(unsigned)grid, 256, 0, st>>>(q, n, host_codebook(), out);
+    return cudaGetLastError();
+}
+
+}  // namespace qnf4

@@ -1,0 +1,156 @@
+/*
+ * qlora_nf4.h - C ABI of the QLoRA NF4 + double-quantisation linear layer
+ * (sm_100a, one GPU).
+ *
+ * The method is the one summarised in "QLoRA: put the large model in memory,
+ * then change it with a small adapter" (wq-win.github.io/llm/074-qlora):
+ *   section 1 (equation)  Y = X W^ + s X A B,  W^ = Dequant(W4, scales); the
+ *                         frozen base gets no gradient, dX flows through W^ transposed;
+ *   section 2             NF4 codes for 64-weight absmax blocks (16 normal-quantile
+ *                         values, exact zero), 8-bit first-level constants with an
+ *                         offset, one fp32 second-level constant per 256 constants;
+ *   section 3             quantise W first, then the constants; dequantise to BF16
+ *                         on demand.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer argument of a tensor is DEVICE memory owned by the caller,
+ *   16-byte aligned unless stated otherwise. The library never allocates or
+ *   frees device memory; scratch comes from a caller-provided workspace whose
+ *   size the matching *_workspace() query returns.
+ * - bf16 tensors are passed as void pointers to IEEE bfloat16 bit patterns.
+ * - The stored weight uses the nn.Linear layout [rows = d_out, cols = d_in],
+ *   row-major. The W^ of the layer equation is its transpose.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream). The return value covers host-side argument checks and launch
+ *   errors. Conditions found on the device (a non-finite weight, a bounded
+ *   wait that ran out) are recorded in a per-device status word that
+ *   qlora_get_device_status() reads and clears. Kernels never trap.
+ * - Arithmetic of the encoding is fixed: one IEEE binary32 operation per step,
+ *   round-to-nearest-even, no fused multiply-add, denormals kept; bf16 and int8
+ *   conversions round to nearest even. Codes, constants and dequantised values
+ *   are therefore bit-for-bit reproducible.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QLORA_OK = 0,
+    QLORA_ERR_INVALID_ARG = 1,       /* null / misaligned pointer, bad dtype or scale */
+    QLORA_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside the rules stated per entry point */
+    QLORA_ERR_WORKSPACE = 3,         /* workspace pointer null or smaller than required */
+    QLORA_ERR_NONFINITE = 4,         /* device: a weight handed to the quantiser was NaN/Inf */
+    QLORA_ERR_TIMEOUT = 5,           /* device: a bounded wait ran out; outputs undefined */
+    QLORA_ERR_CUDA = 6               /* a CUDA runtime/driver call failed */
+} qlora_status;
+
+typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
+
+/* A cudaStream_t passed through the ABI without the CUDA headers. */
+typedef void *qlora_stream_t;
+
+/*
+ * The stored NF4 + double-quantised tensor (section 2 of the page). n = rows*cols
+ * weights flattened row-major; nb = ceil(n/64) first-level blocks (block b holds
+ * weights 64b .. 64b+63); nb2 = ceil(nb/256) second-level blocks.
+ *   codes   ceil(n/2) bytes; byte k = (code[2k] << 4) | code[2k+1]; for odd n the
+ *           missing low nibble is 7, the zero code;
+ *   scale8  nb int8 first-level constants, linear symmetric about the offset;
+ *   scale2  nb2 fp32 second-level constants (max |c1 - offset| of the group);
+ *   offset  one fp32: the mean of all first-level absmax constants.
+ * All four are device pointers owned by the caller (see qlora_nf4_storage_bytes).
+ */
+typedef struct {
+    int64_t rows, cols;
+    uint8_t *codes;
+    int8_t *scale8;
+    float *scale2;
+    float *offset;
+} qlora_nf4_tensor;
+
+/* Bytes of the four buffers of a [rows, cols] tensor: ceil(n/2) + nb + 4*nb2 + 4.
+ * Returns 0 for rows < 1 or cols < 1. */
+size_t qlora_nf4_storage_bytes(int64_t rows, int64_t cols);
+
+/* Workspace bytes qlora_nf4_quantize needs: nb fp32 exact absmax constants and
+ * nb2 fp64 partial sums of the offset, each region 256-byte aligned. */
+size_t qlora_nf4_quantize_workspace(int64_t rows, int64_t cols);
+
+/*
+ * Quantise W (rows*cols values of dtype dt, row-major) into `out`
+ * (page section 2 and the section 3 order: codes from the exact fp32 absmax,
+ * then the offset, then the 8-bit constants and the second-level constants).
+ *   W    device, 16-byte aligned; any rows, cols >= 1.
+ *   out  host struct whose device buffers receive the result; out->rows/cols
+ *        must equal rows/cols of W.
+ *   ws   device workspace of at least qlora_nf4_quantize_workspace() bytes.
+ * Three kernel launches on `stream`. A NaN/Inf weight sets QLORA_ERR_NONFINITE
+ * in the device status word; the outputs are then undefined.
+ */
+qlora_status qlora_nf4_quantize(const void *W, qlora_dtype dt, const qlora_nf4_tensor *out,
+                                void *ws, size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * Dequantise to bf16 (page section 3, "dequantise to BF16 on demand"):
+ *   step_j = fl(scale2[j] / 127), c^_b = fl(fl(scale8[b] * step_j) + offset),
+ *   W_out[i] = bf16(fl(Q[code_i] * c^_b)).
+ * W_out: device, rows*cols bf16, row-major, 16-byte aligned.
+ */
+qlora_status qlora_nf4_dequant(const qlora_nf4_tensor *q, void *W_out, qlora_stream_t stream);
+
+/*
+ * Forward of the layer (page section 1 equation, with W^ = stored^T):
+ *   Y[M, rows] = X[M, cols] * Dequant(W)^T + s * (X * A) * B
+ *   X  bf16 [M, cols];  A bf16 [cols, r];  B bf16 [r, rows];  Y bf16 [M, rows].
+ *   XA_save  bf16 [M, r] receives X*A (unscaled) for the backward, or NULL.
+ * Shapes: M >= 1, cols % 64 == 0, rows % 16 == 0, 0 <= r <= 256, r % 8 == 0
+ * (r == 0: no adapter; A, B, XA_save ignored). M <= 16 takes the streaming GEMV
+ * kernel, larger M the fused tcgen05 dequant-GEMM.
+ */
+size_t qlora_linear_fwd_workspace(int64_t M, int64_t rows, int64_t cols, int r);
+qlora_status qlora_linear_fwd(const void *X, int64_t M, const qlora_nf4_tensor *W,
+                              const void *A, const void *B, int r, float s,
+                              void *Y, void *XA_save, void *ws, size_t ws_bytes,
+                              qlora_stream_t stream);
+
+/*
+ * Backward of the layer (page section 1: the base weight gets no gradient, the
+ * input gradient flows through W^ transposed; the adapter gets both gradients):
+ *   G  = dY * B^T                          [M, r]
+ *   dX = dY * Dequant(W) + s * G * A^T     bf16 [M, cols]
+ *   dA = s * X^T * G                       fp32 [cols, r]  (overwritten)
+ *   dB = s * (X*A)^T * dY                  fp32 [r, rows]  (overwritten)
+ *   XA  bf16 [M, r] saved by the forward, or NULL to recompute it.
+ * Shapes as for the forward, with M >= 1.
+ */
+size_t qlora_linear_bwd_workspace(int64_t M, int64_t rows, int64_t cols, int r);
+qlora_status qlora_linear_bwd(const void *X, const void *dY, int64_t M, const qlora_nf4_tensor *W,
+                              const void *A, const void *B, int r, float s, const void *XA,
+                              void *dX, float *dA, float *dB, void *ws, size_t ws_bytes,
+                              qlora_stream_t stream);
+
+/* Synchronises `stream`, returns the first condition recorded on the current
+ * device since the last call (QLORA_OK if none) and clears it. */
+qlora_status qlora_get_device_status(qlora_stream_t stream);
+
+/* Static description of a status code. */
+const char *qlora_status_string(qlora_status s);
+
+/* The library's own fp32 NF4 codebook (ascending, Q[7] = +0, Q[0] = -1,
+ * Q[15] = +1), derived on the host from its definition: 8 positive and 7
+ * negative standard-normal quantiles at equally spaced probabilities up to
+ * delta = 1 - (1/32 + 1/30)/2, divided by the quantile at delta (the
+ * construction of Dettmers et al. 2023, which the page summarises). */
+void qlora_nf4_codebook(float out[16]);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_NF4_H */

@@ -273,9 +273,14 @@ def linear_bwd(X, dY, Ws, A, B, s: float):
     X, dY, Ws, A, B = map(_f64, (X, dY, Ws, A, B))
     G = dY @ B.T
     dX = dY @ Ws + s * (G @ A.T)
-    dA = s * (X.T @ G)
-    dB = s * ((X @ A).T @ dY)
+    dA, dB = adapter_grads(X, dY, A, B, s)
     return dX, dA, dB
+
+
+def adapter_grads(X, dY, A, B, s: float):
+    """dA = s X^T (dY B^T), dB = s (X A)^T dY (the adapter half of linear_bwd)."""
+    X, dY, A, B = map(_f64, (X, dY, A, B))
+    return s * (X.T @ (dY @ B.T)), s * ((X @ A).T @ dY)
 
 
 def lora_param_count(d_in: int, d_out: int, r: int) -> int:

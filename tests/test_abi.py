@@ -1,0 +1,100 @@
+"""The C-ABI library loads, exports every declared entry point, and its
+host-side logic (sizes, workspace queries, argument checks, the codebook
+derivation) behaves as declared. No GPU compute is called here."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bit_nf4_quantized_double_b200 as q
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "qlora_nf4.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(qlora_[a-z0-9_]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    L = q.lib()
+    names = declared_functions()
+    assert len(names) >= 11
+    for name in names:
+        assert hasattr(L, name), name
+    # the binding wraps every declared function
+    for name in names:
+        assert name in q._SIGS, name
+
+
+def test_codebook_bit_equal_to_oracle():
+    # the library derives its codebook on the host (Newton on erfc), the
+    # oracle by bisection; the fp32 tables must agree bit for bit
+    lib_q = np.array(q.qlora_nf4_codebook(), dtype=np.float32)
+    assert np.array_equal(lib_q.view(np.uint32), oracle.codebook().view(np.uint32))
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 1), (1, 16384), (512, 256), (4096, 4096), (11008, 4096),
+                                       (3, 16421), (28672, 8192)])
+def test_storage_bytes_match_format(rows, cols):
+    assert q.qlora_nf4_storage_bytes(rows, cols) == oracle.storage_bytes(rows, cols)
+
+
+def test_storage_bytes_invalid():
+    assert q.qlora_nf4_storage_bytes(0, 5) == 0
+    assert q.qlora_nf4_storage_bytes(5, -1) == 0
+
+
+def test_quantize_workspace_size():
+    L = q.lib()
+    n, _, nb, nb2 = q.nf4_sizes(4096, 4096)
+    ws = L.qlora_nf4_quantize_workspace(4096, 4096)
+    assert ws >= nb * 4 + nb2 * 8
+    assert L.qlora_nf4_quantize_workspace(0, 1) == 0
+
+
+def test_workspace_queries_positive():
+    L = q.lib()
+    for M in (1, 16, 17, 4096):
+        assert L.qlora_linear_fwd_workspace(M, 4096, 4096, 64) > 0
+        assert L.qlora_linear_bwd_workspace(M, 4096, 4096, 64) > 0
+    assert L.qlora_linear_bwd_workspace(4096, 4096, 4096, 0) == 0
+
+
+def test_status_strings():
+    for s in range(7):
+        assert len(q.status_string(s)) > 0
+    assert q.status_string(99) == "unknown status"
+
+
+def test_argument_checks_run_on_host():
+    # null and misaligned pointers, bad shapes and a missing workspace are
+    # rejected before any launch, so these calls need no GPU
+    L = q.lib()
+    t = q._Tensor(64, 64, 0, 0, 0, 0)
+    assert L.qlora_nf4_quantize(None, 0, ctypes.byref(t), None, 0, None) == q.QLORA_ERR_INVALID_ARG
+    assert L.qlora_nf4_dequant(ctypes.byref(t), None, None) == q.QLORA_ERR_INVALID_ARG
+    fake = 1 << 20   # never dereferenced: validation fails first
+    good = q._Tensor(64, 64, fake, fake, fake, fake)
+    assert L.qlora_nf4_quantize(ctypes.c_void_p(fake), 7, ctypes.byref(good), None, 0, None) == q.QLORA_ERR_INVALID_ARG
+    assert L.qlora_nf4_quantize(ctypes.c_void_p(fake + 4), 0, ctypes.byref(good), None, 0, None) == q.QLORA_ERR_INVALID_ARG
+    assert L.qlora_nf4_quantize(ctypes.c_void_p(fake), 0, ctypes.byref(good), None, 0, None) == q.QLORA_ERR_WORKSPACE
+    bad_cols = q._Tensor(64, 100, fake, fake, fake, fake)
+    assert L.qlora_linear_fwd(ctypes.c_void_p(fake), 4, ctypes.byref(bad_cols), None, None, 0, 1.0,
+                              ctypes.c_void_p(fake), None, None, 0, None) == q.QLORA_ERR_UNSUPPORTED_SHAPE
+    assert L.qlora_linear_fwd(ctypes.c_void_p(fake), 4, ctypes.byref(good), ctypes.c_void_p(fake),
+                              ctypes.c_void_p(fake), 12, 1.0, ctypes.c_void_p(fake), None, None, 0,
+                              None) == q.QLORA_ERR_UNSUPPORTED_SHAPE          # r % 8 != 0
+    assert L.qlora_linear_fwd(ctypes.c_void_p(fake), 4, ctypes.byref(good), ctypes.c_void_p(fake),
+                              ctypes.c_void_p(fake), 16, float("nan"), ctypes.c_void_p(fake), None, None, 0,
+                              None) == q.QLORA_ERR_INVALID_ARG                # non-finite scale
+    assert L.qlora_linear_fwd(ctypes.c_void_p(fake), 4, ctypes.byref(good), ctypes.c_void_p(fake),
+                              ctypes.c_void_p(fake), 16, 1.0, ctypes.c_void_p(fake), None, None, 0,
+                              None) == q.QLORA_ERR_WORKSPACE
+    assert L.qlora_linear_bwd(None, ctypes.c_void_p(fake), 0, ctypes.byref(good), None, None, 0, 1.0, None,
+                              ctypes.c_void_p(fake), None, None, None, 0, None) == q.QLORA_ERR_UNSUPPORTED_SHAPE

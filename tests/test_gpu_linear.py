@@ -1,0 +1,184 @@
+"""GPU parity of the QLoRA linear forward and backward against the fp64 oracle.
+
+Tolerance (stated for the layer): for each of Y, dX, dA, dB separately,
+max|err| / max|ref| <= 2e-2 and ||err||_F / ||ref||_F <= 5e-3, where the
+reference is the exact (fp64) product of the same bf16 operands and the
+oracle's bf16 dequantised weight."""
+import numpy as np
+import pytest
+import torch
+
+import bit_nf4_quantized_double_b200 as q
+import oracle
+import synth_inputs as si
+
+pytestmark = pytest.mark.gpu
+
+MAX_TOL = 2e-2
+FRO_TOL = 5e-3
+
+
+def f64(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def check(got, ref, name):
+    m, f = oracle.rel_errors(got, ref)
+    assert m <= MAX_TOL and f <= FRO_TOL, f"{name}: max-rel {m:.3e}, fro-rel {f:.3e}"
+
+
+def make_problem(M, rows, cols, r, seed, w_std=0.02, a_std=0.02, b_std=0.02, outliers=0.0):
+    L = si.Layer("p", rows, cols, w_std, r=r, alpha=2.0 * r if r else 0.0, a_std=a_std, b_std=b_std,
+                 outlier_frac=outliers)
+    W = si.weight(L, seed, device="cuda")
+    X = si.normal((M, cols), 1.0, seed + 1, device="cuda", dtype=torch.bfloat16)
+    dY = si.normal((M, rows), 1.0, seed + 2, device="cuda", dtype=torch.bfloat16)
+    A = si.normal((cols, r), a_std, seed + 3, device="cuda", dtype=torch.bfloat16) if r else None
+    B = si.normal((r, rows), b_std, seed + 4, device="cuda", dtype=torch.bfloat16) if r else None
+    return W, X, dY, A, B, (L.s if r else 0.0)
+
+
+def oracle_weight(W):
+    ref = oracle.quantize(W.float().cpu().numpy())
+    return oracle.bf16_bits_to_f32(oracle.dequant(ref)).reshape(W.shape).astype(np.float64)
+
+
+def run_case(M, rows, cols, r, seed, do_bwd=True, sample_rows=None, **kw):
+    W, X, dY, A, B, s = make_problem(M, rows, cols, r, seed, **kw)
+    t = q.qlora_nf4_quantize(W)
+    Y, XA = q.qlora_linear_fwd(X, t, A, B, s)
+    if do_bwd:
+        dX, dA, dB = q.qlora_linear_bwd(X, dY, t, A, B, s, XA=XA)
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    Wh = oracle_weight(W)
+    Xn, dYn = f64(X), f64(dY)
+    An = f64(A) if r else np.zeros((cols, 0))
+    Bn = f64(B) if r else np.zeros((0, rows))
+    idx = np.arange(M) if sample_rows is None else sample_rows
+    Yref = oracle.linear_fwd(Xn[idx], Wh, An, Bn, s)
+    check(f64(Y)[idx], Yref, "Y")
+    if r:
+        check(f64(XA)[idx], Xn[idx] @ An, "XA")
+    if do_bwd:
+        if sample_rows is None:
+            dXr, dAr, dBr = oracle.linear_bwd(Xn, dYn, Wh, An, Bn, s)
+        else:
+            dXr, _, _ = oracle.linear_bwd(Xn[idx], dYn[idx], Wh, An, Bn, s)
+            dAr, dBr = oracle.adapter_grads(Xn, dYn, An, Bn, s)
+        check(f64(dX)[idx], dXr, "dX")
+        if r:
+            check(f64(dA), dAr, "dA")
+            check(f64(dB), dBr, "dB")
+    return Y
+
+
+def test_tiny_layer():
+    # 256 -> 512, 32 tokens, rank 8, alpha 16
+    wl = si.workload("tiny")
+    inp = si.layer_inputs(wl, 0, device="cuda")
+    L = wl.layers[0]
+    t = q.qlora_nf4_quantize(inp["W"])
+    Y, XA = q.qlora_linear_fwd(inp["X"], t, inp["A"], inp["B"], L.s)
+    dX, dA, dB = q.qlora_linear_bwd(inp["X"], inp["dY"], t, inp["A"], inp["B"], L.s, XA=XA)
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    Wh = oracle_weight(inp["W"])
+    Xn, dYn, An, Bn = (f64(inp[k]) for k in ("X", "dY", "A", "B"))
+    check(f64(Y), oracle.linear_fwd(Xn, Wh, An, Bn, L.s), "Y")
+    dXr, dAr, dBr = oracle.linear_bwd(Xn, dYn, Wh, An, Bn, L.s)
+    check(f64(dX), dXr, "dX")
+    check(f64(dA), dAr, "dA")
+    check(f64(dB), dBr, "dB")
+
+
+@pytest.mark.parametrize("M,rows,cols,r", [
+    (300, 400, 320, 24),     # several tiles in every dimension, ragged tails, r % 16 != 0
+    (300, 400, 320, 0),      # no adapter
+    (257, 272, 192, 64),
+    (520, 384, 640, 128),    # two adapter K blocks
+    (17, 128, 128, 16),      # just above the small-M path
+    (1000, 1024, 1088, 8),
+])
+def test_multi_tile_ragged(M, rows, cols, r):
+    run_case(M, rows, cols, r, seed=M + rows + cols + r)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+@pytest.mark.parametrize("r", [0, 16])
+def test_small_m_gemv(M, r):
+    run_case(M, 1024, 2048 + 64, r, seed=100 + M + r)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_layer_full(M):
+    # one Llama-7B-shaped block at decode sizes, forward only (rank 16 on q, k, v, o)
+    wl = si.workload("decode7b", M=M)
+    for li, L in enumerate(wl.layers):
+        inp = si.layer_inputs(wl, li, device="cuda")
+        t = q.qlora_nf4_quantize(inp["W"])
+        Y, _ = q.qlora_linear_fwd(inp["X"], t, inp.get("A"), inp.get("B"), L.s)
+        assert q.qlora_get_device_status() == q.QLORA_OK
+        Wh = oracle_weight(inp["W"])
+        An = f64(inp["A"]) if L.r else np.zeros((L.d_in, 0))
+        Bn = f64(inp["B"]) if L.r else np.zeros((0, L.d_out))
+        check(f64(Y), oracle.linear_fwd(f64(inp["X"]), Wh, An, Bn, L.s), f"Y[{L.name}]")
+
+
+def test_full_4096_layer_sampled():
+    # the 4096 x 4096 layer at 4096 tokens, rank 64, in the bench's launch configuration
+    M = 4096
+    rows_idx = np.unique(np.concatenate([[0, 1, 255, 256, M - 1], np.random.default_rng(0).integers(0, M, 60)]))
+    wl = si.workload("l4096")
+    inp = si.layer_inputs(wl, 0, device="cuda")
+    L = wl.layers[0]
+    t = q.qlora_nf4_quantize(inp["W"])
+    Y, XA = q.qlora_linear_fwd(inp["X"], t, inp["A"], inp["B"], L.s)
+    dX, dA, dB = q.qlora_linear_bwd(inp["X"], inp["dY"], t, inp["A"], inp["B"], L.s, XA=XA)
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    Wh = oracle_weight(inp["W"])
+    Xn, dYn, An, Bn = (f64(inp[k]) for k in ("X", "dY", "A", "B"))
+    check(f64(Y)[rows_idx], oracle.linear_fwd(Xn[rows_idx], Wh, An, Bn, L.s), "Y")
+    dXr, _, _ = oracle.linear_bwd(Xn[rows_idx], dYn[rows_idx], Wh, An, Bn, L.s)
+    check(f64(dX)[rows_idx], dXr, "dX")
+    dAr, dBr = oracle.adapter_grads(Xn, dYn, An, Bn, L.s)
+    check(f64(dA), dAr, "dA")
+    check(f64(dB), dBr, "dB")
+
+
+def test_70b_projections_sampled():
+    # two projections of the 70B-like block at 4096 tokens: the skinny-N k projection
+    # and the long-K down projection
+    wl = si.workload("l70b")
+    M = 4096
+    rows_idx = np.array([0, 1, 1000, 2047, 2048, 4095])
+    for name in ("k", "down"):
+        li = [l.name for l in wl.layers].index(name)
+        L = wl.layers[li]
+        inp = si.layer_inputs(wl, li, device="cuda")
+        t = q.qlora_nf4_quantize(inp["W"])
+        Y, XA = q.qlora_linear_fwd(inp["X"], t, inp["A"], inp["B"], L.s)
+        dX, dA, dB = q.qlora_linear_bwd(inp["X"], inp["dY"], t, inp["A"], inp["B"], L.s, XA=XA)
+        assert q.qlora_get_device_status() == q.QLORA_OK
+        Wh = oracle_weight(inp["W"])
+        Xn, dYn, An, Bn = (f64(inp[k]) for k in ("X", "dY", "A", "B"))
+        check(f64(Y)[rows_idx], oracle.linear_fwd(Xn[rows_idx], Wh, An, Bn, L.s), f"Y[{name}]")
+        dXr, _, _ = oracle.linear_bwd(Xn[rows_idx], dYn[rows_idx], Wh, An, Bn, L.s)
+        check(f64(dX)[rows_idx], dXr, f"dX[{name}]")
+        dAr, dBr = oracle.adapter_grads(Xn, dYn, An, Bn, L.s)
+        check(f64(dA), dAr, f"dA[{name}]")
+        check(f64(dB), dBr, f"dB[{name}]")
+        del inp, t, Y, XA, dX, dA, dB, Wh, Xn, dYn
+        torch.cuda.empty_cache()
+
+
+def test_zero_adapter_equals_plain_product():
+    # B = 0 (or s = 0) leaves the plain dequantised product, checked against
+    # torch.matmul on the dequantised weight
+    W, X, dY, A, B, s = make_problem(384, 256, 512, 16, seed=77)
+    t = q.qlora_nf4_quantize(W)
+    Wh = q.qlora_nf4_dequant(t)
+    Y0, _ = q.qlora_linear_fwd(X, t, A, torch.zeros_like(B), s)
+    Y1, _ = q.qlora_linear_fwd(X, t, A, B, 0.0)
+    ref = torch.matmul(X.double(), Wh.double().T)
+    for Y in (Y0, Y1):
+        m, f = oracle.rel_errors(f64(Y), ref.cpu().numpy())
+        assert m <= MAX_TOL and f <= FRO_TOL
