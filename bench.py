@@ -1,0 +1,520 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA NF4 + double-quant linear layer on B200.
+
+Headline: forward + backward of one 4096 x 4096 QLoRA linear at M = 4096
+tokens, rank 64, alpha 128 (s = 2), W ~ N(0, 0.02) with 0.1 % outliers x 10,
+X and dY ~ N(0, 1) in bf16 -- in TFLOP/s of algorithmic work
+    4 M d_in d_out + 6 M r (d_in + d_out)  per step.
+A step = one qlora_linear_fwd + one qlora_linear_bwd (the frozen weight is
+quantised once, before timing, as in training). With --gpus N > 1 each rank
+runs the same step on its own batch (weak scaling) and the adapter gradients
+dA, dB are summed over ranks with NCCL, the data-parallel exchange.
+
+Also reported ("components", rank 0 at N = 1): the quantise and dequantise
+sweep over 32 Llama-7B-shaped layers (HBM GB/s) and the decode-sized NF4
+GEMV over one Llama-7B block at M in {1, 4, 16} (HBM GB/s).
+
+--impl reference times the CPU oracle (plain C + numpy fp64) on a bounded
+sample of the same workload; it is the reference arm of this repository.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s at M=4096; NF4 GEMV/dequant HBM GB/s"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20        # 2x the 126 MB L2
+
+
+def step_flops(M, d_in, d_out, r):
+    return 4.0 * M * d_in * d_out + 6.0 * M * r * (d_in + d_out)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        loaded = [v for v in sm if mx and v > 0.3 * max(mx)] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def allreduce_adapter_grads(dA, dB, world):
+    """Data-parallel exchange of the adapter gradients (sum over ranks)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(dA)
+        dist.all_reduce(dB)
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    import torch
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ our arm
+def headline_inputs(rank):
+    import synth_inputs as si
+    wl = si.workload("l4096")
+    L = wl.layers[0]
+    inp = si.layer_inputs(wl, 0, device="cuda", w_device="cuda")
+    if rank:
+        # weak scaling: every rank its own batch of tokens
+        inp["X"] = si.normal((wl.M, L.d_in), 1.0, si.seed_of(wl, 0, "X") + 7777 * rank, device="cuda",
+                             dtype=inp["X"].dtype)
+        inp["dY"] = si.normal((wl.M, L.d_out), 1.0, si.seed_of(wl, 0, "dY") + 7777 * rank, device="cuda",
+                              dtype=inp["dY"].dtype)
+    return wl, L, inp
+
+
+def run_ours(args, peaks, peak_kind):
+    import torch
+    import bit_nf4_quantized_double_b200 as q
+
+    world, rank, local = dist_setup(args)
+    wl, L, inp = headline_inputs(rank)
+    M, d_in, d_out, r, s = wl.M, L.d_in, L.d_out, L.r, L.s
+    dev = inp["X"].device
+    t = q.qlora_nf4_quantize(inp["W"])
+    del inp["W"]
+    X, dY, A, B = inp["X"], inp["dY"], inp["A"], inp["B"]
+    Y = torch.empty(M, d_out, dtype=torch.bfloat16, device=dev)
+    XA = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(M, d_in, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(d_in, r, dtype=torch.float32, device=dev)
+    dB = torch.empty(r, d_out, dtype=torch.float32, device=dev)
+    Lb = q.lib()
+    ws_f = torch.empty(max(1, Lb.qlora_linear_fwd_workspace(M, d_out, d_in, r)), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(max(1, Lb.qlora_linear_bwd_workspace(M, d_out, d_in, r)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        q.qlora_linear_fwd(X, t, A, B, s, Y=Y, XA_save=XA, ws=ws_f)
+        q.qlora_linear_bwd(X, dY, t, A, B, s, XA=XA, dX=dX, dA=dA, dB=dB, ws=ws_b)
+        allreduce_adapter_grads(dA, dB, world)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = q.qlora_get_device_status()
+    if status != q.QLORA_OK:
+        raise RuntimeError(f"device status {status} during warm-up")
+
+    stream = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = q.qlora_launch_count()
+    q.qlora_profile_enable(True)
+    for i in range(args.steps):
+        flush.zero_()                     # L2 flush between timed steps (not timed)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    q.qlora_profile_enable(False)
+    launches = q.qlora_launch_count() - launches0
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    total_ms = sum(a.elapsed_time(b) for a, b in evs)
+    total_ms = max_over_ranks(total_ms, world)
+    kern = {}
+    for name in ("k_fused_fwd", "k_fused_dgrad", "k_skinny", "k_reduce_xa", "k_reduce_f32", "k_reduce_f32_t"):
+        kern[name] = q.qlora_profile_read(name)
+    q.qlora_profile_read(None)
+    status = q.qlora_get_device_status()
+    if status != q.QLORA_OK:
+        raise RuntimeError(f"device status {status} during timing")
+
+    flops = step_flops(M, d_in, d_out, r)
+    value = world * args.steps * flops / (total_ms / 1e3) / 1e12
+    # dominant kernel: the fused forward or the fused dgrad, whichever took longer
+    dom = max(("k_fused_fwd", "k_fused_dgrad"), key=lambda k: kern[k][0])
+    dom_flops = 2.0 * M * d_in * d_out + 2.0 * M * r * (d_out if dom == "k_fused_fwd" else d_in)
+    dom_ms, dom_n = kern[dom]
+    achieved = dom_flops / (dom_ms / dom_n / 1e3) / 1e12 if dom_n else None
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+
+    # ---------------------------------------------------------------- e2e
+    Xh = X.cpu().pin_memory()
+    dYh = dY.cpu().pin_memory()
+    dAh = torch.empty(dA.shape, dtype=dA.dtype).pin_memory()
+    dBh = torch.empty(dB.shape, dtype=dB.dtype).pin_memory()
+
+    def e2e_step():
+        X.copy_(Xh, non_blocking=True)
+        dY.copy_(dYh, non_blocking=True)
+        step()
+        dAh.copy_(dA, non_blocking=True)
+        dBh.copy_(dB, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    for i in range(args.steps):
+        flush.zero_()
+        eev[i][0].record(stream)
+        e2e_step()
+        eev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eev), world)
+    e2e = {"value": world * args.steps * flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+           "h2d_bytes_per_step": X.numel() * 2 + dY.numel() * 2,
+           "d2h_bytes_per_step": dA.numel() * 4 + dB.numel() * 4}
+
+    components = None
+    if world == 1 and not args.no_components:
+        del Xh, dYh
+        components = run_components(args, peaks, peak_kind, flush)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(M_sample=args.cpu_sample_tokens)
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, generated on device)",
+        "config": {"workload": "QLoRA linear 4096x4096 (d_in=d_out=4096), M=4096 tokens, r=64, alpha=128 (s=2), "
+                               "W ~ N(0,0.02) fp32 with 0.1% x10 outliers quantised once to NF4+DQ, "
+                               "X,dY ~ N(0,1) bf16; step = fwd + bwd" + (" + NCCL all-reduce of dA,dB"
+                                                                       if world > 1 else ""),
+                   "global_batch_tokens": M * world, "l2": "flushed between timed steps (256 MB write)",
+                   "flops_per_step": flops, "parallelism": f"dp{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2) if achieved else None,
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4) if achieved else None,
+                     "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                     else "fallback 1590 TFLOP/s",
+                     "traffic": None, "flops_per_launch": dom_flops, "launches": dom_n,
+                     "kernel_ms": {k: round(v[0] / max(v[1], 1), 5) for k, v in kern.items()}},
+        "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+    }
+    if components is not None:
+        line["components"] = components
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _time_graph(fn, reps, flush, stream):
+    """Capture fn in a CUDA graph, replay it reps times with an L2 flush before
+    each replay; return the average device milliseconds of one replay."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    for _ in range(2):
+        g.replay()
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(torch.cuda.current_stream())
+        g.replay()
+        b.record(torch.cuda.current_stream())
+        times.append((a, b))
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in times) / reps
+    del g
+    return ms
+
+
+def run_components(args, peaks, peak_kind, flush):
+    import torch
+    import bit_nf4_quantized_double_b200 as q
+    import synth_inputs as si
+
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    out = {"hbm_peak_gbs": hbm, "hbm_peak_source": peak_kind}
+    stream = torch.cuda.current_stream()
+
+    # --- quantise / dequantise sweep over 32 Llama-7B-shaped layers (bf16 weights)
+    n_layers = args.sweep_layers
+    wl = si.workload("llama7b", n_layers=n_layers)
+    Ws, Ts = [], []
+    for li in range(len(wl.layers)):
+        W = si.layer_inputs(wl, li, device="cuda")["W"]
+        Ws.append(W)
+        Ts.append(q.nf4_empty(W.shape[0], W.shape[1]))
+    n_w = sum(W.numel() for W in Ws)
+    maxn = max(W.numel() for W in Ws)
+    wq_ws = torch.empty(q.lib().qlora_nf4_quantize_workspace(1, maxn), dtype=torch.uint8, device="cuda")
+    wh = torch.empty(maxn, dtype=torch.bfloat16, device="cuda")
+    alg_bytes = 2.0 + 0.5 + 1.0 / 64 + 4.0 / 16384       # per weight, bf16 in/out
+
+    def quant_sweep():
+        for W, T in zip(Ws, Ts):
+            q.qlora_nf4_quantize(W, out=T, ws=wq_ws)
+
+    def deq_sweep():
+        for T in Ts:
+            q.qlora_nf4_dequant(T, out=wh[: T.rows * T.cols].view(T.rows, T.cols))
+
+    res = {}
+    for name, fn in (("quantize", quant_sweep), ("dequant", deq_sweep)):
+        fn()
+        torch.cuda.synchronize()
+        q.qlora_profile_enable(True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        q.qlora_profile_enable(False)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        kname = "k_quantize_codes" if name == "quantize" else "k_dequant"
+        kms, kn = q.qlora_profile_read(kname)
+        q.qlora_profile_read(None)
+        gbs = n_w * alg_bytes / (ms / 1e3) / 1e9
+        kgbs = n_w * alg_bytes / (kms / reps / 1e3) / 1e9 if kn else None
+        res[name] = {"workload": f"{n_layers} Llama-7B layers x 7 projections, {n_w} bf16 weights",
+                     "ms_per_sweep": round(ms, 4), "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                     "kernel": kname, "kernel_GB/s": round(kgbs, 1) if kgbs else None,
+                     "kernel_frac": round(kgbs / hbm, 4) if kgbs else None,
+                     "bytes_per_weight": round(alg_bytes, 5), "launches": kn}
+    out["llama7b_sweep"] = res
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    del Ws, Ts, wh, wq_ws
+    torch.cuda.empty_cache()
+
+    # --- decode GEMV: one Llama-7B block at M in {1, 4, 16}, forward only
+    gem = {}
+    for M in (1, 4, 16):
+        wl = si.workload("decode7b", M=M)
+        items = []
+        nbytes = 0
+        for li, L in enumerate(wl.layers):
+            inp = si.layer_inputs(wl, li, device="cuda")
+            T = q.qlora_nf4_quantize(inp["W"])
+            Y = torch.empty(M, L.d_out, dtype=torch.bfloat16, device="cuda")
+            ws = torch.empty(max(1, q.lib().qlora_linear_fwd_workspace(M, L.d_out, L.d_in, L.r)),
+                             dtype=torch.uint8, device="cuda")
+            items.append((inp["X"], T, inp.get("A"), inp.get("B"), L.s, Y, ws))
+            nbytes += T.nbytes + inp["X"].numel() * 2 + Y.numel() * 2
+            if L.r:
+                nbytes += inp["A"].numel() * 2 + inp["B"].numel() * 2
+            del inp
+
+        def layer():
+            for X, T, A, B, s, Y, ws in items:
+                q.qlora_linear_fwd(X, T, A, B, s, Y=Y, XA_save=False, ws=ws)
+
+        ms = _time_graph(layer, 20, flush, stream)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        gem[f"M{M}"] = {"ms_per_layer": round(ms, 5), "bytes": nbytes, "GB/s": round(gbs, 1),
+                        "frac": round(gbs / hbm, 4)}
+        del items
+        torch.cuda.empty_cache()
+    out["decode7b_gemv"] = {"workload": "one Llama-7B block (q,k,v,o 4096x4096; gate,up 11008x4096; "
+                                        "down 4096x11008), r=16 on q,k,v,o, fwd only, CUDA graph replay, "
+                                        "L2 flushed", **gem}
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    return out
+
+
+# ------------------------------------------------------------------ CPU oracle
+def _oracle_problem(M_sample):
+    import numpy as np
+    import torch
+    import oracle
+    import synth_inputs as si
+    wl = si.workload("l4096")
+    L = wl.layers[0]
+    inp = si.layer_inputs(wl, 0, device="cpu")
+    ref = oracle.quantize(inp["W"].numpy())
+    f64 = lambda t: t.to(torch.float64).numpy()
+    return (wl, L, ref, f64(inp["X"][:M_sample]), f64(inp["dY"][:M_sample]), f64(inp["A"]), f64(inp["B"]))
+
+
+def _oracle_step(L, ref, X, dY, A, B):
+    import oracle
+    Wh = oracle.bf16_bits_to_f32(oracle.dequant(ref)).reshape(L.d_out, L.d_in).astype("float64")
+    Y = oracle.linear_fwd(X, Wh, A, B, L.s)
+    dX, dA, dB = oracle.linear_bwd(X, dY, Wh, A, B, L.s)
+    return Y, dX, dA, dB
+
+
+def _cores():
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        blas = os.cpu_count()
+    return max(oracle.threads(), blas)
+
+
+def cpu_baseline(M_sample=512, target_s=10.0):
+    wl, L, ref, X, dY, A, B = _oracle_problem(M_sample)
+    t0 = time.perf_counter()
+    _oracle_step(L, ref, X, dY, A, B)
+    one = time.perf_counter() - t0
+    reps = max(1, min(20, int(target_s / max(one, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        _oracle_step(L, ref, X, dY, A, B)
+    el = time.perf_counter() - t0
+    flops = step_flops(M_sample, L.d_in, L.d_out, L.r)
+    return {"value": round(reps * flops / el / 1e12, 6), "unit": UNIT, "cores": _cores(), "kind": "oracle",
+            "sample": f"{M_sample} of the 4096 tokens, full 4096x4096 weight: oracle dequant (C) + fp64 "
+                      f"fwd + bwd products (numpy), {reps} steps, {el:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl, L, ref, X, dY, A, B = _oracle_problem(args.cpu_sample_tokens)
+    for _ in range(args.warmup):
+        _oracle_step(L, ref, X, dY, A, B)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(L, ref, X, dY, A, B)
+    el = time.perf_counter() - t0
+    flops = step_flops(args.cpu_sample_tokens, L.d_in, L.d_out, L.r)
+    value = args.steps * flops / el / 1e12
+    sample = (f"{args.cpu_sample_tokens} of the 4096 tokens per step, full 4096x4096 weight: oracle dequant (C) "
+              f"+ fp64 fwd + bwd products (numpy)")
+    n = int(os.environ.get("WORLD_SIZE", "1"))
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": n,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)",
+            "config": {"workload": "QLoRA linear 4096x4096, M=4096 tokens, r=64, alpha=128 (s=2); bounded sample "
+                                   "per step", "sample_tokens": args.cpu_sample_tokens},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": _cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-components", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep-layers", type=int, default=32)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=512)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    peaks, kind = load_peaks()
+    run_ours(args, peaks, kind)
+
+
+if __name__ == "__main__":
+    main()

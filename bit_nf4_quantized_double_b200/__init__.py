@@ -65,6 +65,10 @@ _SIGS = {
     "qlora_get_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_nf4_codebook": (None, [ctypes.c_void_p]),
+    "qlora_launch_count": (ctypes.c_ulonglong, []),
+    "qlora_profile_enable": (None, [ctypes.c_int]),
+    "qlora_profile_read": (ctypes.c_int, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
+                                          ctypes.POINTER(ctypes.c_int)]),
 }
 
 
@@ -224,3 +228,20 @@ def qlora_linear_bwd(X: torch.Tensor, dY: torch.Tensor, W: NF4Tensor, A: torch.T
 
 def qlora_get_device_status(stream=None) -> int:
     return int(lib().qlora_get_device_status(_stream(stream)))
+
+
+def qlora_launch_count() -> int:
+    return int(lib().qlora_launch_count())
+
+
+def qlora_profile_enable(on: bool = True) -> None:
+    lib().qlora_profile_enable(1 if on else 0)
+
+
+def qlora_profile_read(kernel: str | None = None):
+    """(total milliseconds, launches) of the recorded launches of `kernel` (None: all)."""
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_int(0)
+    _check(lib().qlora_profile_read(kernel.encode() if kernel else None, ctypes.byref(ms), ctypes.byref(n)),
+           "qlora_profile_read")
+    return float(ms.value), int(n.value)

@@ -73,4 +73,16 @@ inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 const Codebook &host_codebook();
 int num_sms();
+// Launch bookkeeping (profile.cu): counts every launch and, when profiling is
+// enabled, brackets it with CUDA events on its stream.
+void note_launch_begin(const char *name, cudaStream_t st, void **token);
+void note_launch_end(void *token, cudaStream_t st);
 }  // namespace qnf4
+
+#define QNF4_LAUNCH(name, st, ...)                         \
+    do {                                                   \
+        void *qnf4_tok_ = nullptr;                         \
+        ::qnf4::note_launch_begin(name, st, &qnf4_tok_);   \
+        __VA_ARGS__;                                       \
+        ::qnf4::note_launch_end(qnf4_tok_, st);            \
+    } while (0)

@@ -788,7 +788,7 @@ static cudaError_t run_skinny(bool a_mn, const void *a, int64_t a_ld_rows, bool 
 #define QNF4_SK(AM, BM)                                                      \
     e = set_smem(k_skinny<AM, BM>, smem);                                    \
     if (e != cudaSuccess) return e;                                          \
-    k_skinny<AM, BM><<<grid, 128, smem, st>>>(ta, tb, p);
+    QNF4_LAUNCH("k_skinny", st, k_skinny<AM, BM><<<grid, 128, smem, st>>>(ta, tb, p));
     if (a_mn && b_mn) { QNF4_SK(true, true) }
     else if (a_mn) { QNF4_SK(true, false) }
     else if (b_mn) { QNF4_SK(false, true) }
@@ -821,7 +821,7 @@ cudaError_t launch_xa_small(const __nv_bfloat16 *X, int64_t M, int64_t cols, con
     float *part = static_cast<float *>(part_ws);
     cudaError_t e = run_skinny(false, X, M, true, A, M, cols, r, part, &splits, st);
     if (e != cudaSuccess) return e;
-    k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, XA_save, XAs);
+    QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, XA_save, XAs));
     return cudaGetLastError();
 }
 
@@ -860,7 +860,7 @@ static cudaError_t run_fused_fwd(const __nv_bfloat16 *X, int64_t M, const NF4Vie
     const int grid = ntiles < num_sms() ? ntiles : num_sms();
     cudaError_t e = set_smem(k_fused_fwd, fwd::kSmem);
     if (e != cudaSuccess) return e;
-    k_fused_fwd<<<grid, fwd::kThreads, fwd::kSmem, st>>>(tx, tc_, txa, ty, p, host_codebook());
+    QNF4_LAUNCH("k_fused_fwd", st, k_fused_fwd<<<grid, fwd::kThreads, fwd::kSmem, st>>>(tx, tc_, txa, ty, p, host_codebook()));
     return cudaGetLastError();
 }
 
@@ -892,7 +892,7 @@ static cudaError_t run_fused_dgrad(const __nv_bfloat16 *dY, int64_t M, const NF4
     const int grid = ntiles < num_sms() ? ntiles : num_sms();
     cudaError_t e = set_smem(k_fused_dgrad, dg::kSmem);
     if (e != cudaSuccess) return e;
-    k_fused_dgrad<<<grid, dg::kThreads, dg::kSmem, st>>>(tdy, tc_, ta, tg, tdx, p, host_codebook());
+    QNF4_LAUNCH("k_fused_dgrad", st, k_fused_dgrad<<<grid, dg::kThreads, dg::kSmem, st>>>(tdy, tc_, ta, tg, tdx, p, host_codebook()));
     return cudaGetLastError();
 }
 
@@ -906,7 +906,7 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
         int splits = 0;
         cudaError_t e = run_skinny(false, X, M, true, A, M, W.cols, r, part, &splits, st);
         if (e != cudaSuccess) return e;
-        k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, XA_save, XAs);
+        QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, XA_save, XAs));
     }
     return run_fused_fwd(X, M, W, XAs, B, r, Y, st);
 }
@@ -925,13 +925,13 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
         if (!XA) {
             e = run_skinny(false, X, M, true, A, M, W.cols, r, part, &splits, st);
             if (e != cudaSuccess) return e;
-            k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, 1.0f, XAbuf, nullptr);
+            QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, 1.0f, XAbuf, nullptr));
             XA = XAbuf;
         }
         // G = dY B^T -> sG (bf16)
         e = run_skinny(false, dY, M, false, B, M, W.rows, r, part, &splits, st);
         if (e != cudaSuccess) return e;
-        k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, nullptr, Gs);
+        QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, nullptr, Gs));
     }
     e = run_fused_dgrad(dY, M, W, A, Gs, r, dX, st);
     if (e != cudaSuccess) return e;
@@ -941,11 +941,11 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
         // dA = X^T (sG)
         e = run_skinny(true, X, M, true, Gs, W.cols, M, r, part, &splits, st);
         if (e != cudaSuccess) return e;
-        k_reduce_f32<<<reduce_grid(W.cols * r), 256, 0, st>>>(part, splits, W.cols * r, 1.0f, dA);
+        QNF4_LAUNCH("k_reduce_f32", st, k_reduce_f32<<<reduce_grid(W.cols * r), 256, 0, st>>>(part, splits, W.cols * r, 1.0f, dA));
         // dB = s (XA)^T dY, computed as (dY^T XA)^T
         e = run_skinny(true, dY, M, true, XA, W.rows, M, r, part, &splits, st);
         if (e != cudaSuccess) return e;
-        k_reduce_f32_t<<<reduce_grid(W.rows * r), 256, 0, st>>>(part, splits, W.rows, r, s, dB);
+        QNF4_LAUNCH("k_reduce_f32_t", st, k_reduce_f32_t<<<reduce_grid(W.rows * r), 256, 0, st>>>(part, splits, W.rows, r, s, dB));
     }
     return cudaGetLastError();
 }

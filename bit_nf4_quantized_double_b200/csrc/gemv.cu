@@ -211,17 +211,17 @@ cudaError_t launch_linear_fwd(const __nv_bfloat16 *X, int64_t M, const NF4View &
         const size_t sm = gemv_smem(1);
         e = cudaFuncSetAttribute(k_gemv<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
-        k_gemv<1><<<grid, 256, sm, st>>>(W, X, (int)M, host_codebook(), partial);
+        QNF4_LAUNCH("k_gemv", st, k_gemv<1><<<grid, 256, sm, st>>>(W, X, (int)M, host_codebook(), partial));
     } else {
         const size_t sm = gemv_smem(2);
         e = cudaFuncSetAttribute(k_gemv<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
-        k_gemv<2><<<grid, 256, sm, st>>>(W, X, (int)M, host_codebook(), partial);
+        QNF4_LAUNCH("k_gemv", st, k_gemv<2><<<grid, 256, sm, st>>>(W, X, (int)M, host_codebook(), partial));
     }
     const int64_t count = M * W.rows;
     int64_t g = ceil_div(count, 256);
     if (g > (int64_t)num_sms() * 8) g = (int64_t)num_sms() * 8;
-    k_gemv_finish<<<(unsigned)g, 256, 0, st>>>(partial, splits, (int)M, (int)W.rows, XAs, B, r, Y);
+    QNF4_LAUNCH("k_gemv_finish", st, k_gemv_finish<<<(unsigned)g, 256, 0, st>>>(partial, splits, (int)M, (int)W.rows, XAs, B, r, Y));
     return cudaGetLastError();
 }
 

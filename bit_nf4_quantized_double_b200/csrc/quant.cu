@@ -264,11 +264,11 @@ cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlor
     const int64_t nb = ceil_div(n, kBlock1), nb2 = ceil_div(nb, kBlock2);
     const Codebook &cb = host_codebook();
     if (dt == QLORA_F32)
-        k_quantize_codes<float><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const float *>(W), n, nb, cb, c1, part, out.codes);
+        QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<float><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const float *>(W), n, nb, cb, c1, part, out.codes));
     else
-        k_quantize_codes<__nv_bfloat16><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W), n, nb, cb, c1, part, out.codes);
-    k_offset<<<1, 1024, 0, st>>>(part, nb2, nb, out.offset);
-    k_double_quant<<<(unsigned)ceil_div(nb2, 8), 256, 0, st>>>(c1, nb, nb2, out.offset, out.scale8, out.scale2);
+        QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<__nv_bfloat16><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W), n, nb, cb, c1, part, out.codes));
+    QNF4_LAUNCH("k_offset", st, k_offset<<<1, 1024, 0, st>>>(part, nb2, nb, out.offset));
+    QNF4_LAUNCH("k_double_quant", st, k_double_quant<<<(unsigned)ceil_div(nb2, 8), 256, 0, st>>>(c1, nb, nb2, out.offset, out.scale8, out.scale2));
     return cudaGetLastError();
 }
 
@@ -278,7 +278,7 @@ cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st
     int64_t grid = ceil_div(nchunk, 256);
     const int64_t cap = (int64_t)num_sms() * 8;
     if (grid > cap) grid = cap;
-    k_dequant<<<(unsigned)grid, 256, 0, st>>>(q, n, host_codebook(), out);
+    QNF4_LAUNCH("k_dequant", st, k_dequant<<<(unsigned)grid, 256, 0, st>>>(q, n, host_codebook(), out));
     return cudaGetLastError();
 }
 

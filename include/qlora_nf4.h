@@ -150,6 +150,23 @@ const char *qlora_status_string(qlora_status s);
  * construction of Dettmers et al. 2023, which the page summarises). */
 void qlora_nf4_codebook(float out[16]);
 
+/*
+ * Measurement hooks. The page has no counterpart: they let a benchmark count
+ * and time the library's own kernels without a profiler.
+ *   qlora_launch_count    kernel launches issued by this process so far.
+ *   qlora_profile_enable  on != 0: from now on every launch is bracketed by two
+ *                         CUDA events recorded on its stream (a few hundred ns
+ *                         of host time per launch); 0 stops recording.
+ *   qlora_profile_read    waits for the recorded events of the named kernel
+ *                         (NULL: all kernels), returns their summed duration in
+ *                         milliseconds and their count, and forgets them.
+ *                         Returns QLORA_OK or QLORA_ERR_CUDA.
+ * Events belong to the device that was current when they were recorded.
+ */
+unsigned long long qlora_launch_count(void);
+void qlora_profile_enable(int on);
+int qlora_profile_read(const char *kernel, double *total_ms, int *launches);
+
 #ifdef __cplusplus
 }
 #endif
