@@ -151,6 +151,29 @@ const char *qlora_status_string(qlora_status s);
 void qlora_nf4_codebook(float out[16]);
 
 /*
+ * qlora_nf4_quantize without a workspace. The paper has no counterpart: this
+ * is an interface for callers that cannot allocate device memory (code that is
+ * handed only its input and output buffers, an allocator-free runtime, a host
+ * that forbids cudaMalloc once it is running), so they cannot supply the
+ * scratch that qlora_nf4_quantize asks for.
+ *   Computes exactly what qlora_nf4_quantize computes (bit for bit), with the
+ *   same W, dt and out arguments; the scratch is a fixed array inside this
+ *   library (about 4 MiB of device memory on every GPU that loads the library,
+ *   held until the process exits). The call allocates and frees nothing.
+ *   Limit: rows * cols <= 67,108,864 (2^26) weights; larger tensors return
+ *   QLORA_ERR_UNSUPPORTED_SHAPE before anything is launched.
+ *   The first call on each device looks up that device's copy of the array
+ *   (with the device current) and caches it; make that first call before any
+ *   stream capture.
+ *   Every call uses the same array. Calls whose kernels may overlap on the GPU
+ *   (different streams without ordering, several host threads) race on it and
+ *   give undefined results; serialise them. No call depends on what an
+ *   earlier call left in the array.
+ */
+qlora_status qlora_nf4_quantize_noalloc(const void *W, qlora_dtype dt, const qlora_nf4_tensor *out,
+                                        qlora_stream_t stream);
+
+/*
  * Measurement hooks. The page has no counterpart: they let a benchmark count
  * and time the library's own kernels without a profiler.
  *   qlora_launch_count    kernel launches issued by this process so far.
