@@ -92,6 +92,31 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
     }
 }
 
+// Prefetched per-block constants (scale8, scale2) of the next kRing blocks a
+// dequant thread will handle, so their global-memory latency overlaps the
+// work on earlier blocks. Indexed with compile-time slots only.
+constexpr int kRing = 4;
+struct ScaleRing {
+    int8_t q8[kRing];
+    float s2[kRing];
+    __device__ __forceinline__ void load(int slot, const NF4View &w, bool valid, int64_t row, int64_t kbs, int kb,
+                                         int KB) {
+        int8_t a = 0;
+        float b = 0.0f;
+        if (valid && kb < KB) {
+            const int64_t blk = row * kbs + kb;
+            a = __ldg(w.scale8 + blk);
+            b = __ldg(w.scale2 + (blk >> 8));
+        }
+        q8[slot] = a;
+        s2[slot] = b;
+    }
+    __device__ __forceinline__ void load_blk(int slot, const NF4View &w, bool valid, int64_t blk) {
+        q8[slot] = valid ? __ldg(w.scale8 + blk) : (int8_t)0;
+        s2[slot] = valid ? __ldg(w.scale2 + (blk >> 8)) : 0.0f;
+    }
+};
+
 struct FusedParams {
     NF4View w;        // stored weight [rows, cols]
     int M;            // tokens
@@ -105,48 +130,64 @@ struct FusedParams {
 constexpr int kTileRows = 128;   // TMEM lanes / MMA M
 constexpr int kTileTok = 256;    // MMA N
 constexpr int kTokStage = kTileTok * 128;          // 32 KB: 256 tokens x 64 bf16
-constexpr int kStaging = kTileTok * kTileRows * 2; // 64 KB output staging [256 tokens][128 rows]
-
 // Epilogue shared by both fused kernels: TMEM D[row, token] -> bf16 staging
-// [token][row] -> TMA store at (x = row0, y = tok0). Returns false on abort.
-__device__ __forceinline__ void fused_epilogue_tile(uint32_t tmem_d, int q, int lane, int et, uint8_t *staging,
-                                                    const CUtensorMap *tm_out, int row0, int tok0) {
+// [token][row] -> TMA store at (x = row0, y = tok0), in PARTS slices of
+// 256 / PARTS tokens through one staging tile. The accumulator is released
+// (tempty) as soon as its last columns are in registers.
+template <int PARTS>
+__device__ __forceinline__ void fused_epilogue(uint32_t tmem_d, int q, int lane, int et, uint8_t *staging,
+                                               const CUtensorMap *tm_out, int row0, int tok0, uint32_t tempty) {
+    constexpr int kPartTok = kTileTok / PARTS;
     uint16_t *st16 = reinterpret_cast<uint16_t *>(staging);
     const int row_local = q * 32 + lane;
-    if (et == 0) bulk_wait_read0();      // previous store has finished reading the staging tile
-    named_bar_sync(1, 128);
 #pragma unroll 1
-    for (int c = 0; c < kTileTok / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)(32 * c), v);
-        tmem_wait_ld();
+    for (int h = 0; h < PARTS; ++h) {
+        if (et == 0) bulk_wait_read0();      // the previous store has finished reading the staging tile
+        named_bar_sync(1, 128);
+#pragma unroll 1
+        for (int c = 0; c < kPartTok / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * kPartTok + 32 * c), v);
+            tmem_wait_ld();
+            if (h == PARTS - 1 && c == kPartTok / 32 - 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty);
+            }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[i]));
-            st16[(32 * c + i) * kTileRows + row_local] = *reinterpret_cast<const uint16_t *>(&h);
+            for (int i = 0; i < 32; ++i) {
+                const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[i]));
+                st16[(32 * c + i) * kTileRows + row_local] = *reinterpret_cast<const uint16_t *>(&b);
+            }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (et == 0) {
+            tma_store_2d(tm_out, smem_addr(staging), row0, tok0 + h * kPartTok);
+            bulk_commit();
         }
     }
 }
 
-__device__ __forceinline__ void fused_epilogue_finish(int et, uint8_t *staging, const CUtensorMap *tm_out,
-                                                      int row0, int tok0) {
-    fence_proxy_async_smem();
-    named_bar_sync(1, 128);
-    if (et == 0) {
-        tma_store_2d(tm_out, smem_addr(staging), row0, tok0);
-        bulk_commit();
-    }
-}
-
 // ================================================================ forward
+// Warp roles (15 warps): 0 X producer (TMA), 1 MMA issuer + TMEM owner,
+// 2..5 epilogue, 6..13 dequant (two groups of four; group g takes the K blocks
+// of iteration parity g), 14 code-tile producer (TMA). Three decoupled rings:
+// X tiles (SX), code tiles (SC, small, fetched far ahead) and dequantised
+// weight tiles in TMEM (SA), so dequantisation runs up to SA K blocks ahead of
+// the tensor core.
 namespace fwd {
-constexpr int S = 4;                         // pipeline stages (even: stage parity = dequant group)
-constexpr int kCodeStage = kTileRows * 32;   // 4 KB: 128 rows x 32 code bytes
-constexpr int kStage = kTokStage + kCodeStage;
-constexpr int kSmem = 1024 + S * kStage + kStaging;
-constexpr int kThreads = 448;                // 14 warps
+constexpr int SX = 5;
+constexpr int SCG = 4;                       // code-tile slots per dequant group (two rings)
+constexpr int SA = 8;                        // even: each TMEM slot always serves the same group
+constexpr int SC = 2 * SCG;
+constexpr int kCodeStage = kTileRows * 32;   // 4 KB: 128 rows x 32 code bytes (32-byte swizzle)
+constexpr int kParts = 2;                    // output staging: 128 tokens x 128 rows (32 KB)
+constexpr int kStaging = kTileTok / kParts * kTileRows * 2;
+constexpr int kSmem = 1024 + SX * kTokStage + SC * kCodeStage + kStaging;
+constexpr int kThreads = 480;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemD = 0, kTmemA = 256;
+constexpr uint32_t kTmemD = 0, kTmemA = 256;  // A stage s at columns 256 + 32 s
 }  // namespace fwd
 
 __global__ void __launch_bounds__(fwd::kThreads, 1)
@@ -155,27 +196,28 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             FusedParams p, Codebook cb) {
     using namespace fwd;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t bars[3 * S + 3];
+    __shared__ __align__(8) uint64_t bars[2 * (SX + SC + SA) + 3];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *xs = smem;
-    uint8_t *cs = smem + S * kTokStage;
-    uint8_t *staging = cs + S * kCodeStage;
+    uint8_t *cs = xs + SX * kTokStage;
+    uint8_t *staging = cs + SC * kCodeStage;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t bar0 = smem_addr(bars);
-    auto full = [&](int s) { return bar0 + 8u * s; };
-    auto afull = [&](int s) { return bar0 + 8u * (S + s); };
-    auto empty = [&](int s) { return bar0 + 8u * (2 * S + s); };
-    const uint32_t tfull = bar0 + 8u * (3 * S), tempty = tfull + 8u, fin = tfull + 16u;
+    auto x_full = [&](int s) { return bar0 + 8u * s; };
+    auto x_empty = [&](int s) { return bar0 + 8u * (SX + s); };
+    auto c_full = [&](int s) { return bar0 + 8u * (2 * SX + s); };
+    auto c_empty = [&](int s) { return bar0 + 8u * (2 * SX + SC + s); };
+    auto a_full = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SC + s); };
+    auto a_empty = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SC + SA + s); };
+    const uint32_t tfull = bar0 + 8u * (2 * (SX + SC + SA)), tempty = tfull + 8u, fin = tfull + 16u;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(full(s), 1);
-            mbar_init(afull(s), 4);
-            mbar_init(empty(s), 1);
-        }
+        for (int s = 0; s < SX; ++s) { mbar_init(x_full(s), 1); mbar_init(x_empty(s), 1); }
+        for (int s = 0; s < SC; ++s) { mbar_init(c_full(s), 1); mbar_init(c_empty(s), 4); }
+        for (int s = 0; s < SA; ++s) { mbar_init(a_full(s), 4); mbar_init(a_empty(s), 1); }
         mbar_init(tfull, 1);
         mbar_init(tempty, 4);
         mbar_init(fin, 1);
@@ -202,29 +244,45 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     const int ntiles = p.tiles_tok * p.tiles_row;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ X / s*XA producer
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-                const int tok0 = (tile % p.tiles_tok) * kTileTok, row0 = (tile / p.tiles_tok) * kTileRows;
+                const int tok0 = (tile % p.tiles_tok) * kTileTok;
                 for (int kb = 0; kb < KBT; ++kb, ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (it / S) & 1u;
-                    if (!mbar_wait(empty(s), ph ^ 1u, abort)) { ok = false; break; }
-                    if (kb < KB) {
-                        mbar_arrive_expect_tx(full(s), kStage);
-                        tma_load_2d(smem_addr(xs + s * kTokStage), &tm_x, full(s), kb * 64, tok0);
-                        tma_load_2d(smem_addr(cs + s * kCodeStage), &tm_codes, full(s), kb * 32, row0);
-                    } else {
-                        mbar_arrive_expect_tx(full(s), kTokStage);
-                        tma_load_2d(smem_addr(xs + s * kTokStage), &tm_xa, full(s), (kb - KB) * 64, tok0);
-                    }
+                    const int s = it % SX;
+                    if (!mbar_wait(x_empty(s), ((it / SX) & 1u) ^ 1u, abort)) { ok = false; break; }
+                    mbar_arrive_expect_tx(x_full(s), kTokStage);
+                    if (kb < KB) tma_load_2d(smem_addr(xs + s * kTokStage), &tm_x, x_full(s), kb * 64, tok0);
+                    else tma_load_2d(smem_addr(xs + s * kTokStage), &tm_xa, x_full(s), (kb - KB) * 64, tok0);
                 }
             }
-            // every issued copy must land before the CTA can exit
-            const uint32_t first = it > (uint32_t)S ? it - S : 0;
-            for (uint32_t i = first; i < it; ++i) drain_wait(full(i % S), (i / S) & 1u);
+            const uint32_t first = it > (uint32_t)SX ? it - SX : 0;
+            for (uint32_t i = first; i < it; ++i) drain_wait(x_full(i % SX), (i / SX) & 1u);
+        }
+    } else if (warp == 14) {
+        // ------------------------------------------------ code-tile producer
+        if (lane == 0) {
+            // one ring per dequant group: the block of iteration it goes to ring it % 2
+            uint32_t it = 0, ig[2] = {0u, 0u};
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const int row0 = (tile / p.tiles_tok) * kTileRows;
+                for (int kb = 0; kb < KB; ++kb) {
+                    const int gg = (int)((it + (uint32_t)kb) & 1u);
+                    const uint32_t i = ig[gg]++;
+                    const int s = gg * SCG + (int)(i % SCG);
+                    if (!mbar_wait(c_empty(s), ((i / SCG) & 1u) ^ 1u, abort)) { ok = false; break; }
+                    mbar_arrive_expect_tx(c_full(s), kCodeStage);
+                    tma_load_2d(smem_addr(cs + s * kCodeStage), &tm_codes, c_full(s), kb * 32, row0);
+                }
+                it += (uint32_t)KBT;
+            }
+            for (int gg = 0; gg < 2; ++gg) {
+                const uint32_t first = ig[gg] > (uint32_t)SCG ? ig[gg] - SCG : 0;
+                for (uint32_t i = first; i < ig[gg]; ++i) drain_wait(c_full(gg * SCG + (int)(i % SCG)), (i / SCG) & 1u);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -236,21 +294,22 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                 if (!mbar_wait(tempty, (lt & 1u) ^ 1u, abort)) break;
                 tc_fence_after();
                 for (int kb = 0; kb < KBT; ++kb, ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (it / S) & 1u;
-                    if (!mbar_wait(full(s), ph, abort) || !mbar_wait(afull(s), ph, abort)) { ok = false; break; }
+                    const int sx = it % SX, sa = it % SA;
+                    if (!mbar_wait(x_full(sx), (it / SX) & 1u, abort) ||
+                        !mbar_wait(a_full(sa), (it / SA) & 1u, abort)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a = tmem + kTmemA + 32u * s;
-                    const uint32_t xb = smem_addr(xs + s * kTokStage);
+                    const uint32_t a = tmem + kTmemA + 32u * sa;
+                    const uint32_t xb = smem_addr(xs + sx * kTokStage);
                     const int nk = kb < KB ? 4 : min(4, (p.r - (kb - KB) * 64 + 15) / 16);
                     for (int k = 0; k < nk; ++k)
                         mma_ts(tmem + kTmemD, a + 8u * k, sw128_desc(xb + 32u * k, 16, 1024), idesc,
                                (kb | k) != 0 ? 1u : 0u);
-                    mma_commit(empty(s));
+                    mma_commit(x_empty(sx));
+                    mma_commit(a_empty(sa));
                 }
                 if (ok) mma_commit(tfull);
             }
-            mma_commit(fin);          // all MMAs of this CTA complete before TMEM is released
+            mma_commit(fin);          // every MMA of this CTA has completed before TMEM is released
             drain_wait(fin, 0);
         }
     } else if (warp < 6) {
@@ -261,67 +320,86 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             const int tok0 = (tile % p.tiles_tok) * kTileTok, row0 = (tile / p.tiles_tok) * kTileRows;
             if (!mbar_wait(tfull, lt & 1u, abort)) break;
             tc_fence_after();
-            fused_epilogue_tile(tmem + kTmemD, q, lane, et, staging, &tm_y, row0, tok0);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tempty);
-            fused_epilogue_finish(et, staging, &tm_y, row0, tok0);
+            fused_epilogue<kParts>(tmem + kTmemD, q, lane, et, staging, &tm_y, row0, tok0, tempty);
         }
         if (et == 0) bulk_wait0();
     } else {
         // ------------------------------------------------ dequant (warps 6..13)
-        const int g = (warp - 6) >> 2;          // handles iterations with it % 2 == g
+        const int g = (warp - 6) >> 2;          // takes the iterations with it % 2 == g
         const int q = warp & 3;                 // TMEM lane quarter
         const int row_local = q * 32 + lane;
         const float mu = *p.w.offset;
         const int64_t kbs = p.cols / 64;        // 64-blocks per weight row
-        uint32_t it = 0;
+        // code tile rows are 32 bytes, stored with the 32-byte TMA swizzle
+        const uint32_t src_off0 = row_local * 32 + ((0u ^ ((row_local >> 2) & 1u)) << 4);
+        const uint32_t src_off1 = row_local * 32 + ((1u ^ ((row_local >> 2) & 1u)) << 4);
+        uint32_t it = 0, ic = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
             const int row0 = (tile / p.tiles_tok) * kTileRows;
             const int n = row0 + row_local;
             const bool valid = n < p.rows;
-            for (int kb = 0; kb < KBT; ++kb, ++it) {
-                if ((int)(it & 1u) != g) continue;
-                const int s = it % S;
-                const uint32_t ph = (it / S) & 1u;
-                int8_t q8 = 0;
-                float s2 = 0.0f;
-                if (kb < KB && valid) {
-                    const int64_t b = (int64_t)n * kbs + kb;
-                    q8 = p.w.scale8[b];
-                    s2 = p.w.scale2[b >> 8];
-                }
-                if (!mbar_wait(full(s), ph, abort)) { ok = false; break; }
-                uint32_t v[32];
-                if (kb < KB) {
-                    if (valid) {
-                        const uint8_t *src = cs + s * kCodeStage + row_local * 32;
-                        const uint4 c0 = *reinterpret_cast<const uint4 *>(src);
-                        const uint4 c1 = *reinterpret_cast<const uint4 *>(src + 16);
-                        dequant_block(c0, c1, cb, dq_constant(q8, s2, mu), v);
+            const uint32_t it0 = it, ic0 = ic;
+            const int kb_first = (int)((uint32_t)g - it0) & 1;
+            const int J = (KBT - kb_first + 1) / 2;
+            ScaleRing ring;
+#pragma unroll
+            for (int d = 0; d < kRing; ++d) ring.load(d, p.w, valid, n, kbs, kb_first + 2 * d, KB);
+            for (int j0 = 0; j0 < J && ok; j0 += kRing) {
+#pragma unroll
+                for (int u = 0; u < kRing; ++u) {
+                    const int j = j0 + u;
+                    if (j >= J) break;
+                    const int kb = kb_first + 2 * j;
+                    const uint32_t itj = it0 + (uint32_t)kb;
+                    const int sa = itj % SA;
+                    const int8_t q8 = ring.q8[u];
+                    const float s2 = ring.s2[u];
+                    ring.load(u, p.w, valid, n, kbs, kb + 2 * kRing, KB);
+                    uint32_t v[32];
+                    int code_slot = -1;
+                    if (kb < KB) {
+                        const uint32_t icj = ic0 + (uint32_t)j;          // this group's main blocks so far
+                        const int sc = g * SCG + (int)(icj % SCG);
+                        if (!mbar_wait(c_full(sc), (icj / SCG) & 1u, abort)) { ok = false; break; }
+                        const uint8_t *src = cs + sc * kCodeStage;
+                        const uint4 c0 = *reinterpret_cast<const uint4 *>(src + src_off0);
+                        const uint4 c1 = *reinterpret_cast<const uint4 *>(src + src_off1);
+                        code_slot = sc;
+                        if (valid) {
+                            dequant_block(c0, c1, cb, dq_constant(q8, s2, mu), v);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] = 0u;
+                        }
                     } else {
+                        // adapter block: A operand row n = B_lora[:, n] (rank index along K)
+                        const int jr = (kb - KB) * 64;
+                        const uint16_t *bl = reinterpret_cast<const uint16_t *>(p.lora_t);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = 0u;
+                        for (int i = 0; i < 32; ++i) {
+                            const int k = jr + 2 * i;
+                            const uint32_t lo = (valid && k < p.r) ? bl[(int64_t)k * p.rows + n] : 0u;
+                            const uint32_t hi = (valid && k + 1 < p.r) ? bl[(int64_t)(k + 1) * p.rows + n] : 0u;
+                            v[i] = lo | (hi << 16);
+                        }
                     }
-                } else {
-                    // adapter block: A operand row n = B_lora[:, n] (rank index along K)
-                    const int j0 = (kb - KB) * 64;
-                    const uint16_t *bl = reinterpret_cast<const uint16_t *>(p.lora_t);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int k = j0 + 2 * i;
-                        const uint32_t lo = (valid && k < p.r) ? bl[(int64_t)k * p.rows + n] : 0u;
-                        const uint32_t hi = (valid && k + 1 < p.r) ? bl[(int64_t)(k + 1) * p.rows + n] : 0u;
-                        v[i] = lo | (hi << 16);
+                    if (!mbar_wait(a_empty(sa), ((itj / SA) & 1u) ^ 1u, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + kTmemA + 32u * sa, v);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    // the code slot is released only now: the values stored above depend on
+                    // the codes read from it, so those reads have certainly completed
+                    if (lane == 0) {
+                        if (code_slot >= 0) mbar_arrive(c_empty(code_slot));
+                        mbar_arrive(a_full(sa));
                     }
                 }
-                tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + kTmemA + 32u * s, v);
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(afull(s));
             }
+            it = it0 + (uint32_t)KBT;
+            ic = ic0 + (uint32_t)((KB - kb_first + 1) / 2);  // main blocks this group handled
         }
     }
 
@@ -335,13 +413,20 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
 }
 
 // ================================================================ dgrad
+// Same warp roles; the dequant warps write W^ tiles (64 weight rows x 128
+// d_in) into shared memory in the MN-major 128-byte-swizzled layout and the
+// MMA reads them as its A operand; dY tiles come by TMA as B.
 namespace dg {
-constexpr int S = 3;
-constexpr int kAStage = kTileRows * 128;     // 16 KB: 2 MN-chunks (64 d_in) x 64 K rows (d_out) x 128 B
-constexpr int kCodeStage = 64 * 64;          // 4 KB: 64 weight rows x 64 code bytes (128 d_in)
-constexpr int kStage = kAStage + kTokStage + kCodeStage;
-constexpr int kSmem = 1024 + S * kStage + kStaging;
-constexpr int kThreads = 448;
+constexpr int SX = 4;                        // dY / s*G tiles (32 KB); SX <= SA
+constexpr int SCG = 2;                       // code tiles per dequant group (4 KB: 64 rows x 64 bytes, 64-byte swizzle)
+constexpr int SA = 4;                        // dequantised A tiles (16 KB: 2 MN chunks of 64 d_in x 64 K rows); even
+constexpr int SC = 2 * SCG;
+constexpr int kAStage = kTileRows * 128;
+constexpr int kCodeStage = 64 * 64;
+constexpr int kParts = 4;                    // output staging: 64 tokens x 128 rows (16 KB)
+constexpr int kStaging = kTileTok / kParts * kTileRows * 2;
+constexpr int kSmem = 1024 + SA * kAStage + SX * kTokStage + SC * kCodeStage + kStaging;
+constexpr int kThreads = 480;
 constexpr uint32_t kTmemCols = 256;
 }  // namespace dg
 
@@ -351,28 +436,32 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
               const __grid_constant__ CUtensorMap tm_dx, FusedParams p, Codebook cb) {
     using namespace dg;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t bars[3 * S + 3];
+    __shared__ __align__(8) uint64_t bars[2 * (SX + SC + SA) + 3];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *as = smem;
-    uint8_t *bs = smem + S * kAStage;
-    uint8_t *cs = bs + S * kTokStage;
-    uint8_t *staging = cs + S * kCodeStage;
+    uint8_t *bs = as + SA * kAStage;
+    uint8_t *cs = bs + SX * kTokStage;
+    uint8_t *staging = cs + SC * kCodeStage;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t bar0 = smem_addr(bars);
-    auto full = [&](int s) { return bar0 + 8u * s; };
-    auto afull = [&](int s) { return bar0 + 8u * (S + s); };
-    auto empty = [&](int s) { return bar0 + 8u * (2 * S + s); };
-    const uint32_t tfull = bar0 + 8u * (3 * S), tempty = tfull + 8u, fin = tfull + 16u;
+    auto x_full = [&](int s) { return bar0 + 8u * s; };
+    auto x_empty = [&](int s) { return bar0 + 8u * (SX + s); };
+    auto c_full = [&](int s) { return bar0 + 8u * (2 * SX + s); };
+    auto c_empty = [&](int s) { return bar0 + 8u * (2 * SX + SC + s); };
+    auto a_full = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SC + s); };
+    auto a_empty = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SC + SA + s); };
+    const uint32_t tfull = bar0 + 8u * (2 * (SX + SC + SA)), tempty = tfull + 8u, fin = tfull + 16u;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(full(s), 1);
-            mbar_init(afull(s), 4);
-            mbar_init(empty(s), 1);
-        }
+        for (int s = 0; s < SX; ++s) { mbar_init(x_full(s), 1); mbar_init(x_empty(s), 1); }
+        for (int s = 0; s < SC; ++s) { mbar_init(c_full(s), 1); mbar_init(c_empty(s), 4); }
+        // an A stage is filled either by the 4 dequant warps of a group (main
+        // blocks) or by TMA (adapter blocks); the group still arrives for the
+        // latter, and the producer adds the expected bytes
+        for (int s = 0; s < SA; ++s) { mbar_init(a_full(s), 4); mbar_init(a_empty(s), 1); }
         mbar_init(tfull, 1);
         mbar_init(tempty, 4);
         mbar_init(fin, 1);
@@ -400,28 +489,53 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
     const int ntiles = p.tiles_tok * p.tiles_row;
 
     if (warp == 0) {
+        // ------------------------------------------------ dY / s*G producer (+ A_lora for adapter blocks)
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
                 const int tok0 = (tile % p.tiles_tok) * kTileTok, col0 = (tile / p.tiles_tok) * kTileRows;
                 for (int kb = 0; kb < KBT; ++kb, ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (it / S) & 1u;
-                    if (!mbar_wait(empty(s), ph ^ 1u, abort)) { ok = false; break; }
+                    const int s = it % SX;
+                    if (!mbar_wait(x_empty(s), ((it / SX) & 1u) ^ 1u, abort)) { ok = false; break; }
                     if (kb < KB) {
-                        mbar_arrive_expect_tx(full(s), kTokStage + kCodeStage);
-                        tma_load_2d(smem_addr(bs + s * kTokStage), &tm_dy, full(s), kb * 64, tok0);
-                        tma_load_2d(smem_addr(cs + s * kCodeStage), &tm_codes, full(s), col0 / 2, kb * 64);
+                        mbar_arrive_expect_tx(x_full(s), kTokStage);
+                        tma_load_2d(smem_addr(bs + s * kTokStage), &tm_dy, x_full(s), kb * 64, tok0);
                     } else {
-                        mbar_arrive_expect_tx(full(s), kAStage + kTokStage);
-                        tma_load_2d(smem_addr(as + s * kAStage), &tm_alora, full(s), (kb - KB) * 64, col0);
-                        tma_load_2d(smem_addr(bs + s * kTokStage), &tm_gs, full(s), (kb - KB) * 64, tok0);
+                        // the adapter A tile goes into the A ring slot of this iteration,
+                        // which the dequant group has released (it waited a_empty)
+                        const int sa = it % SA;
+                        if (!mbar_wait(a_empty(sa), ((it / SA) & 1u) ^ 1u, abort)) { ok = false; break; }
+                        mbar_arrive_expect_tx(x_full(s), kTokStage + kAStage);
+                        tma_load_2d(smem_addr(as + sa * kAStage), &tm_alora, x_full(s), (kb - KB) * 64, col0);
+                        tma_load_2d(smem_addr(bs + s * kTokStage), &tm_gs, x_full(s), (kb - KB) * 64, tok0);
                     }
                 }
             }
-            const uint32_t first = it > (uint32_t)S ? it - S : 0;
-            for (uint32_t i = first; i < it; ++i) drain_wait(full(i % S), (i / S) & 1u);
+            const uint32_t first = it > (uint32_t)SX ? it - SX : 0;
+            for (uint32_t i = first; i < it; ++i) drain_wait(x_full(i % SX), (i / SX) & 1u);
+        }
+    } else if (warp == 14) {
+        // ------------------------------------------------ code-tile producer
+        if (lane == 0) {
+            uint32_t it = 0, ig[2] = {0u, 0u};
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const int col0 = (tile / p.tiles_tok) * kTileRows;
+                for (int kb = 0; kb < KB; ++kb) {
+                    const int gg = (int)((it + (uint32_t)kb) & 1u);
+                    const uint32_t i = ig[gg]++;
+                    const int s = gg * SCG + (int)(i % SCG);
+                    if (!mbar_wait(c_empty(s), ((i / SCG) & 1u) ^ 1u, abort)) { ok = false; break; }
+                    mbar_arrive_expect_tx(c_full(s), kCodeStage);
+                    tma_load_2d(smem_addr(cs + s * kCodeStage), &tm_codes, c_full(s), col0 / 2, kb * 64);
+                }
+                it += (uint32_t)KBT;
+            }
+            for (int gg = 0; gg < 2; ++gg) {
+                const uint32_t first = ig[gg] > (uint32_t)SCG ? ig[gg] - SCG : 0;
+                for (uint32_t i = first; i < ig[gg]; ++i) drain_wait(c_full(gg * SCG + (int)(i % SCG)), (i / SCG) & 1u);
+            }
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -433,12 +547,12 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
                 if (!mbar_wait(tempty, (lt & 1u) ^ 1u, abort)) break;
                 tc_fence_after();
                 for (int kb = 0; kb < KBT; ++kb, ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (it / S) & 1u;
-                    if (!mbar_wait(full(s), ph, abort) || !mbar_wait(afull(s), ph, abort)) { ok = false; break; }
+                    const int sx = it % SX, sa = it % SA;
+                    if (!mbar_wait(x_full(sx), (it / SX) & 1u, abort) ||
+                        !mbar_wait(a_full(sa), (it / SA) & 1u, abort)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t ab = smem_addr(as + s * kAStage);
-                    const uint32_t bb = smem_addr(bs + s * kTokStage);
+                    const uint32_t ab = smem_addr(as + sa * kAStage);
+                    const uint32_t bb = smem_addr(bs + sx * kTokStage);
                     if (kb < KB) {
                         for (int k = 0; k < 4; ++k)
                             mma_ss(tmem, sw128_desc(ab + 2048u * k, 8192, 1024), sw128_desc(bb + 32u * k, 16, 1024),
@@ -449,7 +563,8 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
                             mma_ss(tmem, sw128_desc(ab + 32u * k, 16, 1024), sw128_desc(bb + 32u * k, 16, 1024),
                                    idesc_lora, (kb | k) != 0 ? 1u : 0u);
                     }
-                    mma_commit(empty(s));
+                    mma_commit(x_empty(sx));
+                    mma_commit(a_empty(sa));
                 }
                 if (ok) mma_commit(tfull);
             }
@@ -463,11 +578,7 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
             const int tok0 = (tile % p.tiles_tok) * kTileTok, col0 = (tile / p.tiles_tok) * kTileRows;
             if (!mbar_wait(tfull, lt & 1u, abort)) break;
             tc_fence_after();
-            fused_epilogue_tile(tmem, q, lane, et, staging, &tm_dx, col0, tok0);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tempty);
-            fused_epilogue_finish(et, staging, &tm_dx, col0, tok0);
+            fused_epilogue<kParts>(tmem, q, lane, et, staging, &tm_dx, col0, tok0, tempty);
         }
         if (et == 0) bulk_wait0();
     } else {
@@ -477,46 +588,87 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         const int n_local = tg & 63, chunk = tg >> 6;
         const float mu = *p.w.offset;
         const int64_t kbs = p.cols / 64;
-        uint32_t it = 0;
+        // code tile rows are 64 bytes, stored with the 64-byte TMA swizzle
+        const uint32_t sw = ((uint32_t)n_local >> 1) & 3u;
+        const uint32_t src_off0 = n_local * 64 + (((2u * chunk) ^ sw) << 4);
+        const uint32_t src_off1 = n_local * 64 + (((2u * chunk + 1u) ^ sw) << 4);
+        uint32_t it = 0, ic = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
             const int col0 = (tile / p.tiles_tok) * kTileRows;
             const int kcol = col0 + 64 * chunk;
-            for (int kb = 0; kb < KBT; ++kb, ++it) {
-                if ((int)(it & 1u) != g) continue;
-                const int s = it % S;
-                const uint32_t ph = (it / S) & 1u;
+            const bool col_ok = kcol < p.cols;
+            const uint32_t it0 = it, ic0 = ic;
+            const int kb_first = (int)((uint32_t)g - it0) & 1;
+            const int J = (KBT - kb_first + 1) / 2;
+            // the block of (row kb*64 + n_local, column chunk kcol/64)
+            auto blk_of = [&](int kb, bool &v) {
                 const int n = kb * 64 + n_local;
-                const bool valid = kb < KB && n < p.rows && kcol < p.cols;
-                int8_t q8 = 0;
-                float s2 = 0.0f;
-                if (valid) {
-                    const int64_t b = (int64_t)n * kbs + kcol / 64;
-                    q8 = p.w.scale8[b];
-                    s2 = p.w.scale2[b >> 8];
-                }
-                if (!mbar_wait(full(s), ph, abort)) { ok = false; break; }
-                if (kb < KB) {
-                    uint32_t v[32];
-                    if (valid) {
-                        const uint8_t *src = cs + s * kCodeStage + n_local * 64 + chunk * 32;
-                        const uint4 c0 = *reinterpret_cast<const uint4 *>(src);
-                        const uint4 c1 = *reinterpret_cast<const uint4 *>(src + 16);
-                        dequant_block(c0, c1, cb, dq_constant(q8, s2, mu), v);
-                    } else {
+                v = kb < KB && n < p.rows && col_ok;
+                return (int64_t)n * kbs + kcol / 64;
+            };
+            ScaleRing ring;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = 0u;
-                    }
-                    uint8_t *dst = as + s * kAStage + chunk * 8192;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<uint4 *>(dst + sw128_offset(n_local, j)) =
-                            make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                    fence_proxy_async_smem();
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(afull(s));
+            for (int d = 0; d < kRing; ++d) {
+                bool v;
+                const int64_t b = blk_of(kb_first + 2 * d, v);
+                ring.load_blk(d, p.w, v, b);
             }
+            for (int j0 = 0; j0 < J && ok; j0 += kRing) {
+#pragma unroll
+                for (int u = 0; u < kRing; ++u) {
+                    const int j = j0 + u;
+                    if (j >= J) break;
+                    const int kb = kb_first + 2 * j;
+                    const uint32_t itj = it0 + (uint32_t)kb;
+                    const int sa = itj % SA;
+                    bool valid;
+                    blk_of(kb, valid);
+                    const int8_t q8 = ring.q8[u];
+                    const float s2 = ring.s2[u];
+                    {
+                        bool v;
+                        const int64_t b = blk_of(kb + 2 * kRing, v);
+                        ring.load_blk(u, p.w, v, b);
+                    }
+                    int code_slot = -1;
+                    if (kb < KB) {
+                        const uint32_t icj = ic0 + (uint32_t)j;          // this group's main blocks so far
+                        const int sc = g * SCG + (int)(icj % SCG);
+                        if (!mbar_wait(c_full(sc), (icj / SCG) & 1u, abort)) { ok = false; break; }
+                        const uint8_t *src = cs + sc * kCodeStage;
+                        const uint4 c0 = *reinterpret_cast<const uint4 *>(src + src_off0);
+                        const uint4 c1 = *reinterpret_cast<const uint4 *>(src + src_off1);
+                        code_slot = sc;
+                        uint32_t v[32];
+                        if (valid) {
+                            dequant_block(c0, c1, cb, dq_constant(q8, s2, mu), v);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] = 0u;
+                        }
+                        if (!mbar_wait(a_empty(sa), ((itj / SA) & 1u) ^ 1u, abort)) { ok = false; break; }
+                        uint8_t *dst = as + sa * kAStage + chunk * 8192;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<uint4 *>(dst + sw128_offset(n_local, c)) =
+                                make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                        fence_proxy_async_smem();
+                    } else {
+                        // adapter block: the producer's TMA fills the A slot
+                        if (!mbar_wait(a_empty(sa), ((itj / SA) & 1u) ^ 1u, abort)) { ok = false; break; }
+                    }
+                    __syncwarp();
+                    // the code slot is released only after the A-tile stores that depend on the
+                    // codes read from it, so those reads have certainly completed
+                    if (lane == 0) {
+                        if (code_slot >= 0) mbar_arrive(c_empty(code_slot));
+                        mbar_arrive(a_full(sa));
+                    }
+                }
+            }
+            it = it0 + (uint32_t)KBT;
+            ic = ic0 + (uint32_t)((KB - kb_first + 1) / 2);  // main blocks this group handled
         }
     }
 
@@ -842,10 +994,11 @@ static cudaError_t run_fused_fwd(const __nv_bfloat16 *X, int64_t M, const NF4Vie
     CUtensorMap tx, tc_, txa, ty;
     bool ok = map_bf16(&tx, X, (uint64_t)W.cols, (uint64_t)M, 64, kTileTok);
     ok = ok && make_map(&tc_, W.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)(W.cols / 2), (uint64_t)W.rows,
-                        (uint64_t)(W.cols / 2), 32, kTileRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+                        (uint64_t)(W.cols / 2), 32, kTileRows, CU_TENSOR_MAP_SWIZZLE_32B);
     if (r > 0) ok = ok && map_bf16(&txa, XAs, (uint64_t)r, (uint64_t)M, 64, kTileTok);
     else txa = tx;
-    ok = ok && map_bf16(&ty, Y, (uint64_t)W.rows, (uint64_t)M, kTileRows, kTileTok, CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok = ok && map_bf16(&ty, Y, (uint64_t)W.rows, (uint64_t)M, kTileRows, kTileTok / fwd::kParts,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return cudaErrorInvalidValue;
     FusedParams p;
     p.w = W;
@@ -869,7 +1022,7 @@ static cudaError_t run_fused_dgrad(const __nv_bfloat16 *dY, int64_t M, const NF4
     CUtensorMap tdy, tc_, ta, tg, tdx;
     bool ok = map_bf16(&tdy, dY, (uint64_t)W.rows, (uint64_t)M, 64, kTileTok);
     ok = ok && make_map(&tc_, W.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)(W.cols / 2), (uint64_t)W.rows,
-                        (uint64_t)(W.cols / 2), 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
+                        (uint64_t)(W.cols / 2), 64, 64, CU_TENSOR_MAP_SWIZZLE_64B);
     if (r > 0) {
         ok = ok && map_bf16(&ta, Alora, (uint64_t)r, (uint64_t)W.cols, 64, kTileRows);
         ok = ok && map_bf16(&tg, Gs, (uint64_t)r, (uint64_t)M, 64, kTileTok);
@@ -877,7 +1030,8 @@ static cudaError_t run_fused_dgrad(const __nv_bfloat16 *dY, int64_t M, const NF4
         ta = tdy;
         tg = tdy;
     }
-    ok = ok && map_bf16(&tdx, dX, (uint64_t)W.cols, (uint64_t)M, kTileRows, kTileTok, CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok = ok && map_bf16(&tdx, dX, (uint64_t)W.cols, (uint64_t)M, kTileRows, kTileTok / dg::kParts,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return cudaErrorInvalidValue;
     FusedParams p;
     p.w = W;

@@ -182,3 +182,23 @@ def test_zero_adapter_equals_plain_product():
     for Y in (Y0, Y1):
         m, f = oracle.rel_errors(f64(Y), ref.cpu().numpy())
         assert m <= MAX_TOL and f <= FRO_TOL
+
+
+@pytest.mark.parametrize("rep", [0, 1])
+def test_many_tiles_per_cta_full(rep):
+    # every CTA of the persistent fused kernels walks several tiles (1024 tiles on
+    # 148 SMs): compare every element, twice, so a race at tile boundaries shows
+    M = 4096
+    for rows, cols in ((1024, 8192), (8192, 1024)):
+        W, X, dY, A, B, s = make_problem(M, rows, cols, 64, seed=300 + rows + rep)
+        t = q.qlora_nf4_quantize(W)
+        Y, XA = q.qlora_linear_fwd(X, t, A, B, s)
+        dX, dA, dB = q.qlora_linear_bwd(X, dY, t, A, B, s, XA=XA)
+        assert q.qlora_get_device_status() == q.QLORA_OK
+        Wh = oracle_weight(W)
+        Xn, dYn, An, Bn = f64(X), f64(dY), f64(A), f64(B)
+        check(f64(Y), oracle.linear_fwd(Xn, Wh, An, Bn, s), f"Y[{rows}x{cols}]")
+        dXr, dAr, dBr = oracle.linear_bwd(Xn, dYn, Wh, An, Bn, s)
+        check(f64(dX), dXr, f"dX[{rows}x{cols}]")
+        check(f64(dA), dAr, f"dA[{rows}x{cols}]")
+        check(f64(dB), dBr, f"dB[{rows}x{cols}]")
