@@ -287,27 +287,47 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
+            // A tcgen05.mma issue returns only once the tensor core has taken the
+            // previous MMA, so any bookkeeping done after a K block's last MMA leaves the
+            // tensor core idle. It is therefore slotted between the MMAs: the previous
+            // block's slots are released after MMA 0 and MMA 1 (each commit covers every
+            // earlier MMA), and the next block's operands are probed without blocking
+            // after MMA 2 and MMA 3; only operands that are actually late are waited for.
             const uint32_t idesc = idesc_bf16(kTileRows, kTileTok, false, false);
             uint32_t it = 0, lt = 0;
             bool ok = true;
+            auto ready = [&](uint32_t i) {
+                return mbar_test(x_full(i % SX), (i / SX) & 1u) && mbar_test(a_full(i % SA), (i / SA) & 1u);
+            };
+            auto wait_operands = [&](uint32_t i) {
+                return mbar_wait(x_full(i % SX), (i / SX) & 1u, abort) && mbar_wait(a_full(i % SA), (i / SA) & 1u, abort);
+            };
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++lt) {
-                if (!mbar_wait(tempty, (lt & 1u) ^ 1u, abort)) break;
+                if (!mbar_wait(tempty, (lt & 1u) ^ 1u, abort) || !wait_operands(it)) { ok = false; break; }
                 tc_fence_after();
                 for (int kb = 0; kb < KBT; ++kb, ++it) {
-                    const int sx = it % SX, sa = it % SA;
-                    if (!mbar_wait(x_full(sx), (it / SX) & 1u, abort) ||
-                        !mbar_wait(a_full(sa), (it / SA) & 1u, abort)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t a = tmem + kTmemA + 32u * sa;
-                    const uint32_t xb = smem_addr(xs + sx * kTokStage);
+                    const uint32_t a = tmem + kTmemA + 32u * (it % SA);
+                    const uint32_t xb = smem_addr(xs + (it % SX) * kTokStage);
                     const int nk = kb < KB ? 4 : min(4, (p.r - (kb - KB) * 64 + 15) / 16);
-                    for (int k = 0; k < nk; ++k)
-                        mma_ts(tmem + kTmemD, a + 8u * k, sw128_desc(xb + 32u * k, 16, 1024), idesc,
-                               (kb | k) != 0 ? 1u : 0u);
-                    mma_commit(x_empty(sx));
-                    mma_commit(a_empty(sa));
+                    const bool has_next = kb + 1 < KBT;
+                    bool next_ready = !has_next;
+                    for (int k = 0; k < 4; ++k) {
+                        if (k < nk)
+                            mma_ts(tmem + kTmemD, a + 8u * k, sw128_desc(xb + 32u * k, 16, 1024), idesc,
+                                   (kb | k) != 0 ? 1u : 0u);
+                        if (k == 0 && kb > 0) mma_commit(x_empty((it - 1) % SX));
+                        else if (k == 1 && kb > 0) mma_commit(a_empty((it - 1) % SA));
+                        else if (k >= 2 && !next_ready) next_ready = ready(it + 1);
+                    }
+                    if (has_next) {
+                        if (!next_ready && !wait_operands(it + 1)) { ok = false; break; }
+                        tc_fence_after();
+                    }
                 }
-                if (ok) mma_commit(tfull);
+                if (!ok) break;
+                mma_commit(x_empty((it - 1) % SX));
+                mma_commit(a_empty((it - 1) % SA));
+                mma_commit(tfull);
             }
             mma_commit(fin);          // every MMA of this CTA has completed before TMEM is released
             drain_wait(fin, 0);
@@ -539,34 +559,47 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         }
     } else if (warp == 1) {
         if (lane == 0) {
+            // bookkeeping slotted between the MMAs, as in the forward kernel
             const uint32_t idesc_main = idesc_bf16(kTileRows, kTileTok, true, false);
             const uint32_t idesc_lora = idesc_bf16(kTileRows, kTileTok, false, false);
             uint32_t it = 0, lt = 0;
             bool ok = true;
+            auto ready = [&](uint32_t i) {
+                return mbar_test(x_full(i % SX), (i / SX) & 1u) && mbar_test(a_full(i % SA), (i / SA) & 1u);
+            };
+            auto wait_operands = [&](uint32_t i) {
+                return mbar_wait(x_full(i % SX), (i / SX) & 1u, abort) && mbar_wait(a_full(i % SA), (i / SA) & 1u, abort);
+            };
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++lt) {
-                if (!mbar_wait(tempty, (lt & 1u) ^ 1u, abort)) break;
+                if (!mbar_wait(tempty, (lt & 1u) ^ 1u, abort) || !wait_operands(it)) { ok = false; break; }
                 tc_fence_after();
                 for (int kb = 0; kb < KBT; ++kb, ++it) {
-                    const int sx = it % SX, sa = it % SA;
-                    if (!mbar_wait(x_full(sx), (it / SX) & 1u, abort) ||
-                        !mbar_wait(a_full(sa), (it / SA) & 1u, abort)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t ab = smem_addr(as + sa * kAStage);
-                    const uint32_t bb = smem_addr(bs + sx * kTokStage);
-                    if (kb < KB) {
-                        for (int k = 0; k < 4; ++k)
-                            mma_ss(tmem, sw128_desc(ab + 2048u * k, 8192, 1024), sw128_desc(bb + 32u * k, 16, 1024),
-                                   idesc_main, (kb | k) != 0 ? 1u : 0u);
-                    } else {
-                        const int nk = min(4, (p.r - (kb - KB) * 64 + 15) / 16);
-                        for (int k = 0; k < nk; ++k)
-                            mma_ss(tmem, sw128_desc(ab + 32u * k, 16, 1024), sw128_desc(bb + 32u * k, 16, 1024),
-                                   idesc_lora, (kb | k) != 0 ? 1u : 0u);
+                    const uint32_t ab = smem_addr(as + (it % SA) * kAStage);
+                    const uint32_t bb = smem_addr(bs + (it % SX) * kTokStage);
+                    const bool main = kb < KB;
+                    const int nk = main ? 4 : min(4, (p.r - (kb - KB) * 64 + 15) / 16);
+                    const bool has_next = kb + 1 < KBT;
+                    bool next_ready = !has_next;
+                    for (int k = 0; k < 4; ++k) {
+                        if (k < nk) {
+                            const uint64_t ad = main ? sw128_desc(ab + 2048u * k, 8192, 1024)
+                                                     : sw128_desc(ab + 32u * k, 16, 1024);
+                            mma_ss(tmem, ad, sw128_desc(bb + 32u * k, 16, 1024), main ? idesc_main : idesc_lora,
+                                   (kb | k) != 0 ? 1u : 0u);
+                        }
+                        if (k == 0 && kb > 0) mma_commit(x_empty((it - 1) % SX));
+                        else if (k == 1 && kb > 0) mma_commit(a_empty((it - 1) % SA));
+                        else if (k >= 2 && !next_ready) next_ready = ready(it + 1);
                     }
-                    mma_commit(x_empty(sx));
-                    mma_commit(a_empty(sa));
+                    if (has_next) {
+                        if (!next_ready && !wait_operands(it + 1)) { ok = false; break; }
+                        tc_fence_after();
+                    }
                 }
-                if (ok) mma_commit(tfull);
+                if (!ok) break;
+                mma_commit(x_empty((it - 1) % SX));
+                mma_commit(a_empty((it - 1) % SA));
+                mma_commit(tfull);
             }
             mma_commit(fin);
             drain_wait(fin, 0);
