@@ -27,10 +27,9 @@
 // Both fused kernels keep the accumulator tile D[row, token] in TMEM and store
 // it transposed (out[token, row]) through a shared-memory staging tile and a
 // TMA store.
-#include <mutex>
-
 #include "launch.h"
 #include "tc.cuh"
+#include "tmap.h"
 
 namespace qnf4 {
 using namespace tc;
@@ -175,7 +174,11 @@ __device__ __forceinline__ void fused_epilogue(uint32_t tmem_d, int q, int lane,
 // of iteration parity g), 14 code-tile producer (TMA). Three decoupled rings:
 // X tiles (SX), code tiles (SC, small, fetched far ahead) and dequantised
 // weight tiles in TMEM (SA), so dequantisation runs up to SA K blocks ahead of
-// the tensor core.
+// the tensor core. The X and weight rings share one pair of barriers per K
+// block (stage ring of SA entries): `full` completes when the X tile has landed
+// and all four dequant warps have stored the weight tile, `empty` when the MMAs
+// of that block have completed. The MMA thread therefore tests one barrier and
+// commits once per block.
 namespace fwd {
 constexpr int SX = 5;
 constexpr int SCG = 4;                       // code-tile slots per dequant group (two rings)
@@ -196,7 +199,7 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             FusedParams p, Codebook cb) {
     using namespace fwd;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t bars[2 * (SX + SC + SA) + 3];
+    __shared__ __align__(8) uint64_t bars[2 * (SA + SC) + 3];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
 
@@ -206,18 +209,17 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     uint8_t *staging = cs + SC * kCodeStage;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t bar0 = smem_addr(bars);
-    auto x_full = [&](int s) { return bar0 + 8u * s; };
-    auto x_empty = [&](int s) { return bar0 + 8u * (SX + s); };
-    auto c_full = [&](int s) { return bar0 + 8u * (2 * SX + s); };
-    auto c_empty = [&](int s) { return bar0 + 8u * (2 * SX + SC + s); };
-    auto a_full = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SC + s); };
-    auto a_empty = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SC + SA + s); };
-    const uint32_t tfull = bar0 + 8u * (2 * (SX + SC + SA)), tempty = tfull + 8u, fin = tfull + 16u;
+    // stage barriers: block `it` uses full/empty(it % SA)
+    auto full = [&](uint32_t s) { return bar0 + 8u * s; };
+    auto empty = [&](uint32_t s) { return bar0 + 8u * (SA + s); };
+    auto c_full = [&](int s) { return bar0 + 8u * (2 * SA + s); };
+    auto c_empty = [&](int s) { return bar0 + 8u * (2 * SA + SC + s); };
+    const uint32_t tfull = bar0 + 8u * (2 * (SA + SC)), tempty = tfull + 8u, fin = tfull + 16u;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < SX; ++s) { mbar_init(x_full(s), 1); mbar_init(x_empty(s), 1); }
+        // full: the X producer's expect_tx arrival plus one arrival per dequant warp
+        for (int s = 0; s < SA; ++s) { mbar_init(full(s), 5); mbar_init(empty(s), 1); }
         for (int s = 0; s < SC; ++s) { mbar_init(c_full(s), 1); mbar_init(c_empty(s), 4); }
-        for (int s = 0; s < SA; ++s) { mbar_init(a_full(s), 4); mbar_init(a_empty(s), 1); }
         mbar_init(tfull, 1);
         mbar_init(tempty, 4);
         mbar_init(fin, 1);
@@ -246,20 +248,26 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     if (warp == 0) {
         // ------------------------------------------------ X / s*XA producer
         if (lane == 0) {
-            uint32_t it = 0;
+            // X slot it % SX is free once block it - SX has been consumed
+            uint32_t it = 0, sx = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
                 const int tok0 = (tile % p.tiles_tok) * kTileTok;
                 for (int kb = 0; kb < KBT; ++kb, ++it) {
-                    const int s = it % SX;
-                    if (!mbar_wait(x_empty(s), ((it / SX) & 1u) ^ 1u, abort)) { ok = false; break; }
-                    mbar_arrive_expect_tx(x_full(s), kTokStage);
-                    if (kb < KB) tma_load_2d(smem_addr(xs + s * kTokStage), &tm_x, x_full(s), kb * 64, tok0);
-                    else tma_load_2d(smem_addr(xs + s * kTokStage), &tm_xa, x_full(s), (kb - KB) * 64, tok0);
+                    if (it >= (uint32_t)SX) {
+                        const uint32_t b = it - SX;
+                        if (!mbar_wait(empty(b % SA), (b / SA) & 1u, abort)) { ok = false; break; }
+                    }
+                    const uint32_t bar = full(it % SA), dst = smem_addr(xs + sx * kTokStage);
+                    mbar_arrive_expect_tx(bar, kTokStage);
+                    if (kb < KB) tma_load_2d(dst, &tm_x, bar, kb * 64, tok0);
+                    else tma_load_2d(dst, &tm_xa, bar, (kb - KB) * 64, tok0);
+                    sx = sx + 1 == (uint32_t)SX ? 0u : sx + 1;
                 }
             }
+            // the last SX copies may still be in flight: wait for their stages
             const uint32_t first = it > (uint32_t)SX ? it - SX : 0;
-            for (uint32_t i = first; i < it; ++i) drain_wait(x_full(i % SX), (i / SX) & 1u);
+            for (uint32_t i = first; i < it; ++i) drain_wait(full(i % SA), (i / SA) & 1u);
         }
     } else if (warp == 14) {
         // ------------------------------------------------ code-tile producer
@@ -287,46 +295,50 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            // A tcgen05.mma issue returns only once the tensor core has taken the
-            // previous MMA, so any bookkeeping done after a K block's last MMA leaves the
-            // tensor core idle. It is therefore slotted between the MMAs: the previous
-            // block's slots are released after MMA 0 and MMA 1 (each commit covers every
-            // earlier MMA), and the next block's operands are probed without blocking
-            // after MMA 2 and MMA 3; only operands that are actually late are waited for.
+            // The tensor core queues only about two MMAs, and each instruction of this
+            // thread costs tens of cycles, so its own work per K block (4 MMAs, ~512 cycles
+            // of tensor work) has to stay small: ring positions are counters, descriptors
+            // advance by constants, one barrier is tested (without blocking, between
+            // MMAs) and one commit releases the previous block's stage.
+            static_assert((SA & (SA - 1)) == 0 && SX <= SA, "stage ring: power of two, at least the X ring");
             const uint32_t idesc = idesc_bf16(kTileRows, kTileTok, false, false);
-            uint32_t it = 0, lt = 0;
+            const uint64_t xdesc0 = sw128_desc(smem_addr(xs), 16, 1024);   // +2048 per 32 KB stage, +2 per K16
+            const uint32_t dD = tmem + kTmemD, dA0 = tmem + kTmemA;
+            uint32_t st = 0, ph = 0, sx = 0;   // stage slot (= TMEM slot) and parity, X slot
+            uint32_t pst = 0;                  // stage slot of the previous block
+            uint32_t lt = 0;
             bool ok = true;
-            auto ready = [&](uint32_t i) {
-                return mbar_test(x_full(i % SX), (i / SX) & 1u) && mbar_test(a_full(i % SA), (i / SA) & 1u);
-            };
-            auto wait_operands = [&](uint32_t i) {
-                return mbar_wait(x_full(i % SX), (i / SX) & 1u, abort) && mbar_wait(a_full(i % SA), (i / SA) & 1u, abort);
-            };
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++lt) {
-                if (!mbar_wait(tempty, (lt & 1u) ^ 1u, abort) || !wait_operands(it)) { ok = false; break; }
+                if (!mbar_wait(tempty, (lt & 1u) ^ 1u, abort) || !mbar_wait(full(st), ph, abort)) { ok = false; break; }
                 tc_fence_after();
-                for (int kb = 0; kb < KBT; ++kb, ++it) {
-                    const uint32_t a = tmem + kTmemA + 32u * (it % SA);
-                    const uint32_t xb = smem_addr(xs + (it % SX) * kTokStage);
-                    const int nk = kb < KB ? 4 : min(4, (p.r - (kb - KB) * 64 + 15) / 16);
-                    const bool has_next = kb + 1 < KBT;
+                for (int kb = 0; kb < KBT; ++kb) {
+                    const uint64_t xd = xdesc0 + ((uint64_t)sx << 11);
+                    const uint32_t ad = dA0 + (st << 5);
+                    const uint32_t nst = (st + 1) & (SA - 1), nph = ph ^ (nst == 0 ? 1u : 0u);
+                    const uint32_t nsx = sx + 1 == (uint32_t)SX ? 0u : sx + 1;
+                    const bool first = kb == 0, has_next = kb + 1 < KBT;
                     bool next_ready = !has_next;
-                    for (int k = 0; k < 4; ++k) {
-                        if (k < nk)
-                            mma_ts(tmem + kTmemD, a + 8u * k, sw128_desc(xb + 32u * k, 16, 1024), idesc,
-                                   (kb | k) != 0 ? 1u : 0u);
-                        if (k == 0 && kb > 0) mma_commit(x_empty((it - 1) % SX));
-                        else if (k == 1 && kb > 0) mma_commit(a_empty((it - 1) % SA));
-                        else if (k >= 2 && !next_ready) next_ready = ready(it + 1);
+                    if (kb < KB) {
+                        mma_ts(dD, ad, xd, idesc, first ? 0u : 1u);
+                        if (!first) mma_commit(empty(pst));
+                        mma_ts(dD, ad + 8u, xd + 2u, idesc, 1u);
+                        if (has_next) next_ready = mbar_test(full(nst), nph);
+                        mma_ts(dD, ad + 16u, xd + 4u, idesc, 1u);
+                        mma_ts(dD, ad + 24u, xd + 6u, idesc, 1u);
+                    } else {
+                        // adapter block (kb >= KB >= 1): up to four K16 steps of the rank
+                        const int nk = min(4, (p.r - (kb - KB) * 64 + 15) / 16);
+                        for (int k = 0; k < nk; ++k) mma_ts(dD, ad + 8u * k, xd + 2u * k, idesc, 1u);
+                        mma_commit(empty(pst));
                     }
                     if (has_next) {
-                        if (!next_ready && !wait_operands(it + 1)) { ok = false; break; }
+                        if (!next_ready && !mbar_wait(full(nst), nph, abort)) { ok = false; break; }
                         tc_fence_after();
                     }
+                    pst = st; st = nst; ph = nph; sx = nsx;
                 }
                 if (!ok) break;
-                mma_commit(x_empty((it - 1) % SX));
-                mma_commit(a_empty((it - 1) % SA));
+                mma_commit(empty(pst));
                 mma_commit(tfull);
             }
             mma_commit(fin);          // every MMA of this CTA has completed before TMEM is released
@@ -372,7 +384,7 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                     if (j >= J) break;
                     const int kb = kb_first + 2 * j;
                     const uint32_t itj = it0 + (uint32_t)kb;
-                    const int sa = itj % SA;
+                    const uint32_t sa = itj % SA;
                     const int8_t q8 = ring.q8[u];
                     const float s2 = ring.s2[u];
                     ring.load(u, p.w, valid, n, kbs, kb + 2 * kRing, KB);
@@ -404,7 +416,7 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                             v[i] = lo | (hi << 16);
                         }
                     }
-                    if (!mbar_wait(a_empty(sa), ((itj / SA) & 1u) ^ 1u, abort)) { ok = false; break; }
+                    if (!mbar_wait(empty(sa), ((itj / SA) & 1u) ^ 1u, abort)) { ok = false; break; }
                     tc_fence_after();
                     tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + kTmemA + 32u * sa, v);
                     tmem_wait_st();
@@ -414,7 +426,7 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                     // the codes read from it, so those reads have certainly completed
                     if (lane == 0) {
                         if (code_slot >= 0) mbar_arrive(c_empty(code_slot));
-                        mbar_arrive(a_full(sa));
+                        mbar_arrive(full(sa));
                     }
                 }
             }
@@ -435,9 +447,10 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
 // ================================================================ dgrad
 // Same warp roles; the dequant warps write W^ tiles (64 weight rows x 128
 // d_in) into shared memory in the MN-major 128-byte-swizzled layout and the
-// MMA reads them as its A operand; dY tiles come by TMA as B.
+// MMA reads them as its A operand; dY tiles come by TMA as B. The dY and W^
+// rings have the same size and share one full/empty barrier pair per K block.
 namespace dg {
-constexpr int SX = 4;                        // dY / s*G tiles (32 KB); SX <= SA
+constexpr int SX = 4;                        // dY / s*G tiles (32 KB); SX == SA
 constexpr int SCG = 2;                       // code tiles per dequant group (4 KB: 64 rows x 64 bytes, 64-byte swizzle)
 constexpr int SA = 4;                        // dequantised A tiles (16 KB: 2 MN chunks of 64 d_in x 64 K rows); even
 constexpr int SC = 2 * SCG;
@@ -456,7 +469,7 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
               const __grid_constant__ CUtensorMap tm_dx, FusedParams p, Codebook cb) {
     using namespace dg;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t bars[2 * (SX + SC + SA) + 3];
+    __shared__ __align__(8) uint64_t bars[2 * (SA + SC) + 3];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
 
@@ -467,21 +480,18 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
     uint8_t *staging = cs + SC * kCodeStage;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t bar0 = smem_addr(bars);
-    auto x_full = [&](int s) { return bar0 + 8u * s; };
-    auto x_empty = [&](int s) { return bar0 + 8u * (SX + s); };
-    auto c_full = [&](int s) { return bar0 + 8u * (2 * SX + s); };
-    auto c_empty = [&](int s) { return bar0 + 8u * (2 * SX + SC + s); };
-    auto a_full = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SC + s); };
-    auto a_empty = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SC + SA + s); };
-    const uint32_t tfull = bar0 + 8u * (2 * (SX + SC + SA)), tempty = tfull + 8u, fin = tfull + 16u;
+    static_assert(SX == SA && (SA & (SA - 1)) == 0, "one stage ring for dY and W^ tiles");
+    auto full = [&](uint32_t s) { return bar0 + 8u * s; };
+    auto empty = [&](uint32_t s) { return bar0 + 8u * (SA + s); };
+    auto c_full = [&](int s) { return bar0 + 8u * (2 * SA + s); };
+    auto c_empty = [&](int s) { return bar0 + 8u * (2 * SA + SC + s); };
+    const uint32_t tfull = bar0 + 8u * (2 * (SA + SC)), tempty = tfull + 8u, fin = tfull + 16u;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < SX; ++s) { mbar_init(x_full(s), 1); mbar_init(x_empty(s), 1); }
+        // full: the producer's expect_tx arrival plus one arrival per dequant warp. The
+        // A tile of an adapter block comes by TMA; its dequant group still arrives.
+        for (int s = 0; s < SA; ++s) { mbar_init(full(s), 5); mbar_init(empty(s), 1); }
         for (int s = 0; s < SC; ++s) { mbar_init(c_full(s), 1); mbar_init(c_empty(s), 4); }
-        // an A stage is filled either by the 4 dequant warps of a group (main
-        // blocks) or by TMA (adapter blocks); the group still arrives for the
-        // latter, and the producer adds the expected bytes
-        for (int s = 0; s < SA; ++s) { mbar_init(a_full(s), 4); mbar_init(a_empty(s), 1); }
         mbar_init(tfull, 1);
         mbar_init(tempty, 4);
         mbar_init(fin, 1);
@@ -516,24 +526,21 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
                 const int tok0 = (tile % p.tiles_tok) * kTileTok, col0 = (tile / p.tiles_tok) * kTileRows;
                 for (int kb = 0; kb < KBT; ++kb, ++it) {
-                    const int s = it % SX;
-                    if (!mbar_wait(x_empty(s), ((it / SX) & 1u) ^ 1u, abort)) { ok = false; break; }
+                    const uint32_t s = it % SA;
+                    if (!mbar_wait(empty(s), ((it / SA) & 1u) ^ 1u, abort)) { ok = false; break; }
                     if (kb < KB) {
-                        mbar_arrive_expect_tx(x_full(s), kTokStage);
-                        tma_load_2d(smem_addr(bs + s * kTokStage), &tm_dy, x_full(s), kb * 64, tok0);
+                        mbar_arrive_expect_tx(full(s), kTokStage);
+                        tma_load_2d(smem_addr(bs + s * kTokStage), &tm_dy, full(s), kb * 64, tok0);
                     } else {
-                        // the adapter A tile goes into the A ring slot of this iteration,
-                        // which the dequant group has released (it waited a_empty)
-                        const int sa = it % SA;
-                        if (!mbar_wait(a_empty(sa), ((it / SA) & 1u) ^ 1u, abort)) { ok = false; break; }
-                        mbar_arrive_expect_tx(x_full(s), kTokStage + kAStage);
-                        tma_load_2d(smem_addr(as + sa * kAStage), &tm_alora, x_full(s), (kb - KB) * 64, col0);
-                        tma_load_2d(smem_addr(bs + s * kTokStage), &tm_gs, x_full(s), (kb - KB) * 64, tok0);
+                        // the adapter A tile goes into the A slot of this stage
+                        mbar_arrive_expect_tx(full(s), kTokStage + kAStage);
+                        tma_load_2d(smem_addr(as + s * kAStage), &tm_alora, full(s), (kb - KB) * 64, col0);
+                        tma_load_2d(smem_addr(bs + s * kTokStage), &tm_gs, full(s), (kb - KB) * 64, tok0);
                     }
                 }
             }
-            const uint32_t first = it > (uint32_t)SX ? it - SX : 0;
-            for (uint32_t i = first; i < it; ++i) drain_wait(x_full(i % SX), (i / SX) & 1u);
+            const uint32_t first = it > (uint32_t)SA ? it - SA : 0;
+            for (uint32_t i = first; i < it; ++i) drain_wait(full(i % SA), (i / SA) & 1u);
         }
     } else if (warp == 14) {
         // ------------------------------------------------ code-tile producer
@@ -559,46 +566,45 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            // bookkeeping slotted between the MMAs, as in the forward kernel
+            // the same lean issue loop as the forward kernel
             const uint32_t idesc_main = idesc_bf16(kTileRows, kTileTok, true, false);
             const uint32_t idesc_lora = idesc_bf16(kTileRows, kTileTok, false, false);
-            uint32_t it = 0, lt = 0;
+            const uint64_t adesc0 = sw128_desc(smem_addr(as), 8192, 1024);   // MN-major W^: +1024 per 16 KB stage, +128 per K16
+            const uint64_t ldesc0 = sw128_desc(smem_addr(as), 16, 1024);     // K-major adapter tile: +2 per K16
+            const uint64_t bdesc0 = sw128_desc(smem_addr(bs), 16, 1024);     // +2048 per 32 KB stage, +2 per K16
+            uint32_t st = 0, ph = 0, pst = 0;
+            uint32_t lt = 0;
             bool ok = true;
-            auto ready = [&](uint32_t i) {
-                return mbar_test(x_full(i % SX), (i / SX) & 1u) && mbar_test(a_full(i % SA), (i / SA) & 1u);
-            };
-            auto wait_operands = [&](uint32_t i) {
-                return mbar_wait(x_full(i % SX), (i / SX) & 1u, abort) && mbar_wait(a_full(i % SA), (i / SA) & 1u, abort);
-            };
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++lt) {
-                if (!mbar_wait(tempty, (lt & 1u) ^ 1u, abort) || !wait_operands(it)) { ok = false; break; }
+                if (!mbar_wait(tempty, (lt & 1u) ^ 1u, abort) || !mbar_wait(full(st), ph, abort)) { ok = false; break; }
                 tc_fence_after();
-                for (int kb = 0; kb < KBT; ++kb, ++it) {
-                    const uint32_t ab = smem_addr(as + (it % SA) * kAStage);
-                    const uint32_t bb = smem_addr(bs + (it % SX) * kTokStage);
-                    const bool main = kb < KB;
-                    const int nk = main ? 4 : min(4, (p.r - (kb - KB) * 64 + 15) / 16);
-                    const bool has_next = kb + 1 < KBT;
+                for (int kb = 0; kb < KBT; ++kb) {
+                    const uint64_t bd = bdesc0 + ((uint64_t)st << 11);
+                    const uint32_t nst = (st + 1) & (SA - 1), nph = ph ^ (nst == 0 ? 1u : 0u);
+                    const bool first = kb == 0, has_next = kb + 1 < KBT;
                     bool next_ready = !has_next;
-                    for (int k = 0; k < 4; ++k) {
-                        if (k < nk) {
-                            const uint64_t ad = main ? sw128_desc(ab + 2048u * k, 8192, 1024)
-                                                     : sw128_desc(ab + 32u * k, 16, 1024);
-                            mma_ss(tmem, ad, sw128_desc(bb + 32u * k, 16, 1024), main ? idesc_main : idesc_lora,
-                                   (kb | k) != 0 ? 1u : 0u);
-                        }
-                        if (k == 0 && kb > 0) mma_commit(x_empty((it - 1) % SX));
-                        else if (k == 1 && kb > 0) mma_commit(a_empty((it - 1) % SA));
-                        else if (k >= 2 && !next_ready) next_ready = ready(it + 1);
+                    if (kb < KB) {
+                        const uint64_t ad = adesc0 + ((uint64_t)st << 10);
+                        mma_ss(tmem, ad, bd, idesc_main, first ? 0u : 1u);
+                        if (!first) mma_commit(empty(pst));
+                        mma_ss(tmem, ad + 128u, bd + 2u, idesc_main, 1u);
+                        if (has_next) next_ready = mbar_test(full(nst), nph);
+                        mma_ss(tmem, ad + 256u, bd + 4u, idesc_main, 1u);
+                        mma_ss(tmem, ad + 384u, bd + 6u, idesc_main, 1u);
+                    } else {
+                        const uint64_t ad = ldesc0 + ((uint64_t)st << 10);
+                        const int nk = min(4, (p.r - (kb - KB) * 64 + 15) / 16);
+                        for (int k = 0; k < nk; ++k) mma_ss(tmem, ad + 2u * k, bd + 2u * k, idesc_lora, 1u);
+                        mma_commit(empty(pst));
                     }
                     if (has_next) {
-                        if (!next_ready && !wait_operands(it + 1)) { ok = false; break; }
+                        if (!next_ready && !mbar_wait(full(nst), nph, abort)) { ok = false; break; }
                         tc_fence_after();
                     }
+                    pst = st; st = nst; ph = nph;
                 }
                 if (!ok) break;
-                mma_commit(x_empty((it - 1) % SX));
-                mma_commit(a_empty((it - 1) % SA));
+                mma_commit(empty(pst));
                 mma_commit(tfull);
             }
             mma_commit(fin);
@@ -654,7 +660,7 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
                     if (j >= J) break;
                     const int kb = kb_first + 2 * j;
                     const uint32_t itj = it0 + (uint32_t)kb;
-                    const int sa = itj % SA;
+                    const uint32_t sa = itj % SA;
                     bool valid;
                     blk_of(kb, valid);
                     const int8_t q8 = ring.q8[u];
@@ -680,7 +686,7 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
 #pragma unroll
                             for (int i = 0; i < 32; ++i) v[i] = 0u;
                         }
-                        if (!mbar_wait(a_empty(sa), ((itj / SA) & 1u) ^ 1u, abort)) { ok = false; break; }
+                        if (!mbar_wait(empty(sa), ((itj / SA) & 1u) ^ 1u, abort)) { ok = false; break; }
                         uint8_t *dst = as + sa * kAStage + chunk * 8192;
 #pragma unroll
                         for (int c = 0; c < 8; ++c)
@@ -688,15 +694,16 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
                                 make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
                         fence_proxy_async_smem();
                     } else {
-                        // adapter block: the producer's TMA fills the A slot
-                        if (!mbar_wait(a_empty(sa), ((itj / SA) & 1u) ^ 1u, abort)) { ok = false; break; }
+                        // adapter block: the producer's TMA fills the A slot; the group only
+                        // keeps the stage's arrival count
+                        if (!mbar_wait(empty(sa), ((itj / SA) & 1u) ^ 1u, abort)) { ok = false; break; }
                     }
                     __syncwarp();
                     // the code slot is released only after the A-tile stores that depend on the
                     // codes read from it, so those reads have certainly completed
                     if (lane == 0) {
                         if (code_slot >= 0) mbar_arrive(c_empty(code_slot));
-                        mbar_arrive(a_full(sa));
+                        mbar_arrive(full(sa));
                     }
                 }
             }
@@ -882,46 +889,6 @@ __global__ void k_reduce_f32_t(const float *__restrict__ part, int splits, int64
 }
 
 // ================================================================ host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-// 2D tensor map: dim0 = inner (contiguous) extent, dim1 = outer extent,
-// row stride in bytes; box {box0, box1}; out-of-range elements read as zero.
-static bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
-                     uint64_t stride_bytes, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {stride_bytes};
-    cuuint32_t box[2] = {box0, box1};
-    cuuint32_t es[2] = {1, 1};
-    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-static bool map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box0, uint32_t box1,
-                     CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
-    return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, inner, outer, inner * 2, box0, box1, sw);
-}
-
-template <typename K>
-static cudaError_t set_smem(K kernel, int bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-}
-
 constexpr int kTargetCtas = 296;   // split-K sizing target (two waves of 148 SMs)
 
 struct SplitPlan { int kb_total, kb_per_split, splits; };
@@ -991,10 +958,19 @@ static unsigned reduce_grid(int64_t count) {
 
 static size_t mr_bytes(int64_t M, int r) { return align256((size_t)M * (size_t)r * 2); }
 
+// From this many tokens on, the layer dequantises W once into bf16 scratch and
+// runs the CTA-pair GEMM: the fused kernel would repeat the dequantisation for
+// every 256-token tile, and at two or more tiles that integer work costs more
+// than writing and re-reading the bf16 copy.
+constexpr int64_t kPairGemmMinM = 512;
+static size_t wd_bytes(int64_t rows, int64_t cols) { return align256((size_t)rows * (size_t)cols * 2); }
+
+static size_t fwd_adapter_bytes(int64_t M, int64_t cols, int r) {
+    return r == 0 ? 0 : mr_bytes(M, r) + partial_bytes(M, cols, r);
+}
+
 size_t fwd_workspace_bytes_large(int64_t M, int64_t rows, int64_t cols, int r) {
-    (void)rows;
-    if (r == 0) return 0;
-    return mr_bytes(M, r) + partial_bytes(M, cols, r);
+    return fwd_adapter_bytes(M, cols, r) + (M >= kPairGemmMinM ? wd_bytes(rows, cols) : 0);
 }
 
 size_t xa_small_workspace(int64_t M, int64_t cols, int r) { return mr_bytes(M, r) + partial_bytes(M, cols, r); }
@@ -1010,7 +986,7 @@ cudaError_t launch_xa_small(const __nv_bfloat16 *X, int64_t M, int64_t cols, con
     return cudaGetLastError();
 }
 
-size_t bwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
+static size_t bwd_adapter_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
     if (r == 0) return 0;
     size_t part = partial_bytes(M, cols, r);                 // X*A
     size_t p2 = partial_bytes(M, rows, r);                   // dY*B^T
@@ -1020,6 +996,10 @@ size_t bwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
     if (p3 > part) part = p3;
     if (p4 > part) part = p4;
     return 2 * mr_bytes(M, r) + part;
+}
+
+size_t bwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
+    return bwd_adapter_bytes(M, rows, cols, r) + (M >= kPairGemmMinM ? wd_bytes(rows, cols) : 0);
 }
 
 static cudaError_t run_fused_fwd(const __nv_bfloat16 *X, int64_t M, const NF4View &W, const __nv_bfloat16 *XAs,
@@ -1095,6 +1075,14 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
         if (e != cudaSuccess) return e;
         QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, XA_save, XAs));
     }
+    if (M >= kPairGemmMinM) {
+        // Y = X W^T + (s XA) B: W^ [d_out, d_in] is the K-major B operand, B_lora [r, d_out]
+        // the MN-major extension
+        __nv_bfloat16 *Wd = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + fwd_adapter_bytes(M, W.cols, r));
+        cudaError_t e = launch_dequant(W, Wd, st);
+        if (e != cudaSuccess) return e;
+        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, st);
+    }
     return run_fused_fwd(X, M, W, XAs, B, r, Y, st);
 }
 
@@ -1120,7 +1108,17 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
         if (e != cudaSuccess) return e;
         QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, nullptr, Gs));
     }
-    e = run_fused_dgrad(dY, M, W, A, Gs, r, dX, st);
+    if (M >= kPairGemmMinM) {
+        // dX = dY W^ + (s G) A^T: W^ [d_out, d_in] read as the MN-major B operand
+        // ([K = d_out][N = d_in]), A_lora [d_in, r] the K-major extension
+        __nv_bfloat16 *Wd = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) +
+                                                              bwd_adapter_bytes(M, W.rows, W.cols, r));
+        e = launch_dequant(W, Wd, st);
+        if (e != cudaSuccess) return e;
+        e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, st);
+    } else {
+        e = run_fused_dgrad(dY, M, W, A, Gs, r, dX, st);
+    }
     if (e != cudaSuccess) return e;
     if (r > 0) {
         float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + 2 * mr_bytes(M, r));

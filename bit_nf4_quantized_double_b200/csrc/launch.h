@@ -9,6 +9,11 @@ cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlor
                             float *c1, double *part, cudaStream_t st);
 cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st);
 
+// Plain bf16 GEMM on CTA pairs (tcgen05 cta_group::2), see gemm2sm.cu.
+cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, const __nv_bfloat16 *B, bool b_mn,
+                           const __nv_bfloat16 *Be, bool be_mn, __nv_bfloat16 *C, int64_t M, int64_t N, int64_t K,
+                           int ke, cudaStream_t st);
+
 size_t fwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r);
 size_t bwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r);
 

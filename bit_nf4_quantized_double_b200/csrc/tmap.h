@@ -1,0 +1,53 @@
+// Host helpers shared by the tcgen05 kernel files: TMA tensor-map encoding
+// (through the driver entry point, so the library needs no -lcuda) and the
+// dynamic shared-memory opt-in.
+#pragma once
+
+#include <cuda.h>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace qnf4 {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2D tensor map: dim0 = inner (contiguous) extent, dim1 = outer extent,
+// row stride in bytes; box {box0, box1}; out-of-range elements read as zero.
+inline bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+                     uint64_t stride_bytes, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {stride_bytes};
+    cuuint32_t box[2] = {box0, box1};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+inline bool map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box0, uint32_t box1,
+                     CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
+    return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, inner, outer, inner * 2, box0, box1, sw);
+}
+
+template <typename K>
+inline cudaError_t set_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+}  // namespace qnf4

@@ -112,7 +112,9 @@ qlora_status qlora_nf4_dequant(const qlora_nf4_tensor *q, void *W_out, qlora_str
  *   XA_save  bf16 [M, r] receives X*A (unscaled) for the backward, or NULL.
  * Shapes: M >= 1, cols % 64 == 0, rows % 16 == 0, 0 <= r <= 256, r % 8 == 0
  * (r == 0: no adapter; A, B, XA_save ignored). M <= 16 takes the streaming GEMV
- * kernel, larger M the fused tcgen05 dequant-GEMM.
+ * kernel, 16 < M < 512 the fused tcgen05 dequant-GEMM, and M >= 512
+ * dequantises W once into bf16 in the workspace (rows * cols * 2 bytes of it)
+ * and runs a CTA-pair tcgen05 GEMM with the adapter term as extra K blocks.
  */
 size_t qlora_linear_fwd_workspace(int64_t M, int64_t rows, int64_t cols, int r);
 qlora_status qlora_linear_fwd(const void *X, int64_t M, const qlora_nf4_tensor *W,
@@ -128,7 +130,8 @@ qlora_status qlora_linear_fwd(const void *X, int64_t M, const qlora_nf4_tensor *
  *   dA = s * X^T * G                       fp32 [cols, r]  (overwritten)
  *   dB = s * (X*A)^T * dY                  fp32 [r, rows]  (overwritten)
  *   XA  bf16 [M, r] saved by the forward, or NULL to recompute it.
- * Shapes as for the forward, with M >= 1.
+ * Shapes as for the forward, with M >= 1. For M >= 512 the workspace also
+ * holds the bf16 dequantised weight (rows * cols * 2 bytes), as in the forward.
  */
 size_t qlora_linear_bwd_workspace(int64_t M, int64_t rows, int64_t cols, int r);
 qlora_status qlora_linear_bwd(const void *X, const void *dY, int64_t M, const qlora_nf4_tensor *W,

@@ -63,7 +63,11 @@ def test_workspace_queries_positive():
     for M in (1, 16, 17, 4096):
         assert L.qlora_linear_fwd_workspace(M, 4096, 4096, 64) > 0
         assert L.qlora_linear_bwd_workspace(M, 4096, 4096, 64) > 0
-    assert L.qlora_linear_bwd_workspace(4096, 4096, 4096, 0) == 0
+    # no adapter and a small batch: nothing to stage
+    assert L.qlora_linear_bwd_workspace(256, 4096, 4096, 0) == 0
+    # from 512 tokens on, the layer keeps a bf16 copy of the dequantised weight
+    assert L.qlora_linear_bwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2
+    assert L.qlora_linear_fwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2
 
 
 def test_status_strings():
