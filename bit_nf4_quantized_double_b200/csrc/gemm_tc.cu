@@ -729,11 +729,12 @@ struct SkinnyParams {
     int Mp, Np, BN;        // output rows, columns (r), MMA N (Np rounded up to 16)
     int kb_total, kb_per_split;
     int stages;
+    int transpose;         // partials as [split][Np][Mp] instead of [split][Mp][Np]
     float *partial;
 };
 
 template <bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128, 2)
 k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, SkinnyParams p) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[2 * 8 + 2];
@@ -831,11 +832,15 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
         tc_fence_after();
         const int row = m0 + warp * 32 + lane;
         float *dst = p.partial + ((int64_t)split * p.Mp + row) * p.Np;
+        float *dst_t = p.partial + (int64_t)split * p.Np * p.Mp + row;   // column j at dst_t[j * Mp]
         for (int c = 0; c < p.BN; c += 16) {
             uint32_t v[16];
             tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
             tmem_wait_ld();
-            if (row < p.Mp) {
+            if (row < p.Mp && p.transpose) {
+                // lanes hold consecutive rows: each column j is one coalesced store per warp
+                for (int i = 0; i < 16 && c + i < p.Np; ++i) dst_t[(int64_t)(c + i) * p.Mp] = __uint_as_float(v[i]);
+            } else if (row < p.Mp) {
                 if (c + 16 <= p.Np) {
 #pragma unroll
                     for (int i = 0; i < 16; i += 4)
@@ -859,44 +864,59 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
 
 // ------------------------------------------------------------------ reduce
 // Sums of split-K partials in split order (deterministic), then scale/convert.
+// Each thread takes four consecutive elements and issues the loads of all
+// splits before adding, so the HBM latencies overlap.
+constexpr int kMaxSplits = 16;
+__device__ __forceinline__ float4 sum_splits4(const float *__restrict__ part, int splits, int64_t count, int64_t i) {
+    float4 v[kMaxSplits];
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp)
+        if (sp < splits) v[sp] = __ldg(reinterpret_cast<const float4 *>(part + sp * count + i));
+    float4 acc = v[0];
+#pragma unroll
+    for (int sp = 1; sp < kMaxSplits; ++sp)
+        if (sp < splits) {
+            acc.x += v[sp].x;
+            acc.y += v[sp].y;
+            acc.z += v[sp].z;
+            acc.w += v[sp].w;
+        }
+    return acc;
+}
+// count % 4 == 0 (counts are multiples of r, itself a multiple of 8)
 __global__ void k_reduce_xa(const float *__restrict__ part, int splits, int64_t count, float s,
                             __nv_bfloat16 *__restrict__ xa, __nv_bfloat16 *__restrict__ xas) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
-        float v = 0.0f;
-        for (int sp = 0; sp < splits; ++sp) v += part[sp * count + i];
-        if (xa) xa[i] = __float2bfloat16_rn(v);
-        if (xas) xas[i] = __float2bfloat16_rn(s * v);
+    for (int64_t i = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < count; i += 4 * (int64_t)gridDim.x * blockDim.x) {
+        const float4 v = sum_splits4(part, splits, count, i);
+        if (xa) {
+            *reinterpret_cast<uint2 *>(xa + i) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+        }
+        if (xas) {
+            *reinterpret_cast<uint2 *>(xas + i) =
+                make_uint2(pack_bf16x2(s * v.x, s * v.y), pack_bf16x2(s * v.z, s * v.w));
+        }
     }
 }
 __global__ void k_reduce_f32(const float *__restrict__ part, int splits, int64_t count, float s,
                              float *__restrict__ out) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
-        float v = 0.0f;
-        for (int sp = 0; sp < splits; ++sp) v += part[sp * count + i];
-        out[i] = s * v;
-    }
-}
-// part [split][rows][r] -> out [r][rows] (transposed), times s
-__global__ void k_reduce_f32_t(const float *__restrict__ part, int splits, int64_t rows, int r, float s,
-                               float *__restrict__ out) {
-    const int64_t count = rows * r;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t j = i / rows, n = i % rows;   // output index [j][n], coalesced over n
-        float v = 0.0f;
-        for (int sp = 0; sp < splits; ++sp) v += part[sp * count + n * r + j];
-        out[i] = s * v;
+    for (int64_t i = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < count; i += 4 * (int64_t)gridDim.x * blockDim.x) {
+        const float4 v = sum_splits4(part, splits, count, i);
+        *reinterpret_cast<float4 *>(out + i) = make_float4(s * v.x, s * v.y, s * v.z, s * v.w);
     }
 }
 
 // ================================================================ host side
-constexpr int kTargetCtas = 296;   // split-K sizing target (two waves of 148 SMs)
+// Split-K sizing: at most two CTAs per SM (each holds at most kSkinnyStages
+// stages), all resident at once, at most kMaxSplits partials per output.
+constexpr int kSkinnyStages = 4;
 
 struct SplitPlan { int kb_total, kb_per_split, splits; };
 static SplitPlan plan_splits(int64_t Mp, int64_t Kp) {
     SplitPlan sp;
     sp.kb_total = (int)ceil_div(Kp, 64);
     const int mt = (int)ceil_div(Mp, 128);
-    int want = (int)ceil_div(kTargetCtas, mt);
+    int want = (2 * num_sms()) / mt;
+    if (want > kMaxSplits) want = kMaxSplits;
     if (want < 1) want = 1;
     if (want > sp.kb_total) want = sp.kb_total;
     sp.kb_per_split = (int)ceil_div(sp.kb_total, want);
@@ -910,7 +930,8 @@ static size_t partial_bytes(int64_t Mp, int64_t Kp, int r) {
 // Launch one skinny product. A operand: K-major [Mp rows, Kp] or MN-major
 // [Kp rows, Mp]; B operand: K-major [r rows, Kp] or MN-major [Kp rows, r].
 static cudaError_t run_skinny(bool a_mn, const void *a, int64_t a_ld_rows, bool b_mn, const void *b, int64_t Mp,
-                              int64_t Kp, int r, float *partial, int *splits_out, cudaStream_t st) {
+                              int64_t Kp, int r, float *partial, int *splits_out, cudaStream_t st,
+                              bool transpose = false) {
     CUtensorMap ta, tb;
     const int BN = (int)ceil_div(r, 16) * 16;
     bool ok;
@@ -928,10 +949,11 @@ static cudaError_t run_skinny(bool a_mn, const void *a, int64_t a_ld_rows, bool 
     p.kb_total = sp.kb_total;
     p.kb_per_split = sp.kb_per_split;
     p.partial = partial;
+    p.transpose = transpose ? 1 : 0;
     const int b_bytes = b_mn ? (int)ceil_div(BN, 64) * 8192 : BN * 128;
     const int stage = 128 * 128 + ((b_bytes + 1023) & ~1023);
-    int stages = (200 * 1024) / stage;
-    if (stages > 8) stages = 8;
+    int stages = (100 * 1024) / stage;
+    if (stages > kSkinnyStages) stages = kSkinnyStages;
     if (stages > sp.kb_per_split) stages = sp.kb_per_split < 2 ? 2 : sp.kb_per_split;
     p.stages = stages;
     const int smem = 1024 + stages * stage;
@@ -951,7 +973,7 @@ static cudaError_t run_skinny(bool a_mn, const void *a, int64_t a_ld_rows, bool 
 }
 
 static unsigned reduce_grid(int64_t count) {
-    int64_t g = ceil_div(count, 256);
+    int64_t g = ceil_div(count, 4 * 256);
     const int64_t cap = (int64_t)num_sms() * 8;
     return (unsigned)(g < 1 ? 1 : (g > cap ? cap : g));
 }
@@ -1127,10 +1149,10 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
         e = run_skinny(true, X, M, true, Gs, W.cols, M, r, part, &splits, st);
         if (e != cudaSuccess) return e;
         QNF4_LAUNCH("k_reduce_f32", st, k_reduce_f32<<<reduce_grid(W.cols * r), 256, 0, st>>>(part, splits, W.cols * r, 1.0f, dA));
-        // dB = s (XA)^T dY, computed as (dY^T XA)^T
-        e = run_skinny(true, dY, M, true, XA, W.rows, M, r, part, &splits, st);
+        // dB = s (XA)^T dY, computed as (dY^T XA)^T with the partials written transposed
+        e = run_skinny(true, dY, M, true, XA, W.rows, M, r, part, &splits, st, true);
         if (e != cudaSuccess) return e;
-        QNF4_LAUNCH("k_reduce_f32_t", st, k_reduce_f32_t<<<reduce_grid(W.rows * r), 256, 0, st>>>(part, splits, W.rows, r, s, dB));
+        QNF4_LAUNCH("k_reduce_f32", st, k_reduce_f32<<<reduce_grid(W.rows * r), 256, 0, st>>>(part, splits, W.rows * r, s, dB));
     }
     return cudaGetLastError();
 }

@@ -218,42 +218,57 @@ k_double_quant(const float *__restrict__ c1, int64_t nb, int64_t nb2, const floa
     }
 }
 
-// Dequantisation: each thread expands 16 code bytes (32 weights, half a
-// block) into 64 bytes of bf16. Codebook in shared memory (16 distinct words,
-// so lookups from a warp never conflict).
+// Dequantisation: each thread expands one 32-bit word of codes (8 weights) into
+// one 16-byte bf16 store, so a warp reads 128 contiguous code bytes and writes
+// 512 contiguous output bytes; four independent words per thread are in flight
+// at once. Codebook in shared memory (16 distinct words: lookups never
+// conflict). A ragged tail (n % 8 != 0) is written element by element.
+constexpr int kDequantUnroll = 4;
 __global__ void __launch_bounds__(256)
 k_dequant(NF4View q, int64_t n, Codebook cb, __nv_bfloat16 *__restrict__ out) {
     __shared__ float s_q[16];
     if (threadIdx.x < 16) s_q[threadIdx.x] = cb.q[threadIdx.x];
     __syncthreads();
     const float mu = *q.offset;
-    const int64_t nchunk = (n + 31) / 32;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < nchunk; c += stride) {
-        const int64_t e0 = c * 32;
-        const int64_t b = e0 / kBlock1;
-        const float ch = dq_constant(q.scale8[b], q.scale2[b / kBlock2], mu);
-        if (e0 + 32 <= n) {
-            const uint4 raw = ldg_nc_v4(q.codes + e0 / 2);
-            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-            uint32_t o[16];
+    const int64_t n8 = n / 8;
+    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+    const uint32_t *codes = reinterpret_cast<const uint32_t *>(q.codes);
+    for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g0 < n8; g0 += kDequantUnroll * nthr) {
+        uint32_t w[kDequantUnroll];
+        int8_t q8[kDequantUnroll];
+        float s2[kDequantUnroll];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+        for (int u = 0; u < kDequantUnroll; ++u) {
+            const int64_t g = g0 + u * nthr;
+            if (g < n8) {
+                const int64_t b = g / (kBlock1 / 8);
+                w[u] = __ldg(codes + g);
+                q8[u] = __ldg(q.scale8 + b);
+                s2[u] = __ldg(q.scale2 + b / kBlock2);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kDequantUnroll; ++u) {
+            const int64_t g = g0 + u * nthr;
+            if (g < n8) {
+                const float ch = dq_constant(q8[u], s2[u], mu);
+                uint32_t o[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const uint32_t byte = (w[i] >> (8 * k)) & 0xffu;
-                    o[4 * i + k] = pack_bf16x2(__fmul_rn(s_q[byte >> 4], ch), __fmul_rn(s_q[byte & 15u], ch));
+                    const uint32_t byte = (w[u] >> (8 * k)) & 0xffu;
+                    o[k] = pack_bf16x2(__fmul_rn(s_q[byte >> 4], ch), __fmul_rn(s_q[byte & 15u], ch));
                 }
+                *reinterpret_cast<uint4 *>(out + 8 * g) = make_uint4(o[0], o[1], o[2], o[3]);
             }
-            uint4 *dst = reinterpret_cast<uint4 *>(out + e0);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-        } else {
-            for (int64_t e = e0; e < n; ++e) {
-                const uint8_t byte = q.codes[e / 2];
-                const uint32_t code = (e % 2 == 0) ? (byte >> 4) : (byte & 15u);
-                out[e] = __float2bfloat16_rn(__fmul_rn(s_q[code], ch));
-            }
+        }
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        for (int64_t e = 8 * n8; e < n; ++e) {
+            const int64_t b = e / kBlock1;
+            const float ch = dq_constant(q.scale8[b], q.scale2[b / kBlock2], mu);
+            const uint8_t byte = q.codes[e / 2];
+            const uint32_t code = (e % 2 == 0) ? (byte >> 4) : (byte & 15u);
+            out[e] = __float2bfloat16_rn(__fmul_rn(s_q[code], ch));
         }
     }
 }
@@ -274,9 +289,9 @@ cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlor
 
 cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st) {
     const int64_t n = q.rows * q.cols;
-    const int64_t nchunk = ceil_div(n, 32);
-    int64_t grid = ceil_div(nchunk, 256);
+    int64_t grid = ceil_div(ceil_div(n, 8 * kDequantUnroll), 256);
     const int64_t cap = (int64_t)num_sms() * 8;
+    if (grid < 1) grid = 1;
     if (grid > cap) grid = cap;
     QNF4_LAUNCH("k_dequant", st, k_dequant<<<(unsigned)grid, 256, 0, st>>>(q, n, host_codebook(), out));
     return cudaGetLastError();
