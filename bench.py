@@ -56,57 +56,78 @@ def load_peaks():
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons of this rank's GPU, polled through
+    NVML every ~2 ms on a background thread (the timed region lasts only a few
+    milliseconds); only samples taken between mark_begin() and mark_end() count.
+    Reads the settings only, changes none. Falls back to nvidia-smi -lms 200."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+        self.samples = []
+        self.t0 = self.t1 = None
+        self.thread = None
+        self.stop_flag = False
+        self.max_mhz = None
+        self.err = None
+
+    def _handle(self, nv):
+        import torch
+        try:
+            pr = torch.cuda.get_device_properties(self.gpu)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.gpu)
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
-        time.sleep(0.3)
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception as e:   # NVML missing: no samples, say why
+            self.err = f"nvml unavailable: {e}"
+            return
+
+        def poll():
+            while not self.stop_flag:
+                try:
+                    t = time.perf_counter()
+                    mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    try:
+                        rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                    except Exception:
+                        rs = int(nv.nvmlDeviceGetCurrentClocksThrottleReasons(h))
+                    self.samples.append((t, mhz, rs))
+                except Exception as e:
+                    self.err = str(e)
+                    return
+                time.sleep(0.002)
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
+        time.sleep(0.01)
+
+    def mark_begin(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
-        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
-        loaded = [v for v in sm if mx and v > 0.3 * max(mx)] or sm
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        self.stop_flag = True
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        t0 = self.t0 if self.t0 is not None else -1e30
+        t1 = self.t1 if self.t1 is not None else 1e30
+        inside = [x for x in self.samples if t0 <= x[0] <= t1]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz,
+                    "reasons": [self.err or "no samples in the timed region"], "samples": 0, "source": "nvml"}
+        reasons = sorted({name for _, _, rs in inside for bit, name in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median(m for _, m, _ in inside), "sm_min_mhz": min(m for _, m, _ in inside),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside), "source": "nvml, 2 ms"}
 
 
 # ------------------------------------------------------------------ distributed
@@ -207,6 +228,7 @@ def run_ours(args, peaks, peak_kind):
     barrier(world)
     torch.cuda.synchronize()
     launches0 = q.qlora_launch_count()
+    clocks.mark_begin()
     for i in range(args.steps):
         flush.zero_()                     # L2 flush between timed steps (not timed)
         evs[i][0].record(stream)
@@ -214,6 +236,7 @@ def run_ours(args, peaks, peak_kind):
         evs[i][1].record(stream)
     launches = q.qlora_launch_count() - launches0
     torch.cuda.synchronize()
+    clocks.mark_end()
     barrier(world)
     clk = clocks.stop()
     total_ms = sum(a.elapsed_time(b) for a, b in evs)

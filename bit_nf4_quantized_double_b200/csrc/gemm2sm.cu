@@ -264,9 +264,12 @@ cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, cons
     p.ke = ke;
     p.tiles_m = (int)ceil_div(M, kTileM);
     p.tiles_n = (int)ceil_div(N, kTileN);
+    // as few pairs as give the same number of tile rounds: the work is as balanced
+    // as it can be, and the SMs left over are free for concurrent kernels
     const int ntiles = p.tiles_m * p.tiles_n;
     const int max_pairs = num_sms() / 2;
-    const int pairs = ntiles < max_pairs ? ntiles : max_pairs;
+    const int rounds = (int)ceil_div(ntiles, max_pairs);
+    const int pairs = (int)ceil_div(ntiles, rounds);
     cudaError_t e;
 #define QNF4_G2(BM, BEM)                                                                                  \
     e = set_smem(k_gemm2sm<BM, BEM>, kSmem);                                                            \

@@ -27,6 +27,8 @@
 // Both fused kernels keep the accumulator tile D[row, token] in TMEM and store
 // it transposed (out[token, row]) through a shared-memory staging tile and a
 // TMA store.
+#include <mutex>
+
 #include "launch.h"
 #include "tc.cuh"
 #include "tmap.h"
@@ -1108,6 +1110,48 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
     return run_fused_fwd(X, M, W, XAs, B, r, Y, st);
 }
 
+// A second stream per device for work that can run beside other kernels: the
+// pair GEMM leaves SMs free (it uses as few CTA pairs as give the same number of
+// tile rounds) and is bound by the tensor pipe, while the adapter products and
+// the dequantisation are bound by memory. The mutex keeps each fork/join
+// sequence of events whole when several host threads call the library.
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+static std::mutex g_side_mu;
+static SideStream *side_stream_locked() {
+    static SideStream tab[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    SideStream &x = tab[dev];
+    if (!x.s) {
+        if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess) {
+            x = SideStream();
+            return nullptr;
+        }
+    }
+    return &x;
+}
+
+// dA = X^T (sG) and dB = s (XA)^T dY on stream `st` (they share the partial buffer,
+// so they run one after the other).
+static cudaError_t adapter_grads(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, int64_t M, const NF4View &W,
+                                 const __nv_bfloat16 *Gs, const __nv_bfloat16 *XA, int r, float s, float *dA,
+                                 float *dB, float *part, cudaStream_t st) {
+    int splits = 0;
+    cudaError_t e = run_skinny(true, X, M, true, Gs, W.cols, M, r, part, &splits, st);
+    if (e != cudaSuccess) return e;
+    QNF4_LAUNCH("k_reduce_f32", st, k_reduce_f32<<<reduce_grid(W.cols * r), 256, 0, st>>>(part, splits, W.cols * r, 1.0f, dA));
+    // computed as (dY^T XA)^T with the partials written transposed
+    e = run_skinny(true, dY, M, true, XA, W.rows, M, r, part, &splits, st, true);
+    if (e != cudaSuccess) return e;
+    QNF4_LAUNCH("k_reduce_f32", st, k_reduce_f32<<<reduce_grid(W.rows * r), 256, 0, st>>>(part, splits, W.rows * r, s, dB));
+    return cudaGetLastError();
+}
+
 cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, int64_t M, const NF4View &W,
                               const __nv_bfloat16 *A, const __nv_bfloat16 *B, int r, float s,
                               const __nv_bfloat16 *XA, __nv_bfloat16 *dX, float *dA, float *dB, void *ws,
@@ -1137,6 +1181,23 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
                                                               bwd_adapter_bytes(M, W.rows, W.cols, r));
         e = launch_dequant(W, Wd, st);
         if (e != cudaSuccess) return e;
+        if (r > 0) {
+            // the adapter gradients need only Gs and XA: they run on the side stream
+            // while the dgrad GEMM occupies the tensor cores
+            std::lock_guard<std::mutex> lock(g_side_mu);
+            SideStream *side = side_stream_locked();
+            if (side) {
+                float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + 2 * mr_bytes(M, r));
+                if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
+                e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, st);
+                if (e != cudaSuccess) return e;
+                if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
+                e = adapter_grads(X, dY, M, W, Gs, XA, r, s, dA, dB, part, side->s);
+                if (e != cudaSuccess) return e;
+                if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess) return e;
+                return cudaStreamWaitEvent(st, side->join, 0);
+            }
+        }
         e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, st);
     } else {
         e = run_fused_dgrad(dY, M, W, A, Gs, r, dX, st);
@@ -1144,15 +1205,7 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
     if (e != cudaSuccess) return e;
     if (r > 0) {
         float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + 2 * mr_bytes(M, r));
-        int splits = 0;
-        // dA = X^T (sG)
-        e = run_skinny(true, X, M, true, Gs, W.cols, M, r, part, &splits, st);
-        if (e != cudaSuccess) return e;
-        QNF4_LAUNCH("k_reduce_f32", st, k_reduce_f32<<<reduce_grid(W.cols * r), 256, 0, st>>>(part, splits, W.cols * r, 1.0f, dA));
-        // dB = s (XA)^T dY, computed as (dY^T XA)^T with the partials written transposed
-        e = run_skinny(true, dY, M, true, XA, W.rows, M, r, part, &splits, st, true);
-        if (e != cudaSuccess) return e;
-        QNF4_LAUNCH("k_reduce_f32", st, k_reduce_f32<<<reduce_grid(W.rows * r), 256, 0, st>>>(part, splits, W.rows * r, s, dB));
+        return adapter_grads(X, dY, M, W, Gs, XA, r, s, dA, dB, part, st);
     }
     return cudaGetLastError();
 }

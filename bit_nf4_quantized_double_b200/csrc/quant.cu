@@ -218,11 +218,11 @@ k_double_quant(const float *__restrict__ c1, int64_t nb, int64_t nb2, const floa
     }
 }
 
-// Dequantisation: each thread expands one 32-bit word of codes (8 weights) into
-// one 16-byte bf16 store, so a warp reads 128 contiguous code bytes and writes
-// 512 contiguous output bytes; four independent words per thread are in flight
-// at once. Codebook in shared memory (16 distinct words: lookups never
-// conflict). A ragged tail (n % 8 != 0) is written element by element.
+// Dequantisation: each thread expands two 32-bit words of codes (16 weights, a
+// quarter block) into two 16-byte bf16 stores; a warp reads 256 contiguous code
+// bytes and writes 1 KB, and four such pairs per thread are in flight at once.
+// Codebook in shared memory (16 distinct words: lookups never conflict). A
+// ragged tail (n % 16 != 0) is written element by element.
 constexpr int kDequantUnroll = 4;
 __global__ void __launch_bounds__(256)
 k_dequant(NF4View q, int64_t n, Codebook cb, __nv_bfloat16 *__restrict__ out) {
@@ -230,18 +230,18 @@ k_dequant(NF4View q, int64_t n, Codebook cb, __nv_bfloat16 *__restrict__ out) {
     if (threadIdx.x < 16) s_q[threadIdx.x] = cb.q[threadIdx.x];
     __syncthreads();
     const float mu = *q.offset;
-    const int64_t n8 = n / 8;
+    const int64_t n16 = n / 16;
     const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
-    const uint32_t *codes = reinterpret_cast<const uint32_t *>(q.codes);
-    for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g0 < n8; g0 += kDequantUnroll * nthr) {
-        uint32_t w[kDequantUnroll];
+    const uint2 *codes = reinterpret_cast<const uint2 *>(q.codes);
+    for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g0 < n16; g0 += kDequantUnroll * nthr) {
+        uint2 w[kDequantUnroll];
         int8_t q8[kDequantUnroll];
         float s2[kDequantUnroll];
 #pragma unroll
         for (int u = 0; u < kDequantUnroll; ++u) {
             const int64_t g = g0 + u * nthr;
-            if (g < n8) {
-                const int64_t b = g / (kBlock1 / 8);
+            if (g < n16) {
+                const int64_t b = g / (kBlock1 / 16);
                 w[u] = __ldg(codes + g);
                 q8[u] = __ldg(q.scale8 + b);
                 s2[u] = __ldg(q.scale2 + b / kBlock2);
@@ -250,20 +250,22 @@ k_dequant(NF4View q, int64_t n, Codebook cb, __nv_bfloat16 *__restrict__ out) {
 #pragma unroll
         for (int u = 0; u < kDequantUnroll; ++u) {
             const int64_t g = g0 + u * nthr;
-            if (g < n8) {
+            if (g < n16) {
                 const float ch = dq_constant(q8[u], s2[u], mu);
-                uint32_t o[4];
+                uint32_t o[8];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint32_t byte = (w[u] >> (8 * k)) & 0xffu;
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t byte = ((k < 4 ? w[u].x : w[u].y) >> (8 * (k & 3))) & 0xffu;
                     o[k] = pack_bf16x2(__fmul_rn(s_q[byte >> 4], ch), __fmul_rn(s_q[byte & 15u], ch));
                 }
-                *reinterpret_cast<uint4 *>(out + 8 * g) = make_uint4(o[0], o[1], o[2], o[3]);
+                uint4 *dst = reinterpret_cast<uint4 *>(out + 16 * g);
+                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
             }
         }
     }
     if (blockIdx.x == 0 && threadIdx.x == 0) {
-        for (int64_t e = 8 * n8; e < n; ++e) {
+        for (int64_t e = 16 * n16; e < n; ++e) {
             const int64_t b = e / kBlock1;
             const float ch = dq_constant(q.scale8[b], q.scale2[b / kBlock2], mu);
             const uint8_t byte = q.codes[e / 2];
@@ -289,7 +291,7 @@ cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlor
 
 cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st) {
     const int64_t n = q.rows * q.cols;
-    int64_t grid = ceil_div(ceil_div(n, 8 * kDequantUnroll), 256);
+    int64_t grid = ceil_div(ceil_div(n, 16 * kDequantUnroll), 256);
     const int64_t cap = (int64_t)num_sms() * 8;
     if (grid < 1) grid = 1;
     if (grid > cap) grid = cap;
