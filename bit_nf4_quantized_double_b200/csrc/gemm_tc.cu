@@ -1087,29 +1087,6 @@ static cudaError_t run_fused_dgrad(const __nv_bfloat16 *dY, int64_t M, const NF4
     return cudaGetLastError();
 }
 
-cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4View &W, const __nv_bfloat16 *A,
-                                    const __nv_bfloat16 *B, int r, float s, __nv_bfloat16 *Y,
-                                    __nv_bfloat16 *XA_save, void *ws, cudaStream_t st) {
-    __nv_bfloat16 *XAs = nullptr;
-    if (r > 0) {
-        XAs = static_cast<__nv_bfloat16 *>(ws);
-        float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + mr_bytes(M, r));
-        int splits = 0;
-        cudaError_t e = run_skinny(false, X, M, true, A, M, W.cols, r, part, &splits, st);
-        if (e != cudaSuccess) return e;
-        QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, XA_save, XAs));
-    }
-    if (M >= kPairGemmMinM) {
-        // Y = X W^T + (s XA) B: W^ [d_out, d_in] is the K-major B operand, B_lora [r, d_out]
-        // the MN-major extension
-        __nv_bfloat16 *Wd = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + fwd_adapter_bytes(M, W.cols, r));
-        cudaError_t e = launch_dequant(W, Wd, st);
-        if (e != cudaSuccess) return e;
-        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, st);
-    }
-    return run_fused_fwd(X, M, W, XAs, B, r, Y, st);
-}
-
 // A second stream per device for work that can run beside other kernels: the
 // pair GEMM leaves SMs free (it uses as few CTA pairs as give the same number of
 // tile rounds) and is bound by the tensor pipe, while the adapter products and
@@ -1136,6 +1113,48 @@ static SideStream *side_stream_locked() {
     return &x;
 }
 
+cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4View &W, const __nv_bfloat16 *A,
+                                    const __nv_bfloat16 *B, int r, float s, __nv_bfloat16 *Y,
+                                    __nv_bfloat16 *XA_save, void *ws, cudaStream_t st) {
+    __nv_bfloat16 *XAs = nullptr;
+    const bool pair = M >= kPairGemmMinM;
+    __nv_bfloat16 *Wd = pair ? reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + fwd_adapter_bytes(M, W.cols, r))
+                             : nullptr;
+    cudaError_t e;
+    std::unique_lock<std::mutex> lock(g_side_mu, std::defer_lock);
+    SideStream *side = nullptr;
+    if (pair && r > 0) {
+        // the dequantisation and X*A are independent memory-bound passes: overlap them
+        lock.lock();
+        side = side_stream_locked();
+        if (side) {
+            if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
+            if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
+            if ((e = launch_dequant(W, Wd, side->s)) != cudaSuccess) return e;
+            if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess) return e;
+        }
+    }
+    if (r > 0) {
+        XAs = static_cast<__nv_bfloat16 *>(ws);
+        float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + mr_bytes(M, r));
+        int splits = 0;
+        e = run_skinny(false, X, M, true, A, M, W.cols, r, part, &splits, st);
+        if (e != cudaSuccess) return e;
+        QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, XA_save, XAs));
+    }
+    if (pair) {
+        // Y = X W^T + (s XA) B: W^ [d_out, d_in] is the K-major B operand, B_lora [r, d_out]
+        // the MN-major extension
+        if (side) {
+            if ((e = cudaStreamWaitEvent(st, side->join, 0)) != cudaSuccess) return e;
+        } else if ((e = launch_dequant(W, Wd, st)) != cudaSuccess) {
+            return e;
+        }
+        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, st);
+    }
+    return run_fused_fwd(X, M, W, XAs, B, r, Y, st);
+}
+
 // dA = X^T (sG) and dB = s (XA)^T dY on stream `st` (they share the partial buffer,
 // so they run one after the other).
 static cudaError_t adapter_grads(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, int64_t M, const NF4View &W,
@@ -1158,6 +1177,24 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
                               cudaStream_t st) {
     __nv_bfloat16 *Gs = nullptr;
     cudaError_t e;
+    const bool pair = M >= kPairGemmMinM;
+    __nv_bfloat16 *Wd = pair ? reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) +
+                                                                bwd_adapter_bytes(M, W.rows, W.cols, r))
+                             : nullptr;
+    std::unique_lock<std::mutex> lock(g_side_mu, std::defer_lock);
+    SideStream *side = nullptr;
+    if (pair && r > 0) {
+        // the dequantisation overlaps the dY*B^T pass; after the dgrad GEMM is
+        // launched, the adapter gradients run beside it
+        lock.lock();
+        side = side_stream_locked();
+        if (side) {
+            if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
+            if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
+            if ((e = launch_dequant(W, Wd, side->s)) != cudaSuccess) return e;
+            if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess) return e;
+        }
+    }
     if (r > 0) {
         Gs = static_cast<__nv_bfloat16 *>(ws);
         __nv_bfloat16 *XAbuf = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + mr_bytes(M, r));
@@ -1174,18 +1211,17 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
         if (e != cudaSuccess) return e;
         QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, nullptr, Gs));
     }
-    if (M >= kPairGemmMinM) {
+    if (pair) {
         // dX = dY W^ + (s G) A^T: W^ [d_out, d_in] read as the MN-major B operand
         // ([K = d_out][N = d_in]), A_lora [d_in, r] the K-major extension
-        __nv_bfloat16 *Wd = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) +
-                                                              bwd_adapter_bytes(M, W.rows, W.cols, r));
-        e = launch_dequant(W, Wd, st);
-        if (e != cudaSuccess) return e;
+        if (side) {
+            if ((e = cudaStreamWaitEvent(st, side->join, 0)) != cudaSuccess) return e;
+        } else if ((e = launch_dequant(W, Wd, st)) != cudaSuccess) {
+            return e;
+        }
         if (r > 0) {
             // the adapter gradients need only Gs and XA: they run on the side stream
             // while the dgrad GEMM occupies the tensor cores
-            std::lock_guard<std::mutex> lock(g_side_mu);
-            SideStream *side = side_stream_locked();
             if (side) {
                 float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + 2 * mr_bytes(M, r));
                 if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
