@@ -209,17 +209,41 @@ def run_ours(args, peaks, peak_kind):
     ws_b = torch.empty(max(1, Lb.qlora_linear_bwd_workspace(M, d_out, d_in, r)), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def step():
+    def layer_step():
         q.qlora_linear_fwd(X, t, A, B, s, Y=Y, XA_save=XA, ws=ws_f)
         q.qlora_linear_bwd(X, dY, t, A, B, s, XA=XA, dX=dX, dA=dA, dB=dB, ws=ws_b)
+
+    def eager_step():
+        layer_step()
         allreduce_adapter_grads(dA, dB, world)
 
     for _ in range(args.warmup):
-        step()
+        eager_step()
     torch.cuda.synchronize()
     status = q.qlora_get_device_status()
     if status != q.QLORA_OK:
         raise RuntimeError(f"device status {status} during warm-up")
+
+    # The layer's fwd + bwd launches are captured once in a CUDA graph and replayed
+    # each step (the same kernels on the same buffers; the graph removes the host
+    # launch cost). The gradient all-reduce stays outside the graph.
+    graph = None
+    launches_per_step = None
+    if not args.no_graph:
+        c0 = q.qlora_launch_count()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layer_step()
+        launches_per_step = q.qlora_launch_count() - c0
+        graph.replay()
+        torch.cuda.synchronize()
+
+    def step():
+        if graph is not None:
+            graph.replay()
+            allreduce_adapter_grads(dA, dB, world)
+        else:
+            eager_step()
 
     stream = torch.cuda.current_stream()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -235,6 +259,8 @@ def run_ours(args, peaks, peak_kind):
         step()
         evs[i][1].record(stream)
     launches = q.qlora_launch_count() - launches0
+    if graph is not None:
+        launches = launches_per_step * args.steps   # replays launch without the host counter
     torch.cuda.synchronize()
     clocks.mark_end()
     barrier(world)
@@ -252,7 +278,7 @@ def run_ours(args, peaks, peak_kind):
     q.qlora_profile_enable(True)
     for i in range(args.steps):
         flush.zero_()
-        step()
+        eager_step()
     q.qlora_profile_enable(False)
     torch.cuda.synchronize()
     kern = {}
@@ -325,7 +351,8 @@ def run_ours(args, peaks, peak_kind):
                                "X,dY ~ N(0,1) bf16; step = fwd + bwd" + (" + NCCL all-reduce of dA,dB"
                                                                        if world > 1 else ""),
                    "global_batch_tokens": M * world, "l2": "flushed between timed steps (256 MB write)",
-                   "flops_per_step": flops, "parallelism": f"dp{world}" if world > 1 else "single GPU"},
+                   "flops_per_step": flops, "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                   "launch": "CUDA graph replay of the layer fwd+bwd" if graph is not None else "eager"},
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2) if achieved else None,
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4) if achieved else None,
                      "peak_source": f"{peak_kind} bf16 sustained (MEASURED_PEAKS.json)" if peak_kind == "measured"
@@ -555,6 +582,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep-layers", type=int, default=32)
     ap.add_argument("--cpu-sample-tokens", type=int, default=512)
+    ap.add_argument("--no-graph", action="store_true", help="launch every step eagerly instead of replaying a CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
