@@ -493,7 +493,57 @@ def run_components(args, peaks, peak_kind, flush):
                                         "down 4096x11008), r=16 on q,k,v,o, fwd only, CUDA graph replay, "
                                         "L2 flushed", **gem}
     assert q.qlora_get_device_status() == q.QLORA_OK
+    out["l70b_layer"] = run_l70b(args, peaks, peak_kind, flush, stream)
     return out
+
+
+def run_l70b(args, peaks, peak_kind, flush, stream):
+    """One 70B-like layer (q,o 8192^2; k,v 1024x8192; gate,up 28672x8192; down
+    8192x28672), r = 64 on all seven projections, M = 4096: fwd + bwd of every
+    projection, replayed from one CUDA graph, L2 flushed between replays."""
+    import torch
+    import bit_nf4_quantized_double_b200 as q
+    import synth_inputs as si
+    wl = si.workload("l70b")
+    M = wl.M
+    items = []
+    flops = 0.0
+    for li, L in enumerate(wl.layers):
+        inp = si.layer_inputs(wl, li, device="cuda")
+        T = q.qlora_nf4_quantize(inp["W"])
+        del inp["W"]
+        lb = q.lib()
+        it = dict(X=inp["X"], dY=inp["dY"], A=inp["A"], B=inp["B"], s=L.s, T=T,
+                  Y=torch.empty(M, L.d_out, dtype=torch.bfloat16, device="cuda"),
+                  XA=torch.empty(M, L.r, dtype=torch.bfloat16, device="cuda"),
+                  dX=torch.empty(M, L.d_in, dtype=torch.bfloat16, device="cuda"),
+                  dA=torch.empty(L.d_in, L.r, dtype=torch.float32, device="cuda"),
+                  dB=torch.empty(L.r, L.d_out, dtype=torch.float32, device="cuda"))
+        items.append(it)
+        flops += step_flops(M, L.d_in, L.d_out, L.r)
+    # one workspace per direction, sized for the largest projection (calls are stream-ordered)
+    wsf = max(lb.qlora_linear_fwd_workspace(M, L.d_out, L.d_in, L.r) for L in wl.layers)
+    wsb = max(lb.qlora_linear_bwd_workspace(M, L.d_out, L.d_in, L.r) for L in wl.layers)
+    ws_f = torch.empty(max(1, wsf), dtype=torch.uint8, device="cuda")
+    ws_b = torch.empty(max(1, wsb), dtype=torch.uint8, device="cuda")
+
+    def layer():
+        for it in items:
+            q.qlora_linear_fwd(it["X"], it["T"], it["A"], it["B"], it["s"], Y=it["Y"], XA_save=it["XA"], ws=ws_f)
+            q.qlora_linear_bwd(it["X"], it["dY"], it["T"], it["A"], it["B"], it["s"], XA=it["XA"], dX=it["dX"],
+                               dA=it["dA"], dB=it["dB"], ws=ws_b)
+
+    reps = max(3, min(args.steps, 10))
+    ms = _time_graph(layer, reps, flush, stream)
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    tf = flops / (ms / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    del items, ws_f, ws_b
+    torch.cuda.empty_cache()
+    return {"workload": "70B-like layer: q,o 8192x8192; k,v 1024x8192; gate,up 28672x8192; down 8192x28672; "
+                        "r=64, alpha=128 on all seven; M=4096; fwd+bwd of each, CUDA graph replay, L2 flushed",
+            "flops_per_step": flops, "ms_per_step": round(ms, 4), "TFLOP/s": round(tf, 1),
+            "frac_of_sustained_bf16": round(tf / peak, 4), "reps": reps}
 
 
 # ------------------------------------------------------------------ CPU oracle

@@ -997,19 +997,6 @@ size_t fwd_workspace_bytes_large(int64_t M, int64_t rows, int64_t cols, int r) {
     return fwd_adapter_bytes(M, cols, r) + (M >= kPairGemmMinM ? wd_bytes(rows, cols) : 0);
 }
 
-size_t xa_small_workspace(int64_t M, int64_t cols, int r) { return mr_bytes(M, r) + partial_bytes(M, cols, r); }
-
-// XA = X A for the small-M path: XA_save = bf16(XA) (optional), XAs = bf16(s XA).
-cudaError_t launch_xa_small(const __nv_bfloat16 *X, int64_t M, int64_t cols, const __nv_bfloat16 *A, int r, float s,
-                            __nv_bfloat16 *XA_save, __nv_bfloat16 *XAs, void *part_ws, cudaStream_t st) {
-    int splits = 0;
-    float *part = static_cast<float *>(part_ws);
-    cudaError_t e = run_skinny(false, X, M, true, A, M, cols, r, part, &splits, st);
-    if (e != cudaSuccess) return e;
-    QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, XA_save, XAs));
-    return cudaGetLastError();
-}
-
 static size_t bwd_adapter_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
     if (r == 0) return 0;
     size_t part = partial_bytes(M, cols, r);                 // X*A

@@ -6,15 +6,18 @@
 // section 1), at decode-sized M where the packed 4-bit codes dominate HBM
 // traffic (section 2: about 4.127 bits per weight).
 //
-// k_gemv streams each weight row's codes once with 8-byte loads (the four
-// threads of a row cover one 32-byte sector per 64-block), turns code bytes
-// into bf16 pairs (Q[hi], Q[lo]) through a 256-entry table replicated once
-// per lane (so a warp's lookups never conflict), and accumulates
-// sum_k Q[code]*x_k per 64-block with mma.sync m16n8k16 (16 weight rows x 8
-// tokens). The block's dequantised constant c^ multiplies each block's partial
-// dot product (sum Q*x) * c^, so the per-weight work is one table lookup.
-// The K dimension is split across CTAs; k_gemv_finish sums the partials in
-// split order, adds the adapter term s*XA*B and rounds to bf16.
+// k_gemv is persistent: each CTA builds, once, a 256-entry table byte ->
+// bf16 pair (Q[hi], Q[lo]) replicated per lane (a warp's lookups never
+// conflict), then takes work units of 128 weight rows x 512 inputs. For a unit
+// it stages the X chunk as mma.sync B fragments, issues every code load (8 bytes
+// per thread per 64-block: the four threads of a row cover one 32-byte sector)
+// and every block-constant load of the unit before any arithmetic, and
+// accumulates sum_k Q[code] x_k per 64-block with mma.sync m16n8k16 (16 weight
+// rows x 8 tokens); the block's dequantised constant c^ then multiplies that
+// block's partial dot product, so the per-weight work is one table lookup.
+// Extra units compute the split-K partials of X*A for the adapter in the same
+// launch. k_gemv_finish sums both kinds of partials in split order (fixed
+// order: reproducible), adds s*(XA)*B and rounds to bf16.
 #include "launch.h"
 
 namespace qnf4 {
@@ -22,14 +25,11 @@ namespace qnf4 {
 cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4View &W, const __nv_bfloat16 *A,
                                     const __nv_bfloat16 *B, int r, float s, __nv_bfloat16 *Y,
                                     __nv_bfloat16 *XA_save, void *ws, cudaStream_t st);
-cudaError_t launch_xa_small(const __nv_bfloat16 *X, int64_t M, int64_t cols, const __nv_bfloat16 *A, int r, float s,
-                            __nv_bfloat16 *XA_save, __nv_bfloat16 *XAs, void *part_ws, cudaStream_t st);
-size_t xa_small_workspace(int64_t M, int64_t cols, int r);
 
 constexpr int kGemvMaxM = 16;
-constexpr int kGemvRows = 128;      // weight rows per CTA (8 warps x 16)
-constexpr int kGemvKChunk = 512;    // K per CTA
-constexpr int kGemvUnroll = 4;      // 64-blocks in flight per thread
+constexpr int kGemvRows = 128;      // weight rows per unit (8 warps x 16)
+constexpr int kGemvKChunk = 512;    // inputs per unit (8 blocks of 64)
+constexpr int kGemvBlk = kGemvKChunk / 64;
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -45,81 +45,161 @@ __device__ __forceinline__ uint2 ldg_nc_v2(const void *p) {
     return r;
 }
 
-// Dequantised block constant of block b, with the second-level step cached
-// while consecutive blocks stay in the same 256-block group.
-struct StepCache {
-    int64_t grp = -1;
-    float step = 0.0f;
-    __device__ __forceinline__ float chat(const NF4View &w, int64_t b, float mu) {
-        const int64_t g = b >> 8;
-        if (g != grp) {
-            grp = g;
-            step = __fdiv_rn(w.scale2[g], 127.0f);
-        }
-        return __fadd_rn(__fmul_rn((float)w.scale8[b], step), mu);
-    }
+__device__ __forceinline__ uint32_t pack2_bf16(const __nv_bfloat16 *p0, const __nv_bfloat16 *p1) {
+    const uint32_t lo = *reinterpret_cast<const uint16_t *>(p0), hi = *reinterpret_cast<const uint16_t *>(p1);
+    return lo | (hi << 16);
+}
+
+struct GemvParams {
+    NF4View w;
+    const __nv_bfloat16 *X;      // [M, K]
+    const __nv_bfloat16 *A;      // [K, r] (adapter down-projection) or null
+    int M, r;
+    int splits, nrb;             // K splits, row blocks
+    float *partial;              // [splits][M][N]
+    float *partial_xa;           // [splits][M][r]
 };
 
-// Token tiles of 8 (NT = 1: M <= 8, NT = 2: M <= 16). Grid: (row blocks, K splits).
+// Token tiles of 8 (NT = 1: M <= 8, NT = 2: M <= 16).
 template <int NT>
-__global__ void __launch_bounds__(256)
-k_gemv(NF4View w, const __nv_bfloat16 *__restrict__ X, int M, Codebook cb, float *__restrict__ partial) {
+__global__ void __launch_bounds__(256, 2)
+k_gemv(GemvParams p, Codebook cb) {
     extern __shared__ __align__(16) uint8_t smem[];
     uint32_t *lut = reinterpret_cast<uint32_t *>(smem);                  // [256 entries][32 lanes]
-    uint2 *xs = reinterpret_cast<uint2 *>(smem + 256 * 32 * 4);           // [NT][nblk][4][32]
-    const int K = (int)w.cols, N = (int)w.rows;
-    const int kbase = blockIdx.y * kGemvKChunk;
-    const int kend = min(K, kbase + kGemvKChunk);
-    const int nblk = (kend - kbase) / 64;
-
-    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
-        const int e = i >> 5;
-        const __nv_bfloat162 pr = __floats2bfloat162_rn(cb.q[e >> 4], cb.q[e & 15]);
-        lut[i] = *reinterpret_cast<const uint32_t *>(&pr);
-    }
-    const int units = NT * nblk * 128;
-    for (int u = threadIdx.x; u < units; u += blockDim.x) {
-        const int nt = u / (nblk * 128), rem = u % (nblk * 128);
-        const int b = rem >> 7, j = (rem >> 5) & 3, ln = rem & 31;
-        const int tok = nt * 8 + (ln >> 2), t = ln & 3;
-        const int k = kbase + b * 64 + 16 * t + 4 * j;
-        uint2 v = make_uint2(0u, 0u);
-        if (tok < M) v = *reinterpret_cast<const uint2 *>(X + (int64_t)tok * K + k);
-        xs[u] = v;
-    }
-    __syncthreads();
-
+    uint2 *xs = reinterpret_cast<uint2 *>(smem + 256 * 32 * 4);           // [NT][kGemvBlk][4][32]
+    __shared__ float s_q[16];
+    const NF4View &w = p.w;
+    const int K = (int)w.cols, N = (int)w.rows, M = p.M;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int r0 = blockIdx.x * kGemvRows + warp * 16 + g, r1 = r0 + 8;
-    const bool v0 = r0 < N, v1 = r1 < N;
+
+    if (threadIdx.x < 16) s_q[threadIdx.x] = cb.q[threadIdx.x];
+    __syncthreads();
+    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
+        const int e = i >> 5;
+        const __nv_bfloat162 pr = __floats2bfloat162_rn(s_q[e >> 4], s_q[e & 15]);
+        lut[i] = *reinterpret_cast<const uint32_t *>(&pr);
+    }
+    const uint32_t *lut_l = lut + lane;
     const int64_t kbs = K / 64;
     const float mu = *w.offset;
-    const uint8_t *c0p = w.codes + ((int64_t)r0 * K + kbase) / 2 + 8 * t;
-    const uint8_t *c1p = w.codes + ((int64_t)r1 * K + kbase) / 2 + 8 * t;
-    const uint32_t *lut_l = lut + lane;
-    StepCache sc0, sc1;
-    float acc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+    const int main_units = p.nrb * p.splits;
+    const int units = main_units + (p.r > 0 ? p.splits : 0);
 
-    for (int b0 = 0; b0 < nblk; b0 += kGemvUnroll) {
-        uint2 u0[kGemvUnroll], u1[kGemvUnroll];
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        const int ks = u < main_units ? u % p.splits : u - main_units;
+        const int kbase = ks * kGemvKChunk;
+        const int nblk = (min(K, kbase + kGemvKChunk) - kbase) / 64;
+        if (u >= main_units) {
+            // ---------------- adapter partial: XA_ks[m][j] = sum over this K chunk of X[m][k] A[k][j]
+            // mma m16n8k16 with X rows (tokens, zero past M) as A and A_lora columns as B.
+            // Warp w takes 16-wide k steps w, w + 8, ...; all loads are issued before the
+            // MMAs, and the eight warps' sums are added in warp order through shared memory.
+            float *red = reinterpret_cast<float *>(xs);           // [8 warps][r / 8 tiles][32 lanes][4]
+            const int ntiles = p.r / 8;
+            const int ksteps = nblk * 4;
+            __syncthreads();                                      // xs is free
+            for (int nt0 = 0; nt0 < ntiles; nt0 += 4) {           // at most 4 tiles per pass (smem)
+                const int nts = min(4, ntiles - nt0);
+                float c[4][4];
 #pragma unroll
-        for (int u = 0; u < kGemvUnroll; ++u) {
-            const bool in = b0 + u < nblk;
-            u0[u] = (in && v0) ? ldg_nc_v2(c0p + 32 * (b0 + u)) : make_uint2(0x77777777u, 0x77777777u);
-            u1[u] = (in && v1) ? ldg_nc_v2(c1p + 32 * (b0 + u)) : make_uint2(0x77777777u, 0x77777777u);
+                for (int q = 0; q < 4; ++q) c[q][0] = c[q][1] = c[q][2] = c[q][3] = 0.0f;
+                for (int kstep = warp; kstep < ksteps; kstep += 8) {
+                    const int k0 = kbase + 16 * kstep;
+                    uint32_t a[4] = {0u, 0u, 0u, 0u};
+                    if (g < M) {
+                        a[0] = *reinterpret_cast<const uint32_t *>(p.X + (int64_t)g * K + k0 + 2 * t);
+                        a[2] = *reinterpret_cast<const uint32_t *>(p.X + (int64_t)g * K + k0 + 8 + 2 * t);
+                    }
+                    if (g + 8 < M) {
+                        a[1] = *reinterpret_cast<const uint32_t *>(p.X + (int64_t)(g + 8) * K + k0 + 2 * t);
+                        a[3] = *reinterpret_cast<const uint32_t *>(p.X + (int64_t)(g + 8) * K + k0 + 8 + 2 * t);
+                    }
+                    uint32_t bb[4][2];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (q < nts) {
+                            const __nv_bfloat16 *ak = p.A + (int64_t)(k0 + 2 * t) * p.r + (nt0 + q) * 8 + g;
+                            bb[q][0] = pack2_bf16(ak, ak + p.r);
+                            bb[q][1] = pack2_bf16(ak + 8 * p.r, ak + 9 * p.r);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        if (q < nts) mma_bf16_16816(c[q], a, bb[q][0], bb[q][1]);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (q < nts)
+                        *reinterpret_cast<float4 *>(red + ((warp * 4 + q) * 32 + lane) * 4) =
+                            make_float4(c[q][0], c[q][1], c[q][2], c[q][3]);
+                __syncthreads();
+                // c[0], c[1]: token g, tile columns 2t, 2t+1; c[2], c[3]: token g + 8
+                for (int i = threadIdx.x; i < nts * 32; i += blockDim.x) {
+                    const int q = i >> 5, ln = i & 31;
+                    float4 v = *reinterpret_cast<const float4 *>(red + (q * 32 + ln) * 4);
+                    for (int ww = 1; ww < 8; ++ww) {
+                        const float4 x = *reinterpret_cast<const float4 *>(red + ((ww * 4 + q) * 32 + ln) * 4);
+                        v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+                    }
+                    const int gg = ln >> 2, tt = ln & 3, j0 = (nt0 + q) * 8 + 2 * tt;
+                    float *dst = p.partial_xa + (int64_t)ks * M * p.r;
+                    if (gg < M) { dst[gg * p.r + j0] = v.x; dst[gg * p.r + j0 + 1] = v.y; }
+                    if (gg + 8 < M) { dst[(gg + 8) * p.r + j0] = v.z; dst[(gg + 8) * p.r + j0 + 1] = v.w; }
+                }
+                __syncthreads();
+            }
+            continue;
         }
+        const int rb = u / p.splits;
+        // ---------------- stage the X chunk as B fragments (k order matches the code bytes below)
+        __syncthreads();   // the previous unit's warps are done with xs
+        for (int i = threadIdx.x; i < NT * nblk * 128; i += blockDim.x) {
+            const int nt = i / (nblk * 128), rem = i % (nblk * 128);
+            const int b = rem >> 7, j = (rem >> 5) & 3, ln = rem & 31;
+            const int tok = nt * 8 + (ln >> 2), tt = ln & 3;
+            const int k = kbase + b * 64 + 16 * tt + 4 * j;
+            uint2 v = make_uint2(0u, 0u);
+            if (tok < M) v = *reinterpret_cast<const uint2 *>(p.X + (int64_t)tok * K + k);
+            xs[((nt * kGemvBlk + b) * 4 + j) * 32 + ln] = v;
+        }
+        __syncthreads();
+
+        const int r0 = rb * kGemvRows + warp * 16 + g, r1 = r0 + 8;
+        const bool v0 = r0 < N, v1 = r1 < N;
+        const uint8_t *c0p = w.codes + ((int64_t)r0 * K + kbase) / 2 + 8 * t;
+        const uint8_t *c1p = w.codes + ((int64_t)r1 * K + kbase) / 2 + 8 * t;
+        // every load of the unit in flight before any arithmetic
+        uint2 u0[kGemvBlk], u1[kGemvBlk];
+        int8_t q0[kGemvBlk], q1[kGemvBlk];
+        const int64_t b0g = (int64_t)r0 * kbs + kbase / 64, b1g = (int64_t)r1 * kbs + kbase / 64;
 #pragma unroll
-        for (int u = 0; u < kGemvUnroll; ++u) {
-            const int b = b0 + u;
+        for (int b = 0; b < kGemvBlk; ++b) {
+            const bool in = b < nblk;
+            u0[b] = (in && v0) ? ldg_nc_v2(c0p + 32 * b) : make_uint2(0x77777777u, 0x77777777u);
+            u1[b] = (in && v1) ? ldg_nc_v2(c1p + 32 * b) : make_uint2(0x77777777u, 0x77777777u);
+            q0[b] = (in && v0) ? __ldg(w.scale8 + b0g + b) : (int8_t)0;
+            q1[b] = (in && v1) ? __ldg(w.scale8 + b1g + b) : (int8_t)0;
+        }
+        // second-level steps: a unit's 8 blocks of one row touch at most two 256-block groups
+        const int64_t g0a = b0g >> 8, g1a = b1g >> 8;
+        const float s0a = v0 ? __fdiv_rn(__ldg(w.scale2 + g0a), 127.0f) : 0.0f;
+        const float s0b = v0 ? __fdiv_rn(__ldg(w.scale2 + ((b0g + nblk - 1) >> 8)), 127.0f) : 0.0f;
+        const float s1a = v1 ? __fdiv_rn(__ldg(w.scale2 + g1a), 127.0f) : 0.0f;
+        const float s1b = v1 ? __fdiv_rn(__ldg(w.scale2 + ((b1g + nblk - 1) >> 8)), 127.0f) : 0.0f;
+
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+#pragma unroll
+        for (int b = 0; b < kGemvBlk; ++b) {
             if (b >= nblk) break;
-            const int64_t kb = kbase / 64 + b;
-            const float ch0 = v0 ? sc0.chat(w, (int64_t)r0 * kbs + kb, mu) : 0.0f;
-            const float ch1 = v1 ? sc1.chat(w, (int64_t)r1 * kbs + kb, mu) : 0.0f;
+            const float st0 = ((b0g + b) >> 8) == g0a ? s0a : s0b;
+            const float st1 = ((b1g + b) >> 8) == g1a ? s1a : s1b;
+            const float ch0 = __fadd_rn(__fmul_rn((float)q0[b], st0), mu);
+            const float ch1 = __fadd_rn(__fmul_rn((float)q1[b], st1), mu);
             float cblk[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
@@ -127,8 +207,8 @@ k_gemv(NF4View w, const __nv_bfloat16 *__restrict__ X, int M, Codebook cb, float
                 for (int i = 0; i < 4; ++i) cblk[nt][i] = 0.0f;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const uint32_t w0 = (j < 2) ? u0[u].x : u0[u].y;
-                const uint32_t w1 = (j < 2) ? u1[u].x : u1[u].y;
+                const uint32_t w0 = (j < 2) ? u0[b].x : u0[b].y;
+                const uint32_t w1 = (j < 2) ? u1[b].x : u1[b].y;
                 const int sh = (j & 1) * 16;
                 uint32_t a[4];
                 a[0] = lut_l[((w0 >> sh) & 0xffu) << 5];
@@ -137,7 +217,7 @@ k_gemv(NF4View w, const __nv_bfloat16 *__restrict__ X, int M, Codebook cb, float
                 a[3] = lut_l[((w1 >> (sh + 8)) & 0xffu) << 5];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const uint2 bx = xs[((nt * nblk + b) * 4 + j) * 32 + lane];
+                    const uint2 bx = xs[((nt * kGemvBlk + b) * 4 + j) * 32 + lane];
                     mma_bf16_16816(cblk[nt], a, bx.x, bx.y);
                 }
             }
@@ -149,39 +229,66 @@ k_gemv(NF4View w, const __nv_bfloat16 *__restrict__ X, int M, Codebook cb, float
                 acc[nt][3] = fmaf(ch1, cblk[nt][3], acc[nt][3]);
             }
         }
-    }
-    float *dst = partial + (int64_t)blockIdx.y * M * N;
+        float *dst = p.partial + (int64_t)ks * M * N;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int t0 = nt * 8 + 2 * t, t1 = t0 + 1;
-        if (v0 && t0 < M) dst[(int64_t)t0 * N + r0] = acc[nt][0];
-        if (v0 && t1 < M) dst[(int64_t)t1 * N + r0] = acc[nt][1];
-        if (v1 && t0 < M) dst[(int64_t)t0 * N + r1] = acc[nt][2];
-        if (v1 && t1 < M) dst[(int64_t)t1 * N + r1] = acc[nt][3];
+        for (int nt = 0; nt < NT; ++nt) {
+            const int t0 = nt * 8 + 2 * t, t1 = t0 + 1;
+            if (v0 && t0 < M) dst[(int64_t)t0 * N + r0] = acc[nt][0];
+            if (v0 && t1 < M) dst[(int64_t)t1 * N + r0] = acc[nt][1];
+            if (v1 && t0 < M) dst[(int64_t)t0 * N + r1] = acc[nt][2];
+            if (v1 && t1 < M) dst[(int64_t)t1 * N + r1] = acc[nt][3];
+        }
     }
 }
 
-// Y[m, n] = bf16( sum_split partial[split][m][n] + sum_j XAs[m, j] * B[j, n] ).
-__global__ void k_gemv_finish(const float *__restrict__ partial, int splits, int M, int N,
-                              const __nv_bfloat16 *__restrict__ XAs, const __nv_bfloat16 *__restrict__ B, int r,
-                              __nv_bfloat16 *__restrict__ Y) {
+// Y[m, n] = bf16( sum_split partial[split][m][n] + sum_j (s XA[m, j]) B[j, n] ),
+// XA[m, j] = sum_split partial_xa[split][m][j] (also written as bf16 to XA_save).
+constexpr int kFinishMaxSplits = 32;
+__global__ void __launch_bounds__(256)
+k_gemv_finish(const float *__restrict__ partial, const float *__restrict__ partial_xa, int splits, int M, int N,
+              int r, float s, const __nv_bfloat16 *__restrict__ B, __nv_bfloat16 *__restrict__ XA_save,
+              __nv_bfloat16 *__restrict__ Y) {
+    extern __shared__ float sxa[];                // [M][r]: s * XA
+    for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
+        float pv[kFinishMaxSplits];
+#pragma unroll
+        for (int sp = 0; sp < kFinishMaxSplits; ++sp)
+            if (sp < splits) pv[sp] = __ldg(partial_xa + sp * M * r + i);
+        float v = 0.0f;
+#pragma unroll
+        for (int sp = 0; sp < kFinishMaxSplits; ++sp)
+            if (sp < splits) v += pv[sp];
+        sxa[i] = s * v;
+        if (XA_save && blockIdx.x == 0) XA_save[i] = __float2bfloat16_rn(v);
+    }
+    __syncthreads();
     const int64_t count = (int64_t)M * N;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
         const int m = (int)(i / N), n = (int)(i % N);
+        float pv[kFinishMaxSplits];
+#pragma unroll
+        for (int sp = 0; sp < kFinishMaxSplits; ++sp)
+            if (sp < splits) pv[sp] = __ldg(partial + sp * count + i);
         float v = 0.0f;
-        for (int sp = 0; sp < splits; ++sp) v += partial[sp * count + i];
-        for (int j = 0; j < r; ++j)
-            v = fmaf(__bfloat162float(XAs[(int64_t)m * r + j]), __bfloat162float(B[(int64_t)j * N + n]), v);
+#pragma unroll
+        for (int sp = 0; sp < kFinishMaxSplits; ++sp)
+            if (sp < splits) v += pv[sp];
+        for (int j = 0; j < r; ++j) v = fmaf(sxa[m * r + j], __bfloat162float(B[(int64_t)j * N + n]), v);
         Y[i] = __float2bfloat16_rn(v);
     }
 }
 
 static int gemv_splits(int64_t cols) { return (int)ceil_div(cols, kGemvKChunk); }
-static size_t gemv_smem(int nt) { return 256 * 32 * 4 + (size_t)nt * (kGemvKChunk / 64) * 128 * 8; }
+// lookup table + the larger of the X fragments and the adapter unit's reduction buffer
+static size_t gemv_smem(int nt) {
+    const size_t xs = (size_t)nt * kGemvBlk * 128 * 8, red = 8 * 4 * 32 * 4 * 4;
+    return 256 * 32 * 4 + (xs > red ? xs : red);
+}
 
 static size_t small_workspace(int64_t M, int64_t rows, int64_t cols, int r) {
-    size_t b = ((size_t)gemv_splits(cols) * M * rows * 4 + 255) & ~size_t(255);
-    if (r > 0) b += xa_small_workspace(M, cols, r);
+    const size_t sp = (size_t)gemv_splits(cols);
+    size_t b = (sp * M * rows * 4 + 255) & ~size_t(255);
+    if (r > 0) b += (sp * M * r * 4 + 255) & ~size_t(255);
     return b;
 }
 
@@ -197,31 +304,40 @@ cudaError_t launch_linear_fwd(const __nv_bfloat16 *X, int64_t M, const NF4View &
                               void *ws, cudaStream_t st) {
     if (M > kGemvMaxM) return launch_linear_fwd_large(X, M, W, A, B, r, s, Y, XA_save, ws, st);
     const int splits = gemv_splits(W.cols);
-    float *partial = static_cast<float *>(ws);
-    char *rest = static_cast<char *>(ws) + (((size_t)splits * M * W.rows * 4 + 255) & ~size_t(255));
-    __nv_bfloat16 *XAs = nullptr;
+    if (splits > kFinishMaxSplits) return cudaErrorInvalidValue;
+    GemvParams p;
+    p.w = W;
+    p.X = X;
+    p.A = A;
+    p.M = (int)M;
+    p.r = r;
+    p.splits = splits;
+    p.nrb = (int)ceil_div(W.rows, kGemvRows);
+    p.partial = static_cast<float *>(ws);
+    p.partial_xa = reinterpret_cast<float *>(static_cast<char *>(ws) +
+                                             (((size_t)splits * M * W.rows * 4 + 255) & ~size_t(255)));
+    const int units = p.nrb * splits + (r > 0 ? splits : 0);
+    int grid = 2 * num_sms();
+    if (grid > units) grid = units;
     cudaError_t e;
-    if (r > 0) {
-        XAs = reinterpret_cast<__nv_bfloat16 *>(rest);
-        e = launch_xa_small(X, M, W.cols, A, r, s, XA_save, XAs, rest + (((size_t)M * r * 2 + 255) & ~size_t(255)), st);
-        if (e != cudaSuccess) return e;
-    }
-    const dim3 grid((unsigned)ceil_div(W.rows, kGemvRows), (unsigned)splits);
     if (M <= 8) {
         const size_t sm = gemv_smem(1);
         e = cudaFuncSetAttribute(k_gemv<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
-        QNF4_LAUNCH("k_gemv", st, k_gemv<1><<<grid, 256, sm, st>>>(W, X, (int)M, host_codebook(), partial));
+        QNF4_LAUNCH("k_gemv", st, k_gemv<1><<<grid, 256, sm, st>>>(p, host_codebook()));
     } else {
         const size_t sm = gemv_smem(2);
         e = cudaFuncSetAttribute(k_gemv<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
-        QNF4_LAUNCH("k_gemv", st, k_gemv<2><<<grid, 256, sm, st>>>(W, X, (int)M, host_codebook(), partial));
+        QNF4_LAUNCH("k_gemv", st, k_gemv<2><<<grid, 256, sm, st>>>(p, host_codebook()));
     }
+    // at least one CTA per SM (32 outputs each at the smallest): the finish is latency bound
     const int64_t count = M * W.rows;
-    int64_t g = ceil_div(count, 256);
-    if (g > (int64_t)num_sms() * 8) g = (int64_t)num_sms() * 8;
-    QNF4_LAUNCH("k_gemv_finish", st, k_gemv_finish<<<(unsigned)g, 256, 0, st>>>(partial, splits, (int)M, (int)W.rows, XAs, B, r, Y));
+    int64_t g = ceil_div(count, 32);
+    if (g > (int64_t)num_sms()) g = ceil_div(count, 256) > num_sms() ? ceil_div(count, 256) : num_sms();
+    if (g > (int64_t)num_sms() * 4) g = (int64_t)num_sms() * 4;
+    const size_t fsm = (size_t)M * (r > 0 ? r : 1) * 4;
+    QNF4_LAUNCH("k_gemv_finish", st, k_gemv_finish<<<(unsigned)g, 256, fsm, st>>>(p.partial, p.partial_xa, splits, (int)M, (int)W.rows, r, s, B, r > 0 ? XA_save : nullptr, Y));
     return cudaGetLastError();
 }
 
