@@ -18,6 +18,7 @@ GEMV over one Llama-7B block at M in {1, 4, 16} (HBM GB/s).
 sample of the same workload; it is the reference arm of this repository.
 """
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -471,17 +472,20 @@ def run_components(args, peaks, peak_kind, flush):
             inp = si.layer_inputs(wl, li, device="cuda")
             T = q.qlora_nf4_quantize(inp["W"])
             Y = torch.empty(M, L.d_out, dtype=torch.bfloat16, device="cuda")
-            ws = torch.empty(max(1, q.lib().qlora_linear_fwd_workspace(M, L.d_out, L.d_in, L.r)),
-                             dtype=torch.uint8, device="cuda")
-            items.append((inp["X"], T, inp.get("A"), inp.get("B"), L.s, Y, ws))
+            items.append({"X": inp["X"], "W": T, "A": inp.get("A"), "B": inp.get("B"), "s": L.s, "Y": Y})
             nbytes += T.nbytes + inp["X"].numel() * 2 + Y.numel() * 2
             if L.r:
                 nbytes += inp["A"].numel() * 2 + inp["B"].numel() * 2
             del inp
+        # the block's seven projections in one grouped call (one GEMV + one finish launch)
+        wsz = q.lib().qlora_linear_fwd_grouped_workspace(
+            M, len(items), (q._LinearDesc * len(items))(*[
+                q._LinearDesc(None, ctypes.pointer(it["W"].ctype()), None, None,
+                              0 if it["A"] is None else it["A"].shape[1], 1.0, None, None) for it in items]))
+        ws = torch.empty(max(1, wsz), dtype=torch.uint8, device="cuda")
 
         def layer():
-            for X, T, A, B, s, Y, ws in items:
-                q.qlora_linear_fwd(X, T, A, B, s, Y=Y, XA_save=False, ws=ws)
+            q.qlora_linear_fwd_grouped(items, ws=ws)
 
         ms = _time_graph(layer, 20, flush, stream)
         gbs = nbytes / (ms / 1e3) / 1e9
@@ -490,8 +494,8 @@ def run_components(args, peaks, peak_kind, flush):
         del items
         torch.cuda.empty_cache()
     out["decode7b_gemv"] = {"workload": "one Llama-7B block (q,k,v,o 4096x4096; gate,up 11008x4096; "
-                                        "down 4096x11008), r=16 on q,k,v,o, fwd only, CUDA graph replay, "
-                                        "L2 flushed", **gem}
+                                        "down 4096x11008), r=16 on q,k,v,o, fwd only, one grouped call "
+                                        "(qlora_linear_fwd_grouped), CUDA graph replay, L2 flushed", **gem}
     assert q.qlora_get_device_status() == q.QLORA_OK
     out["l70b_layer"] = run_l70b(args, peaks, peak_kind, flush, stream)
     return out

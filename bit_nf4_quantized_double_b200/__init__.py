@@ -47,6 +47,13 @@ class _Tensor(ctypes.Structure):
 
 _lib = None
 
+class _LinearDesc(ctypes.Structure):
+    """qlora_linear_desc of the C ABI."""
+    _fields_ = [("X", ctypes.c_void_p), ("W", ctypes.POINTER(_Tensor)), ("A", ctypes.c_void_p),
+                ("B", ctypes.c_void_p), ("r", ctypes.c_int), ("s", ctypes.c_float), ("Y", ctypes.c_void_p),
+                ("XA_save", ctypes.c_void_p)]
+
+
 _SIGS = {
     "qlora_nf4_storage_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
     "qlora_nf4_quantize_workspace": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
@@ -62,6 +69,10 @@ _SIGS = {
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float,
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_linear_fwd_grouped_workspace": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int,
+                                                            ctypes.POINTER(_LinearDesc)]),
+    "qlora_linear_fwd_grouped": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(_LinearDesc),
+                                                ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "qlora_get_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_nf4_codebook": (None, [ctypes.c_void_p]),
@@ -204,6 +215,32 @@ def qlora_linear_fwd(X: torch.Tensor, W: NF4Tensor, A: torch.Tensor | None, B: t
     _check(L.qlora_linear_fwd(_ptr(X), M, ctypes.byref(t), _ptr(A), _ptr(B), r, float(s), _ptr(Y),
                               _ptr(XA_save), _ptr(wsb), wsn, _stream(stream)), "qlora_linear_fwd")
     return Y, XA_save
+
+
+def qlora_linear_fwd_grouped(items, ws: torch.Tensor | None = None, stream=None):
+    """Forward of several projections in one call (all with the same M).
+
+    items: sequence of dicts with keys X, W (NF4Tensor), A, B (or None), s, and
+    optionally Y (output) and XA_save (tensor, or None). Returns the list of Y."""
+    items = list(items)
+    M = items[0]["X"].shape[0]
+    n = len(items)
+    tensors = [it["W"].ctype() for it in items]          # kept alive for the call
+    descs = (_LinearDesc * n)()
+    outs = []
+    for i, it in enumerate(items):
+        X, W, A, B = it["X"], it["W"], it.get("A"), it.get("B")
+        r = 0 if A is None else A.shape[1]
+        Y = it.get("Y")
+        if Y is None:
+            Y = torch.empty(M, W.rows, dtype=torch.bfloat16, device=X.device)
+        outs.append(Y)
+        descs[i] = _LinearDesc(_ptr(X), ctypes.pointer(tensors[i]), _ptr(A), _ptr(B), r, float(it["s"]), _ptr(Y),
+                               _ptr(it.get("XA_save")))
+    L = lib()
+    wsb, wsn = _workspace(int(L.qlora_linear_fwd_grouped_workspace(M, n, descs)), items[0]["X"].device, ws)
+    _check(L.qlora_linear_fwd_grouped(M, n, descs, _ptr(wsb), wsn, _stream(stream)), "qlora_linear_fwd_grouped")
+    return outs
 
 
 def qlora_linear_bwd(X: torch.Tensor, dY: torch.Tensor, W: NF4Tensor, A: torch.Tensor | None,

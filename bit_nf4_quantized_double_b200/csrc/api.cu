@@ -135,6 +135,52 @@ qlora_status qlora_linear_fwd(const void *X, int64_t M, const qlora_nf4_tensor *
                                        ws, static_cast<cudaStream_t>(stream)));
 }
 
+// Validates one grouped item as qlora_linear_fwd validates its arguments and fills
+// the internal descriptor.
+static qlora_status grouped_item(int64_t M, const qlora_linear_desc &in, LinearDesc &out) {
+    if (!in.W) return QLORA_ERR_INVALID_ARG;
+    qlora_status st = check_linear(M, in.W, in.r, in.s);
+    if (st != QLORA_OK) return st;
+    if (!in.X || !in.Y || !aligned16(in.X) || !aligned16(in.Y)) return QLORA_ERR_INVALID_ARG;
+    if (in.r > 0 && (!in.A || !in.B || !aligned16(in.A) || !aligned16(in.B) || (in.XA_save && !aligned16(in.XA_save))))
+        return QLORA_ERR_INVALID_ARG;
+    out.X = static_cast<const __nv_bfloat16 *>(in.X);
+    out.W = view_of(in.W);
+    out.A = static_cast<const __nv_bfloat16 *>(in.A);
+    out.B = static_cast<const __nv_bfloat16 *>(in.B);
+    out.r = in.r;
+    out.s = in.s;
+    out.Y = static_cast<__nv_bfloat16 *>(in.Y);
+    out.XA_save = static_cast<__nv_bfloat16 *>(in.XA_save);
+    return QLORA_OK;
+}
+constexpr int kMaxGrouped = 64;
+
+size_t qlora_linear_fwd_grouped_workspace(int64_t M, int count, const qlora_linear_desc *d) {
+    if (M < 1 || count < 1 || count > kMaxGrouped || !d) return 0;
+    LinearDesc items[kMaxGrouped];
+    for (int i = 0; i < count; ++i) {
+        if (!d[i].W || d[i].W->rows < 1 || d[i].W->cols < 1 || d[i].r < 0) return 0;
+        items[i].W.rows = d[i].W->rows;
+        items[i].W.cols = d[i].W->cols;
+        items[i].r = d[i].r;
+    }
+    return fwd_grouped_workspace_bytes(M, count, items);
+}
+
+qlora_status qlora_linear_fwd_grouped(int64_t M, int count, const qlora_linear_desc *d, void *ws,
+                                      size_t ws_bytes, qlora_stream_t stream) {
+    if (count < 1 || count > kMaxGrouped || !d) return QLORA_ERR_INVALID_ARG;
+    LinearDesc items[kMaxGrouped];
+    for (int i = 0; i < count; ++i) {
+        qlora_status st = grouped_item(M, d[i], items[i]);
+        if (st != QLORA_OK) return st;
+    }
+    const size_t need = fwd_grouped_workspace_bytes(M, count, items);
+    if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return QLORA_ERR_WORKSPACE;
+    return from_cuda(launch_linear_fwd_grouped(M, count, items, ws, static_cast<cudaStream_t>(stream)));
+}
+
 size_t qlora_linear_bwd_workspace(int64_t M, int64_t rows, int64_t cols, int r) {
     if (M < 1 || rows < 1 || cols < 1 || r < 0) return 0;
     return bwd_workspace_bytes(M, rows, cols, r);

@@ -15,6 +15,18 @@ cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, cons
                            int ke, cudaStream_t st);
 
 size_t fwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r);
+
+// One projection of a grouped forward (device pointers; validated by the caller).
+struct LinearDesc {
+    const __nv_bfloat16 *X = nullptr;
+    NF4View W{};
+    const __nv_bfloat16 *A = nullptr, *B = nullptr;
+    int r = 0;
+    float s = 0.0f;
+    __nv_bfloat16 *Y = nullptr, *XA_save = nullptr;
+};
+size_t fwd_grouped_workspace_bytes(int64_t M, int count, const LinearDesc *d);
+cudaError_t launch_linear_fwd_grouped(int64_t M, int count, const LinearDesc *d, void *ws, cudaStream_t st);
 size_t bwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r);
 
 cudaError_t launch_linear_fwd(const __nv_bfloat16 *X, int64_t M, const NF4View &W,

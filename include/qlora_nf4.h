@@ -139,6 +139,34 @@ qlora_status qlora_linear_bwd(const void *X, const void *dY, int64_t M, const ql
                               void *dX, float *dA, float *dB, void *ws, size_t ws_bytes,
                               qlora_stream_t stream);
 
+/*
+ * Forward of several projections at once (the page's equation for each), for
+ * decode-sized batches where one launch per projection would cost more than
+ * streaming its codes. Every item is a separate layer:
+ *   Y_i = X_i * Dequant(W_i)^T + s_i * (X_i * A_i) * B_i
+ * with the shapes, alignment and shape rules of qlora_linear_fwd; all items share M.
+ *   d      host array of `count` descriptors (1 <= count <= 64); W points to a host
+ *          struct as in qlora_linear_fwd.
+ *   ws     one device workspace of qlora_linear_fwd_grouped_workspace() bytes.
+ * M <= 16: the items go through one GEMV launch and one finish launch (per eight
+ * items). Larger M: the items run one after another on the single-item path, and the
+ * workspace is the largest single-item requirement. Results are bit-identical to
+ * calling qlora_linear_fwd on each item.
+ */
+typedef struct {
+    const void *X;                 /* bf16 [M, W->cols] */
+    const qlora_nf4_tensor *W;
+    const void *A;                 /* bf16 [W->cols, r], or NULL when r == 0 */
+    const void *B;                 /* bf16 [r, W->rows], or NULL when r == 0 */
+    int r;
+    float s;
+    void *Y;                       /* bf16 [M, W->rows] */
+    void *XA_save;                 /* bf16 [M, r], or NULL */
+} qlora_linear_desc;
+size_t qlora_linear_fwd_grouped_workspace(int64_t M, int count, const qlora_linear_desc *d);
+qlora_status qlora_linear_fwd_grouped(int64_t M, int count, const qlora_linear_desc *d, void *ws,
+                                      size_t ws_bytes, qlora_stream_t stream);
+
 /* Synchronises `stream`, returns the first condition recorded on the current
  * device since the last call (QLORA_OK if none) and clears it. */
 qlora_status qlora_get_device_status(qlora_stream_t stream);

@@ -70,6 +70,22 @@ def test_workspace_queries_positive():
     assert L.qlora_linear_fwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2
 
 
+def test_grouped_forward_host_checks():
+    # argument checks of the grouped entry point run on the host (no GPU needed)
+    L = q.lib()
+    fake = 1 << 20
+    t = q._Tensor(64, 64, fake, fake, fake, fake)
+    d = (q._LinearDesc * 2)(q._LinearDesc(fake, ctypes.pointer(t), None, None, 0, 1.0, fake, None),
+                            q._LinearDesc(fake, ctypes.pointer(t), None, None, 0, 1.0, fake, None))
+    assert L.qlora_linear_fwd_grouped(1, 0, d, None, 0, None) == q.QLORA_ERR_INVALID_ARG
+    # two 64 x 64 items at M = 1: one split each, M*rows fp32 partials, 256-byte aligned
+    assert L.qlora_linear_fwd_grouped_workspace(1, 2, d) == 2 * 256
+    assert L.qlora_linear_fwd_grouped(1, 2, d, None, 0, None) == q.QLORA_ERR_WORKSPACE
+    bad = (q._LinearDesc * 1)(q._LinearDesc(fake, ctypes.pointer(q._Tensor(64, 100, fake, fake, fake, fake)),
+                                            None, None, 0, 1.0, fake, None))
+    assert L.qlora_linear_fwd_grouped(1, 1, bad, None, 0, None) == q.QLORA_ERR_UNSUPPORTED_SHAPE
+
+
 def test_status_strings():
     for s in range(7):
         assert len(q.status_string(s)) > 0

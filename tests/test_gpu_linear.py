@@ -123,6 +123,34 @@ def test_decode_layer_full(M):
         check(f64(Y), oracle.linear_fwd(f64(inp["X"]), Wh, An, Bn, L.s), f"Y[{L.name}]")
 
 
+@pytest.mark.parametrize("M", [1, 16])
+def test_decode_layer_grouped(M):
+    # the whole block in one grouped call: bit-identical to the per-projection calls
+    # (same units, same fixed-order sums), and within tolerance of the oracle
+    wl = si.workload("decode7b", M=M)
+    items, singles, refs = [], [], []
+    for li, L in enumerate(wl.layers):
+        inp = si.layer_inputs(wl, li, device="cuda")
+        t = q.qlora_nf4_quantize(inp["W"])
+        xa = torch.empty(M, L.r, dtype=torch.bfloat16, device="cuda") if L.r else None
+        items.append({"X": inp["X"], "W": t, "A": inp.get("A"), "B": inp.get("B"), "s": L.s, "XA_save": xa})
+        Ys, XAs = q.qlora_linear_fwd(inp["X"], t, inp.get("A"), inp.get("B"), L.s)
+        singles.append((Ys, XAs))
+        if li in (0, 4):
+            Wh = oracle_weight(inp["W"])
+            An = f64(inp["A"]) if L.r else np.zeros((L.d_in, 0))
+            Bn = f64(inp["B"]) if L.r else np.zeros((0, L.d_out))
+            refs.append((li, oracle.linear_fwd(f64(inp["X"]), Wh, An, Bn, L.s)))
+    Ys = q.qlora_linear_fwd_grouped(items)
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    for (Y1, XA1), Yg, it in zip(singles, Ys, items):
+        assert torch.equal(Y1, Yg)
+        if XA1 is not None:
+            assert torch.equal(XA1, it["XA_save"])
+    for li, ref in refs:
+        check(f64(Ys[li]), ref, f"Y[{wl.layers[li].name}]")
+
+
 def test_full_4096_layer_sampled():
     # the 4096 x 4096 layer at 4096 tokens, rank 64, in the bench's launch configuration
     M = 4096
