@@ -14,6 +14,8 @@
 //   k_offset          one CTA: the upper levels of the fp64 pairwise tree -> mean;
 //   k_double_quant    one warp per group: s2 = max |c1 - mu|, int8 constants.
 
+#include <cmath>
+
 #include "common.cuh"
 
 namespace qnf4 {
@@ -29,6 +31,35 @@ __device__ __forceinline__ int nf4_code(float x, const float *t) {
     c += (x > t[c + 1]) ? 2 : 0;
     c += (x > t[c]) ? 1 : 0;
     return c;
+}
+
+// Code table over 256 equal bins of [-1, 1): bin k = [-1 + k/128, -1 + (k+1)/128)
+// holds base[k] = number of thresholds below the bin and thr[k] = the one
+// threshold inside the bin (4.0 if none). Valid when no threshold lies within
+// kBinMargin of a bin edge (checked on the host).
+struct CodeBins {
+    int base[256];
+    float thr[256];
+};
+constexpr double kBinMargin = 1e-5;
+
+static bool build_code_bins(const Codebook &cb, CodeBins &b) {
+    for (int k = 0; k < 256; ++k) {
+        const double lo = -1.0 + k / 128.0, hi = lo + 1.0 / 128.0;
+        int base = 0;
+        float thr = 4.0f;
+        int inside = 0;
+        for (int t = 0; t < 15; ++t) {
+            const double T = cb.t[t];
+            if (std::fabs(T - lo) < kBinMargin || std::fabs(T - hi) < kBinMargin) return false;
+            if (T < lo) ++base;
+            else if (T < hi) { thr = cb.t[t]; ++inside; }
+        }
+        if (inside > 1) return false;
+        b.base[k] = base;
+        b.thr[k] = thr;
+    }
+    return true;
 }
 
 template <typename T> __device__ __forceinline__ float to_f32(T v);
@@ -51,9 +82,17 @@ __device__ __forceinline__ void load_vec(const T *p, float (&v)[VEC]) {
 // One CTA of 256 threads per second-level group j (blocks 256j .. 256j+255).
 // Warp w handles blocks 256j + 32w .. +31; a 64-block is spread over
 // LPB = 64 / VEC lanes that each load 16 bytes.
-template <typename T>
+//
+// With BINS, a lane divides by one correctly rounded reciprocal of its block's
+// absmax (x' = fl(w * fl(1/c1)), within 1.5 ulp of the exact quotient x =
+// fl(w / c1)) and reads the code from the bin table through the float bits of
+// x' + 3 (in [2, 4): the top 8 mantissa bits are the bin). Where x' lies within
+// 4 ulp of the bin's threshold the exact quotient and the full search decide, so
+// the codes are those of x bit for bit. Without BINS every weight is divided.
+template <typename T, bool BINS>
 __global__ void __launch_bounds__(256)
 k_quantize_codes(const T *__restrict__ W, int64_t n, int64_t nb, Codebook cb,
+                 const __grid_constant__ CodeBins bins,
                  float *__restrict__ c1_out, double *__restrict__ part_out,
                  uint8_t *__restrict__ codes) {
     constexpr int VEC = 16 / sizeof(T);   // elements per 16-byte lane load
@@ -65,9 +104,11 @@ k_quantize_codes(const T *__restrict__ W, int64_t n, int64_t nb, Codebook cb,
     __shared__ float s_t[16];
     __shared__ float s_c1[kBlock2];
     __shared__ double s_part[8];
+    __shared__ int2 s_bin[256];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x < 15) s_t[threadIdx.x] = cb.t[threadIdx.x];
+    if (BINS) s_bin[threadIdx.x] = make_int2(bins.base[threadIdx.x], __float_as_int(bins.thr[threadIdx.x]));
     __syncthreads();
 
     const int64_t group = blockIdx.x;
@@ -101,12 +142,27 @@ k_quantize_codes(const T *__restrict__ W, int64_t n, int64_t nb, Codebook cb,
         }
         // codes of the lane's VEC elements: NBYTES bytes, byte k = hi << 4 | lo
         uint32_t packed = 0;
+        if (BINS) {
+            const float rcp = __frcp_rn(m);
 #pragma unroll
-        for (int k = 0; k < VEC; k += 2) {
-            const float x0 = (m == 0.0f) ? 0.0f : __fdiv_rn(v[k], m);
-            const float x1 = (m == 0.0f) ? 0.0f : __fdiv_rn(v[k + 1], m);
-            const uint32_t byte = ((uint32_t)nf4_code(x0, s_t) << 4) | (uint32_t)nf4_code(x1, s_t);
-            packed |= byte << (8 * (k / 2));
+            for (int k = 0; k < VEC; ++k) {
+                const float xa = __fmul_rn(v[k], rcp);
+                const float y = fminf(fmaxf(__fadd_rn(xa, 3.0f), 2.0f), 3.99999976f);
+                const int2 e = s_bin[(__float_as_uint(y) >> 15) & 0xffu];
+                const float thr = __int_as_float(e.y);
+                int c = e.x + (xa > thr ? 1 : 0);
+                if (fabsf(__fsub_rn(xa, thr)) <= __fmul_rn(fabsf(thr), 0x1p-21f)) c = nf4_code(__fdiv_rn(v[k], m), s_t);
+                if (m == 0.0f) c = 7;
+                packed |= (uint32_t)c << (8 * (k / 2) + ((k & 1) ? 0 : 4));
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < VEC; k += 2) {
+                const float x0 = (m == 0.0f) ? 0.0f : __fdiv_rn(v[k], m);
+                const float x1 = (m == 0.0f) ? 0.0f : __fdiv_rn(v[k + 1], m);
+                const uint32_t byte = ((uint32_t)nf4_code(x0, s_t) << 4) | (uint32_t)nf4_code(x1, s_t);
+                packed |= byte << (8 * (k / 2));
+            }
         }
         const int64_t c0 = e0 / 2;
         if (c0 + NBYTES <= ncode) {
@@ -280,10 +336,19 @@ cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlor
                             float *c1, double *part, cudaStream_t st) {
     const int64_t nb = ceil_div(n, kBlock1), nb2 = ceil_div(nb, kBlock2);
     const Codebook &cb = host_codebook();
-    if (dt == QLORA_F32)
-        QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<float><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const float *>(W), n, nb, cb, c1, part, out.codes));
-    else
-        QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<__nv_bfloat16><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W), n, nb, cb, c1, part, out.codes));
+    static CodeBins bins;
+    static const bool use_bins = build_code_bins(cb, bins);
+    if (dt == QLORA_F32) {
+        if (use_bins)
+            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<float, true><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const float *>(W), n, nb, cb, bins, c1, part, out.codes));
+        else
+            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<float, false><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const float *>(W), n, nb, cb, bins, c1, part, out.codes));
+    } else {
+        if (use_bins)
+            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<__nv_bfloat16, true><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W), n, nb, cb, bins, c1, part, out.codes));
+        else
+            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<__nv_bfloat16, false><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W), n, nb, cb, bins, c1, part, out.codes));
+    }
     QNF4_LAUNCH("k_offset", st, k_offset<<<1, 1024, 0, st>>>(part, nb2, nb, out.offset));
     QNF4_LAUNCH("k_double_quant", st, k_double_quant<<<(unsigned)ceil_div(nb2, 8), 256, 0, st>>>(c1, nb, nb2, out.offset, out.scale8, out.scale2));
     return cudaGetLastError();
