@@ -90,7 +90,7 @@ __device__ __forceinline__ void load_vec(const T *p, float (&v)[VEC]) {
 // 4 ulp of the bin's threshold the exact quotient and the full search decide, so
 // the codes are those of x bit for bit. Without BINS every weight is divided.
 template <typename T, bool BINS>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 k_quantize_codes(const T *__restrict__ W, int64_t n, int64_t nb, Codebook cb,
                  const __grid_constant__ CodeBins bins,
                  float *__restrict__ c1_out, double *__restrict__ part_out,
@@ -116,7 +116,7 @@ k_quantize_codes(const T *__restrict__ W, int64_t n, int64_t nb, Codebook cb,
     const int64_t ncode = (n + 1) / 2;
     bool nonfinite = false;
 
-#pragma unroll 4
+#pragma unroll 2
     for (int it = 0; it < ITERS; ++it) {
         const int local = warp * 32 + it * BPI + sub;          // block index within the group
         const int64_t b = group * kBlock2 + local;
@@ -280,7 +280,7 @@ k_double_quant(const float *__restrict__ c1, int64_t nb, int64_t nb2, const floa
 // Codebook in shared memory (16 distinct words: lookups never conflict). A
 // ragged tail (n % 16 != 0) is written element by element.
 constexpr int kDequantUnroll = 4;
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 k_dequant(NF4View q, int64_t n, Codebook cb, __nv_bfloat16 *__restrict__ out) {
     __shared__ float s_q[16];
     if (threadIdx.x < 16) s_q[threadIdx.x] = cb.q[threadIdx.x];
