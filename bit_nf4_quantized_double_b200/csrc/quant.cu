@@ -116,14 +116,34 @@ k_quantize_codes(const T *__restrict__ W, int64_t n, int64_t nb, Codebook cb,
     const int64_t ncode = (n + 1) / 2;
     bool nonfinite = false;
 
-#pragma unroll 2
-    for (int it = 0; it < ITERS; ++it) {
+    // the lane's 16-byte loads are issued in batches of 8 before any arithmetic
+    // (one memory round trip per batch instead of one per iteration)
+    constexpr int BATCH = ITERS < 8 ? ITERS : 8;
+#pragma unroll 1
+    for (int it0 = 0; it0 < ITERS; it0 += BATCH) {
+    uint4 raw[BATCH];
+#pragma unroll
+    for (int j = 0; j < BATCH; ++j) {
+        const int it = it0 + j;
+        const int64_t e0 = ((group * kBlock2 + warp * 32 + it * BPI + sub) * kBlock1) + (int64_t)li * VEC;
+        raw[j] = (e0 + VEC <= n) ? __ldg(reinterpret_cast<const uint4 *>(W + e0)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < BATCH; ++j) {
+        const int it = it0 + j;
         const int local = warp * 32 + it * BPI + sub;          // block index within the group
         const int64_t b = group * kBlock2 + local;
         const int64_t e0 = b * kBlock1 + (int64_t)li * VEC;     // first element of this lane
         float v[VEC];
         if (e0 + VEC <= n) {
-            load_vec<T, VEC>(W + e0, v);
+            if constexpr (sizeof(T) == 4) {
+                v[0] = __uint_as_float(raw[j].x); v[1] = __uint_as_float(raw[j].y);
+                v[2] = __uint_as_float(raw[j].z); v[3] = __uint_as_float(raw[j].w);
+            } else {
+                const uint32_t w4[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) { v[2 * k] = bf16_lo(w4[k]); v[2 * k + 1] = bf16_hi(w4[k]); }
+            }
         } else {
 #pragma unroll
             for (int k = 0; k < VEC; ++k) v[k] = (e0 + k < n) ? to_f32<T>(W[e0 + k]) : 0.0f;
@@ -173,6 +193,7 @@ k_quantize_codes(const T *__restrict__ W, int64_t n, int64_t nb, Codebook cb,
             for (int k = 0; k < NBYTES; ++k)
                 if (c0 + k < ncode) codes[c0 + k] = (uint8_t)(packed >> (8 * k));
         }
+    }
     }
     if (__any_sync(0xffffffffu, nonfinite) && lane == 0) raise_status(QLORA_ERR_NONFINITE);
     __syncthreads();
