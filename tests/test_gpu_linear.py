@@ -213,9 +213,32 @@ def test_zero_adapter_equals_plain_product():
 
 
 @pytest.mark.parametrize("rep", [0, 1])
+def test_many_tiles_per_cta_fused_full(rep):
+    # below 512 tokens the fused dequant-GEMM kernels run; with 16384 weight rows
+    # (forward) or 16384 inputs (dgrad) every persistent CTA walks several 128 x 256
+    # tiles: compare every element, twice, so a race at tile boundaries shows
+    M = 480
+    for rows, cols in ((16384, 1024), (1024, 16384)):
+        W, X, dY, A, B, s = make_problem(M, rows, cols, 64, seed=500 + rows + rep)
+        t = q.qlora_nf4_quantize(W)
+        Y, XA = q.qlora_linear_fwd(X, t, A, B, s)
+        dX, dA, dB = q.qlora_linear_bwd(X, dY, t, A, B, s, XA=XA)
+        assert q.qlora_get_device_status() == q.QLORA_OK
+        Wh = oracle_weight(W)
+        Xn, dYn, An, Bn = f64(X), f64(dY), f64(A), f64(B)
+        check(f64(Y), oracle.linear_fwd(Xn, Wh, An, Bn, s), f"Y[{rows}x{cols}]")
+        dXr, dAr, dBr = oracle.linear_bwd(Xn, dYn, Wh, An, Bn, s)
+        check(f64(dX), dXr, f"dX[{rows}x{cols}]")
+        check(f64(dA), dAr, f"dA[{rows}x{cols}]")
+        check(f64(dB), dBr, f"dB[{rows}x{cols}]")
+
+
+@pytest.mark.parametrize("rep", [0, 1])
 def test_many_tiles_per_cta_full(rep):
-    # every CTA of the persistent fused kernels walks several tiles (1024 tiles on
-    # 148 SMs): compare every element, twice, so a race at tile boundaries shows
+    # from 512 tokens on the CTA-pair GEMM runs; here the forward of the 8192-row
+    # weight and the dgrad of the 8192-input one give each pair about seven 256 x 256
+    # tiles, so both TMEM accumulators are reused many times: compare every element,
+    # twice, so a race between the epilogue and the next tile's MMAs shows
     M = 4096
     for rows, cols in ((1024, 8192), (8192, 1024)):
         W, X, dY, A, B, s = make_problem(M, rows, cols, 64, seed=300 + rows + rep)
