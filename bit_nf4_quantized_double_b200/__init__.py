@@ -78,6 +78,7 @@ _SIGS = {
     "qlora_nf4_codebook": (None, [ctypes.c_void_p]),
     "qlora_nf4_quantize_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(_Tensor),
                                                   ctypes.c_void_p]),
+    "qlora_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_void_p]),
     "qlora_launch_count": (ctypes.c_ulonglong, []),
     "qlora_profile_enable": (None, [ctypes.c_int]),
     "qlora_profile_read": (ctypes.c_int, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),

@@ -205,6 +205,16 @@ qlora_status qlora_nf4_quantize_noalloc(const void *W, qlora_dtype dt, const qlo
                                         qlora_stream_t stream);
 
 /*
+ * Self-test of the library's failure detection (the page has no counterpart).
+ * Launches one kernel that waits, through the same bounded wait the pipelined
+ * kernels use, on a barrier that nothing completes. After the wait limit (1 s)
+ * the kernel records QLORA_ERR_TIMEOUT in the device status word and returns
+ * normally; qlora_get_device_status() then reports it, and the context stays
+ * usable. Returns QLORA_OK or QLORA_ERR_CUDA (launch failure).
+ */
+qlora_status qlora_selftest_wait_timeout(qlora_stream_t stream);
+
+/*
  * Measurement hooks. The page has no counterpart: they let a benchmark count
  * and time the library's own kernels without a profiler.
  *   qlora_launch_count    kernel launches issued by this process so far.

@@ -96,6 +96,20 @@ def test_nonfinite_sets_status():
     assert q.qlora_get_device_status() == q.QLORA_ERR_NONFINITE
 
 
+def test_bounded_wait_reports_timeout():
+    # a wait that nothing ends gives up after its limit, reports TIMEOUT through the
+    # status word, and leaves the context usable (the next quantisation is exact)
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    assert q.lib().qlora_selftest_wait_timeout(None) == q.QLORA_OK
+    assert q.qlora_get_device_status() == q.QLORA_ERR_TIMEOUT
+    assert q.qlora_get_device_status() == q.QLORA_OK       # read clears it
+    W = si.normal((64, 256), 0.02, seed=9, device="cuda")
+    t = q.qlora_nf4_quantize(W)
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    ref = oracle.quantize(W.cpu().numpy())
+    assert np.array_equal(t.codes.cpu().numpy(), ref.codes)
+
+
 def test_llama7b_layer_full_bf16():
     # every projection of one Llama-7B-shaped block, at full size
     wl = si.workload("llama7b", n_layers=1)
