@@ -71,6 +71,9 @@ def lib() -> ctypes.CDLL:
                                        ctypes.c_void_p, ctypes.c_void_p]
         L.orc_dequant_constant.restype = ctypes.c_float
         L.orc_dequant_constant.argtypes = [ctypes.c_int8, ctypes.c_float, ctypes.c_float]
+        L.orc_merge_bf16.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                     ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p]
+        L.orc_merge_bf16.restype = None
         L.orc_dequant.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
                                   ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
         L.orc_bf16_rne.restype = ctypes.c_uint16
@@ -241,6 +244,20 @@ def dequant(q: NF4Tensor) -> np.ndarray:
     out = np.zeros(q.n, dtype=np.uint16)
     lib().orc_dequant(_ptr(q.codes), _ptr(q.scale8), _ptr(q.scale2), ctypes.c_float(float(q.offset)),
                       q.n, _ptr(codebook()), _ptr(out))
+    return out
+
+
+def merge_bf16(w_hat_bits: np.ndarray, A: np.ndarray, B: np.ndarray, s: float) -> np.ndarray:
+    """Merged BF16 weight w' = bf16(w^ + fl(s * sum_j A[k,j] B[j,n])) (fused multiply-adds in
+    increasing j), as bf16 bits [rows, cols]. w_hat_bits: bf16 bits [rows, cols] of the
+    dequantised weight; A [cols, r], B [r, rows]: fp32 arrays holding bf16 values."""
+    rows, cols = w_hat_bits.shape
+    r = A.shape[1]
+    w = np.ascontiguousarray(w_hat_bits, dtype=np.uint16)
+    a = np.ascontiguousarray(A, dtype=np.float32)
+    b = np.ascontiguousarray(B, dtype=np.float32)
+    out = np.empty((rows, cols), dtype=np.uint16)
+    lib().orc_merge_bf16(_ptr(w), _ptr(a), _ptr(b), rows, cols, r, ctypes.c_float(s), _ptr(out))
     return out
 
 

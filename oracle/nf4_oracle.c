@@ -327,3 +327,28 @@ int orc_max_threads(void)
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------ */
+/* Adapter merge (the page's section 5 notes that merging the adapter into    */
+/* the weight and re-quantising can change outputs; section 6 asks to check   */
+/* it). Reading: the merge is done in BF16, the compute type:                  */
+/*   d[n,k]  = A[k,0]*B[0,n] + ... + A[k,r-1]*B[r-1,n], one fused multiply-add */
+/*             per term in increasing j, starting from 0 (fmaf: the exactly   */
+/*             rounded a*b+c, not a contraction by the compiler);             */
+/*   w'[n,k] = bf16( fl( w^[n,k] + fl(s * d[n,k]) ) ),                         */
+/* with w^ the dequantised BF16 weight [rows, cols] (bf16 bits), A [cols, r]   */
+/* and B [r, rows] widened exactly from bf16 to fp32. Output: bf16 bits.       */
+void orc_merge_bf16(const uint16_t *w_hat, const float *A, const float *B, int64_t rows, int64_t cols,
+                    int r, float s, uint16_t *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < rows; ++n) {
+        for (int64_t k = 0; k < cols; ++k) {
+            float d = 0.0f;
+            for (int j = 0; j < r; ++j) d = fmaf(A[k * r + j], B[(int64_t)j * rows + n], d);
+            const float t = s * d;
+            const float w = orc_bf16_to_f32(w_hat[n * cols + k]) + t;
+            out[n * cols + k] = orc_bf16_rne(w);
+        }
+    }
+}
