@@ -57,15 +57,17 @@ def load_peaks():
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """SM clock, power and clock-event reasons of this rank's GPU, polled through
-    NVML every ~2 ms on a background thread (the timed region lasts only a few
-    milliseconds); only samples taken between mark_begin() and mark_end() count.
-    Reads the settings only, changes none. Falls back to nvidia-smi -lms 200."""
+    """SM clock and clock-event reasons of this rank's GPU, polled through NVML every
+    ~0.5 ms on a background thread (the timed region lasts only a few milliseconds),
+    plus one sample taken synchronously when the region ends (right after the final
+    synchronise, before the clock can relax); only samples between mark_begin() and
+    mark_end() count. Reads the settings only, changes none."""
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.samples = []
+        self.nv = self.h = None
         self.t0 = self.t1 = None
         self.thread = None
         self.stop_flag = False
@@ -91,6 +93,7 @@ class ClockSampler:
         except Exception as e:   # NVML missing: no samples, say why
             self.err = f"nvml unavailable: {e}"
             return
+        self.nv, self.h = nv, h
 
         def poll():
             while not self.stop_flag:
@@ -105,7 +108,7 @@ class ClockSampler:
                 except Exception as e:
                     self.err = str(e)
                     return
-                time.sleep(0.002)
+                time.sleep(0.0005)
         self.thread = threading.Thread(target=poll, daemon=True)
         self.thread.start()
         time.sleep(0.01)
@@ -113,7 +116,22 @@ class ClockSampler:
     def mark_begin(self):
         self.t0 = time.perf_counter()
 
+    def _sample_now(self):
+        nv, h = self.nv, self.h
+        if nv is None:
+            return
+        try:
+            mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+            try:
+                rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+            except Exception:
+                rs = int(nv.nvmlDeviceGetCurrentClocksThrottleReasons(h))
+            self.samples.append((time.perf_counter(), mhz, rs))
+        except Exception as e:
+            self.err = str(e)
+
     def mark_end(self):
+        self._sample_now()
         self.t1 = time.perf_counter()
 
     def stop(self):
@@ -128,7 +146,7 @@ class ClockSampler:
                     "reasons": [self.err or "no samples in the timed region"], "samples": 0, "source": "nvml"}
         reasons = sorted({name for _, _, rs in inside for bit, name in self.REASONS.items() if rs & bit})
         return {"sm_mhz": statistics.median(m for _, m, _ in inside), "sm_min_mhz": min(m for _, m, _ in inside),
-                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside), "source": "nvml, 2 ms"}
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside), "source": "nvml, 0.5 ms"}
 
 
 # ------------------------------------------------------------------ distributed
@@ -496,7 +514,38 @@ def run_components(args, peaks, peak_kind, flush):
                                         "(qlora_linear_fwd_grouped), CUDA graph replay, L2 flushed", **gem}
     assert q.qlora_get_device_status() == q.QLORA_OK
     out["l70b_layer"] = run_l70b(args, peaks, peak_kind, flush, stream)
+    out["merge_4096"] = run_merge(hbm, flush, stream)
     return out
+
+
+def run_merge(hbm, flush, stream):
+    """Adapter merge + re-quantisation of the 4096 x 4096 layer (r = 64): time per call
+    (CUDA-graph replay, L2 flushed) and the change of the layer output it causes."""
+    import torch
+    import bit_nf4_quantized_double_b200 as q
+    import synth_inputs as si
+    wl = si.workload("l4096")
+    L = wl.layers[0]
+    inp = si.layer_inputs(wl, 0, device="cuda")
+    t = q.qlora_nf4_quantize(inp["W"])
+    out = q.nf4_empty(L.d_out, L.d_in)
+    wb = torch.empty(L.d_out, L.d_in, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(q.lib().qlora_nf4_merge_workspace(L.d_out, L.d_in), dtype=torch.uint8, device="cuda")
+    ms = _time_graph(lambda: q.qlora_nf4_merge_adapter(t, inp["A"], inp["B"], L.s, out=out, W_bf16=wb, ws=ws),
+                     10, flush, stream)
+    n = L.d_out * L.d_in
+    # NF4 read, merged bf16 written and read back by the quantiser, NF4 written
+    alg = n * (2 * (0.5 + 1 / 64 + 4 / 16384) + 2 * 2) + (L.d_in + L.d_out) * L.r * 2
+    X = inp["X"][:256]
+    Yu, _ = q.qlora_linear_fwd(X, t, inp["A"], inp["B"], L.s)
+    Ym, _ = q.qlora_linear_fwd(X, out, None, None, 0.0)
+    rel = ((Ym.double() - Yu.double()).norm() / Yu.double().norm()).item()
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    return {"workload": "merge s*(AB)^T into the 4096x4096 NF4 weight in bf16 and re-quantise (r=64), "
+                        "CUDA graph replay, L2 flushed",
+            "ms": round(ms, 4), "GB/s": round(alg / (ms / 1e3) / 1e9, 1), "frac": round(alg / (ms / 1e3) / 1e9 / hbm, 4),
+            "output_rel_change_fro": round(rel, 6),
+            "output_change_sample": "256 tokens: X W'^T (merged, re-quantised) against X W^T + s (XA) B"}
 
 
 def run_l70b(args, peaks, peak_kind, flush, stream):

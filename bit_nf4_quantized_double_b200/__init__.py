@@ -79,6 +79,10 @@ _SIGS = {
     "qlora_nf4_quantize_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(_Tensor),
                                                   ctypes.c_void_p]),
     "qlora_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_void_p]),
+    "qlora_nf4_merge_workspace": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
+    "qlora_nf4_merge_adapter": (ctypes.c_int, [ctypes.POINTER(_Tensor), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                               ctypes.c_float, ctypes.c_void_p, ctypes.POINTER(_Tensor),
+                                               ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "qlora_launch_count": (ctypes.c_ulonglong, []),
     "qlora_profile_enable": (None, [ctypes.c_int]),
     "qlora_profile_read": (ctypes.c_int, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
@@ -216,6 +220,23 @@ def qlora_linear_fwd(X: torch.Tensor, W: NF4Tensor, A: torch.Tensor | None, B: t
     _check(L.qlora_linear_fwd(_ptr(X), M, ctypes.byref(t), _ptr(A), _ptr(B), r, float(s), _ptr(Y),
                               _ptr(XA_save), _ptr(wsb), wsn, _stream(stream)), "qlora_linear_fwd")
     return Y, XA_save
+
+
+def qlora_nf4_merge_adapter(W: NF4Tensor, A: torch.Tensor, B: torch.Tensor, s: float,
+                            out: NF4Tensor | None = None, W_bf16: torch.Tensor | None = None,
+                            ws: torch.Tensor | None = None, stream=None):
+    """Merge the adapter into the weight in BF16 and re-quantise: returns (W_out, W_bf16)
+    with W_bf16 = bf16(Dequant(W) + s (A B)^T) [rows, cols] and W_out its NF4 + DQ form."""
+    if out is None:
+        out = nf4_empty(W.rows, W.cols, W.codes.device)
+    if W_bf16 is None:
+        W_bf16 = torch.empty(W.rows, W.cols, dtype=torch.bfloat16, device=W.codes.device)
+    L = lib()
+    wsb, wsn = _workspace(int(L.qlora_nf4_merge_workspace(W.rows, W.cols)), W.codes.device, ws)
+    t, to = W.ctype(), out.ctype()
+    _check(L.qlora_nf4_merge_adapter(ctypes.byref(t), _ptr(A), _ptr(B), A.shape[1], float(s), _ptr(W_bf16),
+                                     ctypes.byref(to), _ptr(wsb), wsn, _stream(stream)), "qlora_nf4_merge_adapter")
+    return out, W_bf16
 
 
 def qlora_linear_fwd_grouped(items, ws: torch.Tensor | None = None, stream=None):

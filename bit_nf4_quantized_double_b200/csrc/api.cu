@@ -181,6 +181,35 @@ qlora_status qlora_linear_fwd_grouped(int64_t M, int count, const qlora_linear_d
     return from_cuda(launch_linear_fwd_grouped(M, count, items, ws, static_cast<cudaStream_t>(stream)));
 }
 
+size_t qlora_nf4_merge_workspace(int64_t rows, int64_t cols) {
+    if (rows < 1 || cols < 1) return 0;
+    return align256((size_t)rows * (size_t)cols * 2) + qlora_nf4_quantize_workspace(rows, cols);
+}
+
+qlora_status qlora_nf4_merge_adapter(const qlora_nf4_tensor *W, const void *A, const void *B, int r, float s,
+                                     void *W_bf16, const qlora_nf4_tensor *W_out, void *ws, size_t ws_bytes,
+                                     qlora_stream_t stream) {
+    if (!tensor_ok(W) || !tensor_ok(W_out) || W_out->rows != W->rows || W_out->cols != W->cols)
+        return QLORA_ERR_INVALID_ARG;
+    if (W->cols % 64 != 0 || r < 1 || r > 256) return QLORA_ERR_UNSUPPORTED_SHAPE;
+    if (!A || !B || !aligned16(A) || !aligned16(B) || (W_bf16 && !aligned16(W_bf16)) || !std::isfinite(s))
+        return QLORA_ERR_INVALID_ARG;
+    const size_t need = qlora_nf4_merge_workspace(W->rows, W->cols);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return QLORA_ERR_WORKSPACE;
+    const int64_t n = W->rows * W->cols, nb = ceil_div(n, kBlock1), nb2 = ceil_div(nb, kBlock2);
+    if (nb2 > 0x7fffffffLL) return QLORA_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *w = static_cast<char *>(ws);
+    __nv_bfloat16 *merged = W_bf16 ? static_cast<__nv_bfloat16 *>(W_bf16) : reinterpret_cast<__nv_bfloat16 *>(w);
+    w += align256((size_t)n * 2);
+    float *c1 = reinterpret_cast<float *>(w);
+    double *part = reinterpret_cast<double *>(w + align256((size_t)nb * 4));
+    cudaError_t e = launch_merge_bf16(view_of(W), static_cast<const __nv_bfloat16 *>(A),
+                                      static_cast<const __nv_bfloat16 *>(B), r, s, merged, st);
+    if (e != cudaSuccess) return from_cuda(e);
+    return from_cuda(launch_quantize(merged, QLORA_BF16, n, *W_out, c1, part, st));
+}
+
 size_t qlora_linear_bwd_workspace(int64_t M, int64_t rows, int64_t cols, int r) {
     if (M < 1 || rows < 1 || cols < 1 || r < 0) return 0;
     return bwd_workspace_bytes(M, rows, cols, r);

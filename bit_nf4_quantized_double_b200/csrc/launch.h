@@ -8,6 +8,8 @@ namespace qnf4 {
 cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlora_nf4_tensor &out,
                             float *c1, double *part, cudaStream_t st);
 cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st);
+cudaError_t launch_merge_bf16(const NF4View &q, const __nv_bfloat16 *A, const __nv_bfloat16 *B, int r, float s,
+                              __nv_bfloat16 *out, cudaStream_t st);
 
 // Plain bf16 GEMM on CTA pairs (tcgen05 cta_group::2), see gemm2sm.cu.
 cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, const __nv_bfloat16 *B, bool b_mn,

@@ -352,6 +352,85 @@ k_dequant(NF4View q, int64_t n, Codebook cb, __nv_bfloat16 *__restrict__ out) {
     }
 }
 
+// ---------------------------------------------------------------- adapter merge
+// Merged BF16 weight (the page's sections 5 and 6: merging the adapter into the
+// weight and re-quantising can change outputs; the merge is done in BF16):
+//   w'[n,k] = bf16( fl( w^[n,k] + fl(s * d[n,k]) ) ),
+//   d[n,k]  = fused multiply-adds of A[k,j] * B[j,n] over j = 0 .. r-1 in order, from 0,
+// with w^ the dequantised weight computed in place (step 7 of the format). A CTA
+// takes 64 x 64 tiles (rows x inputs: one 64-block per row); the tile's A rows and
+// B columns are staged in shared memory as fp32, transposed so that a thread reads
+// its 16 consecutive inputs of one j with four 16-byte loads.
+__global__ void __launch_bounds__(256)
+k_merge_bf16(NF4View q, const __nv_bfloat16 *__restrict__ A, const __nv_bfloat16 *__restrict__ B, int r, float s,
+             Codebook cb, __nv_bfloat16 *__restrict__ out) {
+    extern __shared__ __align__(16) float msm[];
+    float *As = msm;                 // [r][64]: As[j][kk] = A[k0 + kk][j]
+    float *Bs = msm + r * 64;        // [r][64]: Bs[j][nn] = B[j][n0 + nn]
+    __shared__ float s_q[16];
+    if (threadIdx.x < 16) s_q[threadIdx.x] = cb.q[threadIdx.x];
+    const int64_t rows = q.rows, cols = q.cols, kbs = cols / 64;
+    const float mu = *q.offset;
+    const int nn = threadIdx.x >> 2, kk0 = (threadIdx.x & 3) * 16;
+    const int64_t tiles_n = (rows + 63) / 64, tiles = tiles_n * kbs;
+    for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+        const int64_t n0 = (tile % tiles_n) * 64, k0 = (tile / tiles_n) * 64;
+        __syncthreads();   // previous tile's readers are done
+        for (int i = threadIdx.x; i < r * 64; i += blockDim.x) {
+            const int j = i / 64, c = i % 64;
+            As[j * 64 + c] = __bfloat162float(A[(k0 + c) * r + j]);
+            Bs[j * 64 + c] = (n0 + c < rows) ? __bfloat162float(B[(int64_t)j * rows + n0 + c]) : 0.0f;
+        }
+        __syncthreads();
+        const int64_t n = n0 + nn;
+        if (n >= rows) continue;
+        float d[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) d[e] = 0.0f;
+        for (int j = 0; j < r; ++j) {
+            const float b = Bs[j * 64 + nn];
+            const float4 *a4 = reinterpret_cast<const float4 *>(As + j * 64 + kk0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const float4 a = a4[v];
+                d[4 * v + 0] = fmaf(a.x, b, d[4 * v + 0]);
+                d[4 * v + 1] = fmaf(a.y, b, d[4 * v + 1]);
+                d[4 * v + 2] = fmaf(a.z, b, d[4 * v + 2]);
+                d[4 * v + 3] = fmaf(a.w, b, d[4 * v + 3]);
+            }
+        }
+        // dequantise the 16 weights (one 64-block: block n * kbs + k0 / 64) and add
+        const int64_t e0 = n * cols + k0 + kk0;
+        const int64_t blk = n * kbs + k0 / 64;
+        const float ch = dq_constant(q.scale8[blk], q.scale2[blk / kBlock2], mu);
+        const uint2 cw = *reinterpret_cast<const uint2 *>(q.codes + e0 / 2);
+        uint32_t o[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const uint32_t byte = ((k < 4 ? cw.x : cw.y) >> (8 * (k & 3))) & 0xffu;
+            const float w_hi = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_q[byte >> 4], ch)));
+            const float w_lo = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_q[byte & 15u], ch)));
+            o[k] = pack_bf16x2(__fadd_rn(w_hi, __fmul_rn(s, d[2 * k])), __fadd_rn(w_lo, __fmul_rn(s, d[2 * k + 1])));
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(out + e0);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
+cudaError_t launch_merge_bf16(const NF4View &q, const __nv_bfloat16 *A, const __nv_bfloat16 *B, int r, float s,
+                              __nv_bfloat16 *out, cudaStream_t st) {
+    const int64_t tiles = ceil_div(q.rows, (int64_t)64) * (q.cols / 64);
+    int64_t grid = tiles;
+    const int64_t cap = (int64_t)num_sms() * 4;
+    if (grid > cap) grid = cap;
+    const size_t sm = (size_t)r * 64 * 4 * 2;
+    cudaError_t e = cudaFuncSetAttribute(k_merge_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    QNF4_LAUNCH("k_merge_bf16", st, k_merge_bf16<<<(unsigned)grid, 256, sm, st>>>(q, A, B, r, s, host_codebook(), out));
+    return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlora_nf4_tensor &out,
                             float *c1, double *part, cudaStream_t st) {

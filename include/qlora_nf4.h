@@ -205,6 +205,28 @@ qlora_status qlora_nf4_quantize_noalloc(const void *W, qlora_dtype dt, const qlo
                                         qlora_stream_t stream);
 
 /*
+ * Adapter merge and re-quantisation (the page's sections 5 and 6: merging the
+ * adapter into the weight and re-quantising it can change the outputs, so the
+ * change has to be checked). In BF16, the compute type:
+ *   W'[n,k] = bf16( fl( Dequant(W)[n,k] + fl(s * d[n,k]) ) ),
+ *   d[n,k]  = A[k,0]*B[0,n] + ... + A[k,r-1]*B[r-1,n], one fused multiply-add per
+ *             term in increasing j, starting from 0;
+ * then W_out = the NF4 + double quantisation of W' (qlora_nf4_quantize, bf16 input).
+ *   W      the stored weight [rows, cols]; cols % 64 == 0.
+ *   A, B   bf16 [cols, r] and [r, rows], 1 <= r <= 256, 16-byte aligned.
+ *   W_bf16 optional device buffer (bf16 [rows, cols], 16-byte aligned) that receives
+ *          W'; NULL keeps it in the workspace.
+ *   W_out  receives the re-quantised weight (rows, cols as W); it may be W itself.
+ *   ws     workspace of qlora_nf4_merge_workspace() bytes.
+ * One kernel launch computes W'; the re-quantisation adds three. W' and W_out are
+ * bit-for-bit reproducible. A NaN/Inf in W' sets QLORA_ERR_NONFINITE.
+ */
+size_t qlora_nf4_merge_workspace(int64_t rows, int64_t cols);
+qlora_status qlora_nf4_merge_adapter(const qlora_nf4_tensor *W, const void *A, const void *B, int r, float s,
+                                     void *W_bf16, const qlora_nf4_tensor *W_out, void *ws, size_t ws_bytes,
+                                     qlora_stream_t stream);
+
+/*
  * Self-test of the library's failure detection (the page has no counterpart).
  * Launches one kernel that waits, through the same bounded wait the pipelined
  * kernels use, on a barrier that nothing completes. After the wait limit (1 s)
