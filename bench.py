@@ -35,7 +35,7 @@ UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # the library's kernels, as named by its launch bookkeeping
 KERNELS = ("k_gemm2sm", "k_dequant", "k_fused_fwd", "k_fused_dgrad", "k_skinny", "k_reduce_xa", "k_reduce_f32",
-           "k_gemv", "k_gemv_finish")
+           "k_gemv_xa", "k_gemv_lora", "k_gemv")
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu
 # capture summarised in profiles/k_gemm2sm_l4096.md; update with the kernel.
 TRAFFIC_BYTES = {"k_gemm2sm": 89358336}

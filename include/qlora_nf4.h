@@ -148,10 +148,14 @@ qlora_status qlora_linear_bwd(const void *X, const void *dY, int64_t M, const ql
  *   d      host array of `count` descriptors (1 <= count <= 64); W points to a host
  *          struct as in qlora_linear_fwd.
  *   ws     one device workspace of qlora_linear_fwd_grouped_workspace() bytes.
- * M <= 16: the items go through one GEMV launch and one finish launch (per eight
- * items). Larger M: the items run one after another on the single-item path, and the
- * workspace is the largest single-item requirement. Results are bit-identical to
- * calling qlora_linear_fwd on each item.
+ * M <= 16: per group of up to eight items, three launches: the X*A chunk sums, the
+ * adapter term (s X A) B, and one persistent GEMV over all items' codes (the last two
+ * start early through programmatic dependent launch). Larger M: the items run one after
+ * another on the single-item path, and the workspace is the largest single-item
+ * requirement. XA_save is bit-identical to calling qlora_linear_fwd on each item; Y is
+ * reproducible call to call but, at M <= 16, may differ in the last bits from the
+ * single-item call, because the K chunks of a row block cut between two CTAs are added
+ * in CTA order and the cut depends on the group.
  */
 typedef struct {
     const void *X;                 /* bf16 [M, W->cols] */

@@ -78,8 +78,9 @@ def test_grouped_forward_host_checks():
     d = (q._LinearDesc * 2)(q._LinearDesc(fake, ctypes.pointer(t), None, None, 0, 1.0, fake, None),
                             q._LinearDesc(fake, ctypes.pointer(t), None, None, 0, 1.0, fake, None))
     assert L.qlora_linear_fwd_grouped(1, 0, d, None, 0, None) == q.QLORA_ERR_INVALID_ARG
-    # two 64 x 64 items at M = 1: one split each, M*rows fp32 partials, 256-byte aligned
-    assert L.qlora_linear_fwd_grouped_workspace(1, 2, d) == 2 * 256
+    # two 64 x 64 items at M = 1: one work unit each, so two CTAs; one counter per row
+    # block (256-byte aligned) and two 128-row x M fp32 part slots per CTA
+    assert L.qlora_linear_fwd_grouped_workspace(1, 2, d) == 256 + 2 * 2 * 128 * 1 * 4
     assert L.qlora_linear_fwd_grouped(1, 2, d, None, 0, None) == q.QLORA_ERR_WORKSPACE
     bad = (q._LinearDesc * 1)(q._LinearDesc(fake, ctypes.pointer(q._Tensor(64, 100, fake, fake, fake, fake)),
                                             None, None, 0, 1.0, fake, None))
