@@ -673,6 +673,28 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_decode_profile(M, reps=3):
+    """A small case for an ncu capture of the decode path: one Llama-7B block at M tokens,
+    forward only, through one grouped call, `reps` times with the L2 flushed before each."""
+    import torch
+    import bit_nf4_quantized_double_b200 as q
+    import synth_inputs as si
+    wl = si.workload("decode7b", M=M)
+    items = []
+    for li, L in enumerate(wl.layers):
+        inp = si.layer_inputs(wl, li, device="cuda")
+        items.append({"X": inp["X"], "W": q.qlora_nf4_quantize(inp["W"]), "A": inp.get("A"), "B": inp.get("B"),
+                      "s": L.s, "Y": torch.empty(M, L.d_out, dtype=torch.bfloat16, device="cuda")})
+        del inp
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    for _ in range(reps):
+        flush.zero_()
+        q.qlora_linear_fwd_grouped(items)
+    torch.cuda.synchronize()
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    print(json.dumps({"decode_profile": {"M": M, "reps": reps}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -684,7 +706,12 @@ def main():
     ap.add_argument("--sweep-layers", type=int, default=32)
     ap.add_argument("--cpu-sample-tokens", type=int, default=512)
     ap.add_argument("--no-graph", action="store_true", help="launch every step eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--decode-profile", type=int, default=0, metavar="M",
+                    help="only run the decode block at M tokens three times (a small case for ncu) and exit")
     args = ap.parse_args()
+    if args.decode_profile:
+        run_decode_profile(args.decode_profile)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
