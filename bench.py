@@ -493,7 +493,7 @@ def run_components(args, peaks, peak_kind, flush):
             if L.r:
                 nbytes += inp["A"].numel() * 2 + inp["B"].numel() * 2
             del inp
-        # the block's seven projections in one grouped call (one GEMV + one finish launch)
+        # the block's seven projections in one grouped call (X·A sums, adapter term, one persistent GEMV)
         wsz = q.lib().qlora_linear_fwd_grouped_workspace(
             M, len(items), (q._LinearDesc * len(items))(*[
                 q._LinearDesc(None, ctypes.pointer(it["W"].ctype()), None, None,
