@@ -83,6 +83,10 @@ _SIGS = {
     "qlora_nf4_merge_adapter": (ctypes.c_int, [ctypes.POINTER(_Tensor), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                                ctypes.c_float, ctypes.c_void_p, ctypes.POINTER(_Tensor),
                                                ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_fmt4_quantize": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_fmt4_dequant": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                          ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_launch_count": (ctypes.c_ulonglong, []),
     "qlora_profile_enable": (None, [ctypes.c_int]),
     "qlora_profile_read": (ctypes.c_int, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
@@ -199,6 +203,32 @@ def qlora_nf4_dequant(q: NF4Tensor, out: torch.Tensor | None = None, stream=None
         out = torch.empty(q.rows, q.cols, dtype=torch.bfloat16, device=q.codes.device)
     t = q.ctype()
     _check(lib().qlora_nf4_dequant(ctypes.byref(t), _ptr(out), _stream(stream)), "qlora_nf4_dequant")
+    return out
+
+
+FMT4 = {"int4": 0, "fp4_e2m1": 1, "fp4_e3m0": 2}
+
+
+def qlora_fmt4_quantize(W: torch.Tensor, fmt: str, stream=None):
+    """Blockwise Int4 / FP4 E2M1 / FP4 E3M0 (64-weight absmax blocks) of a fp32 or bf16 tensor.
+    Returns (codes uint8 [ceil(n/2)], two codes per byte; absmax fp32 [ceil(n/64)])."""
+    W = W.contiguous()
+    n = W.numel()
+    dt = {torch.float32: QLORA_F32, torch.bfloat16: QLORA_BF16}[W.dtype]
+    codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=W.device)
+    absmax = torch.empty((n + 63) // 64, dtype=torch.float32, device=W.device)
+    _check(lib().qlora_fmt4_quantize(_ptr(W), dt, n, FMT4[fmt], _ptr(codes), _ptr(absmax), _stream(stream)),
+           "qlora_fmt4_quantize")
+    return codes, absmax
+
+
+def qlora_fmt4_dequant(codes: torch.Tensor, absmax: torch.Tensor, n: int, fmt: str, out: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """bf16 [n] from the codes and block constants of qlora_fmt4_quantize."""
+    if out is None:
+        out = torch.empty(n, dtype=torch.bfloat16, device=codes.device)
+    _check(lib().qlora_fmt4_dequant(_ptr(codes), _ptr(absmax), n, FMT4[fmt], _ptr(out), _stream(stream)),
+           "qlora_fmt4_dequant")
     return out
 
 

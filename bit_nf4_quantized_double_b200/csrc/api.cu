@@ -234,6 +234,28 @@ qlora_status qlora_linear_bwd(const void *X, const void *dY, int64_t M, const ql
                                        ws, static_cast<cudaStream_t>(stream)));
 }
 
+static bool fmt4_ok(qlora_fmt4 f) {
+    return f == QLORA_FMT4_INT4 || f == QLORA_FMT4_FP4_E2M1 || f == QLORA_FMT4_FP4_E3M0;
+}
+
+qlora_status qlora_fmt4_quantize(const void *W, qlora_dtype dt, int64_t n, qlora_fmt4 fmt, uint8_t *codes,
+                                 float *absmax, qlora_stream_t stream) {
+    const uintptr_t wa = reinterpret_cast<uintptr_t>(W);
+    if (!W || !codes || !absmax || n < 1 || !fmt4_ok(fmt) || (dt != QLORA_F32 && dt != QLORA_BF16) ||
+        (wa & (dt == QLORA_F32 ? 3u : 1u)) || (reinterpret_cast<uintptr_t>(absmax) & 3u))
+        return QLORA_ERR_INVALID_ARG;
+    return from_cuda(launch_fmt4_quantize(W, dt, n, fmt, codes, absmax, static_cast<cudaStream_t>(stream)));
+}
+
+qlora_status qlora_fmt4_dequant(const uint8_t *codes, const float *absmax, int64_t n, qlora_fmt4 fmt,
+                                void *W_out, qlora_stream_t stream) {
+    if (!codes || !absmax || !W_out || n < 1 || !fmt4_ok(fmt) || (reinterpret_cast<uintptr_t>(absmax) & 3u) ||
+        (reinterpret_cast<uintptr_t>(W_out) & 3u))
+        return QLORA_ERR_INVALID_ARG;
+    return from_cuda(launch_fmt4_dequant(codes, absmax, n, fmt, static_cast<__nv_bfloat16 *>(W_out),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 qlora_status qlora_get_device_status(qlora_stream_t stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QLORA_ERR_CUDA;
     unsigned int bits = 0, zero = 0;

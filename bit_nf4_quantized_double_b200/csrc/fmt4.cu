@@ -1,0 +1,125 @@
+// Blockwise 4-bit reference formats that the NF4 + double-quantisation format is compared
+// with: Int4, FP4 E2M1 and FP4 E3M0 (page "QLoRA: put the large model in memory, then change
+// it with a small adapter", wq-win.github.io/llm/074-qlora, section 4, evidence 1, the
+// paper's Table 2). The pages name the formats without defining them. This file follows these
+// readings:
+//   64-weight blocks, each scaled by its absmax c (fp32, not double-quantised), with |w| = c
+//     mapped to the format's largest magnitude S;
+//   Int4: magnitudes 0..7 (S = 7);
+//   E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit, with subnormals: magnitudes
+//     0, 0.5, 1, 1.5, 2, 3, 4, 6 (S = 6);
+//   E3M0: sign, 3 exponent bits, exponent field 0 = zero: magnitudes 0 and 2^(e-7) for
+//     e = 1..7 (S = 1);
+//   x' = fl(fl(w / c) * S); the magnitude index is the count of midpoints below |x'|, with a
+//     tie exactly on a midpoint going to the even index; bit 3 holds the sign (none for zero);
+//   w^ = bf16(fl(v * fl(c / S))).
+// Codes are packed two per byte as in the NF4 format: byte k = code[2k] << 4 | code[2k + 1].
+//
+// k_fmt4_quantize: one warp per 64-block, each lane two consecutive weights (one output byte),
+// absmax by a butterfly of shuffles. k_fmt4_dequant: one thread per byte. Both stream HBM.
+#include "launch.h"
+
+namespace qnf4 {
+
+struct Fmt4Table {
+    float mag[8];   // magnitudes, ascending
+    float mid[7];   // midpoints of consecutive magnitudes (exact in fp32)
+    float S;        // largest magnitude
+};
+
+static Fmt4Table fmt4_table(qlora_fmt4 f) {
+    Fmt4Table t;
+    switch (f) {
+        case QLORA_FMT4_INT4:
+            for (int i = 0; i < 8; ++i) t.mag[i] = (float)i;
+            break;
+        case QLORA_FMT4_FP4_E2M1: {
+            const float m[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+            for (int i = 0; i < 8; ++i) t.mag[i] = m[i];
+            break;
+        }
+        default:   // QLORA_FMT4_FP4_E3M0
+            t.mag[0] = 0.0f;
+            for (int e = 1; e <= 7; ++e) t.mag[e] = std::ldexp(1.0f, e - 7);
+            break;
+    }
+    for (int i = 0; i < 7; ++i) t.mid[i] = (t.mag[i] + t.mag[i + 1]) * 0.5f;   // exact for all three
+    t.S = t.mag[7];
+    return t;
+}
+
+__device__ __forceinline__ float load_f32(const float *p) { return __ldg(p); }
+__device__ __forceinline__ float load_f32(const __nv_bfloat16 *p) { return __bfloat162float(p[0]); }
+
+__device__ __forceinline__ uint32_t fmt4_code(float w, float c, const Fmt4Table &t) {
+    const float x = c > 0.0f ? __fmul_rn(__fdiv_rn(w, c), t.S) : 0.0f;
+    const float m = fabsf(x);
+    uint32_t idx = 0;
+#pragma unroll
+    for (int i = 0; i < 7; ++i) idx += (t.mid[i] < m) ? 1u : 0u;
+    if (idx < 7 && (idx & 1u) && m == t.mid[idx]) ++idx;       // a tie goes to the even index
+    return idx | ((x < 0.0f && idx > 0) ? 8u : 0u);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_fmt4_quantize(const T *__restrict__ w, int64_t n, const __grid_constant__ Fmt4Table t,
+                                                      uint8_t *__restrict__ codes, float *__restrict__ absmax) {
+    const int64_t blk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t nb = (n + 63) / 64;
+    if (blk >= nb) return;                                       // whole warps leave together
+    const int64_t i0 = blk * 64 + 2 * lane;
+    const float a = i0 < n ? load_f32(w + i0) : 0.0f;
+    const float b = i0 + 1 < n ? load_f32(w + i0 + 1) : 0.0f;
+    float c = fmaxf(fabsf(a), fabsf(b));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, o));
+    if (i0 < n) codes[i0 >> 1] = (uint8_t)((fmt4_code(a, c, t) << 4) | fmt4_code(b, c, t));
+    if (lane == 0) absmax[blk] = c;
+}
+
+__global__ void __launch_bounds__(256) k_fmt4_dequant(const uint8_t *__restrict__ codes,
+                                                     const float *__restrict__ absmax, int64_t n,
+                                                     const __grid_constant__ Fmt4Table t,
+                                                     __nv_bfloat16 *__restrict__ out) {
+    const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // byte index
+    if (2 * k >= n) return;
+    const uint32_t byte = codes[k];
+    const float step = __fdiv_rn(__ldg(absmax + (2 * k) / 64), t.S);
+    const uint32_t c0 = byte >> 4, c1 = byte & 15u;
+    const float v0 = (c0 & 8u) ? -t.mag[c0 & 7u] : t.mag[c0 & 7u];
+    const float v1 = (c1 & 8u) ? -t.mag[c1 & 7u] : t.mag[c1 & 7u];
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(__fmul_rn(v0, step));
+    if (2 * k + 1 < n) {
+        __nv_bfloat162 p;
+        p.x = h0;
+        p.y = __float2bfloat16_rn(__fmul_rn(v1, step));
+        *reinterpret_cast<__nv_bfloat162 *>(out + 2 * k) = p;
+    } else {
+        out[2 * k] = h0;
+    }
+}
+
+cudaError_t launch_fmt4_quantize(const void *W, qlora_dtype dt, int64_t n, qlora_fmt4 f, uint8_t *codes,
+                                 float *absmax, cudaStream_t st) {
+    const int64_t nb = (n + 63) / 64;
+    const unsigned grid = (unsigned)ceil_div(nb * 32, 256);
+    const Fmt4Table t = fmt4_table(f);
+    if (dt == QLORA_F32)
+        QNF4_LAUNCH("k_fmt4_quantize", st,
+                    k_fmt4_quantize<float><<<grid, 256, 0, st>>>(static_cast<const float *>(W), n, t, codes, absmax));
+    else
+        QNF4_LAUNCH("k_fmt4_quantize", st,
+                    k_fmt4_quantize<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W), n, t,
+                                                                        codes, absmax));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fmt4_dequant(const uint8_t *codes, const float *absmax, int64_t n, qlora_fmt4 f,
+                                __nv_bfloat16 *out, cudaStream_t st) {
+    const unsigned grid = (unsigned)ceil_div((n + 1) / 2, 256);
+    QNF4_LAUNCH("k_fmt4_dequant", st, k_fmt4_dequant<<<grid, 256, 0, st>>>(codes, absmax, n, fmt4_table(f), out));
+    return cudaGetLastError();
+}
+
+}  // namespace qnf4

@@ -8,6 +8,10 @@ namespace qnf4 {
 cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlora_nf4_tensor &out,
                             float *c1, double *part, cudaStream_t st);
 cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st);
+cudaError_t launch_fmt4_quantize(const void *W, qlora_dtype dt, int64_t n, qlora_fmt4 f, uint8_t *codes,
+                                 float *absmax, cudaStream_t st);
+cudaError_t launch_fmt4_dequant(const uint8_t *codes, const float *absmax, int64_t n, qlora_fmt4 f,
+                                __nv_bfloat16 *out, cudaStream_t st);
 cudaError_t launch_merge_bf16(const NF4View &q, const __nv_bfloat16 *A, const __nv_bfloat16 *B, int r, float s,
                               __nv_bfloat16 *out, cudaStream_t st);
 

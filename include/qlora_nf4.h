@@ -241,6 +241,35 @@ qlora_status qlora_nf4_merge_adapter(const qlora_nf4_tensor *W, const void *A, c
 qlora_status qlora_selftest_wait_timeout(qlora_stream_t stream);
 
 /*
+ * Reference 4-bit formats that the page compares NF4 + DQ against: Int4, FP4 E2M1 and FP4 E3M0
+ * (page "QLoRA: put the large model in memory, then change it with a small adapter", section 4,
+ * evidence 1, the paper's Table 2). The page names them without defining them. The readings:
+ *   64-weight blocks, each scaled by its fp32 absmax c (no double quantisation), with |w| = c
+ *   mapped to the largest magnitude S;
+ *   INT4: magnitudes 0..7 (S = 7);
+ *   FP4_E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit, with subnormals:
+ *     magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 (S = 6);
+ *   FP4_E3M0: sign, 3 exponent bits, exponent field 0 = zero: magnitudes 0 and
+ *     2^(e-7) for e = 1..7 (S = 1).
+ * Quantisation: x' = fl(fl(w / c) * S); the code is the count of midpoints of consecutive
+ * magnitudes below |x'|, with a tie exactly on a midpoint going to the even index, plus bit 3
+ * for a negative value (never for zero); an all-zero block gives zero codes.
+ * Dequantisation: w^ = bf16(fl(v * fl(c / S))).
+ *   W       device, n finite values of dtype dt (fp32 4-byte, bf16 2-byte aligned);
+ *   codes   device, ceil(n/2) bytes, byte k = code[2k] << 4 | code[2k+1] (the NF4 packing);
+ *           for odd n the missing low nibble is the zero code;
+ *   absmax  device, ceil(n/64) fp32 block constants, 4-byte aligned;
+ *   W_out   device, n bf16, 4-byte aligned.
+ * One kernel launch each; QLORA_ERR_INVALID_ARG for a null or misaligned pointer, n < 1 or an
+ * unknown format.
+ */
+typedef enum { QLORA_FMT4_INT4 = 0, QLORA_FMT4_FP4_E2M1 = 1, QLORA_FMT4_FP4_E3M0 = 2 } qlora_fmt4;
+qlora_status qlora_fmt4_quantize(const void *W, qlora_dtype dt, int64_t n, qlora_fmt4 fmt, uint8_t *codes,
+                                 float *absmax, qlora_stream_t stream);
+qlora_status qlora_fmt4_dequant(const uint8_t *codes, const float *absmax, int64_t n, qlora_fmt4 fmt,
+                                void *W_out, qlora_stream_t stream);
+
+/*
  * Measurement hooks. The page has no counterpart: they let a benchmark count
  * and time the library's own kernels without a profiler.
  *   qlora_launch_count    kernel launches issued by this process so far.

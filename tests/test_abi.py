@@ -119,3 +119,14 @@ def test_argument_checks_run_on_host():
                               None) == q.QLORA_ERR_WORKSPACE
     assert L.qlora_linear_bwd(None, ctypes.c_void_p(fake), 0, ctypes.byref(good), None, None, 0, 1.0, None,
                               ctypes.c_void_p(fake), None, None, None, 0, None) == q.QLORA_ERR_UNSUPPORTED_SHAPE
+
+
+def test_fmt4_argument_checks_run_on_host():
+    L = q.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.qlora_fmt4_quantize(None, 0, 64, 0, fake, fake, None) == q.QLORA_ERR_INVALID_ARG
+    assert L.qlora_fmt4_quantize(fake, 0, 0, 0, fake, fake, None) == q.QLORA_ERR_INVALID_ARG       # n < 1
+    assert L.qlora_fmt4_quantize(fake, 0, 64, 5, fake, fake, None) == q.QLORA_ERR_INVALID_ARG      # format
+    assert L.qlora_fmt4_quantize(fake, 2, 64, 0, fake, fake, None) == q.QLORA_ERR_INVALID_ARG      # dtype
+    assert L.qlora_fmt4_quantize(ctypes.c_void_p((1 << 20) + 2), 0, 64, 0, fake, fake, None) == q.QLORA_ERR_INVALID_ARG
+    assert L.qlora_fmt4_dequant(fake, fake, 64, 1, ctypes.c_void_p((1 << 20) + 2), None) == q.QLORA_ERR_INVALID_ARG
