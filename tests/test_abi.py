@@ -130,3 +130,23 @@ def test_fmt4_argument_checks_run_on_host():
     assert L.qlora_fmt4_quantize(fake, 2, 64, 0, fake, fake, None) == q.QLORA_ERR_INVALID_ARG      # dtype
     assert L.qlora_fmt4_quantize(ctypes.c_void_p((1 << 20) + 2), 0, 64, 0, fake, fake, None) == q.QLORA_ERR_INVALID_ARG
     assert L.qlora_fmt4_dequant(fake, fake, 64, 1, ctypes.c_void_p((1 << 20) + 2), None) == q.QLORA_ERR_INVALID_ARG
+
+
+def test_grouped_workspace_is_largest_group_of_eight():
+    # more than eight projections go in groups of eight that reuse one workspace, so the
+    # query returns the largest group's need, and a group of one equals the single call's
+    L = q.lib()
+    fake = 1 << 20
+    shapes = [(4096, 4096, 16)] * 4 + [(11008, 4096, 0)] * 2 + [(4096, 11008, 0)] + [(1024, 2048, 64)] * 13
+    ts = [q._Tensor(rows, cols, fake, fake, fake, fake) for rows, cols, _ in shapes]
+    descs = [q._LinearDesc(fake, ctypes.pointer(t), fake, fake, r, 1.0, fake, None) for t, (_, _, r) in zip(ts, shapes)]
+    for M in (1, 16):
+        arr = (q._LinearDesc * len(descs))(*descs)
+        whole = L.qlora_linear_fwd_grouped_workspace(M, len(descs), arr)
+        parts = []
+        for i in range(0, len(descs), 8):
+            sub = (q._LinearDesc * len(descs[i:i + 8]))(*descs[i:i + 8])
+            parts.append(L.qlora_linear_fwd_grouped_workspace(M, len(descs[i:i + 8]), sub))
+        assert whole == max(parts)
+        one = (q._LinearDesc * 1)(descs[0])
+        assert L.qlora_linear_fwd_grouped_workspace(M, 1, one) == L.qlora_linear_fwd_workspace(M, 4096, 4096, 16)
