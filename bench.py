@@ -36,8 +36,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the library's kernels, as named by its launch bookkeeping
 KERNELS = ("k_gemm2sm", "k_dequant", "k_fused_fwd", "k_fused_dgrad", "k_skinny", "k_reduce_xa", "k_reduce_f32",
            "k_gemv_xa", "k_gemv_lora", "k_gemv")
-# DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu
-# capture summarised in profiles/k_gemm2sm_l4096.md; update with the kernel.
+# DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
+# capture of the same kernel and workload; update with the kernel.
 TRAFFIC_BYTES = {"k_gemm2sm": 89358336}
 L2_FLUSH_BYTES = 256 << 20        # 2x the 126 MB L2
 
@@ -193,6 +193,20 @@ def max_over_ranks(x, world):
 
 
 # ------------------------------------------------------------------ our arm
+def rank_batch(wl, li, rank, device):
+    """The data-parallel partition of the tokens: rank k trains on its own batch of
+    wl.M tokens (X, dY), drawn with the workload's seeds shifted by 7777 k, so the
+    global batch of N ranks is the concatenation of the N rank batches in rank order
+    (rank 0's batch is the single-GPU workload itself)."""
+    import torch
+    import synth_inputs as si
+    L = wl.layers[li]
+    X = si.normal((wl.M, L.d_in), 1.0, si.seed_of(wl, li, "X") + 7777 * rank, device=device, dtype=torch.bfloat16)
+    dY = si.normal((wl.M, L.d_out), 1.0, si.seed_of(wl, li, "dY") + 7777 * rank, device=device,
+                   dtype=torch.bfloat16)
+    return X, dY
+
+
 def headline_inputs(rank):
     import synth_inputs as si
     wl = si.workload("l4096")
@@ -200,10 +214,7 @@ def headline_inputs(rank):
     inp = si.layer_inputs(wl, 0, device="cuda", w_device="cuda")
     if rank:
         # weak scaling: every rank its own batch of tokens
-        inp["X"] = si.normal((wl.M, L.d_in), 1.0, si.seed_of(wl, 0, "X") + 7777 * rank, device="cuda",
-                             dtype=inp["X"].dtype)
-        inp["dY"] = si.normal((wl.M, L.d_out), 1.0, si.seed_of(wl, 0, "dY") + 7777 * rank, device="cuda",
-                              dtype=inp["dY"].dtype)
+        inp["X"], inp["dY"] = rank_batch(wl, 0, rank, "cuda")
     return wl, L, inp
 
 

@@ -128,6 +128,18 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _hold(stream, *tensors):
+    """Temporaries made for a call (contiguous copies, a workspace) are freed when the
+    wrapper returns, while the kernels queued on `stream` may still read them. torch's
+    caching allocator only orders reuse on the current stream, so when the call went
+    to another stream the blocks are marked as in use by that stream as well."""
+    if stream is None or stream == torch.cuda.current_stream():
+        return
+    for t in tensors:
+        if t is not None:
+            t.record_stream(stream)
+
+
 @dataclass
 class NF4Tensor:
     """The stored format: four device buffers owned by torch."""
@@ -193,8 +205,10 @@ def qlora_nf4_quantize(W: torch.Tensor, out: NF4Tensor | None = None, ws: torch.
     need = int(L.qlora_nf4_quantize_workspace(rows, cols))
     wsb, wsn = _workspace(need, W.device, ws)
     t = out.ctype()
-    _check(L.qlora_nf4_quantize(_ptr(W.contiguous()), dt, ctypes.byref(t), _ptr(wsb), wsn, _stream(stream)),
+    Wc = W.contiguous()
+    _check(L.qlora_nf4_quantize(_ptr(Wc), dt, ctypes.byref(t), _ptr(wsb), wsn, _stream(stream)),
            "qlora_nf4_quantize")
+    _hold(stream, Wc, wsb)
     return out
 
 
@@ -219,6 +233,7 @@ def qlora_fmt4_quantize(W: torch.Tensor, fmt: str, stream=None):
     absmax = torch.empty((n + 63) // 64, dtype=torch.float32, device=W.device)
     _check(lib().qlora_fmt4_quantize(_ptr(W), dt, n, FMT4[fmt], _ptr(codes), _ptr(absmax), _stream(stream)),
            "qlora_fmt4_quantize")
+    _hold(stream, W)
     return codes, absmax
 
 
@@ -249,6 +264,7 @@ def qlora_linear_fwd(X: torch.Tensor, W: NF4Tensor, A: torch.Tensor | None, B: t
     t = W.ctype()
     _check(L.qlora_linear_fwd(_ptr(X), M, ctypes.byref(t), _ptr(A), _ptr(B), r, float(s), _ptr(Y),
                               _ptr(XA_save), _ptr(wsb), wsn, _stream(stream)), "qlora_linear_fwd")
+    _hold(stream, wsb)
     return Y, XA_save
 
 
@@ -266,6 +282,7 @@ def qlora_nf4_merge_adapter(W: NF4Tensor, A: torch.Tensor, B: torch.Tensor, s: f
     t, to = W.ctype(), out.ctype()
     _check(L.qlora_nf4_merge_adapter(ctypes.byref(t), _ptr(A), _ptr(B), A.shape[1], float(s), _ptr(W_bf16),
                                      ctypes.byref(to), _ptr(wsb), wsn, _stream(stream)), "qlora_nf4_merge_adapter")
+    _hold(stream, wsb)
     return out, W_bf16
 
 
@@ -292,6 +309,7 @@ def qlora_linear_fwd_grouped(items, ws: torch.Tensor | None = None, stream=None)
     L = lib()
     wsb, wsn = _workspace(int(L.qlora_linear_fwd_grouped_workspace(M, n, descs)), items[0]["X"].device, ws)
     _check(L.qlora_linear_fwd_grouped(M, n, descs, _ptr(wsb), wsn, _stream(stream)), "qlora_linear_fwd_grouped")
+    _hold(stream, wsb)
     return outs
 
 
@@ -314,6 +332,7 @@ def qlora_linear_bwd(X: torch.Tensor, dY: torch.Tensor, W: NF4Tensor, A: torch.T
     t = W.ctype()
     _check(L.qlora_linear_bwd(_ptr(X), _ptr(dY), M, ctypes.byref(t), _ptr(A), _ptr(B), r, float(s), _ptr(XA),
                               _ptr(dX), _ptr(dA), _ptr(dB), _ptr(wsb), wsn, _stream(stream)), "qlora_linear_bwd")
+    _hold(stream, wsb)
     return dX, dA, dB
 
 

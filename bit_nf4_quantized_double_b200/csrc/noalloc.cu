@@ -12,8 +12,6 @@
 // Cost of that choice: every GPU that loads the library holds kScratchBytes
 // (about 4 MiB) until the process exits, whether or not the entry point is
 // used; tensors above kNoAllocMaxWeights weights are rejected.
-#include <mutex>
-
 #include "launch.h"
 
 namespace qnf4 {
@@ -26,28 +24,20 @@ constexpr size_t kC1Bytes = (size_t)kNoAllocMaxBlocks * sizeof(float);       // 
 constexpr size_t kScratchBytes = kC1Bytes + (size_t)kNoAllocMaxGroups * sizeof(double);
 
 // The scratch array. In host code this name only stands for the symbol; its
-// device address is looked up per device below and passed to the kernels.
+// device address is looked up below and passed to the kernels.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void *g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and cached.
+// Device address of the scratch array in the current device's context, looked
+// up on every call rather than cached: a context that the caller destroys and
+// re-creates (cudaDeviceReset, a primary-context reset) reloads this library's
+// device code, and the array may then sit at another address. The lookup is a
+// host-side table read once the code is loaded; the first lookup in a context
+// loads it.
 cudaError_t scratch_address(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return cudaSuccess;
 }
 

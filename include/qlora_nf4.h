@@ -197,9 +197,10 @@ void qlora_nf4_codebook(float out[16]);
  *   held until the process exits). The call allocates and frees nothing.
  *   Limit: rows * cols <= 67,108,864 (2^26) weights; larger tensors return
  *   QLORA_ERR_UNSUPPORTED_SHAPE before anything is launched.
- *   The first call on each device looks up that device's copy of the array
- *   (with the device current) and caches it; make that first call before any
- *   stream capture.
+ *   Every call looks up the array's address in the current device's context
+ *   (nothing is cached, so a context that the caller resets and re-creates is
+ *   handled); the first call in a context loads the library's device code
+ *   there, so make that first call before any stream capture.
  *   Every call uses the same array. Calls whose kernels may overlap on the GPU
  *   (different streams without ordering, several host threads) race on it and
  *   give undefined results; serialise them. No call depends on what an
