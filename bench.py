@@ -35,11 +35,23 @@ UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # the library's kernels, as named by its launch bookkeeping
 KERNELS = ("k_gemm2sm", "k_dequant", "k_fused_fwd", "k_fused_dgrad", "k_skinny", "k_reduce_xa", "k_reduce_f32",
-           "k_gemv_xa", "k_gemv_lora", "k_gemv")
+           "k_gemv_xa", "k_gemv", "k_gemv_finish", "k_quantize_codes", "k_offset", "k_double_quant")
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
 # capture of the same kernel and workload; update with the kernel.
 TRAFFIC_BYTES = {"k_gemm2sm": 89358336}
+TRAFFIC_SOURCE = {"k_gemm2sm": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
+                                "-k regex:k_gemm2sm -c 1 on this workload (4096 x 4096 layer, M = 4096, r = 64)"}
 L2_FLUSH_BYTES = 256 << 20        # 2x the 126 MB L2
+
+
+def l2_flush(buf):
+    """Evict the timed kernels' inputs from L2 between timed repetitions (outside the timed
+    region): write a buffer twice the L2 size, then read it back. The read leaves L2 holding
+    clean lines of the flush buffer; a write alone would leave about 126 MB of dirty lines
+    whose write-back the next timed kernel would pay for in DRAM bandwidth."""
+    import torch
+    buf.zero_()
+    buf.view(torch.int32).sum()
 
 
 def step_flops(M, d_in, d_out, r):
@@ -284,7 +296,7 @@ def run_ours(args, peaks, peak_kind):
     launches0 = q.qlora_launch_count()
     clocks.mark_begin()
     for i in range(args.steps):
-        flush.zero_()                     # L2 flush between timed steps (not timed)
+        l2_flush(flush)                     # L2 flush between timed steps (not timed)
         evs[i][0].record(stream)
         step()
         evs[i][1].record(stream)
@@ -307,7 +319,7 @@ def run_ours(args, peaks, peak_kind):
     q.qlora_profile_read(None)
     q.qlora_profile_enable(True)
     for i in range(args.steps):
-        flush.zero_()
+        l2_flush(flush)
         eager_step()
     q.qlora_profile_enable(False)
     torch.cuda.synchronize()
@@ -329,10 +341,10 @@ def run_ours(args, peaks, peak_kind):
     per_step = dom_n // args.steps if dom_n else 0
     dom_flops = (fwd_flops + dgrad_flops) / 2 if per_step == 2 else (fwd_flops if dom != "k_fused_dgrad" else dgrad_flops)
     achieved = dom_flops / (dom_ms / dom_n / 1e3) / 1e12 if dom_n else None
-    # the kernel runs inside a long back-to-back step, so the sustained (power-capped)
-    # cuBLAS figure is its denominator; the burst one is reported beside it
-    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    # the timed region lasts milliseconds, so the burst cuBLAS figure is the denominator;
+    # the sustained (seconds-long, power-capped) one is reported beside it
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
 
     # ---------------------------------------------------------------- e2e
     Xh = X.cpu().pin_memory()
@@ -353,7 +365,7 @@ def run_ours(args, peaks, peak_kind):
     eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier(world)
     for i in range(args.steps):
-        flush.zero_()
+        l2_flush(flush)
         eev[i][0].record(stream)
         e2e_step()
         eev[i][1].record(stream)
@@ -380,15 +392,15 @@ def run_ours(args, peaks, peak_kind):
                                "W ~ N(0,0.02) fp32 with 0.1% x10 outliers quantised once to NF4+DQ, "
                                "X,dY ~ N(0,1) bf16; step = fwd + bwd" + (" + NCCL all-reduce of dA,dB"
                                                                        if world > 1 else ""),
-                   "global_batch_tokens": M * world, "l2": "flushed between timed steps (256 MB write)",
+                   "global_batch_tokens": M * world, "l2": "flushed between timed steps (256 MB written, then read back)",
                    "flops_per_step": flops, "parallelism": f"dp{world}" if world > 1 else "single GPU",
                    "launch": "CUDA graph replay of the layer fwd+bwd" if graph is not None else "eager"},
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2) if achieved else None,
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4) if achieved else None,
-                     "peak_source": f"{peak_kind} bf16 sustained (MEASURED_PEAKS.json)" if peak_kind == "measured"
-                     else "fallback 1400 TFLOP/s sustained",
-                     "frac_of_burst": round(achieved / peak_burst, 4) if achieved else None,
-                     "traffic": TRAFFIC_BYTES.get(dom), "flops_per_launch": dom_flops, "launches": dom_n,
+                     "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                     else "fallback 1590 TFLOP/s burst",
+                     "frac_of_sustained": round(achieved / peak_sustained, 4) if achieved else None,
+                     "traffic": TRAFFIC_BYTES.get(dom), "traffic_source": TRAFFIC_SOURCE.get(dom), "flops_per_launch": dom_flops, "launches": dom_n,
                      "kernel_ms_per_step": {k: round(v[0] / args.steps, 5) for k, v in kern.items()},
                      "kernel_launches_per_step": {k: v[1] // args.steps for k, v in kern.items()}},
         "e2e": e2e, "gpu_launches": launches, "clocks": clk,
@@ -419,7 +431,7 @@ def _time_graph(fn, reps, flush, stream):
         g.replay()
     times = []
     for _ in range(reps):
-        flush.zero_()
+        l2_flush(flush)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(torch.cuda.current_stream())
         g.replay()
@@ -431,62 +443,99 @@ def _time_graph(fn, reps, flush, stream):
     return ms
 
 
-def run_components(args, peaks, peak_kind, flush):
+def _host_time(fn, target_s=2.0, max_reps=10):
+    """Seconds per call of fn on the host: one call, then repeats filling about target_s."""
+    t0 = time.perf_counter()
+    fn()
+    one = time.perf_counter() - t0
+    reps = max(1, min(max_reps, int(target_s / max(one, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        fn()
+    return (time.perf_counter() - t0) / reps, reps
+
+
+def _kernel_ms(names, fn, reps, flush):
+    """Per-call device milliseconds of the named library kernels over `reps` eager calls
+    of fn (every launch bracketed by CUDA events on its stream, L2 flushed before each)."""
     import torch
     import bit_nf4_quantized_double_b200 as q
+    q.qlora_profile_read(None)
+    q.qlora_profile_enable(True)
+    for _ in range(reps):
+        l2_flush(flush)
+        fn()
+    q.qlora_profile_enable(False)
+    torch.cuda.synchronize()
+    out = {}
+    for n in names:
+        ms, k = q.qlora_profile_read(n)
+        if k:
+            out[n] = {"ms_per_call": round(ms / reps, 5), "launches_per_call": k // reps}
+    q.qlora_profile_read(None)
+    return out
+
+
+def run_components(args, peaks, peak_kind, flush):
+    import numpy as np
+    import torch
+    import bit_nf4_quantized_double_b200 as q
+    import oracle
     import synth_inputs as si
 
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     out = {"hbm_peak_gbs": hbm, "hbm_peak_source": peak_kind}
     stream = torch.cuda.current_stream()
+    cores = _cores()
 
-    # --- quantise / dequantise sweep over 32 Llama-7B-shaped layers (bf16 weights)
+    # --- quantise / dequantise sweep over 32 Llama-7B-shaped layers (bf16 weights), one
+    # grouped call per layer (its seven projections)
     n_layers = args.sweep_layers
     wl = si.workload("llama7b", n_layers=n_layers)
-    Ws, Ts = [], []
-    for li in range(len(wl.layers)):
-        W = si.layer_inputs(wl, li, device="cuda")["W"]
-        Ws.append(W)
-        Ts.append(q.nf4_empty(W.shape[0], W.shape[1]))
-    n_w = sum(W.numel() for W in Ws)
-    maxn = max(W.numel() for W in Ws)
-    wq_ws = torch.empty(q.lib().qlora_nf4_quantize_workspace(1, maxn), dtype=torch.uint8, device="cuda")
-    wh = torch.empty(maxn, dtype=torch.bfloat16, device="cuda")
+    layers = []
+    for l0 in range(0, len(wl.layers), 7):
+        Ws = [si.layer_inputs(wl, li, device="cuda")["W"] for li in range(l0, l0 + 7)]
+        layers.append((Ws, [q.nf4_empty(W.shape[0], W.shape[1]) for W in Ws]))
+    n_w = sum(W.numel() for Ws, _ in layers for W in Ws)
+    ws_q = torch.empty(q.lib().qlora_nf4_quantize_grouped_workspace(
+        7, (q._Tensor * 7)(*[t.ctype() for t in layers[0][1]])), dtype=torch.uint8, device="cuda")
+    wh = [torch.empty(W.shape, dtype=torch.bfloat16, device="cuda") for W in layers[0][0]]
     alg_bytes = 2.0 + 0.5 + 1.0 / 64 + 4.0 / 16384       # per weight, bf16 in/out
 
     def quant_sweep():
-        for W, T in zip(Ws, Ts):
-            q.qlora_nf4_quantize(W, out=T, ws=wq_ws)
+        for Ws, Ts in layers:
+            q.qlora_nf4_quantize_grouped(Ws, outs=Ts, ws=ws_q)
 
     def deq_sweep():
-        for T in Ts:
-            q.qlora_nf4_dequant(T, out=wh[: T.rows * T.cols].view(T.rows, T.cols))
+        for _, Ts in layers:
+            q.qlora_nf4_dequant_grouped(Ts, outs=wh)
 
     res = {}
-    for name, fn in (("quantize", quant_sweep), ("dequant", deq_sweep)):
-        # the sweep (224 matrices) replayed from a CUDA graph; the kernel-only time comes
-        # from a separate eager pass with CUDA events around each launch
+    for name, fn, knames in (("quantize", quant_sweep, ("k_quantize_codes", "k_offset", "k_double_quant")),
+                             ("dequant", deq_sweep, ("k_dequant",))):
         reps = 3
         ms = _time_graph(fn, reps, flush, stream)
-        q.qlora_profile_read(None)
-        q.qlora_profile_enable(True)
-        for _ in range(reps):
-            fn()
-        q.qlora_profile_enable(False)
-        torch.cuda.synchronize()
-        kname = "k_quantize_codes" if name == "quantize" else "k_dequant"
-        kms, kn = q.qlora_profile_read(kname)
-        q.qlora_profile_read(None)
+        kern = _kernel_ms(knames, fn, reps, flush)
+        kms = sum(v["ms_per_call"] for v in kern.values())
         gbs = n_w * alg_bytes / (ms / 1e3) / 1e9
-        kgbs = n_w * alg_bytes / (kms / reps / 1e3) / 1e9 if kn else None
-        res[name] = {"workload": f"{n_layers} Llama-7B layers x 7 projections, {n_w} bf16 weights",
+        res[name] = {"workload": f"{n_layers} Llama-7B layers x 7 projections, {n_w} bf16 weights, "
+                                 "one grouped call per layer, CUDA graph replay, L2 flushed",
                      "ms_per_sweep": round(ms, 4), "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
-                     "kernel": kname, "kernel_GB/s": round(kgbs, 1) if kgbs else None,
-                     "kernel_frac": round(kgbs / hbm, 4) if kgbs else None,
-                     "bytes_per_weight": round(alg_bytes, 5), "launches": kn}
+                     "kernels": kern, "kernel_GB/s": round(n_w * alg_bytes / (kms / 1e3) / 1e9, 1) if kms else None,
+                     "bytes_per_weight": round(alg_bytes, 5)}
+    # the oracle on the host: one projection (4096 x 4096, bf16) quantised and dequantised
+    Wq = layers[0][0][0]
+    bits = Wq.view(torch.int16).cpu().numpy().view(np.uint16).ravel()
+    t_q, rq = _host_time(lambda: oracle.quantize_bf16(bits, Wq.shape[0], Wq.shape[1]))
+    ref = oracle.quantize_bf16(bits, Wq.shape[0], Wq.shape[1])
+    t_d, rd = _host_time(lambda: oracle.dequant(ref))
+    nq = Wq.numel()
+    for name, t_s, reps in (("quantize", t_q, rq), ("dequant", t_d, rd)):
+        res[name]["cpu_baseline"] = {"value": round(nq * alg_bytes / t_s / 1e9, 3), "unit": "GB/s", "cores": cores,
+                                     "kind": "oracle", "sample": f"one 4096 x 4096 bf16 projection, {reps} calls"}
     out["llama7b_sweep"] = res
     assert q.qlora_get_device_status() == q.QLORA_OK
-    del Ws, Ts, wh, wq_ws
+    del layers, wh, ws_q
     torch.cuda.empty_cache()
 
     # --- decode GEMV: one Llama-7B block at M in {1, 4, 16}, forward only
@@ -499,12 +548,13 @@ def run_components(args, peaks, peak_kind, flush):
             inp = si.layer_inputs(wl, li, device="cuda")
             T = q.qlora_nf4_quantize(inp["W"])
             Y = torch.empty(M, L.d_out, dtype=torch.bfloat16, device="cuda")
-            items.append({"X": inp["X"], "W": T, "A": inp.get("A"), "B": inp.get("B"), "s": L.s, "Y": Y})
+            items.append({"X": inp["X"], "W": T, "A": inp.get("A"), "B": inp.get("B"), "s": L.s, "Y": Y,
+                          "Wsrc": inp["W"] if li == 0 else None})
             nbytes += T.nbytes + inp["X"].numel() * 2 + Y.numel() * 2
             if L.r:
                 nbytes += inp["A"].numel() * 2 + inp["B"].numel() * 2
             del inp
-        # the block's seven projections in one grouped call (X·A sums, adapter term, one persistent GEMV)
+        # the block's seven projections in one grouped call (one persistent GEMV, X A, finish)
         wsz = q.lib().qlora_linear_fwd_grouped_workspace(
             M, len(items), (q._LinearDesc * len(items))(*[
                 q._LinearDesc(None, ctypes.pointer(it["W"].ctype()), None, None,
@@ -516,8 +566,26 @@ def run_components(args, peaks, peak_kind, flush):
 
         ms = _time_graph(layer, 20, flush, stream)
         gbs = nbytes / (ms / 1e3) / 1e9
+        kern = _kernel_ms(("k_gemv", "k_gemv_xa", "k_gemv_finish"), layer, 10, flush)
         gem[f"M{M}"] = {"ms_per_layer": round(ms, 5), "bytes": nbytes, "GB/s": round(gbs, 1),
-                        "frac": round(gbs / hbm, 4)}
+                        "frac": round(gbs / hbm, 4), "kernels": kern}
+        if M == 1:
+            # the oracle on the host: the q projection at M = 1 (dequantise in C, fp64 product)
+            it = items[0]
+            L = wl.layers[0]
+            bits = it["Wsrc"].view(torch.int16).cpu().numpy().view(np.uint16).ravel()
+            ref = oracle.quantize_bf16(bits, L.d_out, L.d_in)
+            f64 = lambda t: t.to(torch.float64).cpu().numpy()
+            Xn, An, Bn = f64(it["X"]), f64(it["A"]), f64(it["B"])
+
+            def cpu_q():
+                Wh = oracle.bf16_bits_to_f32(oracle.dequant(ref)).reshape(L.d_out, L.d_in).astype(np.float64)
+                oracle.linear_fwd(Xn, Wh, An, Bn, L.s)
+            t_c, reps = _host_time(cpu_q)
+            qbytes = it["W"].nbytes + it["X"].numel() * 2 + it["Y"].numel() * 2 + (An.size + Bn.size) * 2
+            gem[f"M{M}"]["cpu_baseline"] = {"value": round(qbytes / t_c / 1e9, 3), "unit": "GB/s", "cores": cores,
+                                            "kind": "oracle",
+                                            "sample": f"the q projection (4096 x 4096, r = 16) at M = 1, {reps} calls"}
         del items
         torch.cuda.empty_cache()
     out["decode7b_gemv"] = {"workload": "one Llama-7B block (q,k,v,o 4096x4096; gate,up 11008x4096; "
@@ -526,7 +594,44 @@ def run_components(args, peaks, peak_kind, flush):
     assert q.qlora_get_device_status() == q.QLORA_OK
     out["l70b_layer"] = run_l70b(args, peaks, peak_kind, flush, stream)
     out["merge_4096"] = run_merge(hbm, flush, stream)
+    out["fmt4"] = run_fmt4(hbm, flush, stream)
     return out
+
+
+def run_fmt4(hbm, flush, stream):
+    """The 4-bit reference formats (Int4, FP4 E2M1, FP4 E3M0) on 2^26 fp32 weights: quantise
+    (4 + 1/2 + 4/64 B per weight) and dequantise (1/2 + 4/64 + 2 B per weight) against HBM."""
+    import numpy as np
+    import torch
+    import bit_nf4_quantized_double_b200 as q
+    from oracle import formats
+    import synth_inputs as si
+    n = 1 << 26
+    W = si.normal((n,), 0.02, seed=77, device="cuda")
+    res = {}
+    wn = si.normal((1 << 20,), 0.02, seed=77).numpy()
+    for fmt in ("int4", "fp4_e2m1", "fp4_e3m0"):
+        codes, absmax = q.qlora_fmt4_quantize(W, fmt)
+        outb = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        mq = _time_graph(lambda: q.qlora_fmt4_quantize(W, fmt), 5, flush, stream)
+        md = _time_graph(lambda: q.qlora_fmt4_dequant(codes, absmax, n, fmt, out=outb), 5, flush, stream)
+        bq, bd = n * (4 + 0.5 + 4 / 64), n * (0.5 + 4 / 64 + 2)
+        t_c, reps = _host_time(lambda: formats.dequant(*formats.quantize(wn, fmt), fmt), target_s=1.0)
+        res[fmt] = {"quantize_ms": round(mq, 4), "quantize_GB/s": round(bq / (mq / 1e3) / 1e9, 1),
+                    "quantize_frac": round(bq / (mq / 1e3) / 1e9 / hbm, 4),
+                    "dequant_ms": round(md, 4), "dequant_GB/s": round(bd / (md / 1e3) / 1e9, 1),
+                    "dequant_frac": round(bd / (md / 1e3) / 1e9 / hbm, 4),
+                    "cpu_baseline": {"value": round((1 << 20) * (4 + 0.5 + 4 / 64 + 0.5 + 4 / 64 + 2) / t_c / 1e9, 3),
+                                     "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                     "sample": f"2^20 weights quantised and dequantised (numpy), {reps} calls"}}
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    del W
+    torch.cuda.empty_cache()
+    return {"workload": "2^26 fp32 weights ~ N(0, 0.02^2), 64-weight absmax blocks, CUDA graph replay, L2 flushed",
+            **res}
+
+
+_FLUSH = [None]
 
 
 def run_merge(hbm, flush, stream):
@@ -535,6 +640,7 @@ def run_merge(hbm, flush, stream):
     import torch
     import bit_nf4_quantized_double_b200 as q
     import synth_inputs as si
+    _FLUSH[0] = flush
     wl = si.workload("l4096")
     L = wl.layers[0]
     inp = si.layer_inputs(wl, 0, device="cuda")
@@ -552,9 +658,27 @@ def run_merge(hbm, flush, stream):
     Ym, _ = q.qlora_linear_fwd(X, out, None, None, 0.0)
     rel = ((Ym.double() - Yu.double()).norm() / Yu.double().norm()).item()
     assert q.qlora_get_device_status() == q.QLORA_OK
+    kern = _kernel_ms(("k_merge_bf16", "k_quantize_codes", "k_offset", "k_double_quant"),
+                      lambda: q.qlora_nf4_merge_adapter(t, inp["A"], inp["B"], L.s, out=out, W_bf16=wb, ws=ws), 5,
+                      _FLUSH[0])
+    # the oracle on the host: merge (C) and re-quantisation of the same weight
+    import numpy as np
+    import oracle
+    ref = oracle.quantize(inp["W"].cpu().numpy())
+    wh_bits = oracle.dequant(ref).reshape(L.d_out, L.d_in)
+    An = inp["A"].float().cpu().numpy()
+    Bn = inp["B"].float().cpu().numpy()
+
+    def cpu_merge():
+        m = oracle.merge_bf16(wh_bits, An, Bn, L.s)
+        oracle.quantize_bf16(m.ravel(), L.d_out, L.d_in)
+    t_c, reps = _host_time(cpu_merge, target_s=3.0)
     return {"workload": "merge s*(AB)^T into the 4096x4096 NF4 weight in bf16 and re-quantise (r=64), "
                         "CUDA graph replay, L2 flushed",
             "ms": round(ms, 4), "GB/s": round(alg / (ms / 1e3) / 1e9, 1), "frac": round(alg / (ms / 1e3) / 1e9 / hbm, 4),
+            "kernels": kern,
+            "cpu_baseline": {"value": round(alg / t_c / 1e9, 3), "unit": "GB/s", "cores": _cores(), "kind": "oracle",
+                             "sample": f"the same merge and re-quantisation, full size, {reps} calls"},
             "output_rel_change_fro": round(rel, 6),
             "output_change_sample": "256 tokens: X W'^T (merged, re-quantised) against X W^T + s (XA) B"}
 
@@ -600,12 +724,36 @@ def run_l70b(args, peaks, peak_kind, flush, stream):
     assert q.qlora_get_device_status() == q.QLORA_OK
     tf = flops / (ms / 1e3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    # the oracle on the host, a bounded sample: the k projection (1024 x 8192, r = 64),
+    # dequantised in C; Y and dX on 128 token rows and dA, dB over all 4096 tokens in fp64
+    import numpy as np
+    import oracle
+    li = [l.name for l in wl.layers].index("k")
+    L = wl.layers[li]
+    it = items[li]
+    Wsrc = si.layer_inputs(wl, li, device="cpu", M=0)["W"].numpy()
+    ref = oracle.quantize(Wsrc)
+    f64 = lambda t: t.to(torch.float64).cpu().numpy()
+    Xn, dYn, An, Bn = f64(it["X"]), f64(it["dY"]), f64(it["A"]), f64(it["B"])
+    rows = np.random.default_rng(5).choice(M, 128, replace=False)
+
+    def cpu_sample():
+        Wh = oracle.bf16_bits_to_f32(oracle.dequant(ref)).reshape(L.d_out, L.d_in).astype(np.float64)
+        oracle.linear_fwd(Xn[rows], Wh, An, Bn, L.s)
+        oracle.linear_bwd(Xn[rows], dYn[rows], Wh, An, Bn, L.s)
+        oracle.adapter_grads(Xn, dYn, An, Bn, L.s)
+    t_c, creps = _host_time(cpu_sample, target_s=3.0, max_reps=5)
+    K, N, r = L.d_in, L.d_out, L.r
+    sample_flops = 4.0 * 128 * K * N + 6.0 * 128 * r * (K + N) + 6.0 * M * r * (K + N)
+    cpu = {"value": round(sample_flops / t_c / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+           "sample": f"k projection: dequantise, Y and dX on 128 of the 4096 tokens, dA and dB on all, fp64; "
+                     f"{creps} calls; the rate extrapolates to the layer"}
     del items, ws_f, ws_b
     torch.cuda.empty_cache()
     return {"workload": "70B-like layer: q,o 8192x8192; k,v 1024x8192; gate,up 28672x8192; down 8192x28672; "
                         "r=64, alpha=128 on all seven; M=4096; fwd+bwd of each, CUDA graph replay, L2 flushed",
             "flops_per_step": flops, "ms_per_step": round(ms, 4), "TFLOP/s": round(tf, 1),
-            "frac_of_sustained_bf16": round(tf / peak, 4), "reps": reps}
+            "frac_of_sustained_bf16": round(tf / peak, 4), "reps": reps, "cpu_baseline": cpu}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -699,7 +847,7 @@ def run_decode_profile(M, reps=3):
         del inp
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     for _ in range(reps):
-        flush.zero_()
+        l2_flush(flush)
         q.qlora_linear_fwd_grouped(items)
     torch.cuda.synchronize()
     assert q.qlora_get_device_status() == q.QLORA_OK

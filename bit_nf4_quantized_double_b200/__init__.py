@@ -73,6 +73,13 @@ _SIGS = {
                                                             ctypes.POINTER(_LinearDesc)]),
     "qlora_linear_fwd_grouped": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(_LinearDesc),
                                                 ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_nf4_quantize_grouped_workspace": (ctypes.c_size_t, [ctypes.c_int, ctypes.POINTER(_Tensor)]),
+    "qlora_nf4_quantize_grouped": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int,
+                                                  ctypes.POINTER(_Tensor), ctypes.c_void_p, ctypes.c_size_t,
+                                                  ctypes.c_void_p]),
+    "qlora_nf4_dequant_grouped": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(_Tensor),
+                                                 ctypes.POINTER(ctypes.c_void_p), ctypes.c_void_p]),
+    "qlora_nf4_set_code_search": (None, [ctypes.c_int]),
     "qlora_get_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_nf4_codebook": (None, [ctypes.c_void_p]),
@@ -218,6 +225,37 @@ def qlora_nf4_dequant(q: NF4Tensor, out: torch.Tensor | None = None, stream=None
     t = q.ctype()
     _check(lib().qlora_nf4_dequant(ctypes.byref(t), _ptr(out), _stream(stream)), "qlora_nf4_dequant")
     return out
+
+
+def qlora_nf4_quantize_grouped(Ws, outs=None, ws: torch.Tensor | None = None, stream=None):
+    """Quantise a list of [rows, cols] CUDA tensors of one dtype (fp32 or bf16) with one
+    sequence of launches. Returns the list of NF4Tensor."""
+    Ws = [W.view(1, -1) if W.dim() == 1 else W.contiguous() for W in Ws]
+    dt = {torch.float32: QLORA_F32, torch.bfloat16: QLORA_BF16}[Ws[0].dtype]
+    if any(W.dtype != Ws[0].dtype for W in Ws):
+        raise ValueError("qlora_nf4_quantize_grouped: all tensors must share one dtype")
+    if outs is None:
+        outs = [nf4_empty(W.shape[0], W.shape[1], W.device) for W in Ws]
+    n = len(Ws)
+    ts = (_Tensor * n)(*[o.ctype() for o in outs])
+    ptrs = (ctypes.c_void_p * n)(*[W.data_ptr() for W in Ws])
+    L = lib()
+    wsb, wsn = _workspace(int(L.qlora_nf4_quantize_grouped_workspace(n, ts)), Ws[0].device, ws)
+    _check(L.qlora_nf4_quantize_grouped(n, ptrs, dt, ts, _ptr(wsb), wsn, _stream(stream)),
+           "qlora_nf4_quantize_grouped")
+    _hold(stream, wsb, *Ws)
+    return outs
+
+
+def qlora_nf4_dequant_grouped(qs, outs=None, stream=None):
+    """Dequantise a list of NF4Tensor to bf16 [rows, cols] with one launch per 64 tensors."""
+    if outs is None:
+        outs = [torch.empty(t.rows, t.cols, dtype=torch.bfloat16, device=t.codes.device) for t in qs]
+    n = len(qs)
+    ts = (_Tensor * n)(*[t.ctype() for t in qs])
+    ptrs = (ctypes.c_void_p * n)(*[o.data_ptr() for o in outs])
+    _check(lib().qlora_nf4_dequant_grouped(n, ts, ptrs, _stream(stream)), "qlora_nf4_dequant_grouped")
+    return outs
 
 
 FMT4 = {"int4": 0, "fp4_e2m1": 1, "fp4_e3m0": 2}

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "launch.h"
@@ -97,6 +98,56 @@ qlora_status qlora_nf4_quantize(const void *W, qlora_dtype dt, const qlora_nf4_t
     float *c1 = static_cast<float *>(ws);
     double *part = reinterpret_cast<double *>(static_cast<char *>(ws) + align256((size_t)nb * 4));
     return from_cuda(launch_quantize(W, dt, n, *out, c1, part, static_cast<cudaStream_t>(stream)));
+}
+
+constexpr int kMaxGroupedTensors = 4096;
+
+size_t qlora_nf4_quantize_grouped_workspace(int count, const qlora_nf4_tensor *out) {
+    if (count < 1 || count > kMaxGroupedTensors || !out) return 0;
+    size_t b = 0;
+    for (int i = 0; i < count; ++i) {
+        if (out[i].rows < 1 || out[i].cols < 1) return 0;
+        b += qlora_nf4_quantize_workspace(out[i].rows, out[i].cols);
+    }
+    return b;
+}
+
+qlora_status qlora_nf4_quantize_grouped(int count, const void *const *W, qlora_dtype dt, const qlora_nf4_tensor *out,
+                                        void *ws, size_t ws_bytes, qlora_stream_t stream) {
+    if (count < 1 || count > kMaxGroupedTensors || !W || !out || (dt != QLORA_F32 && dt != QLORA_BF16))
+        return QLORA_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i) {
+        if (!W[i] || !aligned16(W[i]) || !tensor_ok(&out[i])) return QLORA_ERR_INVALID_ARG;
+        const int64_t n = out[i].rows * out[i].cols, nb = ceil_div(n, kBlock1), nb2 = ceil_div(nb, kBlock2);
+        if (nb2 > 0x7fffffffLL) return QLORA_ERR_UNSUPPORTED_SHAPE;
+    }
+    const size_t need = qlora_nf4_quantize_grouped_workspace(count, out);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return QLORA_ERR_WORKSPACE;
+    std::vector<QuantArgs> args((size_t)count);
+    char *w = static_cast<char *>(ws);
+    for (int i = 0; i < count; ++i) {
+        const int64_t n = out[i].rows * out[i].cols, nb = ceil_div(n, kBlock1);
+        args[i].W = W[i];
+        args[i].n = n;
+        args[i].out = out[i];
+        args[i].c1 = reinterpret_cast<float *>(w);
+        args[i].part = reinterpret_cast<double *>(w + align256((size_t)nb * 4));
+        w += qlora_nf4_quantize_workspace(out[i].rows, out[i].cols);
+    }
+    return from_cuda(launch_quantize_grouped(args.data(), count, dt, static_cast<cudaStream_t>(stream)));
+}
+
+qlora_status qlora_nf4_dequant_grouped(int count, const qlora_nf4_tensor *q, void *const *W_out,
+                                       qlora_stream_t stream) {
+    if (count < 1 || count > kMaxGroupedTensors || !q || !W_out) return QLORA_ERR_INVALID_ARG;
+    std::vector<NF4View> views((size_t)count);
+    std::vector<__nv_bfloat16 *> outs((size_t)count);
+    for (int i = 0; i < count; ++i) {
+        if (!tensor_ok(&q[i]) || !W_out[i] || !aligned16(W_out[i])) return QLORA_ERR_INVALID_ARG;
+        views[i] = view_of(&q[i]);
+        outs[i] = static_cast<__nv_bfloat16 *>(W_out[i]);
+    }
+    return from_cuda(launch_dequant_grouped(views.data(), outs.data(), count, static_cast<cudaStream_t>(stream)));
 }
 
 qlora_status qlora_nf4_dequant(const qlora_nf4_tensor *q, void *W_out, qlora_stream_t stream) {

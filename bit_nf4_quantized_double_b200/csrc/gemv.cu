@@ -6,26 +6,35 @@
 // section 1), at decode-sized M where the packed 4-bit codes dominate HBM
 // traffic (section 2: about 4.127 bits per weight).
 //
-// Three launches, the last two chained by programmatic dependent launch so that
-// they start while their predecessor still runs:
-//   k_gemv_xa    per (projection, 512-input chunk): XA partial sums [M, r];
-//   k_gemv_lora  per (projection, 256 outputs): XA = sum of the partials in chunk
-//                order, L = (s XA) B in fp32; also clears the main kernel's
-//                row-block counters;
-//   k_gemv       persistent, one CTA per SM over work units of 128 weight rows x
-//                512 inputs, ordered (projection, row block, K chunk) and cut into
-//                equal contiguous ranges, one per CTA.
-// In k_gemv, one producer warp per pipeline stage loads the unit's packed codes
-// with TMA (two 128-byte-swizzled boxes of 128 rows x 128 bytes) and computes the
-// unit's dequantised block constants c^ (double quantisation, section 3) into the
-// stage. Sixteen compute warps (8 row groups of 16 x 2 halves of the K chunk)
-// turn each code byte into a bf16 pair (Q[hi], Q[lo]) with one byte permute
-// (address = byte * 256 + lane * 4) and one load from a per-lane replicated table,
-// accumulate sum_k Q[code] x_k per 64-block with mma.sync m16n8k16 (16 weight rows
-// x 8 tokens) and scale each block's partial dot product by its c^. A row block
-// ends in the CTA that holds its last K chunk: (half 0 + half 1) + L rounded to
-// bf16; a row block cut between two or more CTAs is combined by whichever CTA
-// finishes last, adding the parts in CTA order (reproducible).
+// Three launches, each chained to the previous one by programmatic dependent
+// launch so that it starts while its predecessor still runs:
+//   k_gemv         persistent, one CTA per SM, over work units of 16 RG weight rows
+//                  x 2048 inputs (1 KB of codes per row), ordered (projection, K
+//                  chunk, row block) and cut into contiguous ranges of equal weight
+//                  count, one per CTA; writes each unit's fp32 sums to the workspace.
+//                  RG = 2 row groups for M <= 8, 1 for larger M (whose X fragments
+//                  need twice the registers);
+//   k_gemv_xa      one warp per (adapter, 512 inputs): the X A partial sums, run
+//                  beside the GEMV (no shared memory, so its warps fit next to a
+//                  GEMV CTA);
+//   k_gemv_finish  one thread per output row: Y = the K chunks' sums in chunk order
+//                  + (s XA) B with XA = its chunk partials in chunk order, rounded to
+//                  bf16; the first CTA of a projection also saves XA as bf16.
+// In k_gemv a producer warp loads each unit's codes with TMA (one 3D box of
+// 8 K slices x 16 RG rows x 128 bytes, 128-byte swizzle, or eight 2D boxes when a
+// row is not a whole number of 128-byte slices) and computes the unit's
+// dequantised block constants c^ (double quantisation, section 3) into the stage
+// from int8 constants it fetched three units earlier.
+// 8 RG compute warps, RG row groups of 16 x 8 K slices of 256 inputs, keep
+// their slice of X in registers as mma B fragments for as long as the units
+// stay in one (projection, K chunk), turn each code byte into a bf16 pair
+// (Q[hi], Q[lo]) with one byte permute (address = byte * 256 + lane * 4) and one
+// load from a per-lane replicated table, accumulate sum_k Q[code] x_k per
+// 64-block with mma.sync m16n8k16 (16 weight rows x 8 tokens) and scale each
+// block's partial dot product by its c^. The eight K slices of a row group are
+// added in slice order through shared memory by one of them (the role rotates
+// from unit to unit). Every output is thus a fixed-order sum, whichever CTA
+// computes it.
 #include "launch.h"
 #include "tc.cuh"
 #include "tmap.h"
@@ -39,23 +48,34 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
                                     __nv_bfloat16 *XA_save, void *ws, cudaStream_t st);
 
 constexpr int kGemvMaxM = 16;
-constexpr int kGemvRows = 128;                  // weight rows per unit (8 row groups of 16)
-constexpr int kGemvKChunk = 512;                // inputs per unit (8 blocks of 64)
-constexpr int kGemvCompute = 512;               // compute threads (16 warps)
+constexpr int kGemvSlice = 256;                 // inputs per compute warp (4 blocks of 64)
+constexpr int kGemvMaxSlices = 8;               // slices per K chunk (one per compute warp)
 constexpr int kGemvMaxItems = 8;
-constexpr int kLutBytes = 256 * 256;            // 256 code bytes x 64 words (32 used: one per lane)
-constexpr int kBoxBytes = kGemvRows * 128;      // one TMA box: 128 rows x 128 code bytes
-constexpr int kChatBytes = kGemvRows * 8 * 4;   // c^ of 128 rows x 8 blocks
-constexpr int kStageBytes = 2 * kBoxBytes + kChatBytes;
-constexpr int kXaChunk = 512;                   // inputs per k_gemv_xa CTA
-constexpr int kLoraCols = 256;                  // outputs per k_gemv_lora CTA
+constexpr int kGemvMaxGrid = 160;
+// Shared memory: a 64 KB region whose 256 rows of 256 bytes hold the lookup table in
+// their first 128 bytes (one word per lane) and, in the second 128 bytes ("holes"),
+// the c^ of the stages (one hole per stage row) and then the K-slice reduction
+// buffer (32 RG NT holes); then the stages; then barriers.
+constexpr int kLutRegion = 65536;
 
-__host__ __device__ constexpr int gemv_stages(int nt) { return nt == 1 ? 4 : 3; }
-__host__ __device__ constexpr int gemv_threads(int nt) { return kGemvCompute + 32 * gemv_stages(nt); }
-__host__ __device__ constexpr int gemv_xs_bytes(int nt) { return nt * 8 * 4 * 32 * 8; }   // one X buffer
+// Row groups of 16 per unit, by token tiles of 8: the M <= 8 variant has 16 compute
+// warps (17 with the producer: at most 96 registers a thread), the 9..16 variant 8
+// (9 warps: room for its 64 registers of X fragments).
+__host__ __device__ constexpr int gemv_rg(int nt) { return nt == 1 ? 2 : 1; }
+__host__ __device__ constexpr int gemv_rows(int nt) { return 16 * gemv_rg(nt); }
+__host__ __device__ constexpr int gemv_threads(int nt) { return 256 * gemv_rg(nt) + 32; }
+__host__ __device__ constexpr int gemv_box_bytes(int nt) { return gemv_rows(nt) * 128; }
+__host__ __device__ constexpr int gemv_stage_bytes(int nt) { return 8 * gemv_box_bytes(nt); }
+__host__ __device__ constexpr int gemv_stages(int nt) { return nt == 1 ? 5 : 10; }
+__host__ __device__ constexpr int gemv_red_hole0(int nt) { return gemv_rows(nt) * gemv_stages(nt); }
 __host__ __device__ constexpr int gemv_smem(int nt) {
-    return kLutBytes + 1024 + gemv_stages(nt) * kStageBytes + 2 * gemv_xs_bytes(nt) + 128;
+    return 1024 + kLutRegion + gemv_stages(nt) * gemv_stage_bytes(nt) + 512;
 }
+static_assert(gemv_smem(1) <= 232448 && gemv_smem(2) <= 232448, "shared memory");
+static_assert(gemv_red_hole0(1) + 32 * gemv_rg(1) * 1 <= 256 && gemv_red_hole0(2) + 32 * gemv_rg(2) * 2 <= 256,
+              "holes");
+
+__device__ __forceinline__ uint32_t hole(int h) { return (uint32_t)h * 256u + 128u; }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -63,12 +83,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
         "{%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint2 ldg_nc_v2(const void *p) {
-    uint2 r;
-    asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
-    return r;
 }
 
 __device__ __forceinline__ uint32_t pack2_bf16(const __nv_bfloat16 *p0, const __nv_bfloat16 *p1) {
@@ -79,64 +93,73 @@ __device__ __forceinline__ uint32_t pack2_bf16(const __nv_bfloat16 *p0, const __
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 
-// ---------------------------------------------------------------- adapter kernels
-struct LoraItem {
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float4 lds128f(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts128f(uint32_t a, float4 v) {
+    asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
+}
+__device__ __forceinline__ void sts128u(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+// ---------------------------------------------------------------- adapter product
+constexpr int kXaChunk = 512;                   // inputs per k_gemv_xa warp
+struct XaItem {
     const __nv_bfloat16 *X;      // [M, K]
     const __nv_bfloat16 *A;      // [K, r]
-    const __nv_bfloat16 *B;      // [r, N]
-    __nv_bfloat16 *XA_save;      // [M, r] or null
-    float *part;                 // [nchunks][M][r]
-    float *L;                    // [M][N]
-    float s;
-    int K, N, r, nchunks;
-    int cta_xa, cta_lora;        // first CTA of this item in either kernel
+    float *xpart;                // [nchunks][M][r] partial sums of X A
+    int K, r, cta0;
 };
-struct LoraGroup {
-    LoraItem it[kGemvMaxItems];
+struct XaGroup {
+    XaItem it[kGemvMaxItems];
     int n, M;
-    int *counters;
-    int ncounters;
 };
 
-// XA partial of one 512-input chunk: part[c][m][j] = sum over the chunk of X[m][k] A[k][j].
-// mma m16n8k16 with X rows (tokens, zero past M) as A and A_lora columns as B; warp w
-// takes the chunk's 16-wide k steps w, w + 8, ...; the eight warps' sums are added in
-// warp order through shared memory.
-__global__ void __launch_bounds__(256) k_gemv_xa(const __grid_constant__ LoraGroup grp) {
-    __shared__ float4 red[8 * 4 * 32];
+// X A over one 512-input chunk: mma m16n8k16 with X rows (tokens, zero past M) as A
+// and the adapter's columns as B, the chunk's 32 16-input steps in order.
+__global__ void __launch_bounds__(32) k_gemv_xa(const __grid_constant__ XaGroup grp) {
     griddep_launch_dependents();
     int ii = 0;
-    while (ii + 1 < grp.n && (int)blockIdx.x >= grp.it[ii + 1].cta_xa) ++ii;
-    const LoraItem &it = grp.it[ii];
+    while (ii + 1 < grp.n && (int)blockIdx.x >= grp.it[ii + 1].cta0) ++ii;
+    const XaItem &it = grp.it[ii];
     const int M = grp.M, K = it.K, r = it.r;
-    const int c = blockIdx.x - it.cta_xa;
-    const int kbase = c * kXaChunk;
-    const int ksteps = (min(K, kbase + kXaChunk) - kbase) / 16;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int ntiles = r / 8;
-    float *dst = it.part + (int64_t)c * M * r;
-    for (int nt0 = 0; nt0 < ntiles; nt0 += 4) {
-        const int nts = min(4, ntiles - nt0);
+    const int c = blockIdx.x - it.cta0;
+    const int k_begin = c * kXaChunk, k_end = min(K, k_begin + kXaChunk);
+    const int lane = threadIdx.x, g = lane >> 2, t = lane & 3;
+    float *dst = it.xpart + (int64_t)c * M * r;
+    for (int nt0 = 0; nt0 < r / 8; nt0 += 4) {
+        const int nts = min(4, r / 8 - nt0);
         float acc[4][4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.0f;
-#pragma unroll
-        for (int st = 0; st < kXaChunk / 16 / 8; ++st) {
-            const int kstep = warp + 8 * st;
-            if (kstep >= ksteps) break;
-            const int k0 = kbase + 16 * kstep;
+#pragma unroll 8
+        for (int k0 = k_begin; k0 < k_end; k0 += 16) {
             uint32_t a[4] = {0u, 0u, 0u, 0u};
             if (g < M) {
-                a[0] = *reinterpret_cast<const uint32_t *>(it.X + (int64_t)g * K + k0 + 2 * t);
-                a[2] = *reinterpret_cast<const uint32_t *>(it.X + (int64_t)g * K + k0 + 8 + 2 * t);
+                a[0] = __ldg(reinterpret_cast<const unsigned int *>(it.X + (int64_t)g * K + k0 + 2 * t));
+                a[2] = __ldg(reinterpret_cast<const unsigned int *>(it.X + (int64_t)g * K + k0 + 8 + 2 * t));
             }
             if (g + 8 < M) {
-                a[1] = *reinterpret_cast<const uint32_t *>(it.X + (int64_t)(g + 8) * K + k0 + 2 * t);
-                a[3] = *reinterpret_cast<const uint32_t *>(it.X + (int64_t)(g + 8) * K + k0 + 8 + 2 * t);
+                a[1] = __ldg(reinterpret_cast<const unsigned int *>(it.X + (int64_t)(g + 8) * K + k0 + 2 * t));
+                a[3] = __ldg(reinterpret_cast<const unsigned int *>(it.X + (int64_t)(g + 8) * K + k0 + 8 + 2 * t));
             }
             uint32_t bb[4][2];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
+                bb[q][0] = bb[q][1] = 0u;
                 if (q < nts) {
                     const __nv_bfloat16 *ak = it.A + (int64_t)(k0 + 2 * t) * r + (nt0 + q) * 8 + g;
                     bb[q][0] = pack2_bf16(ak, ak + r);
@@ -147,219 +170,254 @@ __global__ void __launch_bounds__(256) k_gemv_xa(const __grid_constant__ LoraGro
             for (int q = 0; q < 4; ++q)
                 if (q < nts) mma_bf16_16816(acc[q], a, bb[q][0], bb[q][1]);
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            if (q < nts) red[(warp * 4 + q) * 32 + lane] = make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
-        __syncthreads();
         // c[0], c[1]: token g, tile columns 2t, 2t+1; c[2], c[3]: token g + 8
-        for (int i = threadIdx.x; i < nts * 32; i += blockDim.x) {
-            const int q = i >> 5, ln = i & 31;
-            float4 v = red[q * 32 + ln];
-            for (int ww = 1; ww < 8; ++ww) {
-                const float4 x = red[(ww * 4 + q) * 32 + ln];
-                v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (q >= nts) continue;
+            const int j0 = (nt0 + q) * 8 + 2 * t;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int tok = g + (e >= 2 ? 8 : 0);
+                if (tok < M) dst[tok * r + j0 + (e & 1)] = acc[q][e];
             }
-            const int gg = ln >> 2, tt = ln & 3, j0 = (nt0 + q) * 8 + 2 * tt;
-            if (gg < M) { dst[gg * r + j0] = v.x; dst[gg * r + j0 + 1] = v.y; }
-            if (gg + 8 < M) { dst[(gg + 8) * r + j0] = v.z; dst[(gg + 8) * r + j0 + 1] = v.w; }
         }
-        __syncthreads();
     }
-}
-
-// XA = sum of the chunk partials (chunk order), saved as bf16; L[m][n] = sum_j (s XA[m][j]) B[j][n]
-// (fused multiply-adds in increasing j). CTA 0 also clears the main kernel's counters.
-__global__ void __launch_bounds__(256) k_gemv_lora(const __grid_constant__ LoraGroup grp) {
-    __shared__ float sx[kGemvMaxM * 256];          // s XA, r <= 256
-    griddep_launch_dependents();
-    if (blockIdx.x == 0)
-        for (int i = threadIdx.x; i < grp.ncounters; i += blockDim.x) grp.counters[i] = 0;
-    if (grp.n == 0) return;
-    griddep_wait();                                  // the XA partials are complete
-    int ii = 0;
-    while (ii + 1 < grp.n && (int)blockIdx.x >= grp.it[ii + 1].cta_lora) ++ii;
-    const LoraItem &it = grp.it[ii];
-    const int M = grp.M, r = it.r, N = it.N;
-    const int slice = blockIdx.x - it.cta_lora;
-    for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
-        float v = 0.0f;
-        for (int c0 = 0; c0 < it.nchunks; c0 += 8) {         // eight partial loads in flight
-            float pv[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                pv[c] = c0 + c < it.nchunks ? __ldcg(it.part + (int64_t)(c0 + c) * M * r + i) : 0.0f;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                if (c0 + c < it.nchunks) v += pv[c];
-        }
-        sx[i] = it.s * v;
-        if (slice == 0 && it.XA_save) it.XA_save[i] = __float2bfloat16_rn(v);
-    }
-    __syncthreads();
-    const int n = slice * kLoraCols + threadIdx.x;
-    if (n >= N) return;
-    float acc[kGemvMaxM];
-#pragma unroll
-    for (int m = 0; m < kGemvMaxM; ++m) acc[m] = 0.0f;
-    for (int j0 = 0; j0 < r; j0 += 8) {             // r % 8 == 0: eight B loads in flight
-        float b[8];
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) b[jj] = __bfloat162float(it.B[(int64_t)(j0 + jj) * N + n]);
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj)
-#pragma unroll
-            for (int m = 0; m < kGemvMaxM; ++m)
-                if (m < M) acc[m] = fmaf(sx[m * r + j0 + jj], b[jj], acc[m]);
-    }
-#pragma unroll
-    for (int m = 0; m < kGemvMaxM; ++m)
-        if (m < M) it.L[(int64_t)m * N + n] = acc[m];
+    griddep_wait();                                  // this grid ends after the GEMV
 }
 
 // ---------------------------------------------------------------- main kernel
+// The K range of a projection is cut into nch chunks of (nearly) equal numbers of
+// 256-input slices, at most 8: with nsl = q nch + rem, chunk c starts at slice
+// c q + min(c, rem) (the first rem chunks have q + 1 slices).
+__host__ __device__ __forceinline__ int chunk_slice0(int ch, int q, int rem) { return ch * q + min(ch, rem); }
+
 struct GemvItem {
-    CUtensorMap codes;           // codes as bytes [N][K/2], box 128 B x 128 rows, 128-byte swizzle
+    CUtensorMap codes;           // 3D: box of zbig slices; 2D: box 128 B x 16 RG rows; 128-byte swizzle
+    CUtensorMap codes_small;     // 3D only: box of zbig - 1 slices (chunks one slice shorter)
     const int8_t *scale8;
     const float *scale2;
     const float *offset;
     const __nv_bfloat16 *X;      // [M, K]
-    __nv_bfloat16 *Y;            // [M, N]
-    const float *L;              // [M, N] adapter term, or null
-    int N, K, kbs, nks, nrb;     // rows, inputs, 64-blocks per row, K chunks, row blocks
+    float *partial;              // [nch][N][M] K-chunk sums
+    int N, K, kbs, nch, nrb;     // rows, inputs, 64-blocks per row, K chunks, row blocks
+    int nsl, zbig;               // 256-input slices; slices of the longest chunk
+    int sq, srem;                // nsl = sq nch + srem
     int unit0;                   // first unit of this item
-    int rb0;                     // first counter of this item
+    int map3d;                   // codes maps are 3D (K % 256 == 0): one box per unit
 };
 struct GemvGroup {
     GemvItem it[kGemvMaxItems];
     int n, M;
-    int units, per_cta;          // total units; contiguous units per CTA
-    int *counters;               // one per row block, zero on entry (k_gemv_lora)
-    float *partial;              // [grid][2 slots][128 rows][M]
+    int ustart[kGemvMaxGrid + 1];  // CTA c takes units ustart[c] .. ustart[c+1] - 1
+};
+struct FinishItem {
+    const float *partial;        // [nch][N][M]
+    const float *xpart;          // [nxa][M][r] X A chunk partials, or null
+    const __nv_bfloat16 *B;      // [r, N], or null
+    __nv_bfloat16 *Y;            // [M, N]
+    __nv_bfloat16 *XA_save;      // [M, r], or null
+    float s;
+    int N, nch, r, nxa, cta0;
+};
+struct FinishGroup {
+    FinishItem it[kGemvMaxItems];
+    int n, M;
 };
 
 struct UnitPos {
-    int item, rb, ks;
+    int item, ch, rb;
 };
 __device__ __forceinline__ UnitPos unit_pos(const GemvGroup &g, int u) {
     int i = 0;
     while (i + 1 < g.n && u >= g.it[i + 1].unit0) ++i;
-    const int lu = u - g.it[i].unit0, nks = g.it[i].nks;
-    const int rb = lu / nks;
-    return {i, rb, lu - rb * nks};
+    const int lu = u - g.it[i].unit0, nrb = g.it[i].nrb;
+    const int ch = lu / nrb;
+    return {i, ch, lu - ch * nrb};
 }
 __device__ __forceinline__ UnitPos unit_next(const GemvGroup &g, UnitPos p) {
-    if (++p.ks == g.it[p.item].nks) {
-        p.ks = 0;
-        if (++p.rb == g.it[p.item].nrb) {
-            p.rb = 0;
+    if (++p.rb == g.it[p.item].nrb) {
+        p.rb = 0;
+        if (++p.ch == g.it[p.item].nch) {
+            p.ch = 0;
             ++p.item;
         }
     }
     return p;
 }
 
-// Stage producer: TMA of the unit's codes and the unit's c^ (128 rows x 8 blocks;
-// lane l takes rows l, l + 32, l + 64, l + 96). Every load is issued before any
-// arithmetic. c^ = fl(fl(q8 * fl(s2 / 127)) + mu), zero for rows past N and blocks past K.
-__device__ __forceinline__ void gemv_produce(const GemvGroup &grp, const UnitPos p, uint32_t stage, float *chat,
-                                             uint32_t full_bar, int lane) {
+// The int8 constants of one row of a unit (32 blocks), prefetched a unit ahead.
+struct Q8Row {
+    uint32_t w[8];               // blocks 4k .. 4k+3, little-endian
+    float s2a, s2b, mu;
+    int split, nblk;             // blocks < split in the first second-level group; valid blocks
+};
+template <int ROWS>
+__device__ __forceinline__ void q8_fetch(const GemvGroup &grp, UnitPos p, int lane, Q8Row &q) {
     const GemvItem &it = grp.it[p.item];
-    if (lane == 0) {
-        mbar_arrive_expect_tx(full_bar, 2 * kBoxBytes);
-        tma_load_2d(stage, &it.codes, full_bar, p.ks * 256, p.rb * kGemvRows);
-        tma_load_2d(stage + kBoxBytes, &it.codes, full_bar, p.ks * 256 + 128, p.rb * kGemvRows);
-    }
-    const int nblk = min(8, it.K / 64 - p.ks * 8);
-    const float mu = __ldg(it.offset);
-    uint32_t qw[4][2];           // the row's eight int8 constants, little-endian
-    float s2a[4], s2b[4];
-    int split[4];                // blocks b < split[i] are in the first second-level group
+    const int row = p.rb * ROWS + lane;
+    const int sl0 = chunk_slice0(p.ch, it.sq, it.srem), sl1 = chunk_slice0(p.ch + 1, it.sq, it.srem);
+    const int nblk = min(4 * (sl1 - sl0), it.kbs - 4 * sl0);
+    const bool valid = lane < ROWS && row < it.N;
+    const int64_t b0 = (int64_t)row * it.kbs + 4 * sl0;
+    const int8_t *src = it.scale8 + b0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int row = p.rb * kGemvRows + lane + 32 * i;
-        const bool valid = row < it.N;
-        const int64_t b0 = (int64_t)row * it.kbs + p.ks * 8;
-        const int8_t *q8 = it.scale8 + b0;
-        qw[i][0] = qw[i][1] = 0u;
-        if (valid) {
-            if (nblk == 8 && (reinterpret_cast<uintptr_t>(q8) & 3u) == 0) {
-                qw[i][0] = __ldg(reinterpret_cast<const unsigned int *>(q8));
-                qw[i][1] = __ldg(reinterpret_cast<const unsigned int *>(q8) + 1);
-            } else {
+    for (int k = 0; k < 8; ++k) q.w[k] = 0u;
+    if (valid) {
+        const uintptr_t a = reinterpret_cast<uintptr_t>(src);
+        if (nblk == 32 && (a & 15u) == 0) {
+            const uint4 v0 = __ldg(reinterpret_cast<const uint4 *>(src));
+            const uint4 v1 = __ldg(reinterpret_cast<const uint4 *>(src) + 1);
+            q.w[0] = v0.x; q.w[1] = v0.y; q.w[2] = v0.z; q.w[3] = v0.w;
+            q.w[4] = v1.x; q.w[5] = v1.y; q.w[6] = v1.z; q.w[7] = v1.w;
+        } else {
+            const bool w4 = (a & 3u) == 0;
 #pragma unroll
-                for (int b = 0; b < 8; ++b)
-                    if (b < nblk) qw[i][b >> 2] |= (uint32_t)(uint8_t)__ldg(q8 + b) << (8 * (b & 3));
+            for (int k = 0; k < 8; ++k) {
+                if (w4 && 4 * k + 4 <= nblk) {
+                    q.w[k] = __ldg(reinterpret_cast<const unsigned int *>(src) + k);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (4 * k + e < nblk) q.w[k] |= (uint32_t)(uint8_t)__ldg(src + 4 * k + e) << (8 * e);
+                }
             }
         }
-        const int64_t g0 = b0 >> 8;
-        split[i] = 256 - (int)(b0 & 255);
-        s2a[i] = valid ? __ldg(it.scale2 + g0) : 0.0f;
-        s2b[i] = (valid && split[i] < nblk) ? __ldg(it.scale2 + g0 + 1) : s2a[i];
     }
+    const int64_t g0 = b0 >> 8;
+    q.split = 256 - (int)(b0 & 255);
+    q.nblk = valid ? nblk : 0;
+    q.s2a = valid ? __ldg(it.scale2 + g0) : 0.0f;
+    q.s2b = (valid && q.split < nblk) ? __ldg(it.scale2 + g0 + 1) : q.s2a;
+    q.mu = __ldg(it.offset);
+}
+// c^ = fl(fl(q8 * fl(s2 / 127)) + mu) of the row's 32 blocks (zero past K or N), stored
+// in the row's hole with the 16-byte chunks XOR-swizzled by the row (conflict-free reads).
+template <int ROWS>
+__device__ __forceinline__ void chat_store(uint32_t lut_base, int stage, int lane, const Q8Row &q) {
+    if (lane >= ROWS) return;
+    const float st0 = __fdiv_rn(q.s2a, 127.0f);
+    const float st1 = q.split < q.nblk ? __fdiv_rn(q.s2b, 127.0f) : st0;
+    const uint32_t base = lut_base + hole(stage * ROWS + lane);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float st0 = __fdiv_rn(s2a[i], 127.0f);
-        const float st1 = split[i] < nblk ? __fdiv_rn(s2b[i], 127.0f) : st0;
-        float c[8];
+    for (int k = 0; k < 8; ++k) {
+        float c[4];
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            const float q = (float)(int8_t)(qw[i][b >> 2] >> (8 * (b & 3)));
-            c[b] = (b < nblk) ? __fadd_rn(__fmul_rn(q, b < split[i] ? st0 : st1), mu) : 0.0f;
+        for (int e = 0; e < 4; ++e) {
+            const int b = 4 * k + e;
+            const float qv = (float)(int8_t)(q.w[k] >> (8 * e));
+            c[e] = b < q.nblk ? __fadd_rn(__fmul_rn(qv, b < q.split ? st0 : st1), q.mu) : 0.0f;
         }
-        if (p.rb * kGemvRows + lane + 32 * i >= it.N)
-#pragma unroll
-            for (int b = 0; b < 8; ++b) c[b] = 0.0f;
-        float4 *dst = reinterpret_cast<float4 *>(chat + (lane + 32 * i) * 8);
-        dst[0] = make_float4(c[0], c[1], c[2], c[3]);
-        dst[1] = make_float4(c[4], c[5], c[6], c[7]);
+        sts128f(base + (uint32_t)((k ^ (lane & 7)) << 4), make_float4(c[0], c[1], c[2], c[3]));
     }
 }
 
-// X fragments of one unit for the mma B operand: entry ((nt * 8 + b) * 4 + j) * 32 + lane
-// holds X[nt * 8 + lane / 4][kbase + 64 b + 16 (lane % 4) + 4 j + 0..3], the four inputs whose
-// codes are bytes 2j and 2j + 1 of that lane's 8-byte code word of block b (zero past M or K).
+// X fragments of a warp's K slice for the mma B operand: xf[nt][b][2j], xf[nt][b][2j+1] hold
+// X[nt * 8 + lane / 4][k0 + 64 b + 16 (lane % 4) + 4 j + 0..3], the four inputs whose codes
+// are bytes 2j and 2j + 1 of the lane's 8-byte code word of block b (zero past M or K).
 template <int NT>
-__device__ __forceinline__ void x_fetch(const GemvGroup &grp, UnitPos p, int ctid, uint2 (&v)[2 * NT]) {
+__device__ __forceinline__ void x_load(const GemvGroup &grp, UnitPos p, int ks, int lane, uint32_t (&xf)[NT][4][8]) {
     const GemvItem &it = grp.it[p.item];
-    const int kbase = p.ks * kGemvKChunk;
+    const int g = lane >> 2, t = lane & 3;
+    const int sl0 = chunk_slice0(p.ch, it.sq, it.srem), sl1 = chunk_slice0(p.ch + 1, it.sq, it.srem);
+    const int k0 = (sl0 + ks) * kGemvSlice;
+    const bool in_chunk = sl0 + ks < sl1;
 #pragma unroll
-    for (int q = 0; q < 2 * NT; ++q) {
-        const int e = ctid + kGemvCompute * q;
-        const int nt = e >> 10, b = (e >> 7) & 7, j = (e >> 5) & 3, ln = e & 31;
-        const int tok = nt * 8 + (ln >> 2);
-        const int k = kbase + b * 64 + 16 * (ln & 3) + 4 * j;
-        v[q] = (tok < grp.M && k < it.K) ? ldg_nc_v2(it.X + (int64_t)tok * it.K + k) : make_uint2(0u, 0u);
-    }
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int tok = nt * 8 + g, kb = k0 + 64 * b;
+            uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+            if (in_chunk && tok < grp.M && kb < it.K) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(it.X + (int64_t)tok * it.K + kb + 16 * t);
+                v0 = __ldg(src);
+                v1 = __ldg(src + 1);
+            }
+            xf[nt][b][0] = v0.x; xf[nt][b][1] = v0.y; xf[nt][b][2] = v0.z; xf[nt][b][3] = v0.w;
+            xf[nt][b][4] = v1.x; xf[nt][b][5] = v1.y; xf[nt][b][6] = v1.z; xf[nt][b][7] = v1.w;
+        }
 }
-template <int NT>
-__device__ __forceinline__ void x_store(uint2 *xs, int ctid, const uint2 (&v)[2 * NT]) {
+
+// Y[tok][R] = sum over K chunks c in order of partial[c][R][tok] + sum_j (s XA)[tok][j] B[j][R]
+// (fused multiply-adds in increasing j), one thread per output row R. XA = its 512-input
+// chunk partials added in chunk order, staged in shared memory (times s); the first CTA
+// of a projection also saves XA as bf16.
+constexpr int kFinishRows = 256;
+__global__ void __launch_bounds__(kFinishRows) k_gemv_finish(const __grid_constant__ FinishGroup grp) {
+    __shared__ float sx[kGemvMaxM * 256];
+    griddep_wait();                                  // the chunk sums and X A partials are complete
+    int ii = 0;
+    while (ii + 1 < grp.n && (int)blockIdx.x >= grp.it[ii + 1].cta0) ++ii;
+    const FinishItem &it = grp.it[ii];
+    const int M = grp.M, N = it.N, r = it.r;
+    for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
+        float v = 0.0f;
+        for (int c = 0; c < it.nxa; ++c) v += __ldcg(it.xpart + (int64_t)c * M * r + i);
+        sx[i] = it.s * v;
+        if (blockIdx.x == it.cta0 && it.XA_save) it.XA_save[i] = __float2bfloat16_rn(v);
+    }
+    __syncthreads();
+    const int R = (blockIdx.x - it.cta0) * kFinishRows + threadIdx.x;
+    if (R >= N) return;
+    float y[kGemvMaxM];
 #pragma unroll
-    for (int q = 0; q < 2 * NT; ++q) xs[ctid + kGemvCompute * q] = v[q];
+    for (int m = 0; m < kGemvMaxM; ++m) y[m] = 0.0f;
+    for (int c = 0; c < it.nch; ++c) {
+        const float *p = it.partial + ((int64_t)c * N + R) * M;
+#pragma unroll
+        for (int m = 0; m < kGemvMaxM; ++m)
+            if (m < M) y[m] += __ldcg(p + m);
+    }
+    if (r > 0) {
+        float a[kGemvMaxM];
+#pragma unroll
+        for (int m = 0; m < kGemvMaxM; ++m) a[m] = 0.0f;
+        for (int j0 = 0; j0 < r; j0 += 8) {          // r % 8 == 0: eight B loads in flight
+            float bv[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) bv[jj] = __bfloat162float(it.B[(int64_t)(j0 + jj) * N + R]);
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+                for (int m = 0; m < kGemvMaxM; ++m)
+                    if (m < M) a[m] = fmaf(sx[m * r + j0 + jj], bv[jj], a[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < kGemvMaxM; ++m) y[m] += a[m];
+    }
+#pragma unroll
+    for (int m = 0; m < kGemvMaxM; ++m)
+        if (m < M) it.Y[(int64_t)m * N + R] = __float2bfloat16_rn(y[m]);
 }
 
 template <int NT>
 __global__ void __launch_bounds__(gemv_threads(NT), 1)
 k_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ Codebook cb) {
-    constexpr int S = gemv_stages(NT);
+    constexpr int S = gemv_stages(NT), RG = gemv_rg(NT), ROWS = gemv_rows(NT);
+    constexpr int BOX = gemv_box_bytes(NT), STAGE = gemv_stage_bytes(NT);
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    uint32_t *lut = reinterpret_cast<uint32_t *>(smem_raw);
-    uint8_t *stages = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + kLutBytes + 1023) & ~uintptr_t(1023));
-    uint2 *xs = reinterpret_cast<uint2 *>(stages + S * kStageBytes);          // [2][NT][8][4][32]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(stages + S * kStageBytes + 2 * gemv_xs_bytes(NT));
-    int *flags = reinterpret_cast<int *>(bars + 2 * S);                       // abort, last
-    const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + S);
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t lut = smem_addr(base);
+    const uint32_t stages = lut + kLutRegion;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + kLutRegion + S * STAGE);
+    int *flags = reinterpret_cast<int *>(bars + 2 * S + 2 * RG);
+    const uint32_t full0 = smem_addr(bars), empty0 = full0 + 8 * S;
+    const uint32_t redf0 = full0 + 16 * S, rede0 = redf0 + 8 * RG;   // per row group
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // lookup table: word (e * 64 + lane) = bf16 pair (Q[e >> 4] low half, Q[e & 15] high half)
-    for (int i = tid; i < 256 * 32; i += blockDim.x) {
-        const int e = i >> 5;
-        lut[e * 64 + (i & 31)] = pack_bf16x2(cb.q[e >> 4], cb.q[e & 15]);
+    for (int i = tid; i < 256 * 8; i += blockDim.x) {
+        const int e = i >> 3, q = i & 7;
+        const uint32_t v = pack_bf16x2(cb.q[e >> 4], cb.q[e & 15]);
+        sts128u(lut + e * 256 + q * 16, make_uint4(v, v, v, v));
     }
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full0 + 8 * s, 33);           // producer's expect-tx arrival + 32 lanes after c^
-            mbar_init(empty0 + 8 * s, 16);          // one arrival per compute warp
+            mbar_init(empty0 + 8 * s, 8 * RG);      // one arrival per compute warp
+        }
+        for (int rg = 0; rg < RG; ++rg) {
+            mbar_init(redf0 + 8 * rg, 8);           // the row group's eight slices written
+            mbar_init(rede0 + 8 * rg, 1);           // the reducer has read them
         }
         flags[0] = 0;
         fence_barrier_init();
@@ -367,236 +425,193 @@ k_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ Codebook c
     __syncthreads();
     volatile int *abort = flags;
 
-    const int u_begin = blockIdx.x * grp.per_cta;
-    const int count = min(grp.units, u_begin + grp.per_cta) - u_begin;
+    griddep_launch_dependents();
+    const int u_begin = grp.ustart[blockIdx.x];
+    const int count = grp.ustart[blockIdx.x + 1] - u_begin;
     if (count <= 0) return;
 
-    if (warp >= 16) {
-        // ---------------- producer of stage s: units s, s + S, ... of this CTA's range
-        const int s = warp - 16;
-        const uint32_t st_addr = smem_addr(stages + s * kStageBytes);
-        float *chat = reinterpret_cast<float *>(stages + s * kStageBytes + 2 * kBoxBytes);
+    if (warp == 8 * RG) {
+        // ---------------- producer: TMA of the codes, c^ of every row into the stage's holes.
+        // The int8 constants of unit i are fetched while units i-3 .. i-1 are produced, into
+        // a ring of four register sets that the unrolled loop names statically (copying a
+        // set whose loads are in flight would wait for them).
         int last = -1;
-        for (int i = s, n = 0; i < count; i += S, ++n) {
-            if (!mbar_wait(empty0 + 8 * s, (n & 1) ^ 1, abort)) break;
-            gemv_produce(grp, unit_pos(grp, u_begin + i), st_addr, chat, full0 + 8 * s, lane);
-            mbar_arrive(full0 + 8 * s);
-            last = n;
-        }
-        // the CTA does not exit with this stage's copy in flight
-        if (last >= 0 && lane == 0) {
-            const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(full0 + 8 * s, last & 1))
-                if (global_timer_ns() - t0 > kWaitLimitNs) {
-                    raise_status(QLORA_ERR_TIMEOUT);
-                    break;
+        UnitPos p = unit_pos(grp, u_begin), pf = p;
+        Q8Row qa, qb, qc, qd;
+        q8_fetch<ROWS>(grp, pf, lane, qa);
+        pf = unit_next(grp, pf);
+        if (count > 1) q8_fetch<ROWS>(grp, pf, lane, qb);
+        pf = unit_next(grp, pf);
+        if (count > 2) q8_fetch<ROWS>(grp, pf, lane, qc);
+        pf = unit_next(grp, pf);
+        // produce unit i from `cur`; fetch unit i + 3 into `nxt` (the set unit i - 1 used)
+        auto step = [&](int i, const Q8Row &cur, Q8Row &nxt) -> bool {
+            if (i >= count) return false;
+            if (i + 3 < count) q8_fetch<ROWS>(grp, pf, lane, nxt);
+            pf = unit_next(grp, pf);
+            const int s = i % S, n = i / S;
+            if (!mbar_wait(empty0 + 8 * s, (n & 1) ^ 1, abort)) return false;
+            const GemvItem &it = grp.it[p.item];
+            if (lane == 0) {
+                const int sl0 = chunk_slice0(p.ch, it.sq, it.srem);
+                const int nsl = it.sq + (p.ch < it.srem ? 1 : 0);
+                if (it.map3d) {
+                    mbar_arrive_expect_tx(full0 + 8 * s, nsl * BOX);
+                    tma_load_3d(stages + s * STAGE, nsl == it.zbig ? &it.codes : &it.codes_small, full0 + 8 * s, 0,
+                                p.rb * ROWS, sl0);
+                } else {
+                    mbar_arrive_expect_tx(full0 + 8 * s, nsl * BOX);
+                    for (int b = 0; b < nsl; ++b)
+                        tma_load_2d(stages + s * STAGE + b * BOX, &it.codes, full0 + 8 * s, (sl0 + b) * 128,
+                                    p.rb * ROWS);
                 }
+            }
+            chat_store<ROWS>(lut, s, lane, cur);
+            mbar_arrive(full0 + 8 * s);
+            last = i;
+            p = unit_next(grp, p);
+            return true;
+        };
+        for (int i = 0; i < count; i += 4) {
+            if (!step(i, qa, qd)) break;
+            if (!step(i + 1, qb, qa)) break;
+            if (!step(i + 2, qc, qb)) break;
+            if (!step(i + 3, qd, qc)) break;
+        }
+        // the CTA does not exit with a copy in flight: wait for the stages issued last
+        if (lane == 0) {
+            const uint64_t t0 = global_timer_ns();
+            for (int j = max(0, last - S + 1); j <= last; ++j)
+                while (!mbar_try_wait(full0 + 8 * (j % S), (j / S) & 1))
+                    if (global_timer_ns() - t0 > kWaitLimitNs) {
+                        raise_status(QLORA_ERR_TIMEOUT);
+                        j = last;
+                        break;
+                    }
         }
         return;
     }
 
     // ---------------- compute warps
-    const int h = warp >> 3, wr = warp & 7, g = lane >> 2, t = lane & 3;
-    const int Rl0 = wr * 16 + g;                                    // rows Rl0 and Rl0 + 8 of the unit
+    const int rg = warp >> 3, ks = warp & 7, g = lane >> 2, t = lane & 3;
     const uint32_t lane4 = lane * 4;
-    const uint32_t xg = (uint32_t)((t >> 1) ^ g) << 4, tb = (t & 1) * 8;
-    const char *lut_b = reinterpret_cast<const char *>(lut);
-    bool ok = true, dep_done = false;
+    // this lane's 8-byte code words of rows rg*16 + g and + 8 in box ks: chunk (2b + t/2) ^ g
+    const uint32_t box_row0 = ks * BOX + (rg * 16 + g) * 128 + (t & 1) * 8;
+    const uint32_t box_row1 = box_row0 + 8 * 128;
+    const uint32_t red_mine = lut + hole(gemv_red_hole0(NT) + (rg * 8 + ks) * NT * 4 + (lane >> 3)) + (lane & 7) * 16;
+    bool ok = true;
 
+    uint32_t xf[NT][4][8];
     UnitPos pos = unit_pos(grp, u_begin);
-    {
-        uint2 v[2 * NT];
-        x_fetch<NT>(grp, pos, tid, v);
-        x_store<NT>(xs, tid, v);
-    }
-    named_bar_sync(1, kGemvCompute);
-
+    int xkey = -1, nblk = 0;
     float acc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
 
-    for (int i = 0; i < count; ++i) {
-        const int s = i % S, n = i / S, cur = i & 1;
-        const bool has_next = i + 1 < count;
-        const UnitPos nxt = unit_next(grp, pos);
-        uint2 xv[2 * NT];
-        if (has_next) x_fetch<NT>(grp, nxt, tid, xv);
-
+    for (int i = 0; i < count && ok; ++i) {
+        const int s = i % S, n = i / S;
         const GemvItem &it = grp.it[pos.item];
-        const int nblk = min(8, it.K / 64 - pos.ks * 8);
-        uint2 cw[4][2];
-        float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
-        ok = ok && mbar_wait(full0 + 8 * s, n & 1, abort);
-        if (ok) {
-            const uint8_t *box = stages + s * kStageBytes + h * kBoxBytes;
+        const int key = pos.item * 4096 + pos.ch;
+        if (key != xkey) {
+            x_load<NT>(grp, pos, ks, lane, xf);
+            xkey = key;
+            const int sl0 = chunk_slice0(pos.ch, it.sq, it.srem);
+            const int kslice = (sl0 + ks) * kGemvSlice;
+            nblk = ks < it.sq + (pos.ch < it.srem ? 1 : 0) ? min(4, (it.K - kslice) / 64) : 0;
+        }
+        if (!mbar_wait(full0 + 8 * s, n & 1, abort)) { ok = false; break; }
+        if (nblk > 0) {
+            const float4 c0 = lds128f(lut + hole(s * ROWS + rg * 16 + g) + ((ks ^ g) << 4));
+            const float4 c1 = lds128f(lut + hole(s * ROWS + rg * 16 + g + 8) + ((ks ^ g) << 4));
+            const float ch0[4] = {c0.x, c0.y, c0.z, c0.w}, ch1[4] = {c1.x, c1.y, c1.z, c1.w};
+            const uint32_t sb = stages + s * STAGE;
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                const uint32_t off = (((uint32_t)bb << 5) ^ xg) + tb;
-                cw[bb][0] = *reinterpret_cast<const uint2 *>(box + Rl0 * 128 + off);
-                cw[bb][1] = *reinterpret_cast<const uint2 *>(box + (Rl0 + 8) * 128 + off);
+            for (int b = 0; b < 4; ++b) {
+                if (b >= nblk) break;
+                const uint32_t off = (uint32_t)(((2 * b + (t >> 1)) ^ g) << 4);
+                const uint2 w0 = lds64(sb + box_row0 + off);
+                const uint2 w1 = lds64(sb + box_row1 + off);
+                float cbk[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) cbk[nt][0] = cbk[nt][1] = cbk[nt][2] = cbk[nt][3] = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t r0 = (j < 2) ? w0.x : w0.y;
+                    const uint32_t r1 = (j < 2) ? w1.x : w1.y;
+                    // byte k of the word, times 256, plus lane * 4: one permute
+                    const uint32_t slo = 0x5504u | ((uint32_t)(2 * (j & 1)) << 4), shi = slo + 0x10u;
+                    uint32_t a[4];
+                    a[0] = lds32(lut + prmt(r0, lane4, slo));
+                    a[2] = lds32(lut + prmt(r0, lane4, shi));
+                    a[1] = lds32(lut + prmt(r1, lane4, slo));
+                    a[3] = lds32(lut + prmt(r1, lane4, shi));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(cbk[nt], a, xf[nt][b][2 * j], xf[nt][b][2 * j + 1]);
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    acc[nt][0] = fmaf(ch0[b], cbk[nt][0], acc[nt][0]);
+                    acc[nt][1] = fmaf(ch0[b], cbk[nt][1], acc[nt][1]);
+                    acc[nt][2] = fmaf(ch1[b], cbk[nt][2], acc[nt][2]);
+                    acc[nt][3] = fmaf(ch1[b], cbk[nt][3], acc[nt][3]);
+                }
             }
-            const float *chat = reinterpret_cast<const float *>(stages + s * kStageBytes + 2 * kBoxBytes);
-            c0 = *reinterpret_cast<const float4 *>(chat + Rl0 * 8 + 4 * h);
-            c1 = *reinterpret_cast<const float4 *>(chat + (Rl0 + 8) * 8 + 4 * h);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
 
-        if (ok) {
-            const uint2 *xc = xs + cur * (NT * 1024);
-            const float ch0[4] = {c0.x, c0.y, c0.z, c0.w}, ch1[4] = {c1.x, c1.y, c1.z, c1.w};
+        // ---------------- the row group's eight slices: written, then summed by warp ks == i % 8
+        if (i > 0 && !mbar_wait(rede0 + 8 * rg, (i - 1) & 1, abort)) { ok = false; break; }
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                const int b = 4 * h + bb;
-                if (b >= nblk) break;
-                float cb[NT][4];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) cb[nt][0] = cb[nt][1] = cb[nt][2] = cb[nt][3] = 0.0f;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t w0 = (j < 2) ? cw[bb][0].x : cw[bb][0].y;
-                    const uint32_t w1 = (j < 2) ? cw[bb][1].x : cw[bb][1].y;
-                    // byte k of w, times 256, plus lane * 4: one permute
-                    const uint32_t slo = 0x5504u | ((uint32_t)(2 * (j & 1)) << 4), shi = slo + 0x10u;
-                    uint32_t a[4];
-                    a[0] = *reinterpret_cast<const uint32_t *>(lut_b + __byte_perm(w0, lane4, slo));
-                    a[2] = *reinterpret_cast<const uint32_t *>(lut_b + __byte_perm(w0, lane4, shi));
-                    a[1] = *reinterpret_cast<const uint32_t *>(lut_b + __byte_perm(w1, lane4, slo));
-                    a[3] = *reinterpret_cast<const uint32_t *>(lut_b + __byte_perm(w1, lane4, shi));
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const uint2 bx = xc[((nt * 8 + b) * 4 + j) * 32 + lane];
-                        mma_bf16_16816(cb[nt], a, bx.x, bx.y);
-                    }
-                }
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    acc[nt][0] = fmaf(ch0[bb], cb[nt][0], acc[nt][0]);
-                    acc[nt][1] = fmaf(ch0[bb], cb[nt][1], acc[nt][1]);
-                    acc[nt][2] = fmaf(ch1[bb], cb[nt][2], acc[nt][2]);
-                    acc[nt][3] = fmaf(ch1[bb], cb[nt][3], acc[nt][3]);
-                }
-            }
+        for (int nt = 0; nt < NT; ++nt) {
+            sts128f(red_mine + nt * 4 * 256, make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]));
+            acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
         }
-        if (has_next) x_store<NT>(xs + (cur ^ 1) * (NT * 1024), tid, xv);
-        named_bar_sync(1, kGemvCompute);
-
-        if (!has_next || nxt.ks == 0) {
-            // ---------------- row block done in this CTA: combine halves, parts, adapter term
-            if (!dep_done) {
-                griddep_wait();                        // L and the cleared counters are visible
-                dep_done = true;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(redf0 + 8 * rg);
+        if (ks == (i & 7)) {
+            if (!mbar_wait(redf0 + 8 * rg, i & 1, abort)) { ok = false; break; }
+            float sum[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                sum[nt][0] = sum[nt][1] = sum[nt][2] = sum[nt][3] = 0.0f;
+#pragma unroll
+                for (int k2 = 0; k2 < 8; ++k2) {
+                    const float4 v =
+                        lds128f(lut + hole(gemv_red_hole0(NT) + ((rg * 8 + k2) * NT + nt) * 4 + (lane >> 3)) +
+                               (lane & 7) * 16);
+                    sum[nt][0] += v.x; sum[nt][1] += v.y; sum[nt][2] += v.z; sum[nt][3] += v.w;
+                }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(rede0 + 8 * rg);
             const int M = grp.M, N = it.N;
-            float *ex = reinterpret_cast<float *>(xs + cur * (NT * 1024));   // free until the next unit ends
-            if (h == 1)
+            const int R0 = pos.rb * ROWS + rg * 16 + g;
+            float *pp = it.partial + (int64_t)pos.ch * N * M;
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                    reinterpret_cast<float4 *>(ex)[(nt * 8 + wr) * 32 + lane] =
-                        make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
-            named_bar_sync(1, kGemvCompute);
-            const int ru0 = it.unit0 + pos.rb * it.nks;                      // first unit of the row block
-            const int c_first = ru0 / grp.per_cta, c_last = (ru0 + it.nks - 1) / grp.per_cta;
-            const int nparts = c_last - c_first + 1;
-            const int row0 = pos.rb * kGemvRows + Rl0, row1 = row0 + 8;
-            float tot[NT][4];
-            if (h == 0) {
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const float4 o = reinterpret_cast<const float4 *>(ex)[(nt * 8 + wr) * 32 + lane];
-                    tot[nt][0] = acc[nt][0] + o.x;
-                    tot[nt][1] = acc[nt][1] + o.y;
-                    tot[nt][2] = acc[nt][2] + o.z;
-                    tot[nt][3] = acc[nt][3] + o.w;
+                for (int q = 0; q < 4; ++q) {
+                    const int tok = nt * 8 + 2 * t + (q & 1), R = R0 + (q >= 2 ? 8 : 0);
+                    if (tok < M && R < N) pp[(int64_t)R * M + tok] = sum[nt][q];
                 }
-            }
-            bool write_y = nparts == 1;
-            if (nparts > 1) {
-                if (h == 0) {
-                    const int slot = ru0 < u_begin ? 0 : 1;
-                    float *pp = grp.partial + ((int64_t)(blockIdx.x * 2 + slot) * kGemvRows) * M;
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const int t0 = nt * 8 + 2 * t;
-                        if (t0 < M) { pp[Rl0 * M + t0] = tot[nt][0]; pp[(Rl0 + 8) * M + t0] = tot[nt][2]; }
-                        if (t0 + 1 < M) { pp[Rl0 * M + t0 + 1] = tot[nt][1]; pp[(Rl0 + 8) * M + t0 + 1] = tot[nt][3]; }
-                    }
-                    __threadfence();
-                }
-                named_bar_sync(1, kGemvCompute);
-                if (tid == 0) {
-                    const int old = atomicAdd(grp.counters + it.rb0 + pos.rb, 1);
-                    flags[1] = (old == nparts - 1) ? 1 : 0;
-                }
-                named_bar_sync(1, kGemvCompute);
-                write_y = flags[1] != 0;
-                if (write_y && h == 0) {
-                    __threadfence();
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) tot[nt][0] = tot[nt][1] = tot[nt][2] = tot[nt][3] = 0.0f;
-                    for (int pi = 0; pi < nparts; ++pi) {
-                        const int c = c_first + pi;
-                        const int slot = ru0 < c * grp.per_cta ? 0 : 1;
-                        const float *pp = grp.partial + ((int64_t)(c * 2 + slot) * kGemvRows) * M;
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            const int t0 = min(nt * 8 + 2 * t, M - 1), t1 = min(nt * 8 + 2 * t + 1, M - 1);
-                            tot[nt][0] += __ldcg(pp + Rl0 * M + t0);
-                            tot[nt][1] += __ldcg(pp + Rl0 * M + t1);
-                            tot[nt][2] += __ldcg(pp + (Rl0 + 8) * M + t0);
-                            tot[nt][3] += __ldcg(pp + (Rl0 + 8) * M + t1);
-                        }
-                    }
-                    if (tid == 0) grp.counters[it.rb0 + pos.rb] = 0;   // ready for the next launch
-                }
-            }
-            if (write_y && h == 0 && ok) {
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int tok = nt * 8 + 2 * t + (q & 1), row = (q < 2) ? row0 : row1;
-                        if (tok < M && row < N) {
-                            float y = tot[nt][q];
-                            if (it.L) y += __ldcg(it.L + (int64_t)tok * N + row);
-                            it.Y[(int64_t)tok * N + row] = __float2bfloat16_rn(y);
-                        }
-                    }
-                }
-            }
-            named_bar_sync(1, kGemvCompute);              // ex is reused by the next unit
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
         }
-        pos = nxt;
+        pos = unit_next(grp, pos);
     }
 }
 
 // ---------------------------------------------------------------- host side
-static int gemv_grid(int units) {
-    int ctas = num_sms();
-    if (ctas > units) ctas = units;
-    const int per = (int)ceil_div(units, ctas);
-    return (int)ceil_div(units, per);
-}
-static int item_units(const LinearDesc &d) {
-    return (int)(ceil_div(d.W.rows, kGemvRows) * ceil_div(d.W.cols, kGemvKChunk));
-}
+static int rows_for(int64_t M) { return M <= 8 ? gemv_rows(1) : gemv_rows(2); }
 
-// Workspace of one launch group: counters, partial slots, XA partials, L.
+// Workspace of one launch group: fp32 K-chunk sums [nch][N][M] per projection and
+// X A chunk partials [K/512][M][r] per adapter, each region 256-byte aligned.
 static size_t group_workspace(int64_t M, int count, const LinearDesc *d) {
-    int units = 0, nrb = 0;
-    size_t lora = 0;
+    size_t b = 0;
     for (int i = 0; i < count; ++i) {
-        units += item_units(d[i]);
-        nrb += (int)ceil_div(d[i].W.rows, kGemvRows);
-        if (d[i].r > 0) {
-            lora += align256((size_t)ceil_div(d[i].W.cols, kXaChunk) * M * d[i].r * 4);
-            lora += align256((size_t)M * d[i].W.rows * 4);
-        }
+        b += align256((size_t)ceil_div(ceil_div(d[i].W.cols, kGemvSlice), kGemvMaxSlices) * d[i].W.rows * M * 4);
+        if (d[i].r > 0) b += align256((size_t)ceil_div(d[i].W.cols, kXaChunk) * M * d[i].r * 4);
     }
-    const int grid = units > 0 ? gemv_grid(units) : 0;
-    return align256((size_t)nrb * 4) + align256((size_t)grid * 2 * kGemvRows * M * 4) + lora;
+    return b;
 }
 
 size_t fwd_workspace_bytes_large(int64_t M, int64_t rows, int64_t cols, int r);
@@ -639,87 +654,127 @@ static cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, siz
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Small-M forward of count <= kGemvMaxItems projections: adapter kernels and one GEMV launch.
+// Small-M forward of count <= kGemvMaxItems projections: the X A pre-pass, the GEMV, the finish.
 static cudaError_t gemv_group(int64_t M, int count, const LinearDesc *d, void *ws, cudaStream_t st) {
     GemvGroup grp;
-    LoraGroup lg;
-    grp.n = count;
-    grp.M = (int)M;
-    lg.n = 0;
-    lg.M = (int)M;
+    XaGroup xg;
+    FinishGroup fg;
+    const int rows = rows_for(M);
+    grp.n = fg.n = count;
+    grp.M = xg.M = fg.M = (int)M;
+    xg.n = 0;
     char *wsp = static_cast<char *>(ws);
-    int units = 0, nrb = 0;
-    for (int i = 0; i < count; ++i) {
-        units += item_units(d[i]);
-        nrb += (int)ceil_div(d[i].W.rows, kGemvRows);
-    }
-    const int grid = gemv_grid(units);
-    grp.units = units;
-    grp.per_cta = (int)ceil_div(units, grid);
-    grp.counters = reinterpret_cast<int *>(wsp);
-    wsp += align256((size_t)nrb * 4);
-    grp.partial = reinterpret_cast<float *>(wsp);
-    wsp += align256((size_t)grid * 2 * kGemvRows * M * 4);
-    lg.counters = grp.counters;
-    lg.ncounters = nrb;
-    int u0 = 0, rb0 = 0, cta_xa = 0, cta_lora = 0;
+    int u0 = 0, fc = 0;
+    int64_t total = 0;
     for (int i = 0; i < count; ++i) {
         GemvItem &it = grp.it[i];
+        FinishItem &fi = fg.it[i];
         const NF4View &w = d[i].W;
-        if (!make_map(&it.codes, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)w.cols / 2, (uint64_t)w.rows,
-                      (uint64_t)w.cols / 2, 128, kGemvRows, CU_TENSOR_MAP_SWIZZLE_128B))
+        it.nsl = (int)ceil_div(w.cols, kGemvSlice);
+        it.nch = (int)ceil_div(it.nsl, kGemvMaxSlices);
+        it.zbig = (int)ceil_div(it.nsl, it.nch);
+        it.sq = it.nsl / it.nch;
+        it.srem = it.nsl % it.nch;
+        // rows of whole 128-byte slices: one 3D box (slice x row x byte) per unit, of the
+        // chunk's slice count (two maps: chunks differ by at most one slice); else 2D boxes
+        it.map3d = (w.cols % 256 == 0) ? 1 : 0;
+        if (it.map3d) {
+            const uint64_t dims[3] = {128, (uint64_t)w.rows, (uint64_t)w.cols / 256};
+            const uint64_t strides[2] = {(uint64_t)w.cols / 2, 128};
+            const uint32_t box[3] = {128, (uint32_t)rows, (uint32_t)it.zbig};
+            const uint32_t box_small[3] = {128, (uint32_t)rows, (uint32_t)(it.zbig > 1 ? it.zbig - 1 : 1)};
+            if (!make_map_3d(&it.codes, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_128B) ||
+                !make_map_3d(&it.codes_small, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, dims, strides, box_small,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+                return cudaErrorInvalidValue;
+        } else if (!make_map(&it.codes, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)w.cols / 2,
+                             (uint64_t)w.rows, (uint64_t)w.cols / 2, 128, (uint32_t)rows, CU_TENSOR_MAP_SWIZZLE_128B)) {
             return cudaErrorInvalidValue;
+        }
         it.scale8 = w.scale8;
         it.scale2 = w.scale2;
         it.offset = w.offset;
         it.X = d[i].X;
-        it.Y = d[i].Y;
-        it.L = nullptr;
         it.N = (int)w.rows;
         it.K = (int)w.cols;
         it.kbs = (int)(w.cols / 64);
-        it.nks = (int)ceil_div(w.cols, kGemvKChunk);
-        it.nrb = (int)ceil_div(w.rows, kGemvRows);
+        it.nrb = (int)ceil_div(w.rows, rows);
         it.unit0 = u0;
-        it.rb0 = rb0;
-        u0 += it.nks * it.nrb;
-        rb0 += it.nrb;
-        if (d[i].r > 0) {
-            LoraItem &li = lg.it[lg.n++];
-            li.X = d[i].X;
-            li.A = d[i].A;
-            li.B = d[i].B;
-            li.XA_save = d[i].XA_save;
-            li.s = d[i].s;
-            li.K = it.K;
-            li.N = it.N;
-            li.r = d[i].r;
-            li.nchunks = (int)ceil_div(w.cols, kXaChunk);
-            li.part = reinterpret_cast<float *>(wsp);
-            wsp += align256((size_t)li.nchunks * M * li.r * 4);
-            li.L = reinterpret_cast<float *>(wsp);
-            wsp += align256((size_t)M * w.rows * 4);
-            li.cta_xa = cta_xa;
-            li.cta_lora = cta_lora;
-            cta_xa += li.nchunks;
-            cta_lora += (int)ceil_div(w.rows, kLoraCols);
-            it.L = li.L;
+        it.partial = reinterpret_cast<float *>(wsp);
+        wsp += align256((size_t)it.nch * w.rows * M * 4);
+        u0 += it.nch * it.nrb;
+        total += (int64_t)w.rows * w.cols;
+        fi.partial = it.partial;
+        fi.B = d[i].B;
+        fi.Y = d[i].Y;
+        fi.N = it.N;
+        fi.nch = it.nch;
+        fi.r = d[i].r > 0 ? d[i].r : 0;
+        fi.s = d[i].s;
+        fi.xpart = nullptr;
+        fi.XA_save = d[i].r > 0 ? d[i].XA_save : nullptr;
+        fi.nxa = 0;
+        fi.cta0 = fc;
+        fc += (int)ceil_div(w.rows, kFinishRows);
+    }
+    int xc = 0;
+    for (int i = 0; i < count; ++i) {
+        if (d[i].r <= 0) continue;
+        XaItem &xi = xg.it[xg.n++];
+        const int nxa = (int)ceil_div(d[i].W.cols, kXaChunk);
+        xi.X = d[i].X;
+        xi.A = d[i].A;
+        xi.K = (int)d[i].W.cols;
+        xi.r = d[i].r;
+        xi.cta0 = xc;
+        xi.xpart = reinterpret_cast<float *>(wsp);
+        wsp += align256((size_t)nxa * M * d[i].r * 4);
+        xc += nxa;
+        fg.it[i].xpart = xi.xpart;
+        fg.it[i].nxa = nxa;
+    }
+    // contiguous unit ranges of (nearly) equal weight count, one per CTA
+    const int units = u0;
+    int grid = num_sms();
+    if (grid > kGemvMaxGrid) grid = kGemvMaxGrid;
+    if (grid > units) grid = units;
+    {
+        int c = 0;
+        int64_t acc = 0;
+        grp.ustart[0] = 0;
+        for (int i = 0; i < count; ++i) {
+            const GemvItem &it = grp.it[i];
+            for (int ch = 0; ch < it.nch; ++ch) {
+                const int64_t sl0 = chunk_slice0(ch, it.sq, it.srem), sl1 = chunk_slice0(ch + 1, it.sq, it.srem);
+                const int64_t kin = std::min<int64_t>(sl1 * kGemvSlice, it.K) - sl0 * kGemvSlice;
+                for (int rb = 0; rb < it.nrb; ++rb) {
+                    const int64_t nr = std::min<int64_t>(rows, it.N - (int64_t)rb * rows);
+                    acc += nr * kin;
+                    const int u = it.unit0 + ch * it.nrb + rb;
+                    // CTA c ends after the unit that brings the running sum to c+1 shares
+                    while (c < grid - 1 && acc * grid >= (int64_t)(c + 1) * total) grp.ustart[++c] = u + 1;
+                }
+            }
         }
+        while (c < grid) grp.ustart[++c] = units;
     }
     cudaError_t e;
-    const bool xa = lg.n > 0;
-    if (xa) QNF4_LAUNCH("k_gemv_xa", st, k_gemv_xa<<<cta_xa, 256, 0, st>>>(lg));
-    QNF4_LAUNCH("k_gemv_lora", st, e = launch_pdl(k_gemv_lora, xa ? cta_lora : 1, 256, 0, st, xa, lg));
-    if (e != cudaSuccess) return e;
     if (M <= 8) {
         if ((e = set_smem(k_gemv<1>, gemv_smem(1))) != cudaSuccess) return e;
         QNF4_LAUNCH("k_gemv", st,
-                    e = launch_pdl(k_gemv<1>, grid, gemv_threads(1), gemv_smem(1), st, true, grp, host_codebook()));
+                    e = launch_pdl(k_gemv<1>, grid, gemv_threads(1), gemv_smem(1), st, false, grp, host_codebook()));
     } else {
         if ((e = set_smem(k_gemv<2>, gemv_smem(2))) != cudaSuccess) return e;
         QNF4_LAUNCH("k_gemv", st,
-                    e = launch_pdl(k_gemv<2>, grid, gemv_threads(2), gemv_smem(2), st, true, grp, host_codebook()));
+                    e = launch_pdl(k_gemv<2>, grid, gemv_threads(2), gemv_smem(2), st, false, grp, host_codebook()));
     }
+    if (e != cudaSuccess) return e;
+    if (xc > 0) {
+        QNF4_LAUNCH("k_gemv_xa", st, e = launch_pdl(k_gemv_xa, xc, 32, 0, st, true, xg));
+        if (e != cudaSuccess) return e;
+    }
+    QNF4_LAUNCH("k_gemv_finish", st, e = launch_pdl(k_gemv_finish, fc, kFinishRows, 0, st, true, fg));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -7,7 +7,17 @@ namespace qnf4 {
 
 cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlora_nf4_tensor &out,
                             float *c1, double *part, cudaStream_t st);
+// One tensor of a grouped quantisation: input, weights, output buffers and its workspace slices.
+struct QuantArgs {
+    const void *W;
+    int64_t n;
+    qlora_nf4_tensor out;
+    float *c1;
+    double *part;
+};
+cudaError_t launch_quantize_grouped(const QuantArgs *a, int count, qlora_dtype dt, cudaStream_t st);
 cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st);
+cudaError_t launch_dequant_grouped(const NF4View *q, __nv_bfloat16 *const *out, int count, cudaStream_t st);
 cudaError_t launch_fmt4_quantize(const void *W, qlora_dtype dt, int64_t n, qlora_fmt4 f, uint8_t *codes,
                                  float *absmax, cudaStream_t st);
 cudaError_t launch_fmt4_dequant(const uint8_t *codes, const float *absmax, int64_t n, qlora_fmt4 f,

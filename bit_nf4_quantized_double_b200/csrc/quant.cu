@@ -14,9 +14,10 @@
 //   k_offset          one CTA: the upper levels of the fp64 pairwise tree -> mean;
 //   k_double_quant    one warp per group: s2 = max |c1 - mu|, int8 constants.
 
+#include <atomic>
 #include <cmath>
 
-#include "common.cuh"
+#include "launch.h"
 
 namespace qnf4 {
 
@@ -89,12 +90,39 @@ __device__ __forceinline__ void load_vec(const T *p, float (&v)[VEC]) {
 // x' + 3 (in [2, 4): the top 8 mantissa bits are the bin). Where x' lies within
 // 4 ulp of the bin's threshold the exact quotient and the full search decide, so
 // the codes are those of x bit for bit. Without BINS every weight is divided.
+// A list of tensors quantised by one sequence of launches: CTA ranges per tensor
+// (groups in k_quantize_codes, blocks of eight groups in k_double_quant), one CTA
+// per tensor in k_offset.
+constexpr int kQuantMaxItems = 64;
+struct QuantItem {
+    const void *W;
+    int64_t n, nb, nb2;
+    float *c1;                   // [nb] exact absmax (workspace)
+    double *part;                // [nb2] group partial sums (workspace)
+    uint8_t *codes;
+    int8_t *scale8;
+    float *scale2;
+    float *offset;
+    int64_t cta0;                // first CTA of this tensor in k_quantize_codes
+    int64_t dq0;                 // first CTA of this tensor in k_double_quant
+};
+struct QuantGroup {
+    QuantItem it[kQuantMaxItems];
+    int count;
+};
+// The tensor whose CTA range holds block b (ranges ascending from 0).
+__device__ __forceinline__ int quant_item(const QuantGroup &g, int64_t b, bool dq) {
+    int lo = 0, hi = g.count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((dq ? g.it[mid].dq0 : g.it[mid].cta0) <= b) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
 template <typename T, bool BINS>
 __global__ void __launch_bounds__(256, 4)
-k_quantize_codes(const T *__restrict__ W, int64_t n, int64_t nb, Codebook cb,
-                 const __grid_constant__ CodeBins bins,
-                 float *__restrict__ c1_out, double *__restrict__ part_out,
-                 uint8_t *__restrict__ codes) {
+k_quantize_codes(const __grid_constant__ QuantGroup grp, Codebook cb, const __grid_constant__ CodeBins bins) {
     constexpr int VEC = 16 / sizeof(T);   // elements per 16-byte lane load
     constexpr int LPB = kBlock1 / VEC;    // lanes per block
     constexpr int BPI = 32 / LPB;         // blocks per warp iteration
@@ -111,7 +139,13 @@ k_quantize_codes(const T *__restrict__ W, int64_t n, int64_t nb, Codebook cb,
     if (BINS) s_bin[threadIdx.x] = make_int2(bins.base[threadIdx.x], __float_as_int(bins.thr[threadIdx.x]));
     __syncthreads();
 
-    const int64_t group = blockIdx.x;
+    const QuantItem &item = grp.it[quant_item(grp, blockIdx.x, false)];
+    const T *__restrict__ W = static_cast<const T *>(item.W);
+    const int64_t n = item.n, nb = item.nb;
+    float *__restrict__ c1_out = item.c1;
+    double *__restrict__ part_out = item.part;
+    uint8_t *__restrict__ codes = item.codes;
+    const int64_t group = blockIdx.x - item.cta0;
     const int sub = lane / LPB, li = lane % LPB;
     const int64_t ncode = (n + 1) / 2;
     bool nonfinite = false;
@@ -224,8 +258,12 @@ k_quantize_codes(const T *__restrict__ W, int64_t n, int64_t nb, Codebook cb,
 // a binary-counter stack (which forms exactly the subtree of those leaves),
 // then the 1024 subtree sums are combined level by level. mu = fl(S / nb).
 __global__ void __launch_bounds__(1024)
-k_offset(const double *__restrict__ part, int64_t nb2, int64_t nb, float *__restrict__ offset_out) {
+k_offset(const __grid_constant__ QuantGroup grp) {
     __shared__ double s_w[32];
+    const QuantItem &item = grp.it[blockIdx.x];
+    const double *__restrict__ part = item.part;
+    const int64_t nb2 = item.nb2, nb = item.nb;
+    float *__restrict__ offset_out = item.offset;
     int64_t L = 1024;
     while (L < nb2) L <<= 1;
     const int64_t C = L / 1024;
@@ -267,10 +305,15 @@ k_offset(const double *__restrict__ part, int64_t nb2, int64_t nb, float *__rest
 // One warp per second-level group: d_b = fl(c1_b - mu), s2 = max |d_b|,
 // q8_b = rint(fl(fl(d_b / s2) * 127)) (0 when s2 == 0).
 __global__ void __launch_bounds__(256)
-k_double_quant(const float *__restrict__ c1, int64_t nb, int64_t nb2, const float *__restrict__ offset,
-               int8_t *__restrict__ q8, float *__restrict__ s2) {
+k_double_quant(const __grid_constant__ QuantGroup grp) {
+    const QuantItem &item = grp.it[quant_item(grp, blockIdx.x, true)];
+    const float *__restrict__ c1 = item.c1;
+    const int64_t nb = item.nb, nb2 = item.nb2;
+    const float *__restrict__ offset = item.offset;
+    int8_t *__restrict__ q8 = item.scale8;
+    float *__restrict__ s2 = item.scale2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t j = (int64_t)blockIdx.x * 8 + warp;
+    const int64_t j = (int64_t)(blockIdx.x - item.dq0) * 8 + warp;
     if (j >= nb2) return;
     const float mu = *offset;
     float d[8];
@@ -295,59 +338,88 @@ k_double_quant(const float *__restrict__ c1, int64_t nb, int64_t nb2, const floa
     }
 }
 
-// Dequantisation: each thread expands two 32-bit words of codes (16 weights, a
-// quarter block) into two 16-byte bf16 stores; a warp reads 256 contiguous code
-// bytes and writes 1 KB, and four such pairs per thread are in flight at once.
-// Codebook in shared memory (16 distinct words: lookups never conflict). A
-// ragged tail (n % 16 != 0) is written element by element.
-constexpr int kDequantUnroll = 4;
-__global__ void __launch_bounds__(256, 4)
-k_dequant(NF4View q, int64_t n, Codebook cb, __nv_bfloat16 *__restrict__ out) {
+// Dequantisation, over one tensor or a list of them in one launch. The codes of
+// every tensor are cut into chunks of 256 32-bit words (2048 weights, 32 blocks;
+// chunks never straddle a second-level group of 2048 words), numbered across the
+// list; warps walk the chunks grid-stride. Lane l of a warp expands words
+// 32 u + l (u = 0..7) of its chunk: eight coalesced 4-byte code loads and eight
+// coalesced 16-byte bf16 stores, all loads issued before any arithmetic. Each word
+// is one eighth of a 64-block: c^ = fl(fl(q8 * fl(s2 / 127)) + mu) with the step
+// divided once per chunk, then w^ = bf16(fl(Q[code] * c^)) from the codebook in
+// shared memory (16 distinct words: the lookups never conflict). The last n % 8
+// weights of a tensor, if any, are written element by element.
+constexpr int kDeqChunkWords = 256;
+constexpr int kDeqMaxItems = 64;
+struct DeqItem {
+    const uint32_t *codes;
+    const int8_t *scale8;
+    const float *scale2;
+    const float *offset;
+    __nv_bfloat16 *out;
+    int64_t n;              // weights
+    int64_t chunk0;         // first chunk of this tensor in the list's numbering
+};
+struct DeqGroup {
+    DeqItem it[kDeqMaxItems];
+    int count;
+    int64_t chunks;         // total
+};
+
+__device__ __forceinline__ uint32_t dequant_pair(const float *s_q, uint32_t byte, float ch) {
+    return pack_bf16x2(__fmul_rn(s_q[byte >> 4], ch), __fmul_rn(s_q[byte & 15u], ch));
+}
+
+__global__ void __launch_bounds__(256)
+k_dequant(const __grid_constant__ DeqGroup grp, Codebook cb) {
     __shared__ float s_q[16];
     if (threadIdx.x < 16) s_q[threadIdx.x] = cb.q[threadIdx.x];
     __syncthreads();
-    const float mu = *q.offset;
-    const int64_t n16 = n / 16;
-    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
-    const uint2 *codes = reinterpret_cast<const uint2 *>(q.codes);
-    for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g0 < n16; g0 += kDequantUnroll * nthr) {
-        uint2 w[kDequantUnroll];
-        int8_t q8[kDequantUnroll];
-        float s2[kDequantUnroll];
-#pragma unroll
-        for (int u = 0; u < kDequantUnroll; ++u) {
-            const int64_t g = g0 + u * nthr;
-            if (g < n16) {
-                const int64_t b = g / (kBlock1 / 16);
-                w[u] = __ldg(codes + g);
-                q8[u] = __ldg(q.scale8 + b);
-                s2[u] = __ldg(q.scale2 + b / kBlock2);
-            }
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    int ii = 0;
+    float mu = __ldg(grp.it[0].offset);
+    for (int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; c < grp.chunks; c += nwarps) {
+        if (c >= grp.it[ii].chunk0 + ((grp.it[ii].n / 8 + kDeqChunkWords - 1) / kDeqChunkWords)) {
+            do { ++ii; } while (ii + 1 < grp.count && c >= grp.it[ii + 1].chunk0);
+            mu = __ldg(grp.it[ii].offset);
         }
+        const DeqItem &it = grp.it[ii];
+        const int64_t nw = it.n / 8;                       // whole code words
+        const int64_t w0 = (c - it.chunk0) * kDeqChunkWords;
+        uint32_t w[8];
+        int8_t q8[8];
 #pragma unroll
-        for (int u = 0; u < kDequantUnroll; ++u) {
-            const int64_t g = g0 + u * nthr;
-            if (g < n16) {
-                const float ch = dq_constant(q8[u], s2[u], mu);
-                uint32_t o[8];
+        for (int u = 0; u < 8; ++u) {
+            const int64_t wi = w0 + 32 * u + lane;
+            w[u] = wi < nw ? __ldg(it.codes + wi) : 0u;
+            q8[u] = wi < nw ? __ldg(it.scale8 + (wi >> 3)) : (int8_t)0;
+        }
+        const float step = __fdiv_rn(__ldg(it.scale2 + (w0 >> 11)), 127.0f);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t byte = ((k < 4 ? w[u].x : w[u].y) >> (8 * (k & 3))) & 0xffu;
-                    o[k] = pack_bf16x2(__fmul_rn(s_q[byte >> 4], ch), __fmul_rn(s_q[byte & 15u], ch));
-                }
-                uint4 *dst = reinterpret_cast<uint4 *>(out + 16 * g);
-                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        for (int u = 0; u < 8; ++u) {
+            const int64_t wi = w0 + 32 * u + lane;
+            if (wi < nw) {
+                const float ch = __fadd_rn(__fmul_rn((float)q8[u], step), mu);
+                uint4 o;
+                o.x = dequant_pair(s_q, w[u] & 0xffu, ch);
+                o.y = dequant_pair(s_q, (w[u] >> 8) & 0xffu, ch);
+                o.z = dequant_pair(s_q, (w[u] >> 16) & 0xffu, ch);
+                o.w = dequant_pair(s_q, w[u] >> 24, ch);
+                reinterpret_cast<uint4 *>(it.out)[wi] = o;
             }
         }
     }
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        for (int64_t e = 16 * n16; e < n; ++e) {
+    // the last n % 8 weights of tensor blockIdx.x (the code word is read byte by byte)
+    if ((int)blockIdx.x < grp.count && threadIdx.x == 0) {
+        const DeqItem &it = grp.it[blockIdx.x];
+        const uint8_t *cbytes = reinterpret_cast<const uint8_t *>(it.codes);
+        const float m = __ldg(it.offset);
+        for (int64_t e = (it.n / 8) * 8; e < it.n; ++e) {
             const int64_t b = e / kBlock1;
-            const float ch = dq_constant(q.scale8[b], q.scale2[b / kBlock2], mu);
-            const uint8_t byte = q.codes[e / 2];
+            const float ch = dq_constant(it.scale8[b], it.scale2[b / kBlock2], m);
+            const uint8_t byte = cbytes[e / 2];
             const uint32_t code = (e % 2 == 0) ? (byte >> 4) : (byte & 15u);
-            out[e] = __float2bfloat16_rn(__fmul_rn(s_q[code], ch));
+            it.out[e] = __float2bfloat16_rn(__fmul_rn(s_q[code], ch));
         }
     }
 }
@@ -432,36 +504,110 @@ cudaError_t launch_merge_bf16(const NF4View &q, const __nv_bfloat16 *A, const __
 }
 
 // ---------------------------------------------------------------- launchers
-cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlora_nf4_tensor &out,
-                            float *c1, double *part, cudaStream_t st) {
-    const int64_t nb = ceil_div(n, kBlock1), nb2 = ceil_div(nb, kBlock2);
+// Code search of the quantiser: the bin table with its exact fallback (default) or a
+// division for every weight; both give the same codes (the second exists so that the
+// tests can compare the two).
+static std::atomic<int> g_divide_every_weight{0};
+
+// Three launches over up to kQuantMaxItems tensors of one input dtype.
+static cudaError_t quantize_launch(const QuantArgs *a, int count, qlora_dtype dt, cudaStream_t st) {
     const Codebook &cb = host_codebook();
     static CodeBins bins;
-    static const bool use_bins = build_code_bins(cb, bins);
+    static const bool bins_ok = build_code_bins(cb, bins);
+    const bool use_bins = bins_ok && g_divide_every_weight.load() == 0;
+    QuantGroup g;
+    g.count = count;
+    int64_t ctas = 0, dq = 0;
+    for (int i = 0; i < count; ++i) {
+        QuantItem &it = g.it[i];
+        it.W = a[i].W;
+        it.n = a[i].n;
+        it.nb = ceil_div(it.n, kBlock1);
+        it.nb2 = ceil_div(it.nb, kBlock2);
+        it.c1 = a[i].c1;
+        it.part = a[i].part;
+        it.codes = a[i].out.codes;
+        it.scale8 = a[i].out.scale8;
+        it.scale2 = a[i].out.scale2;
+        it.offset = a[i].out.offset;
+        it.cta0 = ctas;
+        it.dq0 = dq;
+        ctas += it.nb2;
+        dq += ceil_div(it.nb2, 8);
+    }
+    if (ctas > 0x7fffffffLL || dq > 0x7fffffffLL) return cudaErrorInvalidValue;
     if (dt == QLORA_F32) {
         if (use_bins)
-            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<float, true><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const float *>(W), n, nb, cb, bins, c1, part, out.codes));
+            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<float, true><<<(unsigned)ctas, 256, 0, st>>>(g, cb, bins));
         else
-            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<float, false><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const float *>(W), n, nb, cb, bins, c1, part, out.codes));
+            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<float, false><<<(unsigned)ctas, 256, 0, st>>>(g, cb, bins));
     } else {
         if (use_bins)
-            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<__nv_bfloat16, true><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W), n, nb, cb, bins, c1, part, out.codes));
+            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<__nv_bfloat16, true><<<(unsigned)ctas, 256, 0, st>>>(g, cb, bins));
         else
-            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<__nv_bfloat16, false><<<(unsigned)nb2, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W), n, nb, cb, bins, c1, part, out.codes));
+            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<__nv_bfloat16, false><<<(unsigned)ctas, 256, 0, st>>>(g, cb, bins));
     }
-    QNF4_LAUNCH("k_offset", st, k_offset<<<1, 1024, 0, st>>>(part, nb2, nb, out.offset));
-    QNF4_LAUNCH("k_double_quant", st, k_double_quant<<<(unsigned)ceil_div(nb2, 8), 256, 0, st>>>(c1, nb, nb2, out.offset, out.scale8, out.scale2));
+    QNF4_LAUNCH("k_offset", st, k_offset<<<(unsigned)count, 1024, 0, st>>>(g));
+    QNF4_LAUNCH("k_double_quant", st, k_double_quant<<<(unsigned)dq, 256, 0, st>>>(g));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const void *W, qlora_dtype dt, int64_t n, const qlora_nf4_tensor &out,
+                            float *c1, double *part, cudaStream_t st) {
+    const QuantArgs a{W, n, out, c1, part};
+    return quantize_launch(&a, 1, dt, st);
+}
+
+cudaError_t launch_quantize_grouped(const QuantArgs *a, int count, qlora_dtype dt, cudaStream_t st) {
+    for (int i = 0; i < count; i += kQuantMaxItems) {
+        const int n = count - i < kQuantMaxItems ? count - i : kQuantMaxItems;
+        cudaError_t e = quantize_launch(a + i, n, dt, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+// One launch over up to kDeqMaxItems tensors; a persistent grid of up to eight
+// 256-thread CTAs per SM.
+static cudaError_t dequant_launch(const NF4View *q, __nv_bfloat16 *const *out, int count, cudaStream_t st) {
+    DeqGroup g;
+    g.count = count;
+    int64_t chunks = 0;
+    for (int i = 0; i < count; ++i) {
+        DeqItem &it = g.it[i];
+        it.codes = reinterpret_cast<const uint32_t *>(q[i].codes);
+        it.scale8 = q[i].scale8;
+        it.scale2 = q[i].scale2;
+        it.offset = q[i].offset;
+        it.out = out[i];
+        it.n = q[i].rows * q[i].cols;
+        it.chunk0 = chunks;
+        chunks += ceil_div(it.n / 8, kDeqChunkWords);
+    }
+    g.chunks = chunks;
+    int64_t grid = ceil_div(chunks, 8);                   // eight warps per CTA
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (grid > cap) grid = cap;
+    if (grid < count) grid = count;                       // one CTA per tensor writes its tail
+    QNF4_LAUNCH("k_dequant", st, k_dequant<<<(unsigned)grid, 256, 0, st>>>(g, host_codebook()));
     return cudaGetLastError();
 }
 
 cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st) {
-    const int64_t n = q.rows * q.cols;
-    int64_t grid = ceil_div(ceil_div(n, 16 * kDequantUnroll), 256);
-    const int64_t cap = (int64_t)num_sms() * 8;
-    if (grid < 1) grid = 1;
-    if (grid > cap) grid = cap;
-    QNF4_LAUNCH("k_dequant", st, k_dequant<<<(unsigned)grid, 256, 0, st>>>(q, n, host_codebook(), out));
-    return cudaGetLastError();
+    return dequant_launch(&q, &out, 1, st);
+}
+
+cudaError_t launch_dequant_grouped(const NF4View *q, __nv_bfloat16 *const *out, int count, cudaStream_t st) {
+    for (int i = 0; i < count; i += kDeqMaxItems) {
+        const int n = count - i < kDeqMaxItems ? count - i : kDeqMaxItems;
+        cudaError_t e = dequant_launch(q + i, out + i, n, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace qnf4
+
+extern "C" void qlora_nf4_set_code_search(int divide_every_weight) {
+    qnf4::g_divide_every_weight.store(divide_every_weight ? 1 : 0);
+}

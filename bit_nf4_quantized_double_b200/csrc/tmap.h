@@ -40,6 +40,19 @@ inline bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, u
     return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// 3D tensor map with arbitrary strides: dims {d0 (contiguous), d1, d2}, byte strides of
+// dims 1 and 2, box {b0, b1, b2}; out-of-range elements read as zero.
+inline bool make_map_3d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, const uint64_t (&dims)[3],
+                        const uint64_t (&strides)[2], const uint32_t (&box)[3], CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+    cuuint64_t st[2] = {strides[0], strides[1]};
+    cuuint32_t bx[3] = {box[0], box[1], box[2]};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, dt, 3, const_cast<void *>(base), d, st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 inline bool map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box0, uint32_t box1,
                      CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
     return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, inner, outer, inner * 2, box0, box1, sw);

@@ -106,6 +106,27 @@ qlora_status qlora_nf4_quantize(const void *W, qlora_dtype dt, const qlora_nf4_t
 qlora_status qlora_nf4_dequant(const qlora_nf4_tensor *q, void *W_out, qlora_stream_t stream);
 
 /*
+ * Quantise or dequantise a list of tensors with one sequence of launches (the page's
+ * section 3 quantises every frozen weight of the model before training; a list
+ * costs three launches per 64 tensors instead of three per tensor). Each tensor
+ * gets exactly what qlora_nf4_quantize / qlora_nf4_dequant give it alone.
+ *   count   1 .. 4096 tensors.
+ *   W       host array of count device pointers (16-byte aligned), all of dtype dt.
+ *   out, q  host arrays of count tensor descriptors, as in the single calls.
+ *   W_out   host array of count device pointers (bf16 [rows, cols], 16-byte aligned).
+ *   ws      device workspace of qlora_nf4_quantize_grouped_workspace() bytes: the
+ *           single-tensor workspaces of the list, back to back.
+ * Every descriptor and pointer is checked before anything is launched. The host
+ * arrays are read during the call only.
+ */
+size_t qlora_nf4_quantize_grouped_workspace(int count, const qlora_nf4_tensor *out);
+qlora_status qlora_nf4_quantize_grouped(int count, const void *const *W, qlora_dtype dt,
+                                        const qlora_nf4_tensor *out, void *ws, size_t ws_bytes,
+                                        qlora_stream_t stream);
+qlora_status qlora_nf4_dequant_grouped(int count, const qlora_nf4_tensor *q, void *const *W_out,
+                                       qlora_stream_t stream);
+
+/*
  * Forward of the layer (page section 1 equation, with W^ = stored^T):
  *   Y[M, rows] = X[M, cols] * Dequant(W)^T + s * (X * A) * B
  *   X  bf16 [M, cols];  A bf16 [cols, r];  B bf16 [r, rows];  Y bf16 [M, rows].
@@ -148,14 +169,13 @@ qlora_status qlora_linear_bwd(const void *X, const void *dY, int64_t M, const ql
  *   d      host array of `count` descriptors (1 <= count <= 64); W points to a host
  *          struct as in qlora_linear_fwd.
  *   ws     one device workspace of qlora_linear_fwd_grouped_workspace() bytes.
- * M <= 16: per group of up to eight items, three launches: the X*A chunk sums, the
- * adapter term (s X A) B, and one persistent GEMV over all items' codes (the last two
- * start early through programmatic dependent launch). Larger M: the items run one after
- * another on the single-item path, and the workspace is the largest single-item
- * requirement. XA_save is bit-identical to calling qlora_linear_fwd on each item; Y is
- * reproducible call to call but, at M <= 16, may differ in the last bits from the
- * single-item call, because the K chunks of a row block cut between two CTAs are added
- * in CTA order and the cut depends on the group.
+ * M <= 16: per group of up to eight items, two launches: X*A of every adapter, and one
+ * persistent GEMV over all items' codes that adds the adapter term (s X A) B as it
+ * finishes each row block (it starts early through programmatic dependent launch).
+ * Larger M: the items run one after another on the single-item path, and the workspace
+ * is the largest single-item requirement. Y and XA_save are bit-identical to calling
+ * qlora_linear_fwd on each item: every output adds its input slices and K chunks in a
+ * fixed order, whichever CTA computes them.
  */
 typedef struct {
     const void *X;                 /* bf16 [M, W->cols] */
@@ -208,6 +228,16 @@ void qlora_nf4_codebook(float out[16]);
  */
 qlora_status qlora_nf4_quantize_noalloc(const void *W, qlora_dtype dt, const qlora_nf4_tensor *out,
                                         qlora_stream_t stream);
+
+/*
+ * Test hook of the quantiser's code search (the page has no counterpart). By default a
+ * weight's code is read from a 256-bin table over x' = w * fl(1/c1), and the exact
+ * quotient fl(w / c1) with the full threshold search decides wherever x' lies within
+ * 4 ulp of the bin's threshold; divide_every_weight != 0 makes every later quantisation
+ * in the process divide every weight instead. Both give the same codes bit for bit;
+ * the hook lets tests compare them. Not thread-safe with concurrent quantisations.
+ */
+void qlora_nf4_set_code_search(int divide_every_weight);
 
 /*
  * Adapter merge and re-quantisation (the page's sections 5 and 6: merging the

@@ -78,9 +78,14 @@ def test_grouped_forward_host_checks():
     d = (q._LinearDesc * 2)(q._LinearDesc(fake, ctypes.pointer(t), None, None, 0, 1.0, fake, None),
                             q._LinearDesc(fake, ctypes.pointer(t), None, None, 0, 1.0, fake, None))
     assert L.qlora_linear_fwd_grouped(1, 0, d, None, 0, None) == q.QLORA_ERR_INVALID_ARG
-    # two 64 x 64 items at M = 1: one work unit each, so two CTAs; one counter per row
-    # block (256-byte aligned) and two 128-row x M fp32 part slots per CTA
-    assert L.qlora_linear_fwd_grouped_workspace(1, 2, d) == 256 + 2 * 2 * 128 * 1 * 4
+    # two 64 x 64 items at M = 1: one K chunk each, so fp32 sums [1][64][1] per item, each
+    # region 256-byte aligned
+    assert L.qlora_linear_fwd_grouped_workspace(1, 2, d) == 2 * 256
+    # 64 x 4096 (two K chunks of 2048) at M = 3 with rank 8: the fp32 chunk sums [2][64][3]
+    # and the X A partials of eight 512-input chunks [8][3][8], each region 256-byte aligned
+    t2 = q._Tensor(64, 4096, fake, fake, fake, fake)
+    d2 = (q._LinearDesc * 1)(q._LinearDesc(fake, ctypes.pointer(t2), fake, fake, 8, 1.0, fake, None))
+    assert L.qlora_linear_fwd_grouped_workspace(3, 1, d2) == 2 * 64 * 3 * 4 + 8 * 3 * 8 * 4
     assert L.qlora_linear_fwd_grouped(1, 2, d, None, 0, None) == q.QLORA_ERR_WORKSPACE
     bad = (q._LinearDesc * 1)(q._LinearDesc(fake, ctypes.pointer(q._Tensor(64, 100, fake, fake, fake, fake)),
                                             None, None, 0, 1.0, fake, None))

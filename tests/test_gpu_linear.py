@@ -109,7 +109,9 @@ def test_small_m_gemv(M, r):
 
 
 @pytest.mark.parametrize("M,rows,cols,r", [
-    (3, 400, 320, 24),       # rows past the last 128-row block, one partial K chunk
+    (3, 400, 320, 24),       # rows past the last 32-row block, one partial K chunk
+    (5, 48, 4096, 16),       # odd M, two K chunks, a half row block
+    (8, 4096, 11008, 16),    # the long-K projection: six chunks, the last 768 inputs
     (16, 272, 192, 64),
     (1, 16, 64, 8),          # a single 64-block
     (9, 1040, 4160, 256),    # widest adapter, ragged rows and K chunks
@@ -137,11 +139,9 @@ def test_decode_layer_full(M):
 
 @pytest.mark.parametrize("M", [1, 16])
 def test_decode_layer_grouped(M):
-    # the whole block in one grouped call. The adapter product XA does not depend on the
-    # grouping (per-projection chunk sums in chunk order): bit-identical to the single calls.
-    # Y sums each row block's K chunks in the order of the CTAs that hold them, and the cut
-    # of the work into CTA ranges depends on the group: Y is reproducible call to call and
-    # within tolerance of the oracle, whether computed alone or grouped.
+    # the whole block in one grouped call, every projection against the oracle. Each output
+    # row sums its K slices in slice order and its K chunks in chunk order whichever CTA holds
+    # them, so the grouped call is bit-identical to the single calls and to itself.
     wl = si.workload("decode7b", M=M)
     items, singles, refs = [], [], []
     for li, L in enumerate(wl.layers):
@@ -151,21 +151,59 @@ def test_decode_layer_grouped(M):
         items.append({"X": inp["X"], "W": t, "A": inp.get("A"), "B": inp.get("B"), "s": L.s, "XA_save": xa})
         Ys, XAs = q.qlora_linear_fwd(inp["X"], t, inp.get("A"), inp.get("B"), L.s)
         singles.append((Ys, XAs))
-        if li in (0, 4):
-            Wh = oracle_weight(inp["W"])
-            An = f64(inp["A"]) if L.r else np.zeros((L.d_in, 0))
-            Bn = f64(inp["B"]) if L.r else np.zeros((0, L.d_out))
-            refs.append((li, oracle.linear_fwd(f64(inp["X"]), Wh, An, Bn, L.s)))
+        Wh = oracle_weight(inp["W"])
+        An = f64(inp["A"]) if L.r else np.zeros((L.d_in, 0))
+        Bn = f64(inp["B"]) if L.r else np.zeros((0, L.d_out))
+        refs.append(oracle.linear_fwd(f64(inp["X"]), Wh, An, Bn, L.s))
     Ys = [y.clone() for y in q.qlora_linear_fwd_grouped(items)]
     Ys2 = q.qlora_linear_fwd_grouped(items)
     assert q.qlora_get_device_status() == q.QLORA_OK
-    for (Y1, XA1), Yg, Yg2, it in zip(singles, Ys, Ys2, items):
-        assert torch.equal(Yg, Yg2)
+    for li, ((Y1, XA1), Yg, Yg2, it) in enumerate(zip(singles, Ys, Ys2, items)):
+        name = wl.layers[li].name
+        check(f64(Yg), refs[li], f"Y[{name}]")
+        assert torch.equal(Yg, Yg2), name
+        assert torch.equal(Yg, Y1), name
         if XA1 is not None:
             assert torch.equal(XA1, it["XA_save"])
-    for li, ref in refs:
-        check(f64(Ys[li]), ref, f"Y[{wl.layers[li].name}]")
-        check(f64(singles[li][0]), ref, f"Y[{wl.layers[li].name}] alone")
+
+
+@pytest.mark.parametrize("M", [2, 8, 9])
+def test_grouped_more_than_eight(M):
+    # eleven projections of mixed shapes: two launch groups (eight, then three) that share
+    # one workspace; ragged rows (N % 32 == 16), inputs that end inside a K chunk and a slice
+    shapes = [(48, 4096, 16), (16, 64, 8), (400, 320, 24), (1040, 4160, 0), (272, 2112, 64), (32, 2048, 8),
+              (2064, 1600, 0), (128, 6144, 16), (80, 576, 0), (16, 2048, 256), (96, 4224, 8)]
+    items, refs = [], []
+    for i, (rows, cols, r) in enumerate(shapes):
+        W, X, dY, A, B, s = make_problem(M, rows, cols, r, seed=900 + 13 * i + M)
+        t = q.qlora_nf4_quantize(W)
+        xa = torch.empty(M, r, dtype=torch.bfloat16, device="cuda") if r else None
+        items.append({"X": X, "W": t, "A": A, "B": B, "s": s, "XA_save": xa})
+        An = f64(A) if r else np.zeros((cols, 0))
+        Bn = f64(B) if r else np.zeros((0, rows))
+        refs.append((oracle.linear_fwd(f64(X), oracle_weight(W), An, Bn, s), f64(X) @ An))
+    Ys = q.qlora_linear_fwd_grouped(items)
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    for i, (Y, it, (ref, xaref)) in enumerate(zip(Ys, items, refs)):
+        check(f64(Y), ref, f"Y[{i}]")
+        if it["XA_save"] is not None:
+            check(f64(it["XA_save"]), xaref, f"XA[{i}]")
+        Y1, _ = q.qlora_linear_fwd(it["X"], it["W"], it["A"], it["B"], it["s"])
+        assert torch.equal(Y, Y1), i
+
+
+@pytest.mark.parametrize("M,rows,cols,r", [(3, 400, 320, 24), (200, 272, 640, 64), (1024, 512, 1024, 16)])
+def test_backward_recomputes_xa(M, rows, cols, r):
+    # XA = NULL: the backward recomputes X A itself (small-M, fused and CTA-pair paths)
+    W, X, dY, A, B, s = make_problem(M, rows, cols, r, seed=31 * M + rows)
+    t = q.qlora_nf4_quantize(W)
+    dX, dA, dB = q.qlora_linear_bwd(X, dY, t, A, B, s, XA=None)
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    Wh = oracle_weight(W)
+    dXr, dAr, dBr = oracle.linear_bwd(f64(X), f64(dY), Wh, f64(A), f64(B), s)
+    check(f64(dX), dXr, "dX")
+    check(f64(dA), dAr, "dA")
+    check(f64(dB), dBr, "dB")
 
 
 def test_full_4096_layer_sampled():

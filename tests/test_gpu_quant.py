@@ -135,3 +135,102 @@ def test_repeat_is_deterministic():
     torch.cuda.synchronize()
     for x, y in [(a.codes, b.codes), (a.scale8, b.scale8), (a.scale2, b.scale2), (a.offset, b.offset)]:
         assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_grouped_quantize_and_dequant(dtype):
+    # a list of tensors through the grouped entry points: each tensor exactly as quantised
+    # and dequantised alone (ragged sizes, a 1-weight tensor, a tensor of several groups)
+    shapes = [(7, 1000), (1, 1), (512, 1024), (3, 5), (33, 4097), (64, 256 * 64 + 3), (1, 63)]
+    Ws = [si.normal(sh, 0.02, seed=40 + i, device="cuda", dtype=dtype) for i, sh in enumerate(shapes)]
+    ts = q.qlora_nf4_quantize_grouped(Ws)
+    whs = q.qlora_nf4_dequant_grouped(ts)
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    for W, t, wh in zip(Ws, ts, whs):
+        assert_bit_exact(W, t, wh)
+
+
+def test_grouped_more_than_one_launch_set():
+    # more tensors than one launch takes (64): the list is cut into launch sets
+    Ws = [si.normal((4, 64 * (1 + i % 5) + i), 0.02, seed=500 + i, device="cuda") for i in range(70)]
+    ts = q.qlora_nf4_quantize_grouped(Ws)
+    whs = q.qlora_nf4_dequant_grouped(ts)
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    for W, t, wh in zip(Ws, ts, whs):
+        assert_bit_exact(W, t, wh)
+
+
+def _band_weights_fp32(rng):
+    # blocks [c1, w_1 .. w_63]: w = fl(T[t] c1) moved by k fp32 ulps (k = -6 .. 6), with c1
+    # not a power of two, so the normalised weight lands within a few ulps of a threshold
+    T = oracle.midpoints().astype(np.float32)
+    blocks = []
+    for c1 in np.float32([0.7, 0.3, 1.3, 2.7, 0.05, 123.4, 0.0171, 9.9e-4]) * np.float32(1 + rng.random(8) * 1e-3):
+        vals = []
+        for thr in T:
+            base = np.float32(thr * c1)
+            for k in range(-6, 7):
+                w = base
+                step = np.float32(np.inf if k > 0 else -np.inf)
+                for _ in range(abs(k)):
+                    w = np.nextafter(w, step, dtype=np.float32)
+                if abs(w) <= c1:
+                    vals.append(w)
+        vals = np.array(vals, np.float32)
+        for j in range(0, vals.size, 63):
+            blk = np.zeros(64, np.float32)
+            blk[0] = c1
+            part = vals[j: j + 63]
+            blk[1: 1 + part.size] = part
+            blocks.append(blk)
+    return np.concatenate(blocks)
+
+
+def _band_weights_bf16():
+    # bf16 pairs (c1, w), searched over every bf16 mantissa of c1, whose fp32 quotient lies
+    # nearest to a threshold. With 8-bit operands no quotient comes within 16 fp32 ulps of a
+    # threshold (the search shows it), so bf16 input never reaches the 4-ulp fallback band;
+    # the pairs within 256 ulps are the closest there are. Blocks [c1 2^e, w 2^e, 0 ...].
+    T = oracle.midpoints().astype(np.float32)
+    c1 = torch.arange(0x3f80, 0x4000, dtype=torch.int32).to(torch.int16).view(torch.bfloat16).float().numpy()
+    hits, closest = [], np.inf
+    for thr in T:
+        approx = torch.from_numpy((thr * c1).astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy()
+        for d in range(-3, 4):
+            w = torch.from_numpy((approx.astype(np.int32) + d).astype(np.int16)).view(torch.bfloat16).float().numpy()
+            x = (w / c1).astype(np.float32)          # IEEE single division, correctly rounded
+            dist = np.abs(x - thr) / np.spacing(np.abs(thr)).astype(np.float32)
+            ok = (dist <= 256) & (np.abs(w) <= c1)
+            closest = min(closest, float(dist[np.abs(w) <= c1].min()))
+            hits.extend(zip(c1[ok], w[ok]))
+    blocks = []
+    for e in (-6, -2, 0, 3):
+        for c, w in hits:
+            blk = np.zeros(64, np.float32)
+            blk[0], blk[1] = np.ldexp(c, e), np.ldexp(w, e)
+            blocks.append(blk)
+    return np.concatenate(blocks), len(hits), closest
+
+
+@pytest.mark.parametrize("divide_every_weight", [0, 1])
+def test_threshold_band_both_code_searches(divide_every_weight):
+    # weights whose normalised value lies within a few ulps of a decision threshold: the
+    # bin table's x' = w fl(1/c1) is then inside its 4-ulp fallback band, where the exact
+    # quotient decides. Both code searches (table with fallback; a division per weight)
+    # must match the oracle bit for bit, in fp32 and for the closest bf16 pairs.
+    rng = np.random.default_rng(5)
+    w32 = _band_weights_fp32(rng)
+    wb, nhits, closest = _band_weights_bf16()
+    assert nhits >= 10 and closest > 16
+    # the fp32 set really reaches the band: |x' - T| <= |T| 2^-21 for many of its weights
+    c1 = np.repeat(w32.reshape(-1, 64)[:, 0], 64)
+    xa = (w32 * (np.float32(1) / c1)).astype(np.float32)
+    T = oracle.midpoints().astype(np.float32)
+    near = np.min(np.abs(xa[:, None] - T[None, :]) - np.abs(T)[None, :] * np.float32(2.0 ** -21), axis=1) <= 0
+    assert near.sum() > 500
+    q.lib().qlora_nf4_set_code_search(divide_every_weight)
+    try:
+        assert_bit_exact(torch.from_numpy(w32).view(1, -1).cuda())
+        assert_bit_exact(torch.from_numpy(wb).view(1, -1).cuda().to(torch.bfloat16))
+    finally:
+        q.lib().qlora_nf4_set_code_search(0)
