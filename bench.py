@@ -35,7 +35,7 @@ UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # the library's kernels, as named by its launch bookkeeping
 KERNELS = ("k_gemm2sm", "k_dequant", "k_fused_fwd", "k_fused_dgrad", "k_skinny", "k_reduce_xa", "k_reduce_f32",
-           "k_gemv_xa", "k_gemv", "k_gemv_finish", "k_quantize_codes", "k_offset", "k_double_quant")
+           "k_gemv_xa", "k_gemv", "k_gemv_finish", "k_quantize_codes", "k_offset", "k_double_quant", "k_adamw")
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
 # capture of the same kernel and workload; update with the kernel.
 TRAFFIC_BYTES = {"k_gemm2sm": 89358336}
@@ -595,7 +595,51 @@ def run_components(args, peaks, peak_kind, flush):
     out["l70b_layer"] = run_l70b(args, peaks, peak_kind, flush, stream)
     out["merge_4096"] = run_merge(hbm, flush, stream)
     out["fmt4"] = run_fmt4(hbm, flush, stream)
+    out["adamw"] = run_adamw(hbm, flush, stream)
     return out
+
+
+def run_adamw(hbm, flush, stream, layers=80):
+    """The adapter's optimizer step (AdamW, fp32 state) over the adapters of 80 70B-like
+    layers (r = 64 on all seven projections: 10.35 M parameters a layer), in device memory
+    and in managed memory brought to the GPU beforehand; 30 bytes per parameter."""
+    import numpy as np
+    import torch
+    import bit_nf4_quantized_double_b200 as q
+    import oracle
+    import synth_inputs as si
+    wl = si.workload("l70b")
+    per_layer = sum(L.r * (L.d_in + L.d_out) for L in wl.layers)
+    n = per_layer * layers
+    res = {"workload": f"AdamW step over the r=64 adapters of {layers} 70B-like layers ({n} fp32 parameters), "
+                       "CUDA graph replay", "params": n, "bytes_per_param": 30}
+    g = torch.randn(n, device="cuda") * 1e-3
+    for kind in ("device", "managed"):
+        if kind == "device":
+            theta, m, v = torch.zeros(n, device="cuda"), torch.zeros(n, device="cuda"), torch.zeros(n, device="cuda")
+            tb = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        else:
+            theta, m, v, tb = q.managed_empty(n), q.managed_empty(n), q.managed_empty(n), q.managed_empty(n, torch.bfloat16)
+            for x in (theta, m, v):
+                x.zero_()
+            for x in (theta, m, v, tb):
+                q.qlora_adamw_prefetch(x, to_device=True)
+        ms = _time_graph(lambda: q.qlora_adamw_step(theta, g, m, v, 1, 1e-3, theta_bf16=tb), 5, flush, stream)
+        gbs = n * 30 / (ms / 1e3) / 1e9
+        res[kind] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4)}
+        del theta, m, v, tb
+        torch.cuda.empty_cache()
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    del g
+    torch.cuda.empty_cache()
+    rng = np.random.default_rng(0)
+    th = rng.normal(0, 0.02, per_layer).astype(np.float32)
+    gg = rng.normal(0, 1e-3, per_layer).astype(np.float32)
+    mm, vv = np.zeros(per_layer, np.float32), np.zeros(per_layer, np.float32)
+    t_c, reps = _host_time(lambda: oracle.adamw_step(th, gg, mm, vv, 1, 1e-3, want_bf16=True))
+    res["cpu_baseline"] = {"value": round(per_layer * 30 / t_c / 1e9, 3), "unit": "GB/s", "cores": _cores(),
+                           "kind": "oracle", "sample": f"one layer's adapters ({per_layer} parameters), {reps} calls"}
+    return res
 
 
 def run_fmt4(hbm, flush, stream):

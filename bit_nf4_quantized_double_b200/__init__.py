@@ -80,6 +80,9 @@ _SIGS = {
     "qlora_nf4_dequant_grouped": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(_Tensor),
                                                  ctypes.POINTER(ctypes.c_void_p), ctypes.c_void_p]),
     "qlora_nf4_set_code_search": (None, [ctypes.c_int]),
+    "qlora_adamw_step": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_adamw_prefetch": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]),
     "qlora_get_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_nf4_codebook": (None, [ctypes.c_void_p]),
@@ -256,6 +259,69 @@ def qlora_nf4_dequant_grouped(qs, outs=None, stream=None):
     ptrs = (ctypes.c_void_p * n)(*[o.data_ptr() for o in outs])
     _check(lib().qlora_nf4_dequant_grouped(n, ts, ptrs, _stream(stream)), "qlora_nf4_dequant_grouped")
     return outs
+
+
+class AdamwHparams(ctypes.Structure):
+    """qlora_adamw_hparams of the C ABI."""
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+                ("weight_decay", ctypes.c_float), ("step", ctypes.c_int64)]
+
+
+def qlora_adamw_step(theta: torch.Tensor, grad: torch.Tensor, m: torch.Tensor, v: torch.Tensor, step: int,
+                     lr: float, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+                     weight_decay: float = 0.0, theta_bf16: torch.Tensor | None = None, stream=None):
+    """One AdamW step in place on fp32 CUDA (or managed) tensors theta, m, v with gradient grad;
+    theta_bf16, when given, receives bf16(theta)."""
+    n = theta.numel()
+    for t in (grad, m, v):
+        assert t.numel() == n and t.dtype == torch.float32 and t.is_contiguous()
+    h = AdamwHparams(lr, beta1, beta2, eps, weight_decay, int(step))
+    _check(lib().qlora_adamw_step(_ptr(theta), _ptr(grad), _ptr(m), _ptr(v), n, ctypes.byref(h), _ptr(theta_bf16),
+                                  _stream(stream)), "qlora_adamw_step")
+
+
+def qlora_adamw_prefetch(t: torch.Tensor, to_device: bool = True, stream=None):
+    """Move the managed pages of tensor t to the current GPU (or back to host memory)."""
+    _check(lib().qlora_adamw_prefetch(_ptr(t), t.numel() * t.element_size(), 1 if to_device else 0, _stream(stream)),
+           "qlora_adamw_prefetch")
+
+
+class _Managed:
+    """A block of CUDA managed (unified) memory exposed to torch through the CUDA array
+    interface, freed when the last tensor viewing it is gone. Plumbing for paged optimizer
+    state; the library itself never allocates."""
+    _cudart = None
+
+    def __init__(self, nbytes: int):
+        if _Managed._cudart is None:
+            torch.cuda.init()
+            _Managed._cudart = ctypes.CDLL("libcudart.so.12")
+        p = ctypes.c_void_p()
+        if _Managed._cudart.cudaMallocManaged(ctypes.byref(p), ctypes.c_size_t(max(nbytes, 16)), 1) != 0:
+            raise MemoryError("cudaMallocManaged failed")
+        self.ptr, self.nbytes = p.value, nbytes
+
+    def __del__(self):
+        if self.ptr and _Managed._cudart is not None:
+            _Managed._cudart.cudaFree(ctypes.c_void_p(self.ptr))
+            self.ptr = None
+
+
+def managed_empty(n: int, dtype=torch.float32) -> torch.Tensor:
+    """A 1-D tensor of n elements in CUDA managed memory (pages move between host and GPU on
+    demand, or by qlora_adamw_prefetch)."""
+    esz = torch.empty(0, dtype=dtype).element_size()
+    blk = _Managed(n * esz)
+    typestr = {torch.float32: "<f4", torch.bfloat16: "<V2", torch.int8: "|i1", torch.uint8: "|u1"}[dtype]
+
+    class _View:
+        __cuda_array_interface__ = {"shape": (n,), "typestr": typestr if dtype != torch.bfloat16 else "<i2",
+                                    "data": (blk.ptr, False), "version": 2}
+    t = torch.as_tensor(_View(), device="cuda")
+    if dtype == torch.bfloat16:
+        t = t.view(torch.bfloat16)
+    t._qlora_managed = blk            # the memory lives as long as the tensor
+    return t
 
 
 FMT4 = {"int4": 0, "fp4_e2m1": 1, "fp4_e3m0": 2}

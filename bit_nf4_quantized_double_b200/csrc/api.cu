@@ -285,6 +285,23 @@ qlora_status qlora_linear_bwd(const void *X, const void *dY, int64_t M, const ql
                                        ws, static_cast<cudaStream_t>(stream)));
 }
 
+qlora_status qlora_adamw_step(float *theta, const float *grad, float *m, float *v, int64_t n,
+                              const qlora_adamw_hparams *h, void *theta_bf16, qlora_stream_t stream) {
+    if (!theta || !grad || !m || !v || !h || !aligned16(theta) || !aligned16(grad) || !aligned16(m) || !aligned16(v) ||
+        (theta_bf16 && !aligned16(theta_bf16)) || n < 1)
+        return QLORA_ERR_INVALID_ARG;
+    if (h->step < 1 || !std::isfinite(h->lr) || !std::isfinite(h->eps) || !std::isfinite(h->weight_decay) ||
+        !(h->beta1 >= 0.0f && h->beta1 < 1.0f) || !(h->beta2 >= 0.0f && h->beta2 < 1.0f) || h->eps < 0.0f)
+        return QLORA_ERR_INVALID_ARG;
+    return from_cuda(launch_adamw(theta, grad, m, v, n, h->lr, h->beta1, h->beta2, h->eps, h->weight_decay, h->step,
+                                  static_cast<__nv_bfloat16 *>(theta_bf16), static_cast<cudaStream_t>(stream)));
+}
+
+qlora_status qlora_adamw_prefetch(const void *ptr, size_t bytes, int to_device, qlora_stream_t stream) {
+    if (!ptr || bytes == 0) return QLORA_ERR_INVALID_ARG;
+    return from_cuda(launch_prefetch(ptr, bytes, to_device != 0, static_cast<cudaStream_t>(stream)));
+}
+
 static bool fmt4_ok(qlora_fmt4 f) {
     return f == QLORA_FMT4_INT4 || f == QLORA_FMT4_FP4_E2M1 || f == QLORA_FMT4_FP4_E3M0;
 }

@@ -205,7 +205,7 @@ k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
 
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem = align1024(smem_raw);
     uint8_t *xs = smem;
     uint8_t *cs = xs + SX * kTokStage;
     uint8_t *staging = cs + SC * kCodeStage;
@@ -475,7 +475,7 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
 
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem = align1024(smem_raw);
     uint8_t *as = smem;
     uint8_t *bs = as + SA * kAStage;
     uint8_t *cs = bs + SX * kTokStage;
@@ -742,7 +742,7 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
     __shared__ __align__(8) uint64_t bars[2 * 8 + 2];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem = align1024(smem_raw);
     const int S = p.stages;
     const int a_bytes = 128 * 128;
     const int b_chunks = B_MN ? (p.BN + 63) / 64 : 1;
@@ -993,8 +993,18 @@ static size_t fwd_adapter_bytes(int64_t M, int64_t cols, int r) {
     return r == 0 ? 0 : mr_bytes(M, r) + partial_bytes(M, cols, r);
 }
 
+// CTA pairs of the pair GEMM: every SM, except beside a concurrent side-stream job, where
+// the GEMM takes as few pairs as give the same number of tile rounds and leaves the rest.
+static int side_job_pairs(int64_t M, int64_t N) {
+    const int64_t ntiles = ceil_div(M, 256) * ceil_div(N, 256);
+    const int max_pairs = gemm2sm_pairs(0);
+    const int64_t rounds = ceil_div(ntiles, max_pairs);
+    return (int)ceil_div(ntiles, rounds);
+}
+static size_t g2_bytes() { return gemm2sm_workspace_bytes(gemm2sm_pairs(0)); }
+
 size_t fwd_workspace_bytes_large(int64_t M, int64_t rows, int64_t cols, int r) {
-    return fwd_adapter_bytes(M, cols, r) + (M >= kPairGemmMinM ? wd_bytes(rows, cols) : 0);
+    return fwd_adapter_bytes(M, cols, r) + (M >= kPairGemmMinM ? wd_bytes(rows, cols) + g2_bytes() : 0);
 }
 
 static size_t bwd_adapter_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
@@ -1010,7 +1020,7 @@ static size_t bwd_adapter_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
 }
 
 size_t bwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
-    return bwd_adapter_bytes(M, rows, cols, r) + (M >= kPairGemmMinM ? wd_bytes(rows, cols) : 0);
+    return bwd_adapter_bytes(M, rows, cols, r) + (M >= kPairGemmMinM ? wd_bytes(rows, cols) + g2_bytes() : 0);
 }
 
 static cudaError_t run_fused_fwd(const __nv_bfloat16 *X, int64_t M, const NF4View &W, const __nv_bfloat16 *XAs,
@@ -1137,7 +1147,8 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
         } else if ((e = launch_dequant(W, Wd, st)) != cudaSuccess) {
             return e;
         }
-        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, st);
+        void *g2ws = reinterpret_cast<char *>(Wd) + wd_bytes(W.rows, W.cols);
+        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, gemm2sm_pairs(0), g2ws, st);
     }
     return run_fused_fwd(X, M, W, XAs, B, r, Y, st);
 }
@@ -1212,7 +1223,8 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
             if (side) {
                 float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + 2 * mr_bytes(M, r));
                 if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
-                e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, st);
+                e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, side_job_pairs(M, W.cols),
+                                   reinterpret_cast<char *>(Wd) + wd_bytes(W.rows, W.cols), st);
                 if (e != cudaSuccess) return e;
                 if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
                 e = adapter_grads(X, dY, M, W, Gs, XA, r, s, dA, dB, part, side->s);
@@ -1221,7 +1233,8 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
                 return cudaStreamWaitEvent(st, side->join, 0);
             }
         }
-        e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, st);
+        e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, gemm2sm_pairs(0),
+                           reinterpret_cast<char *>(Wd) + wd_bytes(W.rows, W.cols), st);
     } else {
         e = run_fused_dgrad(dY, M, W, A, Gs, r, dX, st);
     }

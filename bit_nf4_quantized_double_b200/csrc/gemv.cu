@@ -63,7 +63,8 @@ constexpr int kLutRegion = 65536;
 // (9 warps: room for its 64 registers of X fragments).
 __host__ __device__ constexpr int gemv_rg(int nt) { return nt == 1 ? 2 : 1; }
 __host__ __device__ constexpr int gemv_rows(int nt) { return 16 * gemv_rg(nt); }
-__host__ __device__ constexpr int gemv_threads(int nt) { return 256 * gemv_rg(nt) + 32; }
+constexpr int kGemvProducers = 2;              // producer warps, taking alternate units
+__host__ __device__ constexpr int gemv_threads(int nt) { return 256 * gemv_rg(nt) + 32 * kGemvProducers; }
 __host__ __device__ constexpr int gemv_box_bytes(int nt) { return gemv_rows(nt) * 128; }
 __host__ __device__ constexpr int gemv_stage_bytes(int nt) { return 8 * gemv_box_bytes(nt); }
 __host__ __device__ constexpr int gemv_stages(int nt) { return nt == 1 ? 5 : 10; }
@@ -78,8 +79,7 @@ static_assert(gemv_red_hole0(1) + 32 * gemv_rg(1) * 1 <= 256 && gemv_red_hole0(2
 __device__ __forceinline__ uint32_t hole(int h) { return (uint32_t)h * 256u + 128u; }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -93,21 +93,6 @@ __device__ __forceinline__ uint32_t pack2_bf16(const __nv_bfloat16 *p0, const __
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-    uint2 v;
-    asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ float4 lds128f(uint32_t a) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
-    return v;
-}
 __device__ __forceinline__ void sts128f(uint32_t a, float4 v) {
     asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
 }
@@ -389,13 +374,140 @@ __global__ void __launch_bounds__(kFinishRows) k_gemv_finish(const __grid_consta
         if (m < M) it.Y[(int64_t)m * N + R] = __float2bfloat16_rn(y[m]);
 }
 
+// Compute warps of k_gemv (warp w < 8 RG): row group w / 8, K slice w % 8.
+template <int NT>
+__device__ __forceinline__ void gemv_compute(const GemvGroup &grp, const uint8_t *base, uint32_t full0,
+                                             uint32_t empty0, uint32_t redf0, uint32_t rede0, volatile int *abort,
+                                             int u_begin, int count, int warp, int lane) {
+    constexpr int S = gemv_stages(NT), ROWS = gemv_rows(NT);
+    constexpr int BOX = gemv_box_bytes(NT), STAGE = gemv_stage_bytes(NT);
+    // shared memory is read through ordinary loads, which the compiler may interleave
+    // (they are ordered after the barrier waits, whose asm clobbers memory)
+    const uint8_t *lut = base;
+    const uint8_t *stages = base + kLutRegion;
+    auto ld32 = [&](uint32_t off) { return *reinterpret_cast<const uint32_t *>(lut + off); };
+    auto ld128 = [&](uint32_t off) { return *reinterpret_cast<const float4 *>(lut + off); };
+    const int rg = warp >> 3, ks = warp & 7, g = lane >> 2, t = lane & 3;
+    const uint32_t lane4 = lane * 4;
+    // this lane's 8-byte code words of rows rg*16 + g and + 8 in box ks: chunk (2b + t/2) ^ g
+    const uint32_t box_row0 = ks * BOX + (rg * 16 + g) * 128 + (t & 1) * 8;
+    const uint32_t box_row1 = box_row0 + 8 * 128;
+    const uint32_t red_mine = hole(gemv_red_hole0(NT) + (rg * 8 + ks) * NT * 4 + (lane >> 3)) + (lane & 7) * 16;
+    bool ok = true;
+
+    uint32_t xf[NT][4][8];
+    UnitPos pos = unit_pos(grp, u_begin);
+    int xkey = -1, nblk = 0;
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+
+    for (int i = 0; i < count && ok; ++i) {
+        const int s = i % S, n = i / S;
+        const GemvItem &it = grp.it[pos.item];
+        const int key = pos.item * 4096 + pos.ch;
+        if (key != xkey) {
+            x_load<NT>(grp, pos, ks, lane, xf);
+            xkey = key;
+            const int sl0 = chunk_slice0(pos.ch, it.sq, it.srem);
+            const int kslice = (sl0 + ks) * kGemvSlice;
+            nblk = ks < it.sq + (pos.ch < it.srem ? 1 : 0) ? min(4, (it.K - kslice) / 64) : 0;
+        }
+        if (!mbar_wait(full0 + 8 * s, n & 1, abort)) { ok = false; break; }
+        if (nblk > 0) {
+            const float4 c0 = ld128(hole(s * ROWS + rg * 16 + g) + ((ks ^ g) << 4));
+            const float4 c1 = ld128(hole(s * ROWS + rg * 16 + g + 8) + ((ks ^ g) << 4));
+            const float ch0[4] = {c0.x, c0.y, c0.z, c0.w}, ch1[4] = {c1.x, c1.y, c1.z, c1.w};
+            const uint8_t *sb = stages + s * STAGE;
+            // one 64-block: 16 table lookups, 4 NT MMAs, the block's c^ on the partial sums
+            auto block = [&](int b) {
+                const uint32_t off = (uint32_t)(((2 * b + (t >> 1)) ^ g) << 4);
+                const uint2 w0 = *reinterpret_cast<const uint2 *>(sb + box_row0 + off);
+                const uint2 w1 = *reinterpret_cast<const uint2 *>(sb + box_row1 + off);
+                float cbk[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) cbk[nt][0] = cbk[nt][1] = cbk[nt][2] = cbk[nt][3] = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t r0 = (j < 2) ? w0.x : w0.y;
+                    const uint32_t r1 = (j < 2) ? w1.x : w1.y;
+                    // byte k of the word, times 256, plus lane * 4: one permute
+                    const uint32_t slo = 0x5504u | ((uint32_t)(2 * (j & 1)) << 4), shi = slo + 0x10u;
+                    uint32_t a[4];
+                    a[0] = ld32(prmt(r0, lane4, slo));
+                    a[2] = ld32(prmt(r0, lane4, shi));
+                    a[1] = ld32(prmt(r1, lane4, slo));
+                    a[3] = ld32(prmt(r1, lane4, shi));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(cbk[nt], a, xf[nt][b][2 * j], xf[nt][b][2 * j + 1]);
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    acc[nt][0] = fmaf(ch0[b], cbk[nt][0], acc[nt][0]);
+                    acc[nt][1] = fmaf(ch0[b], cbk[nt][1], acc[nt][1]);
+                    acc[nt][2] = fmaf(ch1[b], cbk[nt][2], acc[nt][2]);
+                    acc[nt][3] = fmaf(ch1[b], cbk[nt][3], acc[nt][3]);
+                }
+            };
+            if (nblk == 4) {
+#pragma unroll
+                for (int b = 0; b < 4; ++b) block(b);
+            } else {
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    if (b < nblk) block(b);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * s);
+
+        // ---------------- the row group's eight slices: written, then summed by warp ks == i % 8
+        if (i > 0 && !mbar_wait(rede0 + 8 * rg, (i - 1) & 1, abort)) { ok = false; break; }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            *reinterpret_cast<float4 *>(const_cast<uint8_t *>(lut) + red_mine + nt * 4 * 256) =
+                make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
+            acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(redf0 + 8 * rg);
+        if (ks == (i & 7)) {
+            if (!mbar_wait(redf0 + 8 * rg, i & 1, abort)) { ok = false; break; }
+            float sum[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                sum[nt][0] = sum[nt][1] = sum[nt][2] = sum[nt][3] = 0.0f;
+#pragma unroll
+                for (int k2 = 0; k2 < 8; ++k2) {
+                    const float4 v =
+                        ld128(hole(gemv_red_hole0(NT) + ((rg * 8 + k2) * NT + nt) * 4 + (lane >> 3)) + (lane & 7) * 16);
+                    sum[nt][0] += v.x; sum[nt][1] += v.y; sum[nt][2] += v.z; sum[nt][3] += v.w;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(rede0 + 8 * rg);
+            const int M = grp.M, N = it.N;
+            const int R0 = pos.rb * ROWS + rg * 16 + g;
+            float *pp = it.partial + (int64_t)pos.ch * N * M;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int tok = nt * 8 + 2 * t + (q & 1), R = R0 + (q >= 2 ? 8 : 0);
+                    if (tok < M && R < N) pp[(int64_t)R * M + tok] = sum[nt][q];
+                }
+        }
+        pos = unit_next(grp, pos);
+    }
+}
+
 template <int NT>
 __global__ void __launch_bounds__(gemv_threads(NT), 1)
 k_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ Codebook cb) {
     constexpr int S = gemv_stages(NT), RG = gemv_rg(NT), ROWS = gemv_rows(NT);
     constexpr int BOX = gemv_box_bytes(NT), STAGE = gemv_stage_bytes(NT);
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *base = align1024(smem_raw);
     const uint32_t lut = smem_addr(base);
     const uint32_t stages = lut + kLutRegion;
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + kLutRegion + S * STAGE);
@@ -430,25 +542,36 @@ k_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ Codebook c
     const int count = grp.ustart[blockIdx.x + 1] - u_begin;
     if (count <= 0) return;
 
-    if (warp == 8 * RG) {
-        // ---------------- producer: TMA of the codes, c^ of every row into the stage's holes.
-        // The int8 constants of unit i are fetched while units i-3 .. i-1 are produced, into
-        // a ring of four register sets that the unrolled loop names statically (copying a
-        // set whose loads are in flight would wait for them).
+    if (warp >= 8 * RG) {
+        // ---------------- producers: TMA of the codes, c^ of every row into the stage's holes.
+        // Producer w takes units w, w + 2, ... of the CTA's range. The int8 constants of a unit
+        // are fetched while its three predecessors of the same producer are produced, into a
+        // ring of four register sets that the unrolled loop names statically (copying a set
+        // whose loads are in flight would wait for them).
+        const int pw = warp - 8 * RG;
         int last = -1;
-        UnitPos p = unit_pos(grp, u_begin), pf = p;
+        UnitPos p = unit_pos(grp, u_begin);
+        if (pw < count) {
+            for (int j = 0; j < pw; ++j) p = unit_next(grp, p);
+        }
+        UnitPos pf = p;
+        auto advance = [&](UnitPos x) {
+#pragma unroll
+            for (int j = 0; j < kGemvProducers; ++j) x = unit_next(grp, x);
+            return x;
+        };
         Q8Row qa, qb, qc, qd;
-        q8_fetch<ROWS>(grp, pf, lane, qa);
-        pf = unit_next(grp, pf);
-        if (count > 1) q8_fetch<ROWS>(grp, pf, lane, qb);
-        pf = unit_next(grp, pf);
-        if (count > 2) q8_fetch<ROWS>(grp, pf, lane, qc);
-        pf = unit_next(grp, pf);
-        // produce unit i from `cur`; fetch unit i + 3 into `nxt` (the set unit i - 1 used)
+        if (pw < count) q8_fetch<ROWS>(grp, pf, lane, qa);
+        pf = advance(pf);
+        if (pw + kGemvProducers < count) q8_fetch<ROWS>(grp, pf, lane, qb);
+        pf = advance(pf);
+        if (pw + 2 * kGemvProducers < count) q8_fetch<ROWS>(grp, pf, lane, qc);
+        pf = advance(pf);
+        // produce unit i from `cur`; fetch unit i + 3 producer strides on into `nxt`
         auto step = [&](int i, const Q8Row &cur, Q8Row &nxt) -> bool {
             if (i >= count) return false;
-            if (i + 3 < count) q8_fetch<ROWS>(grp, pf, lane, nxt);
-            pf = unit_next(grp, pf);
+            if (i + 3 * kGemvProducers < count) q8_fetch<ROWS>(grp, pf, lane, nxt);
+            pf = advance(pf);
             const int s = i % S, n = i / S;
             if (!mbar_wait(empty0 + 8 * s, (n & 1) ^ 1, abort)) return false;
             const GemvItem &it = grp.it[p.item];
@@ -469,134 +592,39 @@ k_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ Codebook c
             chat_store<ROWS>(lut, s, lane, cur);
             mbar_arrive(full0 + 8 * s);
             last = i;
-            p = unit_next(grp, p);
+            p = advance(p);
             return true;
         };
-        for (int i = 0; i < count; i += 4) {
+        constexpr int P = kGemvProducers;
+        for (int i = pw; i < count; i += 4 * P) {
             if (!step(i, qa, qd)) break;
-            if (!step(i + 1, qb, qa)) break;
-            if (!step(i + 2, qc, qb)) break;
-            if (!step(i + 3, qd, qc)) break;
+            if (!step(i + P, qb, qa)) break;
+            if (!step(i + 2 * P, qc, qb)) break;
+            if (!step(i + 3 * P, qd, qc)) break;
         }
-        // the CTA does not exit with a copy in flight: wait for the stages issued last
-        if (lane == 0) {
-            const uint64_t t0 = global_timer_ns();
-            for (int j = max(0, last - S + 1); j <= last; ++j)
-                while (!mbar_try_wait(full0 + 8 * (j % S), (j / S) & 1))
-                    if (global_timer_ns() - t0 > kWaitLimitNs) {
-                        raise_status(QLORA_ERR_TIMEOUT);
-                        j = last;
-                        break;
-                    }
-        }
-        return;
+        if (lane == 0) flags[1 + pw] = last;           // the last unit this producer issued
+    } else {
+        gemv_compute<NT>(grp, base, full0, empty0, redf0, rede0, abort, u_begin, count, warp, lane);
     }
-
-    // ---------------- compute warps
-    const int rg = warp >> 3, ks = warp & 7, g = lane >> 2, t = lane & 3;
-    const uint32_t lane4 = lane * 4;
-    // this lane's 8-byte code words of rows rg*16 + g and + 8 in box ks: chunk (2b + t/2) ^ g
-    const uint32_t box_row0 = ks * BOX + (rg * 16 + g) * 128 + (t & 1) * 8;
-    const uint32_t box_row1 = box_row0 + 8 * 128;
-    const uint32_t red_mine = lut + hole(gemv_red_hole0(NT) + (rg * 8 + ks) * NT * 4 + (lane >> 3)) + (lane & 7) * 16;
-    bool ok = true;
-
-    uint32_t xf[NT][4][8];
-    UnitPos pos = unit_pos(grp, u_begin);
-    int xkey = -1, nblk = 0;
-    float acc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
-
-    for (int i = 0; i < count && ok; ++i) {
-        const int s = i % S, n = i / S;
-        const GemvItem &it = grp.it[pos.item];
-        const int key = pos.item * 4096 + pos.ch;
-        if (key != xkey) {
-            x_load<NT>(grp, pos, ks, lane, xf);
-            xkey = key;
-            const int sl0 = chunk_slice0(pos.ch, it.sq, it.srem);
-            const int kslice = (sl0 + ks) * kGemvSlice;
-            nblk = ks < it.sq + (pos.ch < it.srem ? 1 : 0) ? min(4, (it.K - kslice) / 64) : 0;
-        }
-        if (!mbar_wait(full0 + 8 * s, n & 1, abort)) { ok = false; break; }
-        if (nblk > 0) {
-            const float4 c0 = lds128f(lut + hole(s * ROWS + rg * 16 + g) + ((ks ^ g) << 4));
-            const float4 c1 = lds128f(lut + hole(s * ROWS + rg * 16 + g + 8) + ((ks ^ g) << 4));
-            const float ch0[4] = {c0.x, c0.y, c0.z, c0.w}, ch1[4] = {c1.x, c1.y, c1.z, c1.w};
-            const uint32_t sb = stages + s * STAGE;
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                if (b >= nblk) break;
-                const uint32_t off = (uint32_t)(((2 * b + (t >> 1)) ^ g) << 4);
-                const uint2 w0 = lds64(sb + box_row0 + off);
-                const uint2 w1 = lds64(sb + box_row1 + off);
-                float cbk[NT][4];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) cbk[nt][0] = cbk[nt][1] = cbk[nt][2] = cbk[nt][3] = 0.0f;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t r0 = (j < 2) ? w0.x : w0.y;
-                    const uint32_t r1 = (j < 2) ? w1.x : w1.y;
-                    // byte k of the word, times 256, plus lane * 4: one permute
-                    const uint32_t slo = 0x5504u | ((uint32_t)(2 * (j & 1)) << 4), shi = slo + 0x10u;
-                    uint32_t a[4];
-                    a[0] = lds32(lut + prmt(r0, lane4, slo));
-                    a[2] = lds32(lut + prmt(r0, lane4, shi));
-                    a[1] = lds32(lut + prmt(r1, lane4, slo));
-                    a[3] = lds32(lut + prmt(r1, lane4, shi));
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(cbk[nt], a, xf[nt][b][2 * j], xf[nt][b][2 * j + 1]);
-                }
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    acc[nt][0] = fmaf(ch0[b], cbk[nt][0], acc[nt][0]);
-                    acc[nt][1] = fmaf(ch0[b], cbk[nt][1], acc[nt][1]);
-                    acc[nt][2] = fmaf(ch1[b], cbk[nt][2], acc[nt][2]);
-                    acc[nt][3] = fmaf(ch1[b], cbk[nt][3], acc[nt][3]);
-                }
+    // The CTA does not exit with a copy in flight: once every role is done, wait for the last
+    // unit issued on each stage (no later unit reuses a stage, so its phase is the stage's last).
+    __syncthreads();
+    if (tid == 0) {
+        const uint64_t t0 = global_timer_ns();
+        for (int s = 0; s < S; ++s) {
+            int u = -1;
+            for (int pw = 0; pw < kGemvProducers; ++pw) {
+                const int lastp = flags[1 + pw];
+                for (int i = lastp; i >= 0 && i > lastp - S * kGemvProducers; i -= kGemvProducers)
+                    if (i % S == s) { u = max(u, i); break; }
             }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + 8 * s);
-
-        // ---------------- the row group's eight slices: written, then summed by warp ks == i % 8
-        if (i > 0 && !mbar_wait(rede0 + 8 * rg, (i - 1) & 1, abort)) { ok = false; break; }
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            sts128f(red_mine + nt * 4 * 256, make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]));
-            acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(redf0 + 8 * rg);
-        if (ks == (i & 7)) {
-            if (!mbar_wait(redf0 + 8 * rg, i & 1, abort)) { ok = false; break; }
-            float sum[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                sum[nt][0] = sum[nt][1] = sum[nt][2] = sum[nt][3] = 0.0f;
-#pragma unroll
-                for (int k2 = 0; k2 < 8; ++k2) {
-                    const float4 v =
-                        lds128f(lut + hole(gemv_red_hole0(NT) + ((rg * 8 + k2) * NT + nt) * 4 + (lane >> 3)) +
-                               (lane & 7) * 16);
-                    sum[nt][0] += v.x; sum[nt][1] += v.y; sum[nt][2] += v.z; sum[nt][3] += v.w;
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(rede0 + 8 * rg);
-            const int M = grp.M, N = it.N;
-            const int R0 = pos.rb * ROWS + rg * 16 + g;
-            float *pp = it.partial + (int64_t)pos.ch * N * M;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int tok = nt * 8 + 2 * t + (q & 1), R = R0 + (q >= 2 ? 8 : 0);
-                    if (tok < M && R < N) pp[(int64_t)R * M + tok] = sum[nt][q];
+            if (u < 0) continue;
+            while (!mbar_try_wait(full0 + 8 * s, (u / S) & 1))
+                if (global_timer_ns() - t0 > kWaitLimitNs) {
+                    raise_status(QLORA_ERR_TIMEOUT);
+                    return;
                 }
         }
-        pos = unit_next(grp, pos);
     }
 }
 

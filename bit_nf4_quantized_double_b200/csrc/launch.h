@@ -22,13 +22,18 @@ cudaError_t launch_fmt4_quantize(const void *W, qlora_dtype dt, int64_t n, qlora
                                  float *absmax, cudaStream_t st);
 cudaError_t launch_fmt4_dequant(const uint8_t *codes, const float *absmax, int64_t n, qlora_fmt4 f,
                                 __nv_bfloat16 *out, cudaStream_t st);
+cudaError_t launch_adamw(float *theta, const float *g, float *m, float *v, int64_t n, float lr, float b1, float b2,
+                         float eps, float wd, int64_t step, __nv_bfloat16 *out_bf16, cudaStream_t st);
+cudaError_t launch_prefetch(const void *ptr, size_t bytes, bool to_device, cudaStream_t st);
 cudaError_t launch_merge_bf16(const NF4View &q, const __nv_bfloat16 *A, const __nv_bfloat16 *B, int r, float s,
                               __nv_bfloat16 *out, cudaStream_t st);
 
-// Plain bf16 GEMM on CTA pairs (tcgen05 cta_group::2), see gemm2sm.cu.
+// Plain bf16 GEMM on CTA pairs (tcgen05 cta_group::2, stream-K), see gemm2sm.cu.
+size_t gemm2sm_workspace_bytes(int pairs);
+int gemm2sm_pairs(int max_pairs);
 cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, const __nv_bfloat16 *B, bool b_mn,
                            const __nv_bfloat16 *Be, bool be_mn, __nv_bfloat16 *C, int64_t M, int64_t N, int64_t K,
-                           int ke, cudaStream_t st);
+                           int ke, int pairs, void *ws, cudaStream_t st);
 
 size_t fwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r);
 

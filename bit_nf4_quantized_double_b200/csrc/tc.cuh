@@ -16,6 +16,14 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte-aligned byte of a shared-memory array, reached by pointer
+// arithmetic on the array itself: the compiler then still knows the result points
+// into shared memory, so loads and stores through it stay shared-memory accesses
+// (a round trip through an integer would turn them into generic ones).
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return p + ((1024u - (smem_addr(p) & 1023u)) & 1023u);
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

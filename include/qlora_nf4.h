@@ -230,6 +230,38 @@ qlora_status qlora_nf4_quantize_noalloc(const void *W, qlora_dtype dt, const qlo
                                         qlora_stream_t stream);
 
 /*
+ * Optimizer step of the adapter (the page's section 3 procedure ends every batch with
+ * "update LoRA with a paged optimizer"; section 2: a paged optimizer keeps its state in
+ * unified memory that moves between GPU and CPU memory when needed). AdamW with
+ * decoupled weight decay on fp32 master parameters theta and fp32 moments m, v, one
+ * step at step count h->step >= 1, per element and in this order, every operation one
+ * IEEE binary32 operation (round to nearest even, no fused multiply-add):
+ *   m = b1 m + (1 - b1) g;  v = b2 v + (1 - b2) g g;
+ *   upd = (m / bc1) / (sqrt(v / bc2) + eps);  theta = theta - lr (upd + wd theta);
+ * bc1 = 1 - b1^step and bc2 = 1 - b2^step are computed in double and rounded to float.
+ *   theta, m, v   n fp32 each, updated in place; grad n fp32 (dA or dB of
+ *                 qlora_linear_bwd, or both laid out back to back);
+ *   theta_bf16    n bf16 receiving bf16(theta), the adapter copy the layer multiplies
+ *                 with, or NULL;
+ * all 16-byte aligned, device or managed (cudaMallocManaged) memory: state kept in
+ * managed memory is paged in by the step itself, or ahead of it by qlora_adamw_prefetch.
+ * One kernel launch; QLORA_ERR_INVALID_ARG for a null or misaligned pointer, n < 1,
+ * step < 1, betas outside [0, 1), a negative eps or a non-finite lr, eps or weight decay.
+ */
+typedef struct {
+    float lr, beta1, beta2, eps, weight_decay;
+    int64_t step;
+} qlora_adamw_hparams;
+qlora_status qlora_adamw_step(float *theta, const float *grad, float *m, float *v, int64_t n,
+                              const qlora_adamw_hparams *h, void *theta_bf16, qlora_stream_t stream);
+
+/* Paging of optimizer state kept in managed memory: asks the driver to move `bytes` at
+ * `ptr` to the current device (to_device != 0), before the step needs them, or back to
+ * host memory (to_device == 0), to give the GPU memory back between steps. Asynchronous
+ * on `stream`. QLORA_ERR_CUDA when ptr is not managed memory or the move is refused. */
+qlora_status qlora_adamw_prefetch(const void *ptr, size_t bytes, int to_device, qlora_stream_t stream);
+
+/*
  * Test hook of the quantiser's code search (the page has no counterpart). By default a
  * weight's code is read from a 256-bin table over x' = w * fl(1/c1), and the exact
  * quotient fl(w / c1) with the full threshold search decides wherever x' lies within

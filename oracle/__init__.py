@@ -80,6 +80,10 @@ def lib() -> ctypes.CDLL:
         L.orc_bf16_rne.argtypes = [ctypes.c_float]
         L.orc_bf16_array_to_f32.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
         L.orc_max_threads.restype = ctypes.c_int
+        L.orc_adamw_step.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_int64] + [ctypes.c_float] * 7 + [ctypes.c_void_p]
+        L.orc_adamw_bias_corrections.argtypes = [ctypes.c_float, ctypes.c_float, ctypes.c_int64,
+                                                 ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]
         del f32p
         _lib = L
     return _lib
@@ -314,3 +318,29 @@ def rel_errors(got, ref):
     fref = float(np.linalg.norm(ref))
     return (float(np.max(np.abs(err))) / mref if mref > 0 else float(np.max(np.abs(err), initial=0.0)),
             float(np.linalg.norm(err)) / fref if fref > 0 else float(np.linalg.norm(err)))
+
+
+# --------------------------------------------------------------------------
+# Paged AdamW of the adapter (section 3: "update LoRA with a paged optimizer";
+# section 2: the optimizer state lives in unified memory). One step on fp32
+# master parameters, fp32 moments; the operation order is in nf4_oracle.c.
+# --------------------------------------------------------------------------
+def adamw_bias_corrections(b1: float, b2: float, t: int):
+    bc1, bc2 = ctypes.c_float(0.0), ctypes.c_float(0.0)
+    lib().orc_adamw_bias_corrections(b1, b2, int(t), ctypes.byref(bc1), ctypes.byref(bc2))
+    return np.float32(bc1.value), np.float32(bc2.value)
+
+
+def adamw_step(theta: np.ndarray, g: np.ndarray, m: np.ndarray, v: np.ndarray, t: int, lr: float,
+               b1: float = 0.9, b2: float = 0.999, eps: float = 1e-8, wd: float = 0.0, want_bf16: bool = False):
+    """One AdamW step in place on fp32 arrays theta, m, v (gradient g). Returns bf16 bits of
+    the new theta when want_bf16, else None."""
+    for a in (theta, g, m, v):
+        assert a.dtype == np.float32 and a.flags["C_CONTIGUOUS"]
+    n = theta.size
+    bc1, bc2 = adamw_bias_corrections(b1, b2, t)
+    out = np.empty(n, dtype=np.uint16) if want_bf16 else None
+    lib().orc_adamw_step(_ptr(theta), _ptr(g), _ptr(m), _ptr(v), n, lr, b1, b2, eps, wd, float(bc1), float(bc2),
+                         _ptr(out) if want_bf16 else None)
+    return out
+

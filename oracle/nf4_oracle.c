@@ -352,3 +352,48 @@ void orc_merge_bf16(const uint16_t *w_hat, const float *A, const float *B, int64
         }
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Optimizer step of the adapter (the page's section 3 procedure ends every   */
+/* batch with "update LoRA with a paged optimizer"; section 2 says paged      */
+/* optimizers keep their state in unified memory that moves between GPU and  */
+/* CPU when needed). The optimizer is AdamW (decoupled weight decay) on fp32  */
+/* master parameters theta with fp32 moments m, v. Reading: one step at       */
+/* step count t >= 1 is, per element and in this order, every operation one   */
+/* IEEE binary32 operation:                                                   */
+/*   m     = fl( fl(b1 * m) + fl(fl(1 - b1) * g) )                            */
+/*   v     = fl( fl(b2 * v) + fl(fl(1 - b2) * fl(g * g)) )                    */
+/*   mhat  = fl(m / bc1),  vhat = fl(v / bc2)                                 */
+/*   upd   = fl( mhat / fl(fl(sqrt(vhat)) + eps) )                            */
+/*   theta = fl( theta - fl(lr * fl(upd + fl(wd * theta))) )                  */
+/* with the bias corrections bc1 = (float)(1 - b1^t), bc2 = (float)(1 - b2^t) */
+/* computed in double by the caller. theta_bf16 (optional) receives           */
+/* bf16(theta), the adapter copy the layer multiplies with.                   */
+void orc_adamw_step(float *theta, const float *g, float *m, float *v, int64_t n, float lr, float b1,
+                    float b2, float eps, float wd, float bc1, float bc2, uint16_t *theta_bf16)
+{
+    const float c1 = 1.0f - b1, c2 = 1.0f - b2;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        const float gi = g[i];
+        const float mi = b1 * m[i] + c1 * gi;
+        const float gg = gi * gi;
+        const float vi = b2 * v[i] + c2 * gg;
+        const float mhat = mi / bc1, vhat = vi / bc2;
+        const float den = sqrtf(vhat) + eps;
+        const float upd = mhat / den;
+        const float decay = wd * theta[i];
+        const float step = lr * (upd + decay);
+        theta[i] = theta[i] - step;
+        m[i] = mi;
+        v[i] = vi;
+        if (theta_bf16) theta_bf16[i] = orc_bf16_rne(theta[i]);
+    }
+}
+
+/* Bias corrections of step t (double, rounded once to float). */
+void orc_adamw_bias_corrections(float b1, float b2, int64_t t, float *bc1, float *bc2)
+{
+    *bc1 = (float)(1.0 - pow((double)b1, (double)t));
+    *bc2 = (float)(1.0 - pow((double)b2, (double)t));
+}

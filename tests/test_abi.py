@@ -65,9 +65,12 @@ def test_workspace_queries_positive():
         assert L.qlora_linear_bwd_workspace(M, 4096, 4096, 64) > 0
     # no adapter and a small batch: nothing to stage
     assert L.qlora_linear_bwd_workspace(256, 4096, 4096, 0) == 0
-    # from 512 tokens on, the layer keeps a bf16 copy of the dequantised weight
-    assert L.qlora_linear_bwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2
-    assert L.qlora_linear_fwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2
+    # from 512 tokens on, the layer keeps a bf16 copy of the dequantised weight, plus the
+    # pair GEMM's stream-K partials (one 256 x 256 fp32 tile per CTA pair, 74 pairs on 148
+    # SMs, the count assumed without a GPU) and their flags
+    g2 = 74 * 256 * 256 * 4 + 768
+    assert L.qlora_linear_bwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2 + g2
+    assert L.qlora_linear_fwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2 + g2
 
 
 def test_grouped_forward_host_checks():
@@ -155,3 +158,19 @@ def test_grouped_workspace_is_largest_group_of_eight():
         assert whole == max(parts)
         one = (q._LinearDesc * 1)(descs[0])
         assert L.qlora_linear_fwd_grouped_workspace(M, 1, one) == L.qlora_linear_fwd_workspace(M, 4096, 4096, 16)
+
+
+def test_adamw_host_checks():
+    # the optimizer step's argument checks run on the host (no GPU needed)
+    L = q.lib()
+    fake = 1 << 20
+    h = q.AdamwHparams(1e-3, 0.9, 0.999, 1e-8, 0.0, 1)
+    p = ctypes.c_void_p(fake)
+    assert L.qlora_adamw_step(None, p, p, p, 16, ctypes.byref(h), None, None) == q.QLORA_ERR_INVALID_ARG
+    assert L.qlora_adamw_step(p, p, p, ctypes.c_void_p(fake + 4), 16, ctypes.byref(h), None, None) == \
+        q.QLORA_ERR_INVALID_ARG
+    assert L.qlora_adamw_step(p, p, p, p, 0, ctypes.byref(h), None, None) == q.QLORA_ERR_INVALID_ARG
+    for bad in (q.AdamwHparams(1e-3, 0.9, 0.999, 1e-8, 0.0, 0), q.AdamwHparams(1e-3, 1.0, 0.999, 1e-8, 0.0, 1),
+                q.AdamwHparams(float("nan"), 0.9, 0.999, 1e-8, 0.0, 1), q.AdamwHparams(1e-3, 0.9, 0.999, -1.0, 0.0, 1)):
+        assert L.qlora_adamw_step(p, p, p, p, 16, ctypes.byref(bad), None, None) == q.QLORA_ERR_INVALID_ARG
+    assert L.qlora_adamw_prefetch(None, 16, 1, None) == q.QLORA_ERR_INVALID_ARG
