@@ -898,6 +898,65 @@ def run_decode_profile(M, reps=3):
     print(json.dumps({"decode_profile": {"M": M, "reps": reps}}), flush=True)
 
 
+def run_profile_case(name, reps=3):
+    """Small cases for ncu captures of one kernel each (a few launches, inputs above the L2
+    size, the L2 flushed before each launch): decode1 / decode16 (the decode block's grouped
+    forward), layer (one Llama-7B layer quantised and dequantised by the grouped calls),
+    adamw (64 M adapter parameters), merge (the 4096^2 adapter merge), fmt4 (the three
+    4-bit reference formats on 2^26 weights), l4096 (one fwd + bwd step of the headline layer)."""
+    import torch
+    import bit_nf4_quantized_double_b200 as q
+    import synth_inputs as si
+    if name.startswith("decode"):
+        run_decode_profile(int(name[len("decode"):]), reps)
+        return
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    if name == "layer":
+        wl = si.workload("llama7b", n_layers=1)
+        Ws = [si.layer_inputs(wl, li, device="cuda")["W"] for li in range(7)]
+        Ts = q.qlora_nf4_quantize_grouped(Ws)
+        outs = [torch.empty(W.shape, dtype=torch.bfloat16, device="cuda") for W in Ws]
+        for _ in range(reps):
+            l2_flush(flush)
+            q.qlora_nf4_quantize_grouped(Ws, outs=Ts)
+            l2_flush(flush)
+            q.qlora_nf4_dequant_grouped(Ts, outs=outs)
+    elif name == "adamw":
+        n = 64 << 20
+        theta, g, m, v = (torch.zeros(n, device="cuda") for _ in range(4))
+        tb = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        for t in range(1, reps + 1):
+            l2_flush(flush)
+            q.qlora_adamw_step(theta, g, m, v, t, 1e-3, theta_bf16=tb)
+    elif name == "merge":
+        wl = si.workload("l4096")
+        L = wl.layers[0]
+        inp = si.layer_inputs(wl, 0, device="cuda")
+        t = q.qlora_nf4_quantize(inp["W"])
+        for _ in range(reps):
+            l2_flush(flush)
+            q.qlora_nf4_merge_adapter(t, inp["A"], inp["B"], L.s)
+    elif name == "fmt4":
+        W = si.normal((1 << 26,), 0.02, seed=77, device="cuda")
+        for fmt in ("int4", "fp4_e2m1", "fp4_e3m0"):
+            l2_flush(flush)
+            codes, absmax = q.qlora_fmt4_quantize(W, fmt)
+            l2_flush(flush)
+            q.qlora_fmt4_dequant(codes, absmax, W.numel(), fmt)
+    elif name == "l4096":
+        wl, L, inp = headline_inputs(0)
+        t = q.qlora_nf4_quantize(inp["W"])
+        for _ in range(reps):
+            l2_flush(flush)
+            Y, XA = q.qlora_linear_fwd(inp["X"], t, inp["A"], inp["B"], L.s)
+            q.qlora_linear_bwd(inp["X"], inp["dY"], t, inp["A"], inp["B"], L.s, XA=XA)
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    torch.cuda.synchronize()
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    print(json.dumps({"profile_case": name, "reps": reps}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -911,7 +970,13 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch every step eagerly instead of replaying a CUDA graph")
     ap.add_argument("--decode-profile", type=int, default=0, metavar="M",
                     help="only run the decode block at M tokens three times (a small case for ncu) and exit")
+    ap.add_argument("--profile-case", default="", metavar="NAME",
+                    help="only run a small case for an ncu capture (decode1, decode16, layer, adamw, merge, fmt4, "
+                         "l4096) and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args.profile_case)
+        return
     if args.decode_profile:
         run_decode_profile(args.decode_profile)
         return

@@ -20,8 +20,9 @@
 // 128 accumulator rows. Per SM that is 8 KB of operand reads per K16 step, half
 // of what a one-SM 128 x 256 tile with both operands in shared memory needs.
 // Persistent stream-K: the tiles' K blocks, tile after tile, are cut into one
-// contiguous run per pair, equal to within one block, so every SM pair gets the
-// same work whatever the tile count. A pair whose run starts inside a tile (it
+// contiguous run per pair, equal to within one block, so every pair gets the same
+// work whatever the tile count (with a pair count that divides the tiles, each run
+// is whole tiles and no partials are written). A pair whose run starts inside a tile (it
 // holds that tile's last K blocks, and processes them first) writes its fp32
 // accumulator to the workspace and raises a flag; the pair holding the tile's
 // first blocks (its last work) adds those partials in pair order before the

@@ -738,6 +738,7 @@ struct SkinnyParams {
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(128, 2)
 k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, SkinnyParams p) {
+    griddep_launch_dependents();                     // the reduction may be scheduled (it waits for us)
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[2 * 8 + 2];
     __shared__ uint32_t s_tmem;
@@ -888,6 +889,7 @@ __device__ __forceinline__ float4 sum_splits4(const float *__restrict__ part, in
 // count % 4 == 0 (counts are multiples of r, itself a multiple of 8)
 __global__ void k_reduce_xa(const float *__restrict__ part, int splits, int64_t count, float s,
                             __nv_bfloat16 *__restrict__ xa, __nv_bfloat16 *__restrict__ xas) {
+    griddep_wait();                                  // the partials are complete
     for (int64_t i = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < count; i += 4 * (int64_t)gridDim.x * blockDim.x) {
         const float4 v = sum_splits4(part, splits, count, i);
         if (xa) {
@@ -901,6 +903,7 @@ __global__ void k_reduce_xa(const float *__restrict__ part, int splits, int64_t 
 }
 __global__ void k_reduce_f32(const float *__restrict__ part, int splits, int64_t count, float s,
                              float *__restrict__ out) {
+    griddep_wait();                                  // the partials are complete
     for (int64_t i = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < count; i += 4 * (int64_t)gridDim.x * blockDim.x) {
         const float4 v = sum_splits4(part, splits, count, i);
         *reinterpret_cast<float4 *>(out + i) = make_float4(s * v.x, s * v.y, s * v.z, s * v.w);
@@ -993,8 +996,10 @@ static size_t fwd_adapter_bytes(int64_t M, int64_t cols, int r) {
     return r == 0 ? 0 : mr_bytes(M, r) + partial_bytes(M, cols, r);
 }
 
-// CTA pairs of the pair GEMM: every SM, except beside a concurrent side-stream job, where
-// the GEMM takes as few pairs as give the same number of tile rounds and leaves the rest.
+// CTA pairs of the pair GEMM: as few pairs as give the same number of tile rounds. The
+// GEMM is bound by the power cap more than by the SM count (measured: stream-K over every
+// SM was 0.6 % slower at 4096^2 than 64 pairs of four whole tiles), and the SMs left over
+// run the side stream's adapter gradients beside the dgrad GEMM.
 static int side_job_pairs(int64_t M, int64_t N) {
     const int64_t ntiles = ceil_div(M, 256) * ceil_div(N, 256);
     const int max_pairs = gemm2sm_pairs(0);
@@ -1137,8 +1142,8 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
         int splits = 0;
         e = run_skinny(false, X, M, true, A, M, W.cols, r, part, &splits, st);
         if (e != cudaSuccess) return e;
-        QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, XA_save, XAs));
-    }
+        QNF4_LAUNCH("k_reduce_xa", st, e = launch_pdl(k_reduce_xa, (int)reduce_grid(M * r), 256, 0, st, true, part, splits, M * r, s, XA_save, XAs));
+    if (e != cudaSuccess) return e;}
     if (pair) {
         // Y = X W^T + (s XA) B: W^ [d_out, d_in] is the K-major B operand, B_lora [r, d_out]
         // the MN-major extension
@@ -1148,7 +1153,7 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
             return e;
         }
         void *g2ws = reinterpret_cast<char *>(Wd) + wd_bytes(W.rows, W.cols);
-        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, gemm2sm_pairs(0), g2ws, st);
+        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, side_job_pairs(M, W.rows), g2ws, st);
     }
     return run_fused_fwd(X, M, W, XAs, B, r, Y, st);
 }
@@ -1161,12 +1166,12 @@ static cudaError_t adapter_grads(const __nv_bfloat16 *X, const __nv_bfloat16 *dY
     int splits = 0;
     cudaError_t e = run_skinny(true, X, M, true, Gs, W.cols, M, r, part, &splits, st);
     if (e != cudaSuccess) return e;
-    QNF4_LAUNCH("k_reduce_f32", st, k_reduce_f32<<<reduce_grid(W.cols * r), 256, 0, st>>>(part, splits, W.cols * r, 1.0f, dA));
-    // computed as (dY^T XA)^T with the partials written transposed
+    QNF4_LAUNCH("k_reduce_f32", st, e = launch_pdl(k_reduce_f32, (int)reduce_grid(W.cols * r), 256, 0, st, true, part, splits, W.cols * r, 1.0f, dA));
+    if (e != cudaSuccess) return e;// computed as (dY^T XA)^T with the partials written transposed
     e = run_skinny(true, dY, M, true, XA, W.rows, M, r, part, &splits, st, true);
     if (e != cudaSuccess) return e;
-    QNF4_LAUNCH("k_reduce_f32", st, k_reduce_f32<<<reduce_grid(W.rows * r), 256, 0, st>>>(part, splits, W.rows * r, s, dB));
-    return cudaGetLastError();
+    QNF4_LAUNCH("k_reduce_f32", st, e = launch_pdl(k_reduce_f32, (int)reduce_grid(W.rows * r), 256, 0, st, true, part, splits, W.rows * r, s, dB));
+    if (e != cudaSuccess) return e;return cudaGetLastError();
 }
 
 cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, int64_t M, const NF4View &W,
@@ -1201,14 +1206,14 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
         if (!XA) {
             e = run_skinny(false, X, M, true, A, M, W.cols, r, part, &splits, st);
             if (e != cudaSuccess) return e;
-            QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, 1.0f, XAbuf, nullptr));
-            XA = XAbuf;
+            QNF4_LAUNCH("k_reduce_xa", st, e = launch_pdl(k_reduce_xa, (int)reduce_grid(M * r), 256, 0, st, true, part, splits, M * r, 1.0f, XAbuf, nullptr));
+            if (e != cudaSuccess) return e;XA = XAbuf;
         }
         // G = dY B^T -> sG (bf16)
         e = run_skinny(false, dY, M, false, B, M, W.rows, r, part, &splits, st);
         if (e != cudaSuccess) return e;
-        QNF4_LAUNCH("k_reduce_xa", st, k_reduce_xa<<<reduce_grid(M * r), 256, 0, st>>>(part, splits, M * r, s, nullptr, Gs));
-    }
+        QNF4_LAUNCH("k_reduce_xa", st, e = launch_pdl(k_reduce_xa, (int)reduce_grid(M * r), 256, 0, st, true, part, splits, M * r, s, nullptr, Gs));
+    if (e != cudaSuccess) return e;}
     if (pair) {
         // dX = dY W^ + (s G) A^T: W^ [d_out, d_in] read as the MN-major B operand
         // ([K = d_out][N = d_in]), A_lora [d_in, r] the K-major extension

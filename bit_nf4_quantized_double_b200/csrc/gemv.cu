@@ -67,13 +67,15 @@ constexpr int kGemvProducers = 2;              // producer warps, taking alterna
 __host__ __device__ constexpr int gemv_threads(int nt) { return 256 * gemv_rg(nt) + 32 * kGemvProducers; }
 __host__ __device__ constexpr int gemv_box_bytes(int nt) { return gemv_rows(nt) * 128; }
 __host__ __device__ constexpr int gemv_stage_bytes(int nt) { return 8 * gemv_box_bytes(nt); }
-__host__ __device__ constexpr int gemv_stages(int nt) { return nt == 1 ? 5 : 10; }
+__host__ __device__ constexpr int gemv_stages(int nt) { return nt == 1 ? 4 : 8; }
 __host__ __device__ constexpr int gemv_red_hole0(int nt) { return gemv_rows(nt) * gemv_stages(nt); }
+// holes of one of the two reduction buffers (a warp's slice sums: 32 lanes x NT float4)
+__host__ __device__ constexpr int gemv_red_holes(int nt) { return 32 * gemv_rg(nt) * nt; }
 __host__ __device__ constexpr int gemv_smem(int nt) {
     return 1024 + kLutRegion + gemv_stages(nt) * gemv_stage_bytes(nt) + 512;
 }
 static_assert(gemv_smem(1) <= 232448 && gemv_smem(2) <= 232448, "shared memory");
-static_assert(gemv_red_hole0(1) + 32 * gemv_rg(1) * 1 <= 256 && gemv_red_hole0(2) + 32 * gemv_rg(2) * 2 <= 256,
+static_assert(gemv_red_hole0(1) + 2 * gemv_red_holes(1) <= 256 && gemv_red_hole0(2) + 2 * gemv_red_holes(2) <= 256,
               "holes");
 
 __device__ __forceinline__ uint32_t hole(int h) { return (uint32_t)h * 256u + 128u; }
@@ -90,8 +92,6 @@ __device__ __forceinline__ uint32_t pack2_bf16(const __nv_bfloat16 *p0, const __
     return lo | (hi << 16);
 }
 
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 __device__ __forceinline__ void sts128f(uint32_t a, float4 v) {
     asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
@@ -392,7 +392,10 @@ __device__ __forceinline__ void gemv_compute(const GemvGroup &grp, const uint8_t
     // this lane's 8-byte code words of rows rg*16 + g and + 8 in box ks: chunk (2b + t/2) ^ g
     const uint32_t box_row0 = ks * BOX + (rg * 16 + g) * 128 + (t & 1) * 8;
     const uint32_t box_row1 = box_row0 + 8 * 128;
+    // two reduction buffers, used by alternate units: a warp that is ahead waits for the
+    // reducer of the unit before last only
     const uint32_t red_mine = hole(gemv_red_hole0(NT) + (rg * 8 + ks) * NT * 4 + (lane >> 3)) + (lane & 7) * 16;
+    constexpr uint32_t kRedBuf = gemv_red_holes(NT) * 256u;
     bool ok = true;
 
     uint32_t xf[NT][4][8];
@@ -462,17 +465,18 @@ __device__ __forceinline__ void gemv_compute(const GemvGroup &grp, const uint8_t
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
 
         // ---------------- the row group's eight slices: written, then summed by warp ks == i % 8
-        if (i > 0 && !mbar_wait(rede0 + 8 * rg, (i - 1) & 1, abort)) { ok = false; break; }
+        const int rb_ = i & 1, use = i >> 1;             // reduction buffer and its use count
+        if (use > 0 && !mbar_wait(rede0 + 16 * rg + 8 * rb_, (use - 1) & 1, abort)) { ok = false; break; }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            *reinterpret_cast<float4 *>(const_cast<uint8_t *>(lut) + red_mine + nt * 4 * 256) =
+            *reinterpret_cast<float4 *>(const_cast<uint8_t *>(lut) + red_mine + rb_ * kRedBuf + nt * 4 * 256) =
                 make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
             acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(redf0 + 8 * rg);
+        if (lane == 0) mbar_arrive(redf0 + 16 * rg + 8 * rb_);
         if (ks == (i & 7)) {
-            if (!mbar_wait(redf0 + 8 * rg, i & 1, abort)) { ok = false; break; }
+            if (!mbar_wait(redf0 + 16 * rg + 8 * rb_, use & 1, abort)) { ok = false; break; }
             float sum[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -480,12 +484,13 @@ __device__ __forceinline__ void gemv_compute(const GemvGroup &grp, const uint8_t
 #pragma unroll
                 for (int k2 = 0; k2 < 8; ++k2) {
                     const float4 v =
-                        ld128(hole(gemv_red_hole0(NT) + ((rg * 8 + k2) * NT + nt) * 4 + (lane >> 3)) + (lane & 7) * 16);
+                        ld128(hole(gemv_red_hole0(NT) + ((rg * 8 + k2) * NT + nt) * 4 + (lane >> 3)) + (lane & 7) * 16 +
+                              rb_ * kRedBuf);
                     sum[nt][0] += v.x; sum[nt][1] += v.y; sum[nt][2] += v.z; sum[nt][3] += v.w;
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(rede0 + 8 * rg);
+            if (lane == 0) mbar_arrive(rede0 + 16 * rg + 8 * rb_);
             const int M = grp.M, N = it.N;
             const int R0 = pos.rb * ROWS + rg * 16 + g;
             float *pp = it.partial + (int64_t)pos.ch * N * M;
@@ -511,9 +516,9 @@ k_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ Codebook c
     const uint32_t lut = smem_addr(base);
     const uint32_t stages = lut + kLutRegion;
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + kLutRegion + S * STAGE);
-    int *flags = reinterpret_cast<int *>(bars + 2 * S + 2 * RG);
+    int *flags = reinterpret_cast<int *>(bars + 2 * S + 4 * RG);
     const uint32_t full0 = smem_addr(bars), empty0 = full0 + 8 * S;
-    const uint32_t redf0 = full0 + 16 * S, rede0 = redf0 + 8 * RG;   // per row group
+    const uint32_t redf0 = full0 + 16 * S, rede0 = redf0 + 16 * RG;   // per row group and buffer
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // lookup table: word (e * 64 + lane) = bf16 pair (Q[e >> 4] low half, Q[e & 15] high half)
@@ -527,9 +532,9 @@ k_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ Codebook c
             mbar_init(full0 + 8 * s, 33);           // producer's expect-tx arrival + 32 lanes after c^
             mbar_init(empty0 + 8 * s, 8 * RG);      // one arrival per compute warp
         }
-        for (int rg = 0; rg < RG; ++rg) {
-            mbar_init(redf0 + 8 * rg, 8);           // the row group's eight slices written
-            mbar_init(rede0 + 8 * rg, 1);           // the reducer has read them
+        for (int b = 0; b < 2 * RG; ++b) {
+            mbar_init(redf0 + 8 * b, 8);            // the row group's eight slices written
+            mbar_init(rede0 + 8 * b, 1);            // the reducer has read them
         }
         flags[0] = 0;
         fence_barrier_init();
@@ -664,22 +669,6 @@ size_t fwd_grouped_workspace_bytes(int64_t M, int count, const LinearDesc *d) {
         if (x > b) b = x;
     }
     return b;
-}
-
-template <typename... KArgs, typename... Args>
-static cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st, bool pdl,
-                              Args &&...args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3((unsigned)block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Small-M forward of count <= kGemvMaxItems projections: the X A pre-pass, the GEMV, the finish.

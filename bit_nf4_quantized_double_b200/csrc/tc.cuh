@@ -24,6 +24,13 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return p + ((1024u - (smem_addr(p) & 1023u)) & 1023u);
 }
 
+// Programmatic dependent launch: a kernel launched with the programmatic-serialisation
+// attribute may start before its predecessor ends; griddep_wait blocks until the
+// predecessor has completed and its writes are visible, launch_dependents lets the
+// next such kernel start.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
