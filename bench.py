@@ -596,6 +596,47 @@ def run_components(args, peaks, peak_kind, flush):
     out["merge_4096"] = run_merge(hbm, flush, stream)
     out["fmt4"] = run_fmt4(hbm, flush, stream)
     out["adamw"] = run_adamw(hbm, flush, stream)
+    out["large_m_routes"] = run_routes(flush, stream)
+    return out
+
+
+def run_routes(flush, stream):
+    """The headline layer's fwd + bwd (4096 x 4096, M = 4096, r = 64) through each of the two
+    large-M routes: the default (dequantise W once into bf16 scratch, CTA-pair GEMM) and the
+    fused dequant-GEMM kernels forced at every M, which dequantise the codes in the mainloop
+    of each 256-token tile."""
+    import torch
+    import bit_nf4_quantized_double_b200 as q
+    wl, L, inp = headline_inputs(0)
+    M, d_in, d_out, r, s = wl.M, L.d_in, L.d_out, L.r, L.s
+    t = q.qlora_nf4_quantize(inp["W"])
+    X, dY, A, B = inp["X"], inp["dY"], inp["A"], inp["B"]
+    flops = step_flops(M, d_in, d_out, r)
+    out = {"workload": "4096 x 4096 layer, M = 4096, r = 64, fwd + bwd, CUDA graph replay, L2 flushed"}
+    for name, P in (("dequant_then_pair_gemm", 512), ("fused_dequant_gemm", 2 ** 62)):
+        q.lib().qlora_linear_set_pair_min_m(P)
+        try:
+            Y = torch.empty(M, d_out, dtype=torch.bfloat16, device="cuda")
+            XA = torch.empty(M, r, dtype=torch.bfloat16, device="cuda")
+            dX = torch.empty(M, d_in, dtype=torch.bfloat16, device="cuda")
+            dA = torch.empty(d_in, r, dtype=torch.float32, device="cuda")
+            dB = torch.empty(r, d_out, dtype=torch.float32, device="cuda")
+            ws_f = torch.empty(max(1, q.lib().qlora_linear_fwd_workspace(M, d_out, d_in, r)), dtype=torch.uint8,
+                               device="cuda")
+            ws_b = torch.empty(max(1, q.lib().qlora_linear_bwd_workspace(M, d_out, d_in, r)), dtype=torch.uint8,
+                               device="cuda")
+
+            def step():
+                q.qlora_linear_fwd(X, t, A, B, s, Y=Y, XA_save=XA, ws=ws_f)
+                q.qlora_linear_bwd(X, dY, t, A, B, s, XA=XA, dX=dX, dA=dA, dB=dB, ws=ws_b)
+
+            ms = _time_graph(step, 10, flush, stream)
+            kern = _kernel_ms(KERNELS, step, 5, flush)
+            out[name] = {"ms_per_step": round(ms, 5), "TFLOP/s": round(flops / (ms / 1e3) / 1e12, 1),
+                         "kernels": kern}
+        finally:
+            q.lib().qlora_linear_set_pair_min_m(512)
+    assert q.qlora_get_device_status() == q.QLORA_OK
     return out
 
 
@@ -702,7 +743,7 @@ def run_merge(hbm, flush, stream):
     Ym, _ = q.qlora_linear_fwd(X, out, None, None, 0.0)
     rel = ((Ym.double() - Yu.double()).norm() / Yu.double().norm()).item()
     assert q.qlora_get_device_status() == q.QLORA_OK
-    kern = _kernel_ms(("k_merge_bf16", "k_quantize_codes", "k_offset", "k_double_quant"),
+    kern = _kernel_ms(("k_merge_prep", "k_merge_bf16", "k_quantize_codes", "k_offset", "k_double_quant"),
                       lambda: q.qlora_nf4_merge_adapter(t, inp["A"], inp["B"], L.s, out=out, W_bf16=wb, ws=ws), 5,
                       _FLUSH[0])
     # the oracle on the host: merge (C) and re-quantisation of the same weight
@@ -721,10 +762,28 @@ def run_merge(hbm, flush, stream):
                         "CUDA graph replay, L2 flushed",
             "ms": round(ms, 4), "GB/s": round(alg / (ms / 1e3) / 1e9, 1), "frac": round(alg / (ms / 1e3) / 1e9 / hbm, 4),
             "kernels": kern,
+            "k_merge_bf16_roofline": _merge_roofline(kern, n, L.r),
             "cpu_baseline": {"value": round(alg / t_c / 1e9, 3), "unit": "GB/s", "cores": _cores(), "kind": "oracle",
                              "sample": f"the same merge and re-quantisation, full size, {reps} calls"},
             "output_rel_change_fro": round(rel, 6),
             "output_change_sample": "256 tokens: X W'^T (merged, re-quantised) against X W^T + s (XA) B"}
+
+
+# fp32 FMA peak of the merge kernel's bound (its r multiply-adds per weight have a fixed
+# order, so they run on the FP32 pipes): 148 SMs x 128 FMA lanes x 2 flop x 1.965 GHz
+# (the B200's maximum SM clock), a derived figure, not a measured one.
+FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def _merge_roofline(kern, n, r):
+    k = kern.get("k_merge_bf16")
+    if not k or not k.get("ms_per_call"):
+        return None
+    achieved = 2.0 * n * r / (k["ms_per_call"] / 1e3) / 1e12
+    return {"bound": "alu", "achieved": round(achieved, 2), "peak": round(FP32_FMA_PEAK_TFLOPS, 2),
+            "unit": "TFLOP/s", "frac": round(achieved / FP32_FMA_PEAK_TFLOPS, 4),
+            "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz",
+            "work": f"2 x {n} weights x r = {r} flop (one fused multiply-add per weight per j)"}
 
 
 def run_l70b(args, peaks, peak_kind, flush, stream):
@@ -765,6 +824,7 @@ def run_l70b(args, peaks, peak_kind, flush, stream):
 
     reps = max(3, min(args.steps, 10))
     ms = _time_graph(layer, reps, flush, stream)
+    kern = _kernel_ms(KERNELS, layer, 2, flush)
     assert q.qlora_get_device_status() == q.QLORA_OK
     tf = flops / (ms / 1e3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -797,7 +857,7 @@ def run_l70b(args, peaks, peak_kind, flush, stream):
     return {"workload": "70B-like layer: q,o 8192x8192; k,v 1024x8192; gate,up 28672x8192; down 8192x28672; "
                         "r=64, alpha=128 on all seven; M=4096; fwd+bwd of each, CUDA graph replay, L2 flushed",
             "flops_per_step": flops, "ms_per_step": round(ms, 4), "TFLOP/s": round(tf, 1),
-            "frac_of_sustained_bf16": round(tf / peak, 4), "reps": reps, "cpu_baseline": cpu}
+            "frac_of_sustained_bf16": round(tf / peak, 4), "reps": reps, "kernels": kern, "cpu_baseline": cpu}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -903,7 +963,8 @@ def run_profile_case(name, reps=3):
     size, the L2 flushed before each launch): decode1 / decode16 (the decode block's grouped
     forward), layer (one Llama-7B layer quantised and dequantised by the grouped calls),
     adamw (64 M adapter parameters), merge (the 4096^2 adapter merge), fmt4 (the three
-    4-bit reference formats on 2^26 weights), l4096 (one fwd + bwd step of the headline layer)."""
+    4-bit reference formats on 2^26 weights), l4096 (one fwd + bwd step of the headline layer),
+    l4096fused (the same step through the fused dequant-GEMM kernels)."""
     import torch
     import bit_nf4_quantized_double_b200 as q
     import synth_inputs as si
@@ -943,6 +1004,15 @@ def run_profile_case(name, reps=3):
             codes, absmax = q.qlora_fmt4_quantize(W, fmt)
             l2_flush(flush)
             q.qlora_fmt4_dequant(codes, absmax, W.numel(), fmt)
+    elif name == "l4096fused":
+        wl, L, inp = headline_inputs(0)
+        t = q.qlora_nf4_quantize(inp["W"])
+        q.lib().qlora_linear_set_pair_min_m(2 ** 62)
+        for _ in range(reps):
+            l2_flush(flush)
+            Y, XA = q.qlora_linear_fwd(inp["X"], t, inp["A"], inp["B"], L.s)
+            q.qlora_linear_bwd(inp["X"], inp["dY"], t, inp["A"], inp["B"], L.s, XA=XA)
+        q.lib().qlora_linear_set_pair_min_m(512)
     elif name == "l4096":
         wl, L, inp = headline_inputs(0)
         t = q.qlora_nf4_quantize(inp["W"])

@@ -80,6 +80,7 @@ _SIGS = {
     "qlora_nf4_dequant_grouped": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(_Tensor),
                                                  ctypes.POINTER(ctypes.c_void_p), ctypes.c_void_p]),
     "qlora_nf4_set_code_search": (None, [ctypes.c_int]),
+    "qlora_linear_set_pair_min_m": (None, [ctypes.c_int64]),
     "qlora_adamw_step": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_adamw_prefetch": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]),
@@ -89,6 +90,7 @@ _SIGS = {
     "qlora_nf4_quantize_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(_Tensor),
                                                   ctypes.c_void_p]),
     "qlora_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_void_p]),
+    "qlora_selftest_rcp_error": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_nf4_merge_workspace": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
     "qlora_nf4_merge_adapter": (ctypes.c_int, [ctypes.POINTER(_Tensor), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                                ctypes.c_float, ctypes.c_void_p, ctypes.POINTER(_Tensor),

@@ -10,11 +10,12 @@
 // One element per lane, four per thread (16-byte loads and stores), in this
 // order, every step one IEEE binary32 operation (no contraction):
 //   m = fl(fl(b1 m) + fl(c1 g)),  v = fl(fl(b2 v) + fl(c2 fl(g g))),  c = 1 - b
-//   upd = fl(fl(m / bc1) / fl(fl(sqrt(fl(v / bc2))) + eps))
+//   upd = fl(fl(m ib1) / fl(fl(sqrt(fl(v ib2))) + eps))
 //   theta = fl(theta - fl(lr fl(upd + fl(wd theta))))
-// The bias corrections bc1 = 1 - b1^t and bc2 = 1 - b2^t are computed once on
-// the host in double and rounded to float. The kernel is HBM-bound: 30 bytes
-// per parameter (theta, m, v read and written, g read, the bf16 copy written).
+// The inverse bias corrections ib1 = 1 / (1 - b1^t) and ib2 = 1 / (1 - b2^t) are
+// computed once on the host in double and rounded to float, so each parameter
+// costs one division and one square root. The kernel is HBM-bound: 30 bytes per
+// parameter (theta, m, v read and written, g read, the bf16 copy written).
 #include <cmath>
 
 #include "launch.h"
@@ -22,14 +23,14 @@
 namespace qnf4 {
 
 struct AdamwConsts {
-    float lr, b1, b2, c1, c2, eps, wd, bc1, bc2;
+    float lr, b1, b2, c1, c2, eps, wd, ib1, ib2;
 };
 
 __device__ __forceinline__ float adamw_one(float &theta, float g, float &m, float &v, const AdamwConsts &k) {
     const float mi = __fadd_rn(__fmul_rn(k.b1, m), __fmul_rn(k.c1, g));
     const float vi = __fadd_rn(__fmul_rn(k.b2, v), __fmul_rn(k.c2, __fmul_rn(g, g)));
-    const float mhat = __fdiv_rn(mi, k.bc1), vhat = __fdiv_rn(vi, k.bc2);
-    const float upd = __fdiv_rn(mhat, __fadd_rn(__fsqrt_rn(vhat), k.eps));
+    const float den = __fadd_rn(__fsqrt_rn(__fmul_rn(vi, k.ib2)), k.eps);
+    const float upd = __fdiv_rn(__fmul_rn(mi, k.ib1), den);
     const float t = __fsub_rn(theta, __fmul_rn(k.lr, __fadd_rn(upd, __fmul_rn(k.wd, theta))));
     m = mi;
     v = vi;
@@ -79,8 +80,8 @@ cudaError_t launch_adamw(float *theta, const float *g, float *m, float *v, int64
     k.c2 = 1.0f - b2;
     k.eps = eps;
     k.wd = wd;
-    k.bc1 = (float)(1.0 - std::pow((double)b1, (double)step));
-    k.bc2 = (float)(1.0 - std::pow((double)b2, (double)step));
+    k.ib1 = (float)(1.0 / (1.0 - std::pow((double)b1, (double)step)));
+    k.ib2 = (float)(1.0 / (1.0 - std::pow((double)b2, (double)step)));
     int64_t grid = ceil_div(ceil_div(n, 4), 256);
     const int64_t cap = (int64_t)num_sms() * 8;
     if (grid > cap) grid = cap;

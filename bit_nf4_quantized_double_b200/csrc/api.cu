@@ -234,7 +234,8 @@ qlora_status qlora_linear_fwd_grouped(int64_t M, int count, const qlora_linear_d
 
 size_t qlora_nf4_merge_workspace(int64_t rows, int64_t cols) {
     if (rows < 1 || cols < 1) return 0;
-    return align256((size_t)rows * (size_t)cols * 2) + qlora_nf4_quantize_workspace(rows, cols);
+    return align256((size_t)rows * (size_t)cols * 2) + merge_prep_bytes(rows, cols) +
+           qlora_nf4_quantize_workspace(rows, cols);
 }
 
 qlora_status qlora_nf4_merge_adapter(const qlora_nf4_tensor *W, const void *A, const void *B, int r, float s,
@@ -253,10 +254,12 @@ qlora_status qlora_nf4_merge_adapter(const qlora_nf4_tensor *W, const void *A, c
     char *w = static_cast<char *>(ws);
     __nv_bfloat16 *merged = W_bf16 ? static_cast<__nv_bfloat16 *>(W_bf16) : reinterpret_cast<__nv_bfloat16 *>(w);
     w += align256((size_t)n * 2);
+    void *prep = w;
+    w += merge_prep_bytes(W->rows, W->cols);
     float *c1 = reinterpret_cast<float *>(w);
     double *part = reinterpret_cast<double *>(w + align256((size_t)nb * 4));
     cudaError_t e = launch_merge_bf16(view_of(W), static_cast<const __nv_bfloat16 *>(A),
-                                      static_cast<const __nv_bfloat16 *>(B), r, s, merged, st);
+                                      static_cast<const __nv_bfloat16 *>(B), r, s, merged, prep, st);
     if (e != cudaSuccess) return from_cuda(e);
     return from_cuda(launch_quantize(merged, QLORA_BF16, n, *W_out, c1, part, st));
 }
@@ -318,7 +321,7 @@ qlora_status qlora_fmt4_quantize(const void *W, qlora_dtype dt, int64_t n, qlora
 qlora_status qlora_fmt4_dequant(const uint8_t *codes, const float *absmax, int64_t n, qlora_fmt4 fmt,
                                 void *W_out, qlora_stream_t stream) {
     if (!codes || !absmax || !W_out || n < 1 || !fmt4_ok(fmt) || (reinterpret_cast<uintptr_t>(absmax) & 3u) ||
-        (reinterpret_cast<uintptr_t>(W_out) & 3u))
+        !aligned16(codes) || !aligned16(W_out))
         return QLORA_ERR_INVALID_ARG;
     return from_cuda(launch_fmt4_dequant(codes, absmax, n, fmt, static_cast<__nv_bfloat16 *>(W_out),
                                          static_cast<cudaStream_t>(stream)));

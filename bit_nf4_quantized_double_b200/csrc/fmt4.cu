@@ -16,7 +16,8 @@
 // Codes are packed two per byte as in the NF4 format: byte k = code[2k] << 4 | code[2k + 1].
 //
 // k_fmt4_quantize: one warp per 64-block, each lane two consecutive weights (one output byte),
-// absmax by a butterfly of shuffles. k_fmt4_dequant: one thread per byte. Both stream HBM.
+// absmax by a butterfly of shuffles. k_fmt4_dequant: one thread per 16 weights. Both stream
+// HBM.
 #include "launch.h"
 
 namespace qnf4 {
@@ -78,25 +79,38 @@ __global__ void __launch_bounds__(256) k_fmt4_quantize(const T *__restrict__ w, 
     if (lane == 0) absmax[blk] = c;
 }
 
+// Dequantisation: one thread per 16 weights (an 8-byte code word, all of it in one
+// 64-block: one division for the step), signed values from a 16-entry table in shared
+// memory (16 words in 16 banks: lookups never conflict), two 16-byte bf16 stores. The
+// last n % 16 weights are written element by element by thread 0 of CTA 0.
 __global__ void __launch_bounds__(256) k_fmt4_dequant(const uint8_t *__restrict__ codes,
                                                      const float *__restrict__ absmax, int64_t n,
                                                      const __grid_constant__ Fmt4Table t,
                                                      __nv_bfloat16 *__restrict__ out) {
-    const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // byte index
-    if (2 * k >= n) return;
-    const uint32_t byte = codes[k];
-    const float step = __fdiv_rn(__ldg(absmax + (2 * k) / 64), t.S);
-    const uint32_t c0 = byte >> 4, c1 = byte & 15u;
-    const float v0 = (c0 & 8u) ? -t.mag[c0 & 7u] : t.mag[c0 & 7u];
-    const float v1 = (c1 & 8u) ? -t.mag[c1 & 7u] : t.mag[c1 & 7u];
-    const __nv_bfloat16 h0 = __float2bfloat16_rn(__fmul_rn(v0, step));
-    if (2 * k + 1 < n) {
-        __nv_bfloat162 p;
-        p.x = h0;
-        p.y = __float2bfloat16_rn(__fmul_rn(v1, step));
-        *reinterpret_cast<__nv_bfloat162 *>(out + 2 * k) = p;
-    } else {
-        out[2 * k] = h0;
+    __shared__ float s_v[16];   // code c -> sign (bit 3) times magnitude mag[c & 7]
+    if (threadIdx.x < 16) s_v[threadIdx.x] = (threadIdx.x & 8u) ? -t.mag[threadIdx.x & 7u] : t.mag[threadIdx.x & 7u];
+    __syncthreads();
+    const int64_t words = n / 16;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < words; w += stride) {
+        const uint2 cw = __ldg(reinterpret_cast<const uint2 *>(codes) + w);
+        const float step = __fdiv_rn(__ldg(absmax + w / 4), t.S);
+        uint32_t o[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const uint32_t byte = ((k < 4 ? cw.x : cw.y) >> (8 * (k & 3))) & 0xffu;
+            o[k] = pack_bf16x2(__fmul_rn(s_v[byte >> 4], step), __fmul_rn(s_v[byte & 15u], step));
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(out + 16 * w);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        for (int64_t e = words * 16; e < n; ++e) {
+            const uint32_t byte = codes[e / 2];
+            const uint32_t c = (e % 2 == 0) ? (byte >> 4) : (byte & 15u);
+            out[e] = __float2bfloat16_rn(__fmul_rn(s_v[c], __fdiv_rn(absmax[e / 64], t.S)));
+        }
     }
 }
 
@@ -117,8 +131,12 @@ cudaError_t launch_fmt4_quantize(const void *W, qlora_dtype dt, int64_t n, qlora
 
 cudaError_t launch_fmt4_dequant(const uint8_t *codes, const float *absmax, int64_t n, qlora_fmt4 f,
                                 __nv_bfloat16 *out, cudaStream_t st) {
-    const unsigned grid = (unsigned)ceil_div((n + 1) / 2, 256);
-    QNF4_LAUNCH("k_fmt4_dequant", st, k_fmt4_dequant<<<grid, 256, 0, st>>>(codes, absmax, n, fmt4_table(f), out));
+    int64_t grid = ceil_div(n / 16, (int64_t)256);
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    QNF4_LAUNCH("k_fmt4_dequant", st,
+                k_fmt4_dequant<<<(unsigned)grid, 256, 0, st>>>(codes, absmax, n, fmt4_table(f), out));
     return cudaGetLastError();
 }
 

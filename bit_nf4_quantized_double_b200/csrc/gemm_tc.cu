@@ -27,6 +27,7 @@
 // Both fused kernels keep the accumulator tile D[row, token] in TMEM and store
 // it transposed (out[token, row]) through a shared-memory staging tile and a
 // TMA store.
+#include <atomic>
 #include <mutex>
 
 #include "launch.h"
@@ -985,11 +986,13 @@ static unsigned reduce_grid(int64_t count) {
 
 static size_t mr_bytes(int64_t M, int r) { return align256((size_t)M * (size_t)r * 2); }
 
-// From this many tokens on, the layer dequantises W once into bf16 scratch and
-// runs the CTA-pair GEMM: the fused kernel would repeat the dequantisation for
-// every 256-token tile, and at two or more tiles that integer work costs more
-// than writing and re-reading the bf16 copy.
-constexpr int64_t kPairGemmMinM = 512;
+// From this many tokens on (default 512), the layer dequantises W once into bf16
+// scratch and runs the CTA-pair GEMM: the fused kernel would repeat the
+// dequantisation for every 256-token tile, and at two or more tiles that integer
+// work costs more than writing and re-reading the bf16 copy. Settable so that both
+// routes can be compared at any M (qlora_linear_set_pair_min_m).
+static std::atomic<int64_t> g_pair_min_m{512};
+static bool pair_route(int64_t M) { return M >= g_pair_min_m.load(std::memory_order_relaxed); }
 static size_t wd_bytes(int64_t rows, int64_t cols) { return align256((size_t)rows * (size_t)cols * 2); }
 
 static size_t fwd_adapter_bytes(int64_t M, int64_t cols, int r) {
@@ -1009,7 +1012,7 @@ static int side_job_pairs(int64_t M, int64_t N) {
 static size_t g2_bytes() { return gemm2sm_workspace_bytes(gemm2sm_pairs(0)); }
 
 size_t fwd_workspace_bytes_large(int64_t M, int64_t rows, int64_t cols, int r) {
-    return fwd_adapter_bytes(M, cols, r) + (M >= kPairGemmMinM ? wd_bytes(rows, cols) + g2_bytes() : 0);
+    return fwd_adapter_bytes(M, cols, r) + (pair_route(M) ? wd_bytes(rows, cols) + g2_bytes() : 0);
 }
 
 static size_t bwd_adapter_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
@@ -1025,7 +1028,7 @@ static size_t bwd_adapter_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
 }
 
 size_t bwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
-    return bwd_adapter_bytes(M, rows, cols, r) + (M >= kPairGemmMinM ? wd_bytes(rows, cols) + g2_bytes() : 0);
+    return bwd_adapter_bytes(M, rows, cols, r) + (pair_route(M) ? wd_bytes(rows, cols) + g2_bytes() : 0);
 }
 
 static cudaError_t run_fused_fwd(const __nv_bfloat16 *X, int64_t M, const NF4View &W, const __nv_bfloat16 *XAs,
@@ -1119,7 +1122,7 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
                                     const __nv_bfloat16 *B, int r, float s, __nv_bfloat16 *Y,
                                     __nv_bfloat16 *XA_save, void *ws, cudaStream_t st) {
     __nv_bfloat16 *XAs = nullptr;
-    const bool pair = M >= kPairGemmMinM;
+    const bool pair = pair_route(M);
     __nv_bfloat16 *Wd = pair ? reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + fwd_adapter_bytes(M, W.cols, r))
                              : nullptr;
     cudaError_t e;
@@ -1143,7 +1146,8 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
         e = run_skinny(false, X, M, true, A, M, W.cols, r, part, &splits, st);
         if (e != cudaSuccess) return e;
         QNF4_LAUNCH("k_reduce_xa", st, e = launch_pdl(k_reduce_xa, (int)reduce_grid(M * r), 256, 0, st, true, part, splits, M * r, s, XA_save, XAs));
-    if (e != cudaSuccess) return e;}
+        if (e != cudaSuccess) return e;
+    }
     if (pair) {
         // Y = X W^T + (s XA) B: W^ [d_out, d_in] is the K-major B operand, B_lora [r, d_out]
         // the MN-major extension
@@ -1167,11 +1171,13 @@ static cudaError_t adapter_grads(const __nv_bfloat16 *X, const __nv_bfloat16 *dY
     cudaError_t e = run_skinny(true, X, M, true, Gs, W.cols, M, r, part, &splits, st);
     if (e != cudaSuccess) return e;
     QNF4_LAUNCH("k_reduce_f32", st, e = launch_pdl(k_reduce_f32, (int)reduce_grid(W.cols * r), 256, 0, st, true, part, splits, W.cols * r, 1.0f, dA));
-    if (e != cudaSuccess) return e;// computed as (dY^T XA)^T with the partials written transposed
+    if (e != cudaSuccess) return e;
+    // computed as (dY^T XA)^T with the partials written transposed
     e = run_skinny(true, dY, M, true, XA, W.rows, M, r, part, &splits, st, true);
     if (e != cudaSuccess) return e;
     QNF4_LAUNCH("k_reduce_f32", st, e = launch_pdl(k_reduce_f32, (int)reduce_grid(W.rows * r), 256, 0, st, true, part, splits, W.rows * r, s, dB));
-    if (e != cudaSuccess) return e;return cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
 }
 
 cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, int64_t M, const NF4View &W,
@@ -1180,7 +1186,7 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
                               cudaStream_t st) {
     __nv_bfloat16 *Gs = nullptr;
     cudaError_t e;
-    const bool pair = M >= kPairGemmMinM;
+    const bool pair = pair_route(M);
     __nv_bfloat16 *Wd = pair ? reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) +
                                                                 bwd_adapter_bytes(M, W.rows, W.cols, r))
                              : nullptr;
@@ -1207,13 +1213,15 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
             e = run_skinny(false, X, M, true, A, M, W.cols, r, part, &splits, st);
             if (e != cudaSuccess) return e;
             QNF4_LAUNCH("k_reduce_xa", st, e = launch_pdl(k_reduce_xa, (int)reduce_grid(M * r), 256, 0, st, true, part, splits, M * r, 1.0f, XAbuf, nullptr));
-            if (e != cudaSuccess) return e;XA = XAbuf;
+            if (e != cudaSuccess) return e;
+            XA = XAbuf;
         }
         // G = dY B^T -> sG (bf16)
         e = run_skinny(false, dY, M, false, B, M, W.rows, r, part, &splits, st);
         if (e != cudaSuccess) return e;
         QNF4_LAUNCH("k_reduce_xa", st, e = launch_pdl(k_reduce_xa, (int)reduce_grid(M * r), 256, 0, st, true, part, splits, M * r, s, nullptr, Gs));
-    if (e != cudaSuccess) return e;}
+        if (e != cudaSuccess) return e;
+    }
     if (pair) {
         // dX = dY W^ + (s G) A^T: W^ [d_out, d_in] read as the MN-major B operand
         // ([K = d_out][N = d_in]), A_lora [d_in, r] the K-major extension
@@ -1252,3 +1260,7 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
 }
 
 }  // namespace qnf4
+
+extern "C" void qlora_linear_set_pair_min_m(int64_t m) {
+    qnf4::g_pair_min_m.store(m < 17 ? 17 : m, std::memory_order_relaxed);
+}

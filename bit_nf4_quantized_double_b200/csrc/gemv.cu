@@ -17,7 +17,7 @@
 //   k_gemv_xa      one warp per (adapter, 512 inputs): the X A partial sums, run
 //                  beside the GEMV (no shared memory, so its warps fit next to a
 //                  GEMV CTA);
-//   k_gemv_finish  one thread per output row: Y = the K chunks' sums in chunk order
+//   k_gemv_finish  one thread per output element: Y = the K chunks' sums in chunk order
 //                  + (s XA) B with XA = its chunk partials in chunk order, rounded to
 //                  bf16; the first CTA of a projection also saves XA as bf16.
 // In k_gemv a producer warp loads each unit's codes with TMA (one 3D box of
@@ -323,11 +323,12 @@ __device__ __forceinline__ void x_load(const GemvGroup &grp, UnitPos p, int ks, 
 }
 
 // Y[tok][R] = sum over K chunks c in order of partial[c][R][tok] + sum_j (s XA)[tok][j] B[j][R]
-// (fused multiply-adds in increasing j), one thread per output row R. XA = its 512-input
-// chunk partials added in chunk order, staged in shared memory (times s); the first CTA
-// of a projection also saves XA as bf16.
-constexpr int kFinishRows = 256;
-__global__ void __launch_bounds__(kFinishRows) k_gemv_finish(const __grid_constant__ FinishGroup grp) {
+// (fused multiply-adds in increasing j), one thread per output element (R, tok), tok
+// fastest. XA = its X A chunk partials added in chunk order, staged in shared memory
+// (times s); the first CTA of a projection also saves XA as bf16. Every sum issues its
+// loads (up to eight) before the adds, so a thread waits for memory about three times.
+constexpr int kFinishThreads = 256;
+__global__ void __launch_bounds__(kFinishThreads) k_gemv_finish(const __grid_constant__ FinishGroup grp) {
     __shared__ float sx[kGemvMaxM * 256];
     griddep_wait();                                  // the chunk sums and X A partials are complete
     int ii = 0;
@@ -336,42 +337,44 @@ __global__ void __launch_bounds__(kFinishRows) k_gemv_finish(const __grid_consta
     const int M = grp.M, N = it.N, r = it.r;
     for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
         float v = 0.0f;
-        for (int c = 0; c < it.nxa; ++c) v += __ldcg(it.xpart + (int64_t)c * M * r + i);
+        for (int c0 = 0; c0 < it.nxa; c0 += 8) {
+            float pv[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                pv[c] = c0 + c < it.nxa ? __ldcg(it.xpart + (int64_t)(c0 + c) * M * r + i) : 0.0f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                if (c0 + c < it.nxa) v += pv[c];
+        }
         sx[i] = it.s * v;
         if (blockIdx.x == it.cta0 && it.XA_save) it.XA_save[i] = __float2bfloat16_rn(v);
     }
     __syncthreads();
-    const int R = (blockIdx.x - it.cta0) * kFinishRows + threadIdx.x;
-    if (R >= N) return;
-    float y[kGemvMaxM];
+    const int64_t e = (int64_t)(blockIdx.x - it.cta0) * kFinishThreads + threadIdx.x;
+    if (e >= (int64_t)N * M) return;
+    const int R = (int)(e / M), m = (int)(e - (int64_t)R * M);
+    float y = 0.0f;
+    for (int c0 = 0; c0 < it.nch; c0 += 8) {
+        float pv[8];
 #pragma unroll
-    for (int m = 0; m < kGemvMaxM; ++m) y[m] = 0.0f;
-    for (int c = 0; c < it.nch; ++c) {
-        const float *p = it.partial + ((int64_t)c * N + R) * M;
+        for (int c = 0; c < 8; ++c)
+            pv[c] = c0 + c < it.nch ? __ldcg(it.partial + ((int64_t)(c0 + c) * N + R) * M + m) : 0.0f;
 #pragma unroll
-        for (int m = 0; m < kGemvMaxM; ++m)
-            if (m < M) y[m] += __ldcg(p + m);
+        for (int c = 0; c < 8; ++c)
+            if (c0 + c < it.nch) y += pv[c];
     }
     if (r > 0) {
-        float a[kGemvMaxM];
-#pragma unroll
-        for (int m = 0; m < kGemvMaxM; ++m) a[m] = 0.0f;
+        float a = 0.0f;
         for (int j0 = 0; j0 < r; j0 += 8) {          // r % 8 == 0: eight B loads in flight
             float bv[8];
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) bv[jj] = __bfloat162float(it.B[(int64_t)(j0 + jj) * N + R]);
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-#pragma unroll
-                for (int m = 0; m < kGemvMaxM; ++m)
-                    if (m < M) a[m] = fmaf(sx[m * r + j0 + jj], bv[jj], a[m]);
+            for (int jj = 0; jj < 8; ++jj) a = fmaf(sx[m * r + j0 + jj], bv[jj], a);
         }
-#pragma unroll
-        for (int m = 0; m < kGemvMaxM; ++m) y[m] += a[m];
+        y += a;
     }
-#pragma unroll
-    for (int m = 0; m < kGemvMaxM; ++m)
-        if (m < M) it.Y[(int64_t)m * N + R] = __float2bfloat16_rn(y[m]);
+    it.Y[(int64_t)m * N + R] = __float2bfloat16_rn(y);
 }
 
 // Compute warps of k_gemv (warp w < 8 RG): row group w / 8, K slice w % 8.
@@ -733,7 +736,7 @@ static cudaError_t gemv_group(int64_t M, int count, const LinearDesc *d, void *w
         fi.XA_save = d[i].r > 0 ? d[i].XA_save : nullptr;
         fi.nxa = 0;
         fi.cta0 = fc;
-        fc += (int)ceil_div(w.rows, kFinishRows);
+        fc += (int)ceil_div(w.rows * M, (int64_t)kFinishThreads);
     }
     int xc = 0;
     for (int i = 0; i < count; ++i) {
@@ -791,7 +794,7 @@ static cudaError_t gemv_group(int64_t M, int count, const LinearDesc *d, void *w
         QNF4_LAUNCH("k_gemv_xa", st, e = launch_pdl(k_gemv_xa, xc, 32, 0, st, true, xg));
         if (e != cudaSuccess) return e;
     }
-    QNF4_LAUNCH("k_gemv_finish", st, e = launch_pdl(k_gemv_finish, fc, kFinishRows, 0, st, true, fg));
+    QNF4_LAUNCH("k_gemv_finish", st, e = launch_pdl(k_gemv_finish, fc, kFinishThreads, 0, st, true, fg));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -25,8 +25,11 @@ cudaError_t launch_fmt4_dequant(const uint8_t *codes, const float *absmax, int64
 cudaError_t launch_adamw(float *theta, const float *g, float *m, float *v, int64_t n, float lr, float b1, float b2,
                          float eps, float wd, int64_t step, __nv_bfloat16 *out_bf16, cudaStream_t st);
 cudaError_t launch_prefetch(const void *ptr, size_t bytes, bool to_device, cudaStream_t st);
+// Adapter merge: k_merge_prep (A^T and B widened to fp32 into `prep`, merge_prep_bytes)
+// then k_merge_bf16.
+size_t merge_prep_bytes(int64_t rows, int64_t cols);
 cudaError_t launch_merge_bf16(const NF4View &q, const __nv_bfloat16 *A, const __nv_bfloat16 *B, int r, float s,
-                              __nv_bfloat16 *out, cudaStream_t st);
+                              __nv_bfloat16 *out, void *prep, cudaStream_t st);
 
 // Plain bf16 GEMM on CTA pairs (tcgen05 cta_group::2, stream-K), see gemm2sm.cu.
 size_t gemm2sm_workspace_bytes(int pairs);

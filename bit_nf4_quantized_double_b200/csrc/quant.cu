@@ -7,15 +7,19 @@
 // constants; dequantise to BF16 on demand).
 //
 // Launch sequence of a quantisation (all HBM-bound):
-//   k_quantize_codes  one CTA per second-level group (256 blocks = 16384 weights):
-//                     absmax per 64-block by warp shuffles, IEEE division, 4-step
-//                     threshold search, nibble packing; writes the exact fp32
-//                     absmax and the group's fp64 pairwise partial sum;
-//   k_offset          one CTA: the upper levels of the fp64 pairwise tree -> mean;
+//   k_quantize_codes  persistent CTAs over the second-level groups (256 blocks =
+//                     16384 weights): absmax per 64-block by warp shuffles, codes
+//                     from a bin table with an exact-quotient fallback, nibble
+//                     packing; writes the exact fp32 absmax and the group's fp64
+//                     pairwise partial sum;
+//   k_offset          one CTA per tensor: the upper levels of the fp64 pairwise
+//                     tree -> mean;
 //   k_double_quant    one warp per group: s2 = max |c1 - mu|, int8 constants.
 
 #include <atomic>
 #include <cmath>
+#include <cstring>
+#include <type_traits>
 
 #include "launch.h"
 
@@ -34,65 +38,111 @@ __device__ __forceinline__ int nf4_code(float x, const float *t) {
     return c;
 }
 
-// Code table over 256 equal bins of [-1, 1): bin k = [-1 + k/128, -1 + (k+1)/128)
-// holds base[k] = number of thresholds below the bin and thr[k] = the one
-// threshold inside the bin (4.0 if none). Valid when no threshold lies within
-// kBinMargin of a bin edge (checked on the host).
-struct CodeBins {
-    int base[256];
+// Code table of the quantiser's fast path. A weight's normalised value x' (see
+// k_quantize_codes) is mapped to u = sat(fl(x' / 2 + 1/2)) in [0, 1] (NaN to 0) and
+// to its bin k = z - 2^23 with z = fl(u 255 + 2^23), an integer in [0, 255]. Both
+// roundings are monotone, so each bin holds an interval of x'. Entry k holds the
+// one threshold T inside bin k (4.0 if none) and base = the number of thresholds
+// below bin k, both as floats; the code of x' is base + (x' > T). Valid when no
+// bin holds two thresholds and every threshold's neighbourhood T +- 2^-16 lies
+// inside its own bin (checked on the host), so that a threshold can sit between
+// x' and the exact quotient only if it is the threshold of x''s bin.
+struct CodeTable {
     float thr[256];
+    float base[256];
 };
-constexpr double kBinMargin = 1e-5;
 
-static bool build_code_bins(const Codebook &cb, CodeBins &b) {
+static int host_bin(float x) {
+    float u = std::fmaf(x, 0.5f, 0.5f);
+    u = u < 0.0f ? 0.0f : (u > 1.0f ? 1.0f : u);
+    return (int)(std::fmaf(u, 255.0f, 8388608.0f) - 8388608.0f);
+}
+
+static bool build_code_table(const Codebook &cb, CodeTable &tb) {
+    int owner[256];
+    for (int k = 0; k < 256; ++k) owner[k] = -1;
+    for (int t = 0; t < 15; ++t) {
+        const float T = cb.t[t];
+        const int k = host_bin(T);
+        if (host_bin(T - 0x1p-16f) != k || host_bin(T + 0x1p-16f) != k) return false;
+        if (owner[k] != -1) return false;
+        if (!(std::fabs(T) >= 0x1p-5f && std::fabs(T) < 1.0f)) return false;   // the band below assumes it
+        owner[k] = t;
+    }
     for (int k = 0; k < 256; ++k) {
-        const double lo = -1.0 + k / 128.0, hi = lo + 1.0 / 128.0;
         int base = 0;
-        float thr = 4.0f;
-        int inside = 0;
-        for (int t = 0; t < 15; ++t) {
-            const double T = cb.t[t];
-            if (std::fabs(T - lo) < kBinMargin || std::fabs(T - hi) < kBinMargin) return false;
-            if (T < lo) ++base;
-            else if (T < hi) { thr = cb.t[t]; ++inside; }
-        }
-        if (inside > 1) return false;
-        b.base[k] = base;
-        b.thr[k] = thr;
+        for (int t = 0; t < 15; ++t) base += host_bin(cb.t[t]) < k ? 1 : 0;
+        if (owner[k] >= 0 && owner[k] != base) return false;
+        tb.thr[k] = owner[k] >= 0 ? cb.t[owner[k]] : 4.0f;
+        tb.base[k] = (float)base;
     }
     return true;
+}
+
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+    float d;
+    asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ float mul_sat(float a, float b) {
+    float d;
+    asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+
+__device__ __forceinline__ void lds_f2(uint32_t addr, float &x, float &y) {
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(x), "=f"(y) : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
 }
 
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-template <typename T, int VEC>
-__device__ __forceinline__ void load_vec(const T *p, float (&v)[VEC]) {
-    const uint4 raw = *reinterpret_cast<const uint4 *>(p);
-    if constexpr (sizeof(T) == 4) {
-        v[0] = __uint_as_float(raw.x); v[1] = __uint_as_float(raw.y);
-        v[2] = __uint_as_float(raw.z); v[3] = __uint_as_float(raw.w);
-    } else {
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// 16 input bytes of a lane from element e0 on, zero past n (the partial lane of a
+// tensor's tail).
+template <typename T>
+__device__ __forceinline__ uint4 load_partial(const T *W, int64_t e0, int64_t n) {
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    constexpr int VEC = 16 / sizeof(T);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) { v[2 * k] = bf16_lo(w[k]); v[2 * k + 1] = bf16_hi(w[k]); }
+    for (int k = 0; k < VEC; ++k) {
+        if (e0 + k < n) {
+            if constexpr (sizeof(T) == 4) w[k] = __float_as_uint(reinterpret_cast<const float *>(W)[e0 + k]);
+            else w[k / 2] |= (uint32_t)__bfloat16_as_ushort(W[e0 + k]) << (16 * (k & 1));
+        }
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Store a lane's NBYTES code bytes at code byte c0 (bytes past ncode are dropped).
+template <int NBYTES>
+__device__ __forceinline__ void store_codes(uint8_t *codes, int64_t c0, int64_t ncode, uint32_t packed) {
+    if (c0 + NBYTES <= ncode) {
+        if constexpr (NBYTES == 4) *reinterpret_cast<uint32_t *>(codes + c0) = packed;
+        else *reinterpret_cast<uint16_t *>(codes + c0) = (uint16_t)packed;
+    } else {
+#pragma unroll
+        for (int k = 0; k < NBYTES; ++k)
+            if (c0 + k < ncode) codes[c0 + k] = (uint8_t)(packed >> (8 * k));
     }
 }
 
-// One CTA of 256 threads per second-level group j (blocks 256j .. 256j+255).
-// Warp w handles blocks 256j + 32w .. +31; a 64-block is spread over
-// LPB = 64 / VEC lanes that each load 16 bytes.
-//
-// With BINS, a lane divides by one correctly rounded reciprocal of its block's
-// absmax (x' = fl(w * fl(1/c1)), within 1.5 ulp of the exact quotient x =
-// fl(w / c1)) and reads the code from the bin table through the float bits of
-// x' + 3 (in [2, 4): the top 8 mantissa bits are the bin). Where x' lies within
-// 4 ulp of the bin's threshold the exact quotient and the full search decide, so
-// the codes are those of x bit for bit. Without BINS every weight is divided.
-// A list of tensors quantised by one sequence of launches: CTA ranges per tensor
-// (groups in k_quantize_codes, blocks of eight groups in k_double_quant), one CTA
-// per tensor in k_offset.
+// A list of tensors quantised by one sequence of launches: group ranges per tensor
+// (second-level groups in k_quantize_codes, blocks of eight groups in
+// k_double_quant), one CTA per tensor in k_offset.
 constexpr int kQuantMaxItems = 64;
 struct QuantItem {
     const void *W;
@@ -103,14 +153,15 @@ struct QuantItem {
     int8_t *scale8;
     float *scale2;
     float *offset;
-    int64_t cta0;                // first CTA of this tensor in k_quantize_codes
+    int64_t cta0;                // first group of this tensor in k_quantize_codes' numbering
     int64_t dq0;                 // first CTA of this tensor in k_double_quant
 };
 struct QuantGroup {
     QuantItem it[kQuantMaxItems];
     int count;
+    int64_t groups;              // total second-level groups of the list
 };
-// The tensor whose CTA range holds block b (ranges ascending from 0).
+// The tensor whose range holds unit b (ranges ascending from 0).
 __device__ __forceinline__ int quant_item(const QuantGroup &g, int64_t b, bool dq) {
     int lo = 0, hi = g.count - 1;
     while (lo < hi) {
@@ -120,116 +171,178 @@ __device__ __forceinline__ int quant_item(const QuantGroup &g, int64_t b, bool d
     return lo;
 }
 
+// Codes, exact absmax and group partial sums. A persistent grid of 256-thread CTAs
+// walks the second-level groups (256 blocks = 16384 weights); warp w handles blocks
+// 32w .. 32w+31 of a group, a 64-block spread over LPB = 64 / VEC lanes that each
+// load 16 bytes, eight loads in flight per lane before any arithmetic.
+//
+// Absmax c1 = max |w| is taken on the weights' bit patterns with the sign cleared
+// (integer order equals float order there; inf and NaN compare above every finite
+// value, which also flags a non-finite block).
+//
+// With BINS (default), a lane multiplies by an approximate reciprocal r of c1
+// (within 1 ulp): x' = fl(w r) lies within 3 ulp of the exact quotient
+// x = fl(w / c1), and the code is base + (x' > T) from the lane's own copy of the
+// code table (entry k of lane l at byte 256 k + 8 l: the 32 lanes never meet in one
+// bank; the address is one integer multiply-add of z's bit pattern). The per-weight
+// work stays on the FMA pipe: the compare is sat(fl(x' - T) 2^100), the codes are
+// summed into the mantissa of 2^23 (16 bits per float, joined by one byte
+// permutation), and "near" is sat(|x' - T| 2^100 - 2^79) = 0, i.e. |x' - T| <= 2^-21
+// (thresholds lie in [2^-5, 1), where 3 ulp <= 3 2^-24). Outside that band x and x'
+// are on the same side of every threshold and the code is that of x bit for bit.
+// Inside it, or where c1 is outside [2^-126, 2^125) (a reciprocal that is not a
+// normal number), the lane's 8 or 4 codes are recomputed after the batch from the
+// exact quotient and the threshold search, out of the unrolled path. Without BINS
+// every weight is divided.
 template <typename T, bool BINS>
-__global__ void __launch_bounds__(256, 4)
-k_quantize_codes(const __grid_constant__ QuantGroup grp, Codebook cb, const __grid_constant__ CodeBins bins) {
+__global__ void __launch_bounds__(256, 3)
+k_quantize_codes(const __grid_constant__ QuantGroup grp, Codebook cb, const __grid_constant__ CodeTable tab) {
     constexpr int VEC = 16 / sizeof(T);   // elements per 16-byte lane load
     constexpr int LPB = kBlock1 / VEC;    // lanes per block
     constexpr int BPI = 32 / LPB;         // blocks per warp iteration
     constexpr int ITERS = 32 / BPI;       // iterations per warp (32 blocks)
     constexpr int NBYTES = VEC / 2;       // code bytes per lane per iteration
+    constexpr int BATCH = ITERS < 8 ? ITERS : 8;
 
     __shared__ float s_t[16];
     __shared__ float s_c1[kBlock2];
     __shared__ double s_part[8];
-    __shared__ int2 s_bin[256];
+    extern __shared__ __align__(16) float2 s_tab[];   // BINS: [256][32] (64 KB)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x < 15) s_t[threadIdx.x] = cb.t[threadIdx.x];
-    if (BINS) s_bin[threadIdx.x] = make_int2(bins.base[threadIdx.x], __float_as_int(bins.thr[threadIdx.x]));
+    if constexpr (BINS) {
+        for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) s_tab[i] = make_float2(tab.thr[i >> 5], tab.base[i >> 5]);
+    }
     __syncthreads();
-
-    const QuantItem &item = grp.it[quant_item(grp, blockIdx.x, false)];
-    const T *__restrict__ W = static_cast<const T *>(item.W);
-    const int64_t n = item.n, nb = item.nb;
-    float *__restrict__ c1_out = item.c1;
-    double *__restrict__ part_out = item.part;
-    uint8_t *__restrict__ codes = item.codes;
-    const int64_t group = blockIdx.x - item.cta0;
+    // z's bit pattern is 0x4B000000 + k and 0x4B000000 * 256 = 0 mod 2^32, so
+    // bits(z) * 256 + tab_lane is the byte address of entry k of this lane
+    const uint32_t tab_lane = static_cast<uint32_t>(__cvta_generic_to_shared(s_tab)) + (uint32_t)lane * 8u;
     const int sub = lane / LPB, li = lane % LPB;
-    const int64_t ncode = (n + 1) / 2;
     bool nonfinite = false;
 
-    // the lane's 16-byte loads are issued in batches of 8 before any arithmetic
-    // (one memory round trip per batch instead of one per iteration)
-    constexpr int BATCH = ITERS < 8 ? ITERS : 8;
+    for (int64_t unit = blockIdx.x; unit < grp.groups; unit += gridDim.x) {
+    const QuantItem &item = grp.it[quant_item(grp, unit, false)];
+    const T *__restrict__ W = static_cast<const T *>(item.W);
+    const int64_t n = item.n, nb = item.nb;
+    const int64_t group = unit - item.cta0;
+    const int64_t ncode = (n + 1) / 2;
+
+    // FULL: the whole group lies inside the tensor (every group but a tensor's last):
+    // no bounds checks, fixed offsets from per-lane base pointers
+    auto run_group = [&](auto full_tag) {
+    constexpr bool FULL = decltype(full_tag)::value;
+    const int64_t lane_e = (group * kBlock2 + warp * 32 + sub) * kBlock1 + (int64_t)li * VEC;
+    const T *__restrict__ Wl = W + lane_e;
+    uint8_t *__restrict__ cl = item.codes + lane_e / 2;
 #pragma unroll 1
     for (int it0 = 0; it0 < ITERS; it0 += BATCH) {
-    uint4 raw[BATCH];
+        uint4 raw[BATCH];
 #pragma unroll
-    for (int j = 0; j < BATCH; ++j) {
-        const int it = it0 + j;
-        const int64_t e0 = ((group * kBlock2 + warp * 32 + it * BPI + sub) * kBlock1) + (int64_t)li * VEC;
-        raw[j] = (e0 + VEC <= n) ? __ldg(reinterpret_cast<const uint4 *>(W + e0)) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int j = 0; j < BATCH; ++j) {
-        const int it = it0 + j;
-        const int local = warp * 32 + it * BPI + sub;          // block index within the group
-        const int64_t b = group * kBlock2 + local;
-        const int64_t e0 = b * kBlock1 + (int64_t)li * VEC;     // first element of this lane
-        float v[VEC];
-        if (e0 + VEC <= n) {
-            if constexpr (sizeof(T) == 4) {
-                v[0] = __uint_as_float(raw[j].x); v[1] = __uint_as_float(raw[j].y);
-                v[2] = __uint_as_float(raw[j].z); v[3] = __uint_as_float(raw[j].w);
+        for (int j = 0; j < BATCH; ++j) {
+            const int off = (it0 + j) * BPI * kBlock1;
+            if constexpr (FULL) {
+                raw[j] = __ldg(reinterpret_cast<const uint4 *>(Wl + off));
             } else {
-                const uint32_t w4[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k) { v[2 * k] = bf16_lo(w4[k]); v[2 * k + 1] = bf16_hi(w4[k]); }
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < VEC; ++k) v[k] = (e0 + k < n) ? to_f32<T>(W[e0 + k]) : 0.0f;
-        }
-        float m = 0.0f;
-#pragma unroll
-        for (int k = 0; k < VEC; ++k) {
-            nonfinite |= !isfinite(v[k]);
-            m = fmaxf(m, fabsf(v[k]));
-        }
-#pragma unroll
-        for (int o = LPB / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (li == 0) {
-            s_c1[local] = m;
-            if (b < nb) c1_out[b] = m;
-        }
-        // codes of the lane's VEC elements: NBYTES bytes, byte k = hi << 4 | lo
-        uint32_t packed = 0;
-        if (BINS) {
-            const float rcp = __frcp_rn(m);
-#pragma unroll
-            for (int k = 0; k < VEC; ++k) {
-                const float xa = __fmul_rn(v[k], rcp);
-                const float y = fminf(fmaxf(__fadd_rn(xa, 3.0f), 2.0f), 3.99999976f);
-                const int2 e = s_bin[(__float_as_uint(y) >> 15) & 0xffu];
-                const float thr = __int_as_float(e.y);
-                int c = e.x + (xa > thr ? 1 : 0);
-                if (fabsf(__fsub_rn(xa, thr)) <= __fmul_rn(fabsf(thr), 0x1p-21f)) c = nf4_code(__fdiv_rn(v[k], m), s_t);
-                if (m == 0.0f) c = 7;
-                packed |= (uint32_t)c << (8 * (k / 2) + ((k & 1) ? 0 : 4));
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < VEC; k += 2) {
-                const float x0 = (m == 0.0f) ? 0.0f : __fdiv_rn(v[k], m);
-                const float x1 = (m == 0.0f) ? 0.0f : __fdiv_rn(v[k + 1], m);
-                const uint32_t byte = ((uint32_t)nf4_code(x0, s_t) << 4) | (uint32_t)nf4_code(x1, s_t);
-                packed |= byte << (8 * (k / 2));
+                const int64_t e0 = lane_e + off;
+                raw[j] = (e0 + VEC <= n) ? __ldg(reinterpret_cast<const uint4 *>(W + e0))
+                                         : (e0 < n ? load_partial<T>(W, e0, n) : make_uint4(0u, 0u, 0u, 0u));
             }
         }
-        const int64_t c0 = e0 / 2;
-        if (c0 + NBYTES <= ncode) {
-            if constexpr (NBYTES == 4) *reinterpret_cast<uint32_t *>(codes + c0) = packed;
-            else *reinterpret_cast<uint16_t *>(codes + c0) = (uint16_t)packed;
-        } else {
+        [[maybe_unused]] uint32_t redo = 0;
 #pragma unroll
-            for (int k = 0; k < NBYTES; ++k)
-                if (c0 + k < ncode) codes[c0 + k] = (uint8_t)(packed >> (8 * k));
+        for (int j = 0; j < BATCH; ++j) {
+            const int local = warp * 32 + (it0 + j) * BPI + sub;   // block index within the group
+            const int off = (it0 + j) * BPI * kBlock1;             // elements from the lane's first
+            const uint32_t r4[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+            float v[VEC];
+            uint32_t mbits;
+            if constexpr (sizeof(T) == 4) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v[k] = __uint_as_float(r4[k]);
+                mbits = max(max(r4[0] & 0x7fffffffu, r4[1] & 0x7fffffffu), max(r4[2] & 0x7fffffffu, r4[3] & 0x7fffffffu));
+#pragma unroll
+                for (int o = LPB / 2; o >= 1; o >>= 1) mbits = max(mbits, __shfl_xor_sync(0xffffffffu, mbits, o));
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) { v[2 * k] = bf16_lo(r4[k]); v[2 * k + 1] = bf16_hi(r4[k]); }
+                uint32_t h = vmax_u16x2(vmax_u16x2(r4[0] & 0x7fff7fffu, r4[1] & 0x7fff7fffu),
+                                        vmax_u16x2(r4[2] & 0x7fff7fffu, r4[3] & 0x7fff7fffu));
+#pragma unroll
+                for (int o = LPB / 2; o >= 1; o >>= 1) h = vmax_u16x2(h, __shfl_xor_sync(0xffffffffu, h, o));
+                mbits = max(h & 0xffffu, h >> 16) << 16;
+            }
+            const float m = __uint_as_float(mbits);
+            nonfinite |= mbits >= 0x7f800000u;
+            if (li == 0) {
+                s_c1[local] = m;
+                const int64_t b = group * kBlock2 + local;
+                if (FULL || b < nb) item.c1[b] = m;
+            }
+            // codes of the lane's VEC elements: NBYTES bytes, byte k = hi << 4 | lo
+            uint32_t packed = 0;
+            if constexpr (BINS) {
+                const float rcp = mbits == 0u ? 0.0f : rcp_approx(m);
+                const bool odd = mbits != 0u && (mbits - 0x00800000u) >= (0x7e000000u - 0x00800000u);
+                constexpr float kNibble[4] = {16.0f, 1.0f, 4096.0f, 256.0f};   // byte = code(2i) << 4 | code(2i+1)
+                float pf[(VEC + 3) / 4];
+#pragma unroll
+                for (int h = 0; h < (VEC + 3) / 4; ++h) pf[h] = 8388608.0f;
+                float acc = 1.0f;
+#pragma unroll
+                for (int k = 0; k < VEC; ++k) {
+                    const float xa = __fmul_rn(v[k], rcp);
+                    const float u = fma_sat(xa, 0.5f, 0.5f);
+                    const float z = __fmaf_rn(u, 255.0f, 8388608.0f);
+                    float thr, base;
+                    lds_f2(__float_as_uint(z) * 256u + tab_lane, thr, base);
+                    const float d = __fsub_rn(xa, thr);
+                    const float c = __fadd_rn(base, mul_sat(d, 0x1p100f));
+                    pf[k / 4] = __fmaf_rn(c, kNibble[k % 4], pf[k / 4]);
+                    acc = __fmul_rn(acc, fma_sat(fabsf(d), 0x1p100f, -0x1p79f));
+                }
+                if constexpr (VEC == 8) packed = prmt(__float_as_uint(pf[0]), __float_as_uint(pf[1]), 0x5410u);
+                else packed = __float_as_uint(pf[0]) & 0xffffu;
+                redo |= (odd || acc < 1.0f) ? (1u << j) : 0u;
+            } else {
+#pragma unroll
+                for (int k = 0; k < VEC; k += 2) {
+                    const float x0 = (m == 0.0f) ? 0.0f : __fdiv_rn(v[k], m);
+                    const float x1 = (m == 0.0f) ? 0.0f : __fdiv_rn(v[k + 1], m);
+                    const uint32_t byte = ((uint32_t)nf4_code(x0, s_t) << 4) | (uint32_t)nf4_code(x1, s_t);
+                    packed |= byte << (8 * (k / 2));
+                }
+            }
+            if constexpr (FULL) {
+                if constexpr (NBYTES == 4) *reinterpret_cast<uint32_t *>(cl + off / 2) = packed;
+                else *reinterpret_cast<uint16_t *>(cl + off / 2) = (uint16_t)packed;
+            } else {
+                store_codes<NBYTES>(item.codes, (lane_e + off) / 2, ncode, packed);
+            }
+        }
+        if constexpr (BINS) {
+            __syncwarp();
+            // exact codes of the lanes whose normalised weights came near a threshold
+#pragma unroll 1
+            for (; redo != 0u; redo &= redo - 1u) {
+                const int j = __ffs(redo) - 1;
+                const int local = warp * 32 + (it0 + j) * BPI + sub;
+                const int64_t e0 = lane_e + (it0 + j) * BPI * kBlock1;
+                const float m = s_c1[local];
+                uint32_t packed = 0;
+#pragma unroll 1
+                for (int k = 0; k < VEC; ++k) {
+                    const float w = (e0 + k < n) ? to_f32<T>(W[e0 + k]) : 0.0f;
+                    const float x = (m == 0.0f) ? 0.0f : __fdiv_rn(w, m);
+                    packed |= (uint32_t)nf4_code(x, s_t) << (8 * (k / 2) + ((k & 1) ? 0 : 4));
+                }
+                store_codes<NBYTES>(item.codes, e0 / 2, ncode, packed);
+            }
         }
     }
-    }
-    if (__any_sync(0xffffffffu, nonfinite) && lane == 0) raise_status(QLORA_ERR_NONFINITE);
+    };
+    if ((group + 1) * (int64_t)(kBlock1 * kBlock2) <= n) run_group(std::true_type{});
+    else run_group(std::false_type{});
     __syncthreads();
 
     // fp64 pairwise tree over the group's 256 leaves (blocks past nb are 0):
@@ -249,8 +362,10 @@ k_quantize_codes(const __grid_constant__ QuantGroup grp, Codebook cb, const __gr
             const double u = __shfl_down_sync(0xffffffffu, v, o);
             if ((lane & (2 * o - 1)) == 0) v = v + u;
         }
-        if (lane == 0) part_out[group] = v;
+        if (lane == 0) item.part[group] = v;
     }
+    }
+    if (__any_sync(0xffffffffu, nonfinite) && lane == 0) raise_status(QLORA_ERR_NONFINITE);
 }
 
 // Upper levels of the pairwise tree over the nb2 group partials, zero-padded
@@ -429,77 +544,174 @@ k_dequant(const __grid_constant__ DeqGroup grp, Codebook cb) {
 // weight and re-quantising can change outputs; the merge is done in BF16):
 //   w'[n,k] = bf16( fl( w^[n,k] + fl(s * d[n,k]) ) ),
 //   d[n,k]  = fused multiply-adds of A[k,j] * B[j,n] over j = 0 .. r-1 in order, from 0,
-// with w^ the dequantised weight computed in place (step 7 of the format). A CTA
-// takes 64 x 64 tiles (rows x inputs: one 64-block per row); the tile's A rows and
-// B columns are staged in shared memory as fp32, transposed so that a thread reads
-// its 16 consecutive inputs of one j with four 16-byte loads.
-__global__ void __launch_bounds__(256)
-k_merge_bf16(NF4View q, const __nv_bfloat16 *__restrict__ A, const __nv_bfloat16 *__restrict__ B, int r, float s,
+// with w^ the dequantised weight computed in place (step 7 of the format). The fixed
+// order of the r multiply-adds keeps this on the fp32 FMA pipes (r FMAs per weight;
+// the bound is the FMA rate, not HBM).
+//
+// k_merge_prep widens A and B to fp32 once, A transposed (At[j][k]) and B with rows
+// padded to a multiple of four (Bf[j][n]), so that k_merge_bf16 stages both with
+// 16-byte asynchronous copies. k_merge_bf16: persistent, two 256-thread CTAs per SM
+// over 128 x 128 tiles of W; each thread keeps an 8 x 8 block of d in registers (rows
+// 8t..8t+7, inputs 4t..4t+3 and 64+4t..+3 of the tile, so that a warp's 16-byte
+// shared loads of At are contiguous). At and Bf come in chunks of 32 j through two
+// shared-memory buffers: the copies of the next (tile, chunk) step are in flight
+// while the current one is multiplied (four 16-byte shared loads per 64 FMAs).
+constexpr int kMergeTile = 128;
+constexpr int kMergeJ = 32;
+constexpr int kMergeBuf = kMergeJ * kMergeTile;                       // floats per operand per buffer
+constexpr size_t kMergeSmem = (size_t)2 * 2 * kMergeBuf * sizeof(float);   // 64 KB
+
+__global__ void k_merge_prep(const __nv_bfloat16 *__restrict__ A, const __nv_bfloat16 *__restrict__ B, int r,
+                             int64_t K, int64_t N, int64_t ldb, float *__restrict__ At, float *__restrict__ Bf) {
+    const int64_t j = blockIdx.y;                   // one adapter rank per grid row
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < K; k += stride)
+        At[j * K + k] = __bfloat162float(A[k * r + j]);
+    for (int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; n < ldb; n += stride)
+        Bf[j * ldb + n] = n < N ? __bfloat162float(B[j * N + n]) : 0.0f;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__global__ void __launch_bounds__(256, 2)
+k_merge_bf16(NF4View q, const float *__restrict__ At, const float *__restrict__ Bf, int64_t ldb, int r, float s,
              Codebook cb, __nv_bfloat16 *__restrict__ out) {
-    extern __shared__ __align__(16) float msm[];
-    float *As = msm;                 // [r][64]: As[j][kk] = A[k0 + kk][j]
-    float *Bs = msm + r * 64;        // [r][64]: Bs[j][nn] = B[j][n0 + nn]
+    extern __shared__ __align__(16) float msm[];   // [buf][At chunk | Bf chunk], each [kMergeJ][kMergeTile]
     __shared__ float s_q[16];
+    __shared__ float s_ch[2 * kMergeTile];         // c^ of (row n0 + i, 64-block g of the tile) at 2 i + g
     if (threadIdx.x < 16) s_q[threadIdx.x] = cb.q[threadIdx.x];
     const int64_t rows = q.rows, cols = q.cols, kbs = cols / 64;
-    const float mu = *q.offset;
-    const int nn = threadIdx.x >> 2, kk0 = (threadIdx.x & 3) * 16;
-    const int64_t tiles_n = (rows + 63) / 64, tiles = tiles_n * kbs;
-    for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-        const int64_t n0 = (tile % tiles_n) * 64, k0 = (tile / tiles_n) * 64;
-        __syncthreads();   // previous tile's readers are done
-        for (int i = threadIdx.x; i < r * 64; i += blockDim.x) {
-            const int j = i / 64, c = i % 64;
-            As[j * 64 + c] = __bfloat162float(A[(k0 + c) * r + j]);
-            Bs[j * 64 + c] = (n0 + c < rows) ? __bfloat162float(B[(int64_t)j * rows + n0 + c]) : 0.0f;
-        }
-        __syncthreads();
-        const int64_t n = n0 + nn;
-        if (n >= rows) continue;
-        float d[16];
+    const float mu = __ldg(q.offset);
+    const int tn = threadIdx.x >> 4, tk = threadIdx.x & 15;
+    const int64_t tiles_n = (rows + kMergeTile - 1) / kMergeTile;
+    const int64_t tiles_k = (cols + kMergeTile - 1) / kMergeTile;
+    const int64_t tiles = tiles_n * tiles_k;
+    const int nj = (r + kMergeJ - 1) / kMergeJ;
+    const uint32_t sm0 = static_cast<uint32_t>(__cvta_generic_to_shared(msm));
+
+    // copies of step (tile, chunk) into buffer buf: 2048 16-byte pieces, 8 per thread
+    auto issue = [&](int64_t tile, int c, int buf) {
+        const int64_t n0 = (tile % tiles_n) * kMergeTile, k0 = (tile / tiles_n) * kMergeTile;
+        const int j0 = c * kMergeJ;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) d[e] = 0.0f;
-        for (int j = 0; j < r; ++j) {
-            const float b = Bs[j * 64 + nn];
-            const float4 *a4 = reinterpret_cast<const float4 *>(As + j * 64 + kk0);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const float4 a = a4[v];
-                d[4 * v + 0] = fmaf(a.x, b, d[4 * v + 0]);
-                d[4 * v + 1] = fmaf(a.y, b, d[4 * v + 1]);
-                d[4 * v + 2] = fmaf(a.z, b, d[4 * v + 2]);
-                d[4 * v + 3] = fmaf(a.w, b, d[4 * v + 3]);
+        for (int u = 0; u < 8; ++u) {
+            const int piece = threadIdx.x + 256 * (u & 3);          // [jj][c4] of one operand
+            const int jj = piece >> 5, c4 = piece & 31;
+            const int j = j0 + jj;
+            const uint32_t dst = sm0 + (uint32_t)(((buf * 2 + (u >> 2)) * kMergeBuf + jj * kMergeTile + 4 * c4) * 4);
+            if (u < 4) {
+                const int64_t k = k0 + 4 * c4;
+                const bool ok = j < r && k < cols;
+                cp_async16(dst, ok ? At + (int64_t)j * cols + k : At, ok ? 16u : 0u);
+            } else {
+                const int64_t n = n0 + 4 * c4;
+                const bool ok = j < r && n < ldb;
+                cp_async16(dst, ok ? Bf + (int64_t)j * ldb + n : Bf, ok ? 16u : 0u);
             }
         }
-        // dequantise the 16 weights (one 64-block: block n * kbs + k0 / 64) and add
-        const int64_t e0 = n * cols + k0 + kk0;
-        const int64_t blk = n * kbs + k0 / 64;
-        const float ch = dq_constant(q.scale8[blk], q.scale2[blk / kBlock2], mu);
-        const uint2 cw = *reinterpret_cast<const uint2 *>(q.codes + e0 / 2);
-        uint32_t o[8];
+        cp_async_commit();
+    };
+
+    int64_t tile = blockIdx.x;
+    if (tile < tiles) issue(tile, 0, 0);
+    int step = 0;
+    for (; tile < tiles; tile += gridDim.x) {
+        const int64_t n0 = (tile % tiles_n) * kMergeTile, k0 = (tile / tiles_n) * kMergeTile;
+        float d[8][8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const uint32_t byte = ((k < 4 ? cw.x : cw.y) >> (8 * (k & 3))) & 0xffu;
-            const float w_hi = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_q[byte >> 4], ch)));
-            const float w_lo = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_q[byte & 15u], ch)));
-            o[k] = pack_bf16x2(__fadd_rn(w_hi, __fmul_rn(s, d[2 * k])), __fadd_rn(w_lo, __fmul_rn(s, d[2 * k + 1])));
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) d[i][c] = 0.0f;
+        for (int c = 0; c < nj; ++c, ++step) {
+            // the next step's copies go out before this step's wait
+            const bool more = c + 1 < nj || tile + gridDim.x < tiles;
+            if (more) {
+                if (c + 1 < nj) issue(tile, c + 1, (step + 1) & 1);
+                else issue(tile + gridDim.x, 0, (step + 1) & 1);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            __syncthreads();   // this step's buffer is complete for every thread
+            if (c == 0) {
+                const int64_t n = n0 + (threadIdx.x >> 1), blkk = k0 / 64 + (threadIdx.x & 1);
+                s_ch[threadIdx.x] = (n < rows && blkk < kbs)
+                                        ? dq_constant(q.scale8[n * kbs + blkk], q.scale2[(n * kbs + blkk) / kBlock2], mu)
+                                        : 0.0f;
+            }
+            const float *As = msm + (size_t)((step & 1) * 2) * kMergeBuf;
+            const float *Bs = As + kMergeBuf;
+            const int jn = r - c * kMergeJ < kMergeJ ? r - c * kMergeJ : kMergeJ;
+#pragma unroll 2
+            for (int jj = 0; jj < jn; ++jj) {
+                const float4 a0 = *reinterpret_cast<const float4 *>(As + jj * kMergeTile + 4 * tk);
+                const float4 a1 = *reinterpret_cast<const float4 *>(As + jj * kMergeTile + 64 + 4 * tk);
+                const float4 b0 = *reinterpret_cast<const float4 *>(Bs + jj * kMergeTile + 8 * tn);
+                const float4 b1 = *reinterpret_cast<const float4 *>(Bs + jj * kMergeTile + 8 * tn + 4);
+                const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) d[i][cc] = fmaf(a[cc], b[i], d[i][cc]);
+            }
+            __syncthreads();   // every thread is done with this buffer before it is refilled
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(out + e0);
-        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        // dequantise the thread's weights and add: rows n0 + 8 tn + i, inputs
+        // k0 + 64 g + 4 tk .. + 3 (g = 0, 1; each group inside one 64-block)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int64_t n = n0 + 8 * tn + i;
+            if (n >= rows) break;
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                const int64_t k = k0 + 64 * g + 4 * tk;
+                if (k >= cols) continue;
+                const int64_t e0 = n * cols + k;
+                const float ch = s_ch[2 * (8 * tn + i) + g];
+                const uint32_t cw = *reinterpret_cast<const uint16_t *>(q.codes + e0 / 2);
+                uint32_t o[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t byte = (cw >> (8 * h)) & 0xffu;
+                    const float w_hi = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_q[byte >> 4], ch)));
+                    const float w_lo = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_q[byte & 15u], ch)));
+                    o[h] = pack_bf16x2(__fadd_rn(w_hi, __fmul_rn(s, d[i][4 * g + 2 * h])),
+                                       __fadd_rn(w_lo, __fmul_rn(s, d[i][4 * g + 2 * h + 1])));
+                }
+                *reinterpret_cast<uint2 *>(out + e0) = make_uint2(o[0], o[1]);
+            }
+        }
     }
 }
 
+size_t merge_prep_bytes(int64_t rows, int64_t cols) {
+    return align256((size_t)256 * (size_t)cols * 4) + align256((size_t)256 * (size_t)((rows + 3) / 4 * 4) * 4);
+}
+
 cudaError_t launch_merge_bf16(const NF4View &q, const __nv_bfloat16 *A, const __nv_bfloat16 *B, int r, float s,
-                              __nv_bfloat16 *out, cudaStream_t st) {
-    const int64_t tiles = ceil_div(q.rows, (int64_t)64) * (q.cols / 64);
+                              __nv_bfloat16 *out, void *prep, cudaStream_t st) {
+    const int64_t ldb = (q.rows + 3) / 4 * 4;
+    float *At = static_cast<float *>(prep);
+    float *Bf = reinterpret_cast<float *>(static_cast<char *>(prep) + align256((size_t)256 * (size_t)q.cols * 4));
+    int64_t px = ceil_div(q.cols > ldb ? q.cols : ldb, (int64_t)256);
+    if (px > 64) px = 64;
+    QNF4_LAUNCH("k_merge_prep", st,
+                k_merge_prep<<<dim3((unsigned)px, (unsigned)r), 256, 0, st>>>(A, B, r, q.cols, q.rows, ldb, At, Bf));
+    const int64_t tiles = ceil_div(q.rows, (int64_t)kMergeTile) * ceil_div(q.cols, (int64_t)kMergeTile);
     int64_t grid = tiles;
-    const int64_t cap = (int64_t)num_sms() * 4;
+    const int64_t cap = (int64_t)num_sms() * 2;
     if (grid > cap) grid = cap;
-    const size_t sm = (size_t)r * 64 * 4 * 2;
-    cudaError_t e = cudaFuncSetAttribute(k_merge_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e != cudaSuccess) return e;
-    QNF4_LAUNCH("k_merge_bf16", st, k_merge_bf16<<<(unsigned)grid, 256, sm, st>>>(q, A, B, r, s, host_codebook(), out));
+    static const cudaError_t attr =
+        cudaFuncSetAttribute(k_merge_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMergeSmem);
+    if (attr != cudaSuccess) return attr;
+    QNF4_LAUNCH("k_merge_bf16", st,
+                k_merge_bf16<<<(unsigned)grid, 256, kMergeSmem, st>>>(q, At, Bf, ldb, r, s, host_codebook(), out));
     return cudaGetLastError();
 }
 
@@ -512,12 +724,12 @@ static std::atomic<int> g_divide_every_weight{0};
 // Three launches over up to kQuantMaxItems tensors of one input dtype.
 static cudaError_t quantize_launch(const QuantArgs *a, int count, qlora_dtype dt, cudaStream_t st) {
     const Codebook &cb = host_codebook();
-    static CodeBins bins;
-    static const bool bins_ok = build_code_bins(cb, bins);
-    const bool use_bins = bins_ok && g_divide_every_weight.load() == 0;
+    static CodeTable table;
+    static const bool table_ok = build_code_table(cb, table);
+    const bool use_bins = table_ok && g_divide_every_weight.load() == 0;
     QuantGroup g;
     g.count = count;
-    int64_t ctas = 0, dq = 0;
+    int64_t groups = 0, dq = 0;
     for (int i = 0; i < count; ++i) {
         QuantItem &it = g.it[i];
         it.W = a[i].W;
@@ -530,22 +742,36 @@ static cudaError_t quantize_launch(const QuantArgs *a, int count, qlora_dtype dt
         it.scale8 = a[i].out.scale8;
         it.scale2 = a[i].out.scale2;
         it.offset = a[i].out.offset;
-        it.cta0 = ctas;
+        it.cta0 = groups;
         it.dq0 = dq;
-        ctas += it.nb2;
+        groups += it.nb2;
         dq += ceil_div(it.nb2, 8);
     }
-    if (ctas > 0x7fffffffLL || dq > 0x7fffffffLL) return cudaErrorInvalidValue;
+    g.groups = groups;
+    if (dq > 0x7fffffffLL) return cudaErrorInvalidValue;
+    // persistent: three 256-thread CTAs per SM (65 KB of shared memory each)
+    int64_t grid = groups;
+    const int64_t cap = (int64_t)num_sms() * 3;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    const unsigned gx = (unsigned)grid;
+    const size_t tab_bytes = (size_t)256 * 32 * sizeof(float2);
+    static const bool attr_ok =
+        cudaFuncSetAttribute(k_quantize_codes<float, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tab_bytes) == cudaSuccess &&
+        cudaFuncSetAttribute(k_quantize_codes<__nv_bfloat16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tab_bytes) == cudaSuccess;
+    if (!attr_ok) return cudaErrorInvalidValue;
     if (dt == QLORA_F32) {
         if (use_bins)
-            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<float, true><<<(unsigned)ctas, 256, 0, st>>>(g, cb, bins));
+            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<float, true><<<gx, 256, tab_bytes, st>>>(g, cb, table));
         else
-            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<float, false><<<(unsigned)ctas, 256, 0, st>>>(g, cb, bins));
+            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<float, false><<<gx, 256, 0, st>>>(g, cb, table));
     } else {
         if (use_bins)
-            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<__nv_bfloat16, true><<<(unsigned)ctas, 256, 0, st>>>(g, cb, bins));
+            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<__nv_bfloat16, true><<<gx, 256, tab_bytes, st>>>(g, cb, table));
         else
-            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<__nv_bfloat16, false><<<(unsigned)ctas, 256, 0, st>>>(g, cb, bins));
+            QNF4_LAUNCH("k_quantize_codes", st, k_quantize_codes<__nv_bfloat16, false><<<gx, 256, 0, st>>>(g, cb, table));
     }
     QNF4_LAUNCH("k_offset", st, k_offset<<<(unsigned)count, 1024, 0, st>>>(g));
     QNF4_LAUNCH("k_double_quant", st, k_double_quant<<<(unsigned)dq, 256, 0, st>>>(g));

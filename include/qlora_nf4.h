@@ -18,6 +18,17 @@
  *   16-byte aligned unless stated otherwise. The library never allocates or
  *   frees device memory; scratch comes from a caller-provided workspace whose
  *   size the matching *_workspace() query returns.
+ * - Two resources are the library's own. (1) On the first qlora_linear_fwd or
+ *   qlora_linear_bwd call on a device with M >= P (512 by default, see
+ *   qlora_linear_set_pair_min_m) and r > 0, it creates one non-blocking side
+ *   stream and two events for that device, kept until the process exits: those
+ *   calls fork the memory-bound adapter products and the dequantisation onto it
+ *   and join back before they return control of `stream`. (2) A process-wide
+ *   mutex is held for the host-side duration of each such fork/join sequence
+ *   (the launches, not the GPU work), so host threads that issue M >= P calls
+ *   concurrently are serialised while they enqueue. Calls with M < P or r = 0,
+ *   the quantiser, dequantisation, merge, optimizer and grouped forward take no
+ *   lock and create nothing.
  * - bf16 tensors are passed as void pointers to IEEE bfloat16 bit patterns.
  * - The stored weight uses the nn.Linear layout [rows = d_out, cols = d_in],
  *   row-major. The W^ of the layer equation is its transpose.
@@ -133,9 +144,10 @@ qlora_status qlora_nf4_dequant_grouped(int count, const qlora_nf4_tensor *q, voi
  *   XA_save  bf16 [M, r] receives X*A (unscaled) for the backward, or NULL.
  * Shapes: M >= 1, cols % 64 == 0, rows % 16 == 0, 0 <= r <= 256, r % 8 == 0
  * (r == 0: no adapter; A, B, XA_save ignored). M <= 16 takes the streaming GEMV
- * kernel, 16 < M < 512 the fused tcgen05 dequant-GEMM, and M >= 512
- * dequantises W once into bf16 in the workspace (rows * cols * 2 bytes of it)
- * and runs a CTA-pair tcgen05 GEMM with the adapter term as extra K blocks.
+ * kernel, 16 < M < P the fused tcgen05 dequant-GEMM, and M >= P dequantises W
+ * once into bf16 in the workspace (rows * cols * 2 bytes of it) and runs a
+ * CTA-pair tcgen05 GEMM with the adapter term as extra K blocks; P = 512 unless
+ * qlora_linear_set_pair_min_m changed it.
  */
 size_t qlora_linear_fwd_workspace(int64_t M, int64_t rows, int64_t cols, int r);
 qlora_status qlora_linear_fwd(const void *X, int64_t M, const qlora_nf4_tensor *W,
@@ -151,7 +163,7 @@ qlora_status qlora_linear_fwd(const void *X, int64_t M, const qlora_nf4_tensor *
  *   dA = s * X^T * G                       fp32 [cols, r]  (overwritten)
  *   dB = s * (X*A)^T * dY                  fp32 [r, rows]  (overwritten)
  *   XA  bf16 [M, r] saved by the forward, or NULL to recompute it.
- * Shapes as for the forward, with M >= 1. For M >= 512 the workspace also
+ * Shapes as for the forward, with M >= 1. For M >= P the workspace also
  * holds the bf16 dequantised weight (rows * cols * 2 bytes), as in the forward.
  */
 size_t qlora_linear_bwd_workspace(int64_t M, int64_t rows, int64_t cols, int r);
@@ -159,6 +171,16 @@ qlora_status qlora_linear_bwd(const void *X, const void *dY, int64_t M, const ql
                               const void *A, const void *B, int r, float s, const void *XA,
                               void *dX, float *dA, float *dB, void *ws, size_t ws_bytes,
                               qlora_stream_t stream);
+
+/*
+ * Tuning hook of the two large-M routes (the page has no counterpart): sets P, the
+ * token count from which qlora_linear_fwd / qlora_linear_bwd dequantise W once and run
+ * the CTA-pair GEMM instead of the fused dequant-GEMM (default 512; values below 17
+ * are raised to 17, INT64_MAX keeps every M > 16 on the fused kernels). Both routes
+ * compute the same layer; the workspace queries follow P, so query after setting it.
+ * Process-wide; not synchronised with calls in flight on other host threads.
+ */
+void qlora_linear_set_pair_min_m(int64_t m);
 
 /*
  * Forward of several projections at once (the page's equation for each), for
@@ -237,8 +259,9 @@ qlora_status qlora_nf4_quantize_noalloc(const void *W, qlora_dtype dt, const qlo
  * step at step count h->step >= 1, per element and in this order, every operation one
  * IEEE binary32 operation (round to nearest even, no fused multiply-add):
  *   m = b1 m + (1 - b1) g;  v = b2 v + (1 - b2) g g;
- *   upd = (m / bc1) / (sqrt(v / bc2) + eps);  theta = theta - lr (upd + wd theta);
- * bc1 = 1 - b1^step and bc2 = 1 - b2^step are computed in double and rounded to float.
+ *   upd = (m ib1) / (sqrt(v ib2) + eps);  theta = theta - lr (upd + wd theta);
+ * ib1 = 1 / (1 - b1^step) and ib2 = 1 / (1 - b2^step) are computed in double and rounded
+ * to float.
  *   theta, m, v   n fp32 each, updated in place; grad n fp32 (dA or dB of
  *                 qlora_linear_bwd, or both laid out back to back);
  *   theta_bf16    n bf16 receiving bf16(theta), the adapter copy the layer multiplies
@@ -263,11 +286,13 @@ qlora_status qlora_adamw_prefetch(const void *ptr, size_t bytes, int to_device, 
 
 /*
  * Test hook of the quantiser's code search (the page has no counterpart). By default a
- * weight's code is read from a 256-bin table over x' = w * fl(1/c1), and the exact
- * quotient fl(w / c1) with the full threshold search decides wherever x' lies within
- * 4 ulp of the bin's threshold; divide_every_weight != 0 makes every later quantisation
- * in the process divide every weight instead. Both give the same codes bit for bit;
- * the hook lets tests compare them. Not thread-safe with concurrent quantisations.
+ * weight's code is read from a 256-bin table over x' = fl(w * r), r an approximate
+ * reciprocal of c1 (within 1 ulp), and the exact quotient fl(w / c1) with the full
+ * threshold search decides wherever x' lies within 2^-21 of its bin's threshold (or c1
+ * is outside [2^-126, 2^125)); divide_every_weight != 0 makes
+ * every later quantisation in the process divide every weight instead. Both give the
+ * same codes bit for bit; the hook lets tests compare them. Not thread-safe with
+ * concurrent quantisations.
  */
 void qlora_nf4_set_code_search(int divide_every_weight);
 
@@ -284,8 +309,10 @@ void qlora_nf4_set_code_search(int divide_every_weight);
  *   W_bf16 optional device buffer (bf16 [rows, cols], 16-byte aligned) that receives
  *          W'; NULL keeps it in the workspace.
  *   W_out  receives the re-quantised weight (rows, cols as W); it may be W itself.
- *   ws     workspace of qlora_nf4_merge_workspace() bytes.
- * One kernel launch computes W'; the re-quantisation adds three. W' and W_out are
+ *   ws     workspace of qlora_nf4_merge_workspace() bytes: W' when W_bf16 is NULL,
+ *          fp32 copies of A^T and B (sized for r = 256), the quantiser's scratch.
+ * Two kernel launches compute W' (the fp32 copies, then the merge); the
+ * re-quantisation adds three. W' and W_out are
  * bit-for-bit reproducible. A NaN/Inf in W' sets QLORA_ERR_NONFINITE.
  */
 size_t qlora_nf4_merge_workspace(int64_t rows, int64_t cols);
@@ -304,6 +331,16 @@ qlora_status qlora_nf4_merge_adapter(const qlora_nf4_tensor *W, const void *A, c
 qlora_status qlora_selftest_wait_timeout(qlora_stream_t stream);
 
 /*
+ * Self-test of the reciprocal approximation behind the quantiser's fast code search
+ * (the page has no counterpart; the search is exact only while the approximation
+ * stays within a few ulps). Measures |r - 1/m| over every fp32 mantissa m in [1, 2),
+ * exactly in double, in units of r's ulp, and stores the maximum times 1024
+ * (1024 = one ulp) in *max_err_1024, a device word (zeroed first on the stream).
+ * Returns QLORA_ERR_INVALID_ARG for a NULL pointer, QLORA_ERR_CUDA on a launch failure.
+ */
+qlora_status qlora_selftest_rcp_error(unsigned int *max_err_1024, qlora_stream_t stream);
+
+/*
  * Reference 4-bit formats that the page compares NF4 + DQ against: Int4, FP4 E2M1 and FP4 E3M0
  * (page "QLoRA: put the large model in memory, then change it with a small adapter", section 4,
  * evidence 1, the paper's Table 2). The page names them without defining them. The readings:
@@ -320,9 +357,10 @@ qlora_status qlora_selftest_wait_timeout(qlora_stream_t stream);
  * Dequantisation: w^ = bf16(fl(v * fl(c / S))).
  *   W       device, n finite values of dtype dt (fp32 4-byte, bf16 2-byte aligned);
  *   codes   device, ceil(n/2) bytes, byte k = code[2k] << 4 | code[2k+1] (the NF4 packing);
- *           for odd n the missing low nibble is the zero code;
+ *           for odd n the missing low nibble is the zero code; 16-byte aligned for the
+ *           dequantisation;
  *   absmax  device, ceil(n/64) fp32 block constants, 4-byte aligned;
- *   W_out   device, n bf16, 4-byte aligned.
+ *   W_out   device, n bf16, 16-byte aligned.
  * One kernel launch each; QLORA_ERR_INVALID_ARG for a null or misaligned pointer, n < 1 or an
  * unknown format.
  */

@@ -326,9 +326,10 @@ def rel_errors(got, ref):
 # master parameters, fp32 moments; the operation order is in nf4_oracle.c.
 # --------------------------------------------------------------------------
 def adamw_bias_corrections(b1: float, b2: float, t: int):
-    bc1, bc2 = ctypes.c_float(0.0), ctypes.c_float(0.0)
-    lib().orc_adamw_bias_corrections(b1, b2, int(t), ctypes.byref(bc1), ctypes.byref(bc2))
-    return np.float32(bc1.value), np.float32(bc2.value)
+    """Inverse bias corrections (1 / (1 - b1^t), 1 / (1 - b2^t)) in double, rounded once to fp32."""
+    ib1, ib2 = ctypes.c_float(0.0), ctypes.c_float(0.0)
+    lib().orc_adamw_bias_corrections(b1, b2, int(t), ctypes.byref(ib1), ctypes.byref(ib2))
+    return np.float32(ib1.value), np.float32(ib2.value)
 
 
 def adamw_step(theta: np.ndarray, g: np.ndarray, m: np.ndarray, v: np.ndarray, t: int, lr: float,
@@ -338,9 +339,9 @@ def adamw_step(theta: np.ndarray, g: np.ndarray, m: np.ndarray, v: np.ndarray, t
     for a in (theta, g, m, v):
         assert a.dtype == np.float32 and a.flags["C_CONTIGUOUS"]
     n = theta.size
-    bc1, bc2 = adamw_bias_corrections(b1, b2, t)
+    ib1, ib2 = adamw_bias_corrections(b1, b2, t)
     out = np.empty(n, dtype=np.uint16) if want_bf16 else None
-    lib().orc_adamw_step(_ptr(theta), _ptr(g), _ptr(m), _ptr(v), n, lr, b1, b2, eps, wd, float(bc1), float(bc2),
+    lib().orc_adamw_step(_ptr(theta), _ptr(g), _ptr(m), _ptr(v), n, lr, b1, b2, eps, wd, float(ib1), float(ib2),
                          _ptr(out) if want_bf16 else None)
     return out
 

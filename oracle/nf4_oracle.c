@@ -363,14 +363,16 @@ void orc_merge_bf16(const uint16_t *w_hat, const float *A, const float *B, int64
 /* IEEE binary32 operation:                                                   */
 /*   m     = fl( fl(b1 * m) + fl(fl(1 - b1) * g) )                            */
 /*   v     = fl( fl(b2 * v) + fl(fl(1 - b2) * fl(g * g)) )                    */
-/*   mhat  = fl(m / bc1),  vhat = fl(v / bc2)                                 */
-/*   upd   = fl( mhat / fl(fl(sqrt(vhat)) + eps) )                            */
+/*   den   = fl( fl(sqrt(fl(v * ib2))) + eps )                                */
+/*   upd   = fl( fl(m * ib1) / den )                                          */
 /*   theta = fl( theta - fl(lr * fl(upd + fl(wd * theta))) )                  */
-/* with the bias corrections bc1 = (float)(1 - b1^t), bc2 = (float)(1 - b2^t) */
-/* computed in double by the caller. theta_bf16 (optional) receives           */
-/* bf16(theta), the adapter copy the layer multiplies with.                   */
+/* with the inverse bias corrections ib1 = 1 / (1 - b1^t) and                 */
+/* ib2 = 1 / (1 - b2^t) computed by the caller in double and rounded once to  */
+/* float (one division and one square root per element). theta_bf16          */
+/* (optional) receives bf16(theta), the adapter copy the layer multiplies     */
+/* with.                                                                      */
 void orc_adamw_step(float *theta, const float *g, float *m, float *v, int64_t n, float lr, float b1,
-                    float b2, float eps, float wd, float bc1, float bc2, uint16_t *theta_bf16)
+                    float b2, float eps, float wd, float ib1, float ib2, uint16_t *theta_bf16)
 {
     const float c1 = 1.0f - b1, c2 = 1.0f - b2;
 #pragma omp parallel for schedule(static)
@@ -379,9 +381,8 @@ void orc_adamw_step(float *theta, const float *g, float *m, float *v, int64_t n,
         const float mi = b1 * m[i] + c1 * gi;
         const float gg = gi * gi;
         const float vi = b2 * v[i] + c2 * gg;
-        const float mhat = mi / bc1, vhat = vi / bc2;
-        const float den = sqrtf(vhat) + eps;
-        const float upd = mhat / den;
+        const float den = sqrtf(vi * ib2) + eps;
+        const float upd = (mi * ib1) / den;
         const float decay = wd * theta[i];
         const float step = lr * (upd + decay);
         theta[i] = theta[i] - step;
@@ -391,9 +392,9 @@ void orc_adamw_step(float *theta, const float *g, float *m, float *v, int64_t n,
     }
 }
 
-/* Bias corrections of step t (double, rounded once to float). */
-void orc_adamw_bias_corrections(float b1, float b2, int64_t t, float *bc1, float *bc2)
+/* Inverse bias corrections of step t (double, rounded once to float). */
+void orc_adamw_bias_corrections(float b1, float b2, int64_t t, float *ib1, float *ib2)
 {
-    *bc1 = (float)(1.0 - pow((double)b1, (double)t));
-    *bc2 = (float)(1.0 - pow((double)b2, (double)t));
+    *ib1 = (float)(1.0 / (1.0 - pow((double)b1, (double)t)));
+    *ib2 = (float)(1.0 / (1.0 - pow((double)b2, (double)t)));
 }

@@ -138,6 +138,7 @@ def test_fmt4_argument_checks_run_on_host():
     assert L.qlora_fmt4_quantize(fake, 2, 64, 0, fake, fake, None) == q.QLORA_ERR_INVALID_ARG      # dtype
     assert L.qlora_fmt4_quantize(ctypes.c_void_p((1 << 20) + 2), 0, 64, 0, fake, fake, None) == q.QLORA_ERR_INVALID_ARG
     assert L.qlora_fmt4_dequant(fake, fake, 64, 1, ctypes.c_void_p((1 << 20) + 2), None) == q.QLORA_ERR_INVALID_ARG
+    assert L.qlora_fmt4_dequant(ctypes.c_void_p((1 << 20) + 8), fake, 64, 1, fake, None) == q.QLORA_ERR_INVALID_ARG
 
 
 def test_grouped_workspace_is_largest_group_of_eight():

@@ -308,3 +308,18 @@ def test_many_tiles_per_cta_full(rep):
         check(f64(dX), dXr, f"dX[{rows}x{cols}]")
         check(f64(dA), dAr, f"dA[{rows}x{cols}]")
         check(f64(dB), dBr, f"dB[{rows}x{cols}]")
+
+
+@pytest.mark.parametrize("P,M,rows,cols,r", [
+    (2 ** 62, 1024, 512, 1024, 16),   # the fused dequant-GEMM at four token tiles
+    (2 ** 62, 4096, 256, 512, 64),    # ... and at the headline's 4096 tokens
+    (17, 100, 400, 320, 24),          # the dequant + CTA-pair route below one 256-token tile
+    (17, 300, 272, 192, 64),
+])
+def test_routes_forced_either_way(P, M, rows, cols, r):
+    # both large-M routes compute the same layer at any token count
+    q.lib().qlora_linear_set_pair_min_m(P)
+    try:
+        run_case(M, rows, cols, r, seed=M + rows + r + 7)
+    finally:
+        q.lib().qlora_linear_set_pair_min_m(512)

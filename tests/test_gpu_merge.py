@@ -36,7 +36,8 @@ def check_merge(W, A, B, s, in_place=False):
     return out
 
 
-@pytest.mark.parametrize("rows,cols,r", [(100, 192, 8), (64, 64, 1), (257, 320, 24), (128, 256, 256)])
+@pytest.mark.parametrize("rows,cols,r", [(100, 192, 8), (64, 64, 1), (257, 320, 24), (128, 256, 256),
+                                         (300, 448, 40), (1, 64, 33)])
 def test_merge_small_ragged(rows, cols, r):
     W = si.normal((rows, cols), 0.02, seed=rows + cols, device="cuda")
     A = si.normal((cols, r), 0.05, seed=rows + 1, device="cuda", dtype=torch.bfloat16)

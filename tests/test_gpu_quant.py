@@ -67,6 +67,22 @@ def test_special_blocks():
     assert_bit_exact(W)
 
 
+def test_extreme_absmax_blocks():
+    # blocks whose absmax has no normal reciprocal (subnormal, or above 2^125) take the
+    # exact path; blocks just inside the range take the table; all match the oracle
+    rng = np.random.default_rng(11)
+    scales = [1e-45, 3e-40, 2.9e-39, 1.2e-38, 3e-38, 1e-30, 1.0, 4.2e37, 4.3e37, 1e38, 3.3e38]
+    blocks = []
+    for c in scales:
+        b = (rng.standard_normal(64) * 0.3).astype(np.float32)
+        b[rng.integers(64)] = 1.0
+        blocks.append((b * np.float32(c)).astype(np.float32))
+    w = np.concatenate(blocks)
+    W = torch.from_numpy(w).view(1, -1).cuda()
+    assert np.isfinite(w).all()
+    assert_bit_exact(W)
+
+
 def test_outliers_full_4096():
     wl = si.workload("l4096")
     W = si.layer_inputs(wl, 0, device="cuda", M=0)["W"]
@@ -108,6 +124,16 @@ def test_bounded_wait_reports_timeout():
     assert q.qlora_get_device_status() == q.QLORA_OK
     ref = oracle.quantize(W.cpu().numpy())
     assert np.array_equal(t.codes.cpu().numpy(), ref.codes)
+
+
+def test_reciprocal_approximation_within_one_ulp():
+    # the fast code search is exact only while the hardware reciprocal stays within a few
+    # ulps (its band is sized for 4); every mantissa of [1, 2) is measured
+    out = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert q.lib().qlora_selftest_rcp_error(out.data_ptr(), None) == q.QLORA_OK
+    torch.cuda.synchronize()
+    err_ulps = int(out.item()) / 1024.0
+    assert err_ulps <= 1.0, err_ulps
 
 
 def test_llama7b_layer_full_bf16():
@@ -215,8 +241,8 @@ def _band_weights_bf16():
 @pytest.mark.parametrize("divide_every_weight", [0, 1])
 def test_threshold_band_both_code_searches(divide_every_weight):
     # weights whose normalised value lies within a few ulps of a decision threshold: the
-    # bin table's x' = w fl(1/c1) is then inside its 4-ulp fallback band, where the exact
-    # quotient decides. Both code searches (table with fallback; a division per weight)
+    # bin table's x' (w times an approximate 1/c1) is then inside its fallback band
+    # (|x' - T| <= 2^-21), where the exact quotient decides. Both code searches (table with fallback; a division per weight)
     # must match the oracle bit for bit, in fp32 and for the closest bf16 pairs.
     rng = np.random.default_rng(5)
     w32 = _band_weights_fp32(rng)
