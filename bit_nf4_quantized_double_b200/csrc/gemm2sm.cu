@@ -19,15 +19,10 @@
 // issued by rank 0 reads both CTAs' halves, and each CTA's TMEM receives its
 // 128 accumulator rows. Per SM that is 8 KB of operand reads per K16 step, half
 // of what a one-SM 128 x 256 tile with both operands in shared memory needs.
-// Persistent stream-K: the tiles' K blocks, tile after tile, are cut into one
-// contiguous run per pair, equal to within one block, so every pair gets the same
-// work whatever the tile count (with a pair count that divides the tiles, each run
-// is whole tiles and no partials are written). A pair whose run starts inside a tile (it
-// holds that tile's last K blocks, and processes them first) writes its fp32
-// accumulator to the workspace and raises a flag; the pair holding the tile's
-// first blocks (its last work) adds those partials in pair order before the
-// epilogue. Two accumulators in TMEM let the epilogue of one tile overlap the
-// main loop of the next.
+// Persistent: pair p takes whole tiles p, p + pairs, p + 2 pairs, ..., so that at any
+// moment the pairs work on neighbouring tiles, which share the operand panels in L2.
+// Two accumulators in TMEM let the epilogue of one tile overlap the main loop of the
+// next.
 #include "launch.h"
 #include "tc.cuh"
 #include "tmap.h"
@@ -52,32 +47,7 @@ struct G2Params {
     int KB, KBE;       // main and extension K blocks of 64
     int ke;            // extension K extent (the extension blocks' MMAs stop at it)
     int tiles_m, tiles_n;
-    int64_t iters;     // tiles x (KB + KBE): the K blocks of all tiles, cut into one run per pair
-    float *partial;    // [pairs][2 CTAs][256 columns][128 rows] fp32 accumulators of runs that start mid-tile
-    int *flags;        // [pairs][2 CTAs]: 1 once that partial is written (zero before the launch)
 };
-
-// The run of pair q: K-block iterations [run_begin(q), run_begin(q + 1)).
-__device__ __forceinline__ int64_t run_begin(const G2Params &p, int q, int npairs) {
-    return p.iters * q / npairs;
-}
-// The segments of a pair's run, one per tile it touches: tile, first and end K block.
-struct Seg {
-    int tile, kb0, kb1;
-};
-__device__ __forceinline__ bool next_seg(const G2Params &p, int KBT, int64_t &g, int64_t e, Seg &sg) {
-    if (g >= e) return false;
-    sg.tile = (int)(g / KBT);
-    sg.kb0 = (int)(g - (int64_t)sg.tile * KBT);
-    sg.kb1 = (int)min((int64_t)KBT, e - (int64_t)sg.tile * KBT);
-    g = (int64_t)sg.tile * KBT + sg.kb1;
-    return true;
-}
-__device__ __forceinline__ int ld_acquire(const int *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 
 template <bool B_MN, bool BE_MN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(g2::kThreads, 1)
@@ -126,6 +96,7 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
     volatile int *abort = &s_abort;
 
     const int KBT = p.KB + p.KBE;
+    const int ntiles = p.tiles_m * p.tiles_n;
     const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
 
     if (warp == 0) {
@@ -133,14 +104,10 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
         if (lane == 0) {
             uint32_t st = 0, ph = 0;
             bool ok = true;
-            int64_t g = run_begin(p, pair, npairs);
-            const int64_t ge = run_begin(p, pair + 1, npairs);
-            Seg sg;
-            while (ok && next_seg(p, KBT, g, ge, sg)) {
-                const int tile = sg.tile;
+            for (int tile = pair; tile < ntiles && ok; tile += npairs) {
                 const int m0 = (tile % p.tiles_m) * kTileM + (int)rank * kHalf;
                 const int n0 = (tile / p.tiles_m) * kTileN + (int)rank * kHalf;
-                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+                for (int kb = 0; kb < KBT; ++kb) {
                     if (!mbar_wait(empty(st), ph ^ 1u, abort)) { ok = false; break; }
                     const uint32_t fb = map_to_rank(full(st), 0);
                     if (rank == 0) mbar_arrive_expect_tx(full(st), 2 * kStage);
@@ -179,15 +146,12 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
             constexpr uint32_t kStageDesc = kStage >> 4;
             uint32_t st = 0, ph = 0, lt = 0;
             bool ok = true;
-            int64_t g = run_begin(p, pair, npairs);
-            const int64_t ge = run_begin(p, pair + 1, npairs);
-            Seg sg;
-            for (; ok && next_seg(p, KBT, g, ge, sg); ++lt) {
+            for (int tile = pair; tile < ntiles && ok; tile += npairs, ++lt) {
                 const uint32_t acc = lt & 1u, use = lt >> 1;
                 if (!mbar_wait_cluster(tempty(acc), (use & 1u) ^ 1u, abort)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + acc * 256u;
-                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+                for (int kb = 0; kb < KBT; ++kb) {
                     if (!mbar_wait(full(st), ph, abort)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t ad = adesc0 + st * kStageDesc;
@@ -196,13 +160,13 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
                             mma_pair_ss(d, ad + 2u * k, bd + (B_MN ? 128u : 2u) * k, idesc_main,
-                                        (kb != sg.kb0 || k != 0) ? 1u : 0u);
+                                        (kb != 0 || k != 0) ? 1u : 0u);
                     } else {
                         const uint64_t bd = (BE_MN ? bm0 : bk0) + st * kStageDesc;
                         const int nk = min(4, (p.ke - (kb - p.KB) * 64 + 15) / 16);
                         for (int k = 0; k < nk; ++k)
                             mma_pair_ss(d, ad + 2u * k, bd + (BE_MN ? 128u : 2u) * k, idesc_ext,
-                                        (kb != sg.kb0 || k != 0) ? 1u : 0u);
+                                        (kb != 0 || k != 0) ? 1u : 0u);
                     }
                     mma_pair_commit(empty(st), 0x3);
                     if (++st == (uint32_t)kStages) { st = 0; ph ^= 1u; }
@@ -222,35 +186,13 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
         const int row = q * 32 + lane;                 // TMEM lane = tile row within this CTA
         const uint32_t tempty0 = map_to_rank(tempty(0), 0), tempty1 = map_to_rank(tempty(1), 0);
         uint32_t lt = 0;
-        int64_t g = run_begin(p, pair, npairs);
-        const int64_t ge = run_begin(p, pair + 1, npairs);
-        Seg sg;
-        for (; next_seg(p, KBT, g, ge, sg); ++lt) {
-            const int tile = sg.tile;
+        for (int tile = pair; tile < ntiles; tile += npairs, ++lt) {
             const uint32_t acc = lt & 1u, use = lt >> 1;
             if (!mbar_wait(tfull(acc), use & 1u, abort)) break;
             tc_fence_after();
             const int m0 = (tile % p.tiles_m) * kTileM + (int)rank * kHalf;
             const int n0 = (tile / p.tiles_m) * kTileN;
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * 256u;
-            // this run started inside the tile: its accumulator goes to the workspace
-            const bool to_partial = sg.kb0 > 0;
-            // this run holds the tile's first blocks but not its last: later runs' partials are added
-            const bool add_partials = sg.kb0 == 0 && sg.kb1 < KBT;
-            const int64_t tile_end = (int64_t)(tile + 1) * KBT;
-            if (add_partials) {
-                // every later pair whose run reaches into this tile has written (and flagged) its part
-                const uint64_t t0 = global_timer_ns();
-                for (int qq = pair + 1; qq < npairs && run_begin(p, qq, npairs) < tile_end; ++qq)
-                    while (ld_acquire(p.flags + 2 * qq + rank) == 0) {
-                        if (*abort) break;
-                        if (global_timer_ns() - t0 > kWaitLimitNs) {
-                            *abort = 1;
-                            raise_status(QLORA_ERR_TIMEOUT);
-                            break;
-                        }
-                    }
-            }
 #pragma unroll 1
             for (int part = 0; part < 4; ++part) {     // 64 output columns each
                 uint32_t v[32], w[32];
@@ -262,26 +204,6 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(acc ? tempty1 : tempty0);
-                }
-                if (to_partial) {
-                    // column-major [256][128]: each column's 32 rows of a warp are one 128-byte store
-                    float *dst = p.partial + ((int64_t)(2 * pair + (int)rank) * 256 + part * 64) * 128 + row;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        dst[(int64_t)i * 128] = __uint_as_float(v[i]);
-                        dst[(int64_t)(32 + i) * 128] = __uint_as_float(w[i]);
-                    }
-                    continue;
-                }
-                if (add_partials) {
-                    for (int qq = pair + 1; qq < npairs && run_begin(p, qq, npairs) < tile_end; ++qq) {
-                        const float *src = p.partial + ((int64_t)(2 * qq + (int)rank) * 256 + part * 64) * 128 + row;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            v[i] = __float_as_uint(__uint_as_float(v[i]) + __ldcg(src + (int64_t)i * 128));
-                            w[i] = __float_as_uint(__uint_as_float(w[i]) + __ldcg(src + (int64_t)(32 + i) * 128));
-                        }
-                    }
                 }
                 uint8_t *stg = staging + (part & 1) * kPart;
                 if (et == 0) bulk_wait_read1();        // the store that last read this buffer is done
@@ -302,12 +224,6 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
                     bulk_commit();
                 }
             }
-            if (to_partial) {
-                // all four epilogue warps' stores are visible before the flag
-                __threadfence();
-                named_bar_sync(1, 128);
-                if (et == 0) atomicExch(p.flags + 2 * pair + (int)rank, 1);
-            }
         }
         if (et == 0) bulk_wait0();
     }
@@ -321,11 +237,6 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
     }
 }
 
-// Workspace of launch_gemm2sm with `pairs` CTA pairs: the fp32 accumulators of runs that
-// start inside a tile ([pairs][2][256][128]) and their flags ([pairs][2] ints).
-size_t gemm2sm_workspace_bytes(int pairs) {
-    return align256((size_t)pairs * 2 * 256 * 128 * 4) + align256((size_t)pairs * 2 * 4);
-}
 int gemm2sm_pairs(int max_pairs) {
     const int all = num_sms() / 2;
     return (max_pairs > 0 && max_pairs < all) ? max_pairs : all;
@@ -335,13 +246,12 @@ int gemm2sm_pairs(int max_pairs) {
 // A, Ae: K-major bf16 (row strides K and ke). B: K-major [N][K] or, with
 // b_mn, stored [K][N]. Be likewise with be_mn. ke == 0: no extension.
 // K, N, ke multiples of 8 (16-byte row strides); all pointers 16-byte aligned.
-// `pairs` CTA pairs (gemm2sm_pairs) share the work stream-K; ws holds
-// gemm2sm_workspace_bytes(pairs) bytes.
+// `pairs` CTA pairs (at most gemm2sm_pairs(0)) share the tiles.
 cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, const __nv_bfloat16 *B, bool b_mn,
                            const __nv_bfloat16 *Be, bool be_mn, __nv_bfloat16 *C, int64_t M, int64_t N, int64_t K,
-                           int ke, int pairs, void *ws, cudaStream_t st) {
+                           int ke, int pairs, cudaStream_t st) {
     using namespace g2;
-    if (M < 1 || N < 1 || K < 1 || K % 8 != 0 || N % 8 != 0 || ke < 0 || ke % 8 != 0 || pairs < 1 || !ws)
+    if (M < 1 || N < 1 || K < 1 || K % 8 != 0 || N % 8 != 0 || ke < 0 || ke % 8 != 0 || pairs < 1)
         return cudaErrorInvalidValue;
     CUtensorMap ta, tae, tb, tbe, tcm;
     bool ok = map_bf16(&ta, A, (uint64_t)K, (uint64_t)M, 64, kHalf);
@@ -365,12 +275,9 @@ cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, cons
     p.ke = ke;
     p.tiles_m = (int)ceil_div(M, kTileM);
     p.tiles_n = (int)ceil_div(N, kTileN);
-    p.iters = (int64_t)p.tiles_m * p.tiles_n * (p.KB + p.KBE);
-    p.partial = static_cast<float *>(ws);
-    p.flags = reinterpret_cast<int *>(static_cast<char *>(ws) + align256((size_t)pairs * 2 * 256 * 128 * 4));
-    if (p.iters < pairs) pairs = (int)p.iters;     // at least one K block per pair
-    cudaError_t e = cudaMemsetAsync(p.flags, 0, (size_t)pairs * 2 * sizeof(int), st);
-    if (e != cudaSuccess) return e;
+    const int ntiles = p.tiles_m * p.tiles_n;
+    if (pairs > ntiles) pairs = ntiles;            // at least one tile per pair
+    cudaError_t e;
 #define QNF4_G2(BM, BEM)                                                                                  \
     e = set_smem(k_gemm2sm<BM, BEM>, kSmem);                                                            \
     if (e != cudaSuccess) return e;                                                                      \

@@ -1000,19 +1000,20 @@ static size_t fwd_adapter_bytes(int64_t M, int64_t cols, int r) {
 }
 
 // CTA pairs of the pair GEMM: as few pairs as give the same number of tile rounds. The
-// GEMM is bound by the power cap more than by the SM count (measured: stream-K over every
-// SM was 0.6 % slower at 4096^2 than 64 pairs of four whole tiles), and the SMs left over
-// run the side stream's adapter gradients beside the dgrad GEMM.
+// GEMM is bound by the power cap more than by the SM count (measured: a stream-K split of
+// the K blocks over every SM was 0.6 % slower at 4096^2 than 64 pairs of four whole tiles,
+// and its contiguous per-pair runs lost the L2 reuse of the strided tile order on the
+// 70B-like projections), and the SMs left over run the side stream's adapter gradients
+// beside the dgrad GEMM.
 static int side_job_pairs(int64_t M, int64_t N) {
     const int64_t ntiles = ceil_div(M, 256) * ceil_div(N, 256);
     const int max_pairs = gemm2sm_pairs(0);
     const int64_t rounds = ceil_div(ntiles, max_pairs);
     return (int)ceil_div(ntiles, rounds);
 }
-static size_t g2_bytes() { return gemm2sm_workspace_bytes(gemm2sm_pairs(0)); }
 
 size_t fwd_workspace_bytes_large(int64_t M, int64_t rows, int64_t cols, int r) {
-    return fwd_adapter_bytes(M, cols, r) + (pair_route(M) ? wd_bytes(rows, cols) + g2_bytes() : 0);
+    return fwd_adapter_bytes(M, cols, r) + (pair_route(M) ? wd_bytes(rows, cols) : 0);
 }
 
 static size_t bwd_adapter_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
@@ -1028,7 +1029,7 @@ static size_t bwd_adapter_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
 }
 
 size_t bwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
-    return bwd_adapter_bytes(M, rows, cols, r) + (pair_route(M) ? wd_bytes(rows, cols) + g2_bytes() : 0);
+    return bwd_adapter_bytes(M, rows, cols, r) + (pair_route(M) ? wd_bytes(rows, cols) : 0);
 }
 
 static cudaError_t run_fused_fwd(const __nv_bfloat16 *X, int64_t M, const NF4View &W, const __nv_bfloat16 *XAs,
@@ -1156,8 +1157,7 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
         } else if ((e = launch_dequant(W, Wd, st)) != cudaSuccess) {
             return e;
         }
-        void *g2ws = reinterpret_cast<char *>(Wd) + wd_bytes(W.rows, W.cols);
-        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, side_job_pairs(M, W.rows), g2ws, st);
+        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, side_job_pairs(M, W.rows), st);
     }
     return run_fused_fwd(X, M, W, XAs, B, r, Y, st);
 }
@@ -1236,8 +1236,7 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
             if (side) {
                 float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + 2 * mr_bytes(M, r));
                 if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
-                e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, side_job_pairs(M, W.cols),
-                                   reinterpret_cast<char *>(Wd) + wd_bytes(W.rows, W.cols), st);
+                e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, side_job_pairs(M, W.cols), st);
                 if (e != cudaSuccess) return e;
                 if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
                 e = adapter_grads(X, dY, M, W, Gs, XA, r, s, dA, dB, part, side->s);
@@ -1246,8 +1245,7 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
                 return cudaStreamWaitEvent(st, side->join, 0);
             }
         }
-        e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, gemm2sm_pairs(0),
-                           reinterpret_cast<char *>(Wd) + wd_bytes(W.rows, W.cols), st);
+        e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, side_job_pairs(M, W.cols), st);
     } else {
         e = run_fused_dgrad(dY, M, W, A, Gs, r, dX, st);
     }

@@ -14,7 +14,7 @@
 //                  count, one per CTA; writes each unit's fp32 sums to the workspace.
 //                  RG = 2 row groups for M <= 8, 1 for larger M (whose X fragments
 //                  need twice the registers);
-//   k_gemv_xa      one warp per (adapter, 512 inputs): the X A partial sums, run
+//   k_gemv_xa      one warp per (adapter, 128 inputs): the X A partial sums, run
 //                  beside the GEMV (no shared memory, so its warps fit next to a
 //                  GEMV CTA);
 //   k_gemv_finish  one thread per output element: Y = the K chunks' sums in chunk order
@@ -101,7 +101,7 @@ __device__ __forceinline__ void sts128u(uint32_t a, uint4 v) {
 }
 
 // ---------------------------------------------------------------- adapter product
-constexpr int kXaChunk = 512;                   // inputs per k_gemv_xa warp
+constexpr int kXaChunk = 128;                   // inputs per k_gemv_xa warp
 struct XaItem {
     const __nv_bfloat16 *X;      // [M, K]
     const __nv_bfloat16 *A;      // [K, r]
@@ -113,7 +113,7 @@ struct XaGroup {
     int n, M;
 };
 
-// X A over one 512-input chunk: mma m16n8k16 with X rows (tokens, zero past M) as A
+// X A over one 128-input chunk: mma m16n8k16 with X rows (tokens, zero past M) as A
 // and the adapter's columns as B, the chunk's 32 16-input steps in order.
 __global__ void __launch_bounds__(32) k_gemv_xa(const __grid_constant__ XaGroup grp) {
     griddep_launch_dependents();
@@ -425,43 +425,55 @@ __device__ __forceinline__ void gemv_compute(const GemvGroup &grp, const uint8_t
             const float4 c1 = ld128(hole(s * ROWS + rg * 16 + g + 8) + ((ks ^ g) << 4));
             const float ch0[4] = {c0.x, c0.y, c0.z, c0.w}, ch1[4] = {c1.x, c1.y, c1.z, c1.w};
             const uint8_t *sb = stages + s * STAGE;
-            // one 64-block: 16 table lookups, 4 NT MMAs, the block's c^ on the partial sums
-            auto block = [&](int b) {
-                const uint32_t off = (uint32_t)(((2 * b + (t >> 1)) ^ g) << 4);
-                const uint2 w0 = *reinterpret_cast<const uint2 *>(sb + box_row0 + off);
-                const uint2 w1 = *reinterpret_cast<const uint2 *>(sb + box_row1 + off);
-                float cbk[NT][4];
+            // IB 64-blocks at a time: their code words loaded first, then for each of the four
+            // 16-input steps the lookups and MMAs of every block, so the blocks' MMA chains
+            // (one accumulator per block, since each block has its own c^) overlap
+            constexpr int IB = NT == 1 ? 4 : 2;
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) cbk[nt][0] = cbk[nt][1] = cbk[nt][2] = cbk[nt][3] = 0.0f;
+            for (int b0 = 0; b0 < 4; b0 += IB) {
+                uint2 w0[IB], w1[IB];
+#pragma unroll
+                for (int bi = 0; bi < IB; ++bi) {
+                    const uint32_t off = (uint32_t)(((2 * (b0 + bi) + (t >> 1)) ^ g) << 4);
+                    w0[bi] = *reinterpret_cast<const uint2 *>(sb + box_row0 + off);
+                    w1[bi] = *reinterpret_cast<const uint2 *>(sb + box_row1 + off);
+                }
+                float cbk[IB][NT][4];
+#pragma unroll
+                for (int bi = 0; bi < IB; ++bi)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) cbk[bi][nt][0] = cbk[bi][nt][1] = cbk[bi][nt][2] = cbk[bi][nt][3] = 0.0f;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const uint32_t r0 = (j < 2) ? w0.x : w0.y;
-                    const uint32_t r1 = (j < 2) ? w1.x : w1.y;
                     // byte k of the word, times 256, plus lane * 4: one permute
                     const uint32_t slo = 0x5504u | ((uint32_t)(2 * (j & 1)) << 4), shi = slo + 0x10u;
-                    uint32_t a[4];
-                    a[0] = ld32(prmt(r0, lane4, slo));
-                    a[2] = ld32(prmt(r0, lane4, shi));
-                    a[1] = ld32(prmt(r1, lane4, slo));
-                    a[3] = ld32(prmt(r1, lane4, shi));
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(cbk[nt], a, xf[nt][b][2 * j], xf[nt][b][2 * j + 1]);
+                    for (int bi = 0; bi < IB; ++bi) {
+                        if (b0 + bi >= nblk) continue;
+                        const uint32_t r0 = (j < 2) ? w0[bi].x : w0[bi].y;
+                        const uint32_t r1 = (j < 2) ? w1[bi].x : w1[bi].y;
+                        uint32_t a[4];
+                        a[0] = ld32(prmt(r0, lane4, slo));
+                        a[2] = ld32(prmt(r0, lane4, shi));
+                        a[1] = ld32(prmt(r1, lane4, slo));
+                        a[3] = ld32(prmt(r1, lane4, shi));
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+                            mma_bf16_16816(cbk[bi][nt], a, xf[nt][b0 + bi][2 * j], xf[nt][b0 + bi][2 * j + 1]);
+                    }
                 }
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    acc[nt][0] = fmaf(ch0[b], cbk[nt][0], acc[nt][0]);
-                    acc[nt][1] = fmaf(ch0[b], cbk[nt][1], acc[nt][1]);
-                    acc[nt][2] = fmaf(ch1[b], cbk[nt][2], acc[nt][2]);
-                    acc[nt][3] = fmaf(ch1[b], cbk[nt][3], acc[nt][3]);
+                for (int bi = 0; bi < IB; ++bi) {
+                    if (b0 + bi >= nblk) continue;
+                    const int b = b0 + bi;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        acc[nt][0] = fmaf(ch0[b], cbk[bi][nt][0], acc[nt][0]);
+                        acc[nt][1] = fmaf(ch0[b], cbk[bi][nt][1], acc[nt][1]);
+                        acc[nt][2] = fmaf(ch1[b], cbk[bi][nt][2], acc[nt][2]);
+                        acc[nt][3] = fmaf(ch1[b], cbk[bi][nt][3], acc[nt][3]);
+                    }
                 }
-            };
-            if (nblk == 4) {
-#pragma unroll
-                for (int b = 0; b < 4; ++b) block(b);
-            } else {
-#pragma unroll
-                for (int b = 0; b < 4; ++b)
-                    if (b < nblk) block(b);
             }
         }
         __syncwarp();
@@ -640,7 +652,7 @@ k_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ Codebook c
 static int rows_for(int64_t M) { return M <= 8 ? gemv_rows(1) : gemv_rows(2); }
 
 // Workspace of one launch group: fp32 K-chunk sums [nch][N][M] per projection and
-// X A chunk partials [K/512][M][r] per adapter, each region 256-byte aligned.
+// X A chunk partials [K/128][M][r] per adapter, each region 256-byte aligned.
 static size_t group_workspace(int64_t M, int count, const LinearDesc *d) {
     size_t b = 0;
     for (int i = 0; i < count; ++i) {

@@ -65,12 +65,9 @@ def test_workspace_queries_positive():
         assert L.qlora_linear_bwd_workspace(M, 4096, 4096, 64) > 0
     # no adapter and a small batch: nothing to stage
     assert L.qlora_linear_bwd_workspace(256, 4096, 4096, 0) == 0
-    # from 512 tokens on, the layer keeps a bf16 copy of the dequantised weight, plus the
-    # pair GEMM's stream-K partials (one 256 x 256 fp32 tile per CTA pair, 74 pairs on 148
-    # SMs, the count assumed without a GPU) and their flags
-    g2 = 74 * 256 * 256 * 4 + 768
-    assert L.qlora_linear_bwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2 + g2
-    assert L.qlora_linear_fwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2 + g2
+    # from 512 tokens on, the layer keeps a bf16 copy of the dequantised weight
+    assert L.qlora_linear_bwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2
+    assert L.qlora_linear_fwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2
 
 
 def test_grouped_forward_host_checks():
@@ -85,10 +82,10 @@ def test_grouped_forward_host_checks():
     # region 256-byte aligned
     assert L.qlora_linear_fwd_grouped_workspace(1, 2, d) == 2 * 256
     # 64 x 4096 (two K chunks of 2048) at M = 3 with rank 8: the fp32 chunk sums [2][64][3]
-    # and the X A partials of eight 512-input chunks [8][3][8], each region 256-byte aligned
+    # and the X A partials of 32 128-input chunks [32][3][8], each region 256-byte aligned
     t2 = q._Tensor(64, 4096, fake, fake, fake, fake)
     d2 = (q._LinearDesc * 1)(q._LinearDesc(fake, ctypes.pointer(t2), fake, fake, 8, 1.0, fake, None))
-    assert L.qlora_linear_fwd_grouped_workspace(3, 1, d2) == 2 * 64 * 3 * 4 + 8 * 3 * 8 * 4
+    assert L.qlora_linear_fwd_grouped_workspace(3, 1, d2) == 2 * 64 * 3 * 4 + 32 * 3 * 8 * 4
     assert L.qlora_linear_fwd_grouped(1, 2, d, None, 0, None) == q.QLORA_ERR_WORKSPACE
     bad = (q._LinearDesc * 1)(q._LinearDesc(fake, ctypes.pointer(q._Tensor(64, 100, fake, fake, fake, fake)),
                                             None, None, 0, 1.0, fake, None))
