@@ -425,55 +425,43 @@ __device__ __forceinline__ void gemv_compute(const GemvGroup &grp, const uint8_t
             const float4 c1 = ld128(hole(s * ROWS + rg * 16 + g + 8) + ((ks ^ g) << 4));
             const float ch0[4] = {c0.x, c0.y, c0.z, c0.w}, ch1[4] = {c1.x, c1.y, c1.z, c1.w};
             const uint8_t *sb = stages + s * STAGE;
-            // IB 64-blocks at a time: their code words loaded first, then for each of the four
-            // 16-input steps the lookups and MMAs of every block, so the blocks' MMA chains
-            // (one accumulator per block, since each block has its own c^) overlap
-            constexpr int IB = NT == 1 ? 4 : 2;
+            // one 64-block: 16 table lookups, 4 NT MMAs, the block's c^ on the partial sums
+            auto block = [&](int b) {
+                const uint32_t off = (uint32_t)(((2 * b + (t >> 1)) ^ g) << 4);
+                const uint2 w0 = *reinterpret_cast<const uint2 *>(sb + box_row0 + off);
+                const uint2 w1 = *reinterpret_cast<const uint2 *>(sb + box_row1 + off);
+                float cbk[NT][4];
 #pragma unroll
-            for (int b0 = 0; b0 < 4; b0 += IB) {
-                uint2 w0[IB], w1[IB];
-#pragma unroll
-                for (int bi = 0; bi < IB; ++bi) {
-                    const uint32_t off = (uint32_t)(((2 * (b0 + bi) + (t >> 1)) ^ g) << 4);
-                    w0[bi] = *reinterpret_cast<const uint2 *>(sb + box_row0 + off);
-                    w1[bi] = *reinterpret_cast<const uint2 *>(sb + box_row1 + off);
-                }
-                float cbk[IB][NT][4];
-#pragma unroll
-                for (int bi = 0; bi < IB; ++bi)
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) cbk[bi][nt][0] = cbk[bi][nt][1] = cbk[bi][nt][2] = cbk[bi][nt][3] = 0.0f;
+                for (int nt = 0; nt < NT; ++nt) cbk[nt][0] = cbk[nt][1] = cbk[nt][2] = cbk[nt][3] = 0.0f;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
+                    const uint32_t r0 = (j < 2) ? w0.x : w0.y;
+                    const uint32_t r1 = (j < 2) ? w1.x : w1.y;
                     // byte k of the word, times 256, plus lane * 4: one permute
                     const uint32_t slo = 0x5504u | ((uint32_t)(2 * (j & 1)) << 4), shi = slo + 0x10u;
+                    uint32_t a[4];
+                    a[0] = ld32(prmt(r0, lane4, slo));
+                    a[2] = ld32(prmt(r0, lane4, shi));
+                    a[1] = ld32(prmt(r1, lane4, slo));
+                    a[3] = ld32(prmt(r1, lane4, shi));
 #pragma unroll
-                    for (int bi = 0; bi < IB; ++bi) {
-                        if (b0 + bi >= nblk) continue;
-                        const uint32_t r0 = (j < 2) ? w0[bi].x : w0[bi].y;
-                        const uint32_t r1 = (j < 2) ? w1[bi].x : w1[bi].y;
-                        uint32_t a[4];
-                        a[0] = ld32(prmt(r0, lane4, slo));
-                        a[2] = ld32(prmt(r0, lane4, shi));
-                        a[1] = ld32(prmt(r1, lane4, slo));
-                        a[3] = ld32(prmt(r1, lane4, shi));
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-                            mma_bf16_16816(cbk[bi][nt], a, xf[nt][b0 + bi][2 * j], xf[nt][b0 + bi][2 * j + 1]);
-                    }
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(cbk[nt], a, xf[nt][b][2 * j], xf[nt][b][2 * j + 1]);
                 }
 #pragma unroll
-                for (int bi = 0; bi < IB; ++bi) {
-                    if (b0 + bi >= nblk) continue;
-                    const int b = b0 + bi;
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        acc[nt][0] = fmaf(ch0[b], cbk[bi][nt][0], acc[nt][0]);
-                        acc[nt][1] = fmaf(ch0[b], cbk[bi][nt][1], acc[nt][1]);
-                        acc[nt][2] = fmaf(ch1[b], cbk[bi][nt][2], acc[nt][2]);
-                        acc[nt][3] = fmaf(ch1[b], cbk[bi][nt][3], acc[nt][3]);
-                    }
+                for (int nt = 0; nt < NT; ++nt) {
+                    acc[nt][0] = fmaf(ch0[b], cbk[nt][0], acc[nt][0]);
+                    acc[nt][1] = fmaf(ch0[b], cbk[nt][1], acc[nt][1]);
+                    acc[nt][2] = fmaf(ch1[b], cbk[nt][2], acc[nt][2]);
+                    acc[nt][3] = fmaf(ch1[b], cbk[nt][3], acc[nt][3]);
                 }
+            };
+            if (nblk == 4) {
+#pragma unroll
+                for (int b = 0; b < 4; ++b) block(b);
+            } else {
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    if (b < nblk) block(b);
             }
         }
         __syncwarp();
