@@ -34,7 +34,7 @@ METRIC = "QLoRA linear fwd+bwd TFLOP/s at M=4096; NF4 GEMV/dequant HBM GB/s"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # the library's kernels, as named by its launch bookkeeping
-KERNELS = ("k_gemm2sm", "k_dequant", "k_fused_fwd", "k_fused_dgrad", "k_skinny", "k_reduce_xa", "k_reduce_f32",
+KERNELS = ("k_gemm2sm", "k_dequant", "k_fused_fwd", "k_fused_dgrad", "k_skinny",
            "k_gemv_xa", "k_gemv", "k_gemv_finish", "k_quantize_codes", "k_offset", "k_double_quant", "k_adamw")
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
 # capture of the same kernel and workload; update with the kernel.

@@ -103,11 +103,19 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
         // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
             uint32_t st = 0, ph = 0;
-            bool ok = true;
+            bool ok = true, ext_ready = false;
             for (int tile = pair; tile < ntiles && ok; tile += npairs) {
                 const int m0 = (tile % p.tiles_m) * kTileM + (int)rank * kHalf;
                 const int n0 = (tile / p.tiles_m) * kTileN + (int)rank * kHalf;
                 for (int kb = 0; kb < KBT; ++kb) {
+                    if (kb >= p.KB && !ext_ready) {
+                        // the extension operand (s XA or s G) comes from the kernel launched just
+                        // before this one, which may still run (programmatic dependent launch):
+                        // the main K blocks above needed only inputs that were complete
+                        griddep_wait();
+                        fence_proxy_async_global();
+                        ext_ready = true;
+                    }
                     if (!mbar_wait(empty(st), ph ^ 1u, abort)) { ok = false; break; }
                     const uint32_t fb = map_to_rank(full(st), 0);
                     if (rank == 0) mbar_arrive_expect_tx(full(st), 2 * kStage);
@@ -246,10 +254,12 @@ int gemm2sm_pairs(int max_pairs) {
 // A, Ae: K-major bf16 (row strides K and ke). B: K-major [N][K] or, with
 // b_mn, stored [K][N]. Be likewise with be_mn. ke == 0: no extension.
 // K, N, ke multiples of 8 (16-byte row strides); all pointers 16-byte aligned.
-// `pairs` CTA pairs (at most gemm2sm_pairs(0)) share the tiles.
+// `pairs` CTA pairs (at most gemm2sm_pairs(0)) share the tiles. With pdl, the launch may
+// begin while the previous kernel on the stream still runs, and only the extension operands
+// Ae, Be are read after that kernel completes (it must produce nothing else this GEMM reads).
 cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, const __nv_bfloat16 *B, bool b_mn,
                            const __nv_bfloat16 *Be, bool be_mn, __nv_bfloat16 *C, int64_t M, int64_t N, int64_t K,
-                           int ke, int pairs, cudaStream_t st) {
+                           int ke, int pairs, bool pdl, cudaStream_t st) {
     using namespace g2;
     if (M < 1 || N < 1 || K < 1 || K % 8 != 0 || N % 8 != 0 || ke < 0 || ke % 8 != 0 || pairs < 1)
         return cudaErrorInvalidValue;
@@ -281,7 +291,9 @@ cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, cons
 #define QNF4_G2(BM, BEM)                                                                                  \
     e = set_smem(k_gemm2sm<BM, BEM>, kSmem);                                                            \
     if (e != cudaSuccess) return e;                                                                      \
-    QNF4_LAUNCH("k_gemm2sm", st, k_gemm2sm<BM, BEM><<<2 * pairs, kThreads, kSmem, st>>>(ta, tae, tb, tbe, tcm, p));
+    QNF4_LAUNCH("k_gemm2sm", st,                                                                         \
+                e = launch_pdl(k_gemm2sm<BM, BEM>, 2 * pairs, kThreads, kSmem, st, pdl, ta, tae, tb, tbe, tcm, p)); \
+    if (e != cudaSuccess) return e;
     if (b_mn && be_mn) { QNF4_G2(true, true) }
     else if (b_mn) { QNF4_G2(true, false) }
     else if (be_mn) { QNF4_G2(false, true) }

@@ -22,8 +22,9 @@
 //                 tcgen05.mma reads directly, dY streams through TMA; the extra
 //                 K block multiplies A_lora (TMA) by s*G (TMA).
 //   k_skinny      TMA-fed tcgen05 GEMM for the rank-r products X*A, dY*B^T,
-//                 X^T*(sG), dY^T*XA with split-K partials; k_reduce_* sum the
-//                 partials in a fixed order and apply scale/layout.
+//                 X^T*(sG), dY^T*XA, split over K across the CTAs of a thread-block
+//                 cluster that add their accumulators in a fixed order through
+//                 distributed shared memory and apply scale/layout.
 // Both fused kernels keep the accumulator tile D[row, token] in TMEM and store
 // it transposed (out[token, row]) through a shared-memory staging tile and a
 // TMA store.
@@ -726,20 +727,35 @@ k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
 
 // ================================================================ skinny
 // D[128 x BN] = sum over K of A[128 x K] * B[BN x K]^T, operands by TMA in
-// 128-byte-swizzled tiles of 64 K; A and B each K-major or MN-major. One CTA
-// per (M tile, K split); fp32 partials [split][Mp][Np].
+// 128-byte-swizzled tiles of 64 K; A and B each K-major or MN-major. The K blocks of an
+// M tile are split over the S CTAs of one thread-block cluster (1 x S, S <= 8). Each
+// CTA stages its fp32 accumulator in its own shared memory; CTA q of the cluster then
+// adds rows q/S .. (q+1)/S of the tile over the S accumulators in split order (reading
+// the peers' shared memory), scales, converts and writes the outputs. No partial sums
+// go through HBM and no second kernel runs.
 struct SkinnyParams {
     int Mp, Np, BN;        // output rows, columns (r), MMA N (Np rounded up to 16)
     int kb_total, kb_per_split;
     int stages;
-    int transpose;         // partials as [split][Np][Mp] instead of [split][Mp][Np]
-    float *partial;
+    int transpose;         // the fp32 output as [Np][Mp] instead of [Mp][Np]
+    float s;               // scale of out_s and out_f32
+    __nv_bfloat16 *out;    // bf16 [Mp][Np] of the sum, or null
+    __nv_bfloat16 *out_s;  // bf16 [Mp][Np] of s times the sum, or null
+    float *out_f32;        // fp32 s times the sum, or null
 };
+constexpr int kSkinnyMaxSplits = 8;    // a portable cluster
+
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t caddr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(caddr) : "memory");
+    return v;
+}
 
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(128, 2)
 k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, SkinnyParams p) {
-    griddep_launch_dependents();                     // the reduction may be scheduled (it waits for us)
+    griddep_launch_dependents();                     // a following GEMM may start its main K blocks
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[2 * 8 + 2];
     __shared__ uint32_t s_tmem;
@@ -783,7 +799,8 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
     volatile int *abort = &s_abort;
 
     const int m0 = blockIdx.x * 128;
-    const int split = blockIdx.y;
+    const int split = blockIdx.y;                    // also the CTA's rank in its cluster
+    const int nsplit = gridDim.y;
     const int kb0 = split * p.kb_per_split;
     const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
 
@@ -831,34 +848,66 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
         drain_wait(fin, 0);
     }
     __syncwarp();
-    // epilogue: all 4 warps (warp w reads TMEM lanes 32w..32w+31)
-    if (mbar_wait(done, 0, abort)) {
+    // the accumulator into this CTA's shared memory (the stages are free now): fp32
+    // [128 rows][BN + 4], warp w holding TMEM lanes (rows) 32w .. 32w + 31
+    const int ld = p.BN + 4;
+    float *acc_s = reinterpret_cast<float *>(smem);
+    if (kb1 > kb0 && mbar_wait(done, 0, abort)) {
         tc_fence_after();
-        const int row = m0 + warp * 32 + lane;
-        float *dst = p.partial + ((int64_t)split * p.Mp + row) * p.Np;
-        float *dst_t = p.partial + (int64_t)split * p.Np * p.Mp + row;   // column j at dst_t[j * Mp]
+        const int rl = warp * 32 + lane;
         for (int c = 0; c < p.BN; c += 16) {
             uint32_t v[16];
             tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
             tmem_wait_ld();
-            if (row < p.Mp && p.transpose) {
-                // lanes hold consecutive rows: each column j is one coalesced store per warp
-                for (int i = 0; i < 16 && c + i < p.Np; ++i) dst_t[(int64_t)(c + i) * p.Mp] = __uint_as_float(v[i]);
-            } else if (row < p.Mp) {
-                if (c + 16 <= p.Np) {
 #pragma unroll
-                    for (int i = 0; i < 16; i += 4)
-                        *reinterpret_cast<float4 *>(dst + c + i) =
-                            make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
-                                        __uint_as_float(v[i + 3]));
+            for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<float4 *>(acc_s + rl * ld + c + i) =
+                    make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                                __uint_as_float(v[i + 3]));
+        }
+    } else {
+        // no K blocks for this split (or an expired wait): it adds zero
+        for (int i = threadIdx.x; i < 128 * ld; i += blockDim.x) acc_s[i] = 0.0f;
+    }
+    cluster_sync();   // every CTA's accumulator is in its shared memory
+    {
+        const int rpc = (128 + nsplit - 1) / nsplit;
+        const int r0 = split * rpc, r1 = min(128, r0 + rpc);
+        const int nvec = p.Np / 4;
+        const uint32_t base = smem_addr(acc_s);
+        for (int e = threadIdx.x; e < (r1 - r0) * nvec; e += blockDim.x) {
+            const int rl = r0 + e / nvec, c = (e % nvec) * 4;
+            const int row = m0 + rl;
+            if (row >= p.Mp) continue;
+            const uint32_t off = base + (uint32_t)((rl * ld + c) * 4);
+            float4 v = ld_cluster_f4(map_to_rank(off, 0));
+            for (int k = 1; k < nsplit; ++k) {
+                const float4 w = ld_cluster_f4(map_to_rank(off, (uint32_t)k));
+                v.x += w.x;
+                v.y += w.y;
+                v.z += w.z;
+                v.w += w.w;
+            }
+            const int64_t o = (int64_t)row * p.Np + c;
+            if (p.out) *reinterpret_cast<uint2 *>(p.out + o) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+            if (p.out_s)
+                *reinterpret_cast<uint2 *>(p.out_s + o) =
+                    make_uint2(pack_bf16x2(p.s * v.x, p.s * v.y), pack_bf16x2(p.s * v.z, p.s * v.w));
+            if (p.out_f32) {
+                const float4 w = make_float4(p.s * v.x, p.s * v.y, p.s * v.z, p.s * v.w);
+                if (p.transpose) {
+                    p.out_f32[(int64_t)(c + 0) * p.Mp + row] = w.x;
+                    p.out_f32[(int64_t)(c + 1) * p.Mp + row] = w.y;
+                    p.out_f32[(int64_t)(c + 2) * p.Mp + row] = w.z;
+                    p.out_f32[(int64_t)(c + 3) * p.Mp + row] = w.w;
                 } else {
-                    for (int i = 0; i < 16 && c + i < p.Np; ++i) dst[c + i] = __uint_as_float(v[i]);
+                    *reinterpret_cast<float4 *>(p.out_f32 + o) = w;
                 }
             }
         }
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();   // the peers have read this CTA's shared memory
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
@@ -866,122 +915,91 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
     }
 }
 
-// ------------------------------------------------------------------ reduce
-// Sums of split-K partials in split order (deterministic), then scale/convert.
-// Each thread takes four consecutive elements and issues the loads of all
-// splits before adding, so the HBM latencies overlap.
-constexpr int kMaxSplits = 16;
-__device__ __forceinline__ float4 sum_splits4(const float *__restrict__ part, int splits, int64_t count, int64_t i) {
-    float4 v[kMaxSplits];
-#pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp)
-        if (sp < splits) v[sp] = __ldg(reinterpret_cast<const float4 *>(part + sp * count + i));
-    float4 acc = v[0];
-#pragma unroll
-    for (int sp = 1; sp < kMaxSplits; ++sp)
-        if (sp < splits) {
-            acc.x += v[sp].x;
-            acc.y += v[sp].y;
-            acc.z += v[sp].z;
-            acc.w += v[sp].w;
-        }
-    return acc;
-}
-// count % 4 == 0 (counts are multiples of r, itself a multiple of 8)
-__global__ void k_reduce_xa(const float *__restrict__ part, int splits, int64_t count, float s,
-                            __nv_bfloat16 *__restrict__ xa, __nv_bfloat16 *__restrict__ xas) {
-    griddep_wait();                                  // the partials are complete
-    for (int64_t i = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < count; i += 4 * (int64_t)gridDim.x * blockDim.x) {
-        const float4 v = sum_splits4(part, splits, count, i);
-        if (xa) {
-            *reinterpret_cast<uint2 *>(xa + i) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
-        }
-        if (xas) {
-            *reinterpret_cast<uint2 *>(xas + i) =
-                make_uint2(pack_bf16x2(s * v.x, s * v.y), pack_bf16x2(s * v.z, s * v.w));
-        }
-    }
-}
-__global__ void k_reduce_f32(const float *__restrict__ part, int splits, int64_t count, float s,
-                             float *__restrict__ out) {
-    griddep_wait();                                  // the partials are complete
-    for (int64_t i = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < count; i += 4 * (int64_t)gridDim.x * blockDim.x) {
-        const float4 v = sum_splits4(part, splits, count, i);
-        *reinterpret_cast<float4 *>(out + i) = make_float4(s * v.x, s * v.y, s * v.z, s * v.w);
-    }
-}
-
 // ================================================================ host side
-// Split-K sizing: at most two CTAs per SM (each holds at most kSkinnyStages
-// stages), all resident at once, at most kMaxSplits partials per output.
+// Split-K sizing: at most two CTAs per SM, all resident at once, at most
+// kSkinnyMaxSplits CTAs (one cluster) per M tile.
 constexpr int kSkinnyStages = 4;
 
 struct SplitPlan { int kb_total, kb_per_split, splits; };
-static SplitPlan plan_splits(int64_t Mp, int64_t Kp) {
+static SplitPlan plan_splits(int64_t Mp, int64_t Kp, int sms) {
     SplitPlan sp;
     sp.kb_total = (int)ceil_div(Kp, 64);
     const int mt = (int)ceil_div(Mp, 128);
-    int want = (2 * num_sms()) / mt;
-    if (want > kMaxSplits) want = kMaxSplits;
+    int want = (2 * sms) / mt;
+    if (want > kSkinnyMaxSplits) want = kSkinnyMaxSplits;
     if (want < 1) want = 1;
     if (want > sp.kb_total) want = sp.kb_total;
     sp.kb_per_split = (int)ceil_div(sp.kb_total, want);
     sp.splits = (int)ceil_div(sp.kb_total, sp.kb_per_split);
     return sp;
 }
-static size_t partial_bytes(int64_t Mp, int64_t Kp, int r) {
-    return align256((size_t)plan_splits(Mp, Kp).splits * (size_t)Mp * (size_t)r * 4);
-}
 
-// Launch one skinny product. A operand: K-major [Mp rows, Kp] or MN-major
-// [Kp rows, Mp]; B operand: K-major [r rows, Kp] or MN-major [Kp rows, r].
-static cudaError_t run_skinny(bool a_mn, const void *a, int64_t a_ld_rows, bool b_mn, const void *b, int64_t Mp,
-                              int64_t Kp, int r, float *partial, int *splits_out, cudaStream_t st,
-                              bool transpose = false) {
+// Outputs of one skinny product (any of them may be null): bf16 sum, bf16 s * sum,
+// fp32 s * sum (transposed when f32_transposed).
+struct SkinnyOut {
+    __nv_bfloat16 *bf16 = nullptr, *bf16_s = nullptr;
+    float *f32 = nullptr;
+    bool f32_transposed = false;
+    float s = 1.0f;
+};
+
+// Launch one skinny product on `sms` SMs' worth of CTAs (all of them, or those a
+// concurrent GEMM leaves free). A operand: K-major [Mp rows, Kp] or MN-major [Kp rows, Mp];
+// B operand: K-major [r rows, Kp] or MN-major [Kp rows, r].
+static cudaError_t run_skinny(bool a_mn, const void *a, bool b_mn, const void *b, int64_t Mp, int64_t Kp, int r,
+                              const SkinnyOut &out, cudaStream_t st, int sms = 0) {
     CUtensorMap ta, tb;
     const int BN = (int)ceil_div(r, 16) * 16;
     bool ok;
     if (a_mn) ok = map_bf16(&ta, a, (uint64_t)Mp, (uint64_t)Kp, 64, 64);
     else ok = map_bf16(&ta, a, (uint64_t)Kp, (uint64_t)Mp, 64, 128);
-    (void)a_ld_rows;
     if (b_mn) ok = ok && map_bf16(&tb, b, (uint64_t)r, (uint64_t)Kp, 64, 64);
     else ok = ok && map_bf16(&tb, b, (uint64_t)Kp, (uint64_t)r, 64, (uint32_t)BN);
     if (!ok) return cudaErrorInvalidValue;
-    const SplitPlan sp = plan_splits(Mp, Kp);
+    const SplitPlan sp = plan_splits(Mp, Kp, sms > 0 ? sms : num_sms());
     SkinnyParams p;
     p.Mp = (int)Mp;
     p.Np = r;
     p.BN = BN;
     p.kb_total = sp.kb_total;
     p.kb_per_split = sp.kb_per_split;
-    p.partial = partial;
-    p.transpose = transpose ? 1 : 0;
+    p.transpose = out.f32_transposed ? 1 : 0;
+    p.s = out.s;
+    p.out = out.bf16;
+    p.out_s = out.bf16_s;
+    p.out_f32 = out.f32;
     const int b_bytes = b_mn ? (int)ceil_div(BN, 64) * 8192 : BN * 128;
     const int stage = 128 * 128 + ((b_bytes + 1023) & ~1023);
     int stages = (100 * 1024) / stage;
     if (stages > kSkinnyStages) stages = kSkinnyStages;
     if (stages > sp.kb_per_split) stages = sp.kb_per_split < 2 ? 2 : sp.kb_per_split;
     p.stages = stages;
-    const int smem = 1024 + stages * stage;
-    dim3 grid((unsigned)ceil_div(Mp, 128), (unsigned)sp.splits);
+    const int acc_bytes = 128 * (BN + 4) * 4;       // the staged accumulator reuses the stages
+    const int smem = 1024 + (stages * stage > acc_bytes ? stages * stage : acc_bytes);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ceil_div(Mp, 128), (unsigned)sp.splits);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = (unsigned)sp.splits;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
     cudaError_t e;
 #define QNF4_SK(AM, BM)                                                      \
     e = set_smem(k_skinny<AM, BM>, smem);                                    \
     if (e != cudaSuccess) return e;                                          \
-    QNF4_LAUNCH("k_skinny", st, k_skinny<AM, BM><<<grid, 128, smem, st>>>(ta, tb, p));
+    QNF4_LAUNCH("k_skinny", st, e = cudaLaunchKernelEx(&cfg, k_skinny<AM, BM>, ta, tb, p)); \
+    if (e != cudaSuccess) return e;
     if (a_mn && b_mn) { QNF4_SK(true, true) }
     else if (a_mn) { QNF4_SK(true, false) }
     else if (b_mn) { QNF4_SK(false, true) }
     else { QNF4_SK(false, false) }
 #undef QNF4_SK
-    *splits_out = sp.splits;
     return cudaGetLastError();
-}
-
-static unsigned reduce_grid(int64_t count) {
-    int64_t g = ceil_div(count, 4 * 256);
-    const int64_t cap = (int64_t)num_sms() * 8;
-    return (unsigned)(g < 1 ? 1 : (g > cap ? cap : g));
 }
 
 static size_t mr_bytes(int64_t M, int r) { return align256((size_t)M * (size_t)r * 2); }
@@ -992,11 +1010,15 @@ static size_t mr_bytes(int64_t M, int r) { return align256((size_t)M * (size_t)r
 // work costs more than writing and re-reading the bf16 copy. Settable so that both
 // routes can be compared at any M (qlora_linear_set_pair_min_m).
 static std::atomic<int64_t> g_pair_min_m{512};
+// The dequantisation beside the adapter product runs two 256-thread CTAs per SM (half the
+// registers), so that the product's CTAs are scheduled next to it instead of after it.
+constexpr int kSideDequantCtas = 2;
 static bool pair_route(int64_t M) { return M >= g_pair_min_m.load(std::memory_order_relaxed); }
 static size_t wd_bytes(int64_t rows, int64_t cols) { return align256((size_t)rows * (size_t)cols * 2); }
 
 static size_t fwd_adapter_bytes(int64_t M, int64_t cols, int r) {
-    return r == 0 ? 0 : mr_bytes(M, r) + partial_bytes(M, cols, r);
+    (void)cols;
+    return r == 0 ? 0 : mr_bytes(M, r);                      // s XA
 }
 
 // CTA pairs of the pair GEMM: as few pairs as give the same number of tile rounds. The
@@ -1017,15 +1039,9 @@ size_t fwd_workspace_bytes_large(int64_t M, int64_t rows, int64_t cols, int r) {
 }
 
 static size_t bwd_adapter_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
-    if (r == 0) return 0;
-    size_t part = partial_bytes(M, cols, r);                 // X*A
-    size_t p2 = partial_bytes(M, rows, r);                   // dY*B^T
-    size_t p3 = partial_bytes(cols, M, r);                   // X^T*(sG)
-    size_t p4 = partial_bytes(rows, M, r);                   // dY^T*XA
-    if (p2 > part) part = p2;
-    if (p3 > part) part = p3;
-    if (p4 > part) part = p4;
-    return 2 * mr_bytes(M, r) + part;
+    (void)rows;
+    (void)cols;
+    return r == 0 ? 0 : 2 * mr_bytes(M, r);                  // s G, and X A when it is recomputed
 }
 
 size_t bwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
@@ -1136,46 +1152,48 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
         if (side) {
             if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
             if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
-            if ((e = launch_dequant(W, Wd, side->s)) != cudaSuccess) return e;
+            if ((e = launch_dequant(W, Wd, side->s, kSideDequantCtas)) != cudaSuccess) return e;
             if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess) return e;
         }
     }
+    // the pair GEMM follows the X*A product directly (programmatic dependent launch: its
+    // main K blocks may start while the product finishes), so the dequantised weight is
+    // produced before the product or joined after it
+    if (pair && !side && (e = launch_dequant(W, Wd, st)) != cudaSuccess) return e;
     if (r > 0) {
         XAs = static_cast<__nv_bfloat16 *>(ws);
-        float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + mr_bytes(M, r));
-        int splits = 0;
-        e = run_skinny(false, X, M, true, A, M, W.cols, r, part, &splits, st);
+        SkinnyOut o;
+        o.bf16 = XA_save;
+        o.bf16_s = XAs;
+        o.s = s;
+        e = run_skinny(false, X, true, A, M, W.cols, r, o, st);
         if (e != cudaSuccess) return e;
-        QNF4_LAUNCH("k_reduce_xa", st, e = launch_pdl(k_reduce_xa, (int)reduce_grid(M * r), 256, 0, st, true, part, splits, M * r, s, XA_save, XAs));
-        if (e != cudaSuccess) return e;
+        if (side && (e = cudaStreamWaitEvent(st, side->join, 0)) != cudaSuccess) return e;
     }
     if (pair) {
         // Y = X W^T + (s XA) B: W^ [d_out, d_in] is the K-major B operand, B_lora [r, d_out]
         // the MN-major extension
-        if (side) {
-            if ((e = cudaStreamWaitEvent(st, side->join, 0)) != cudaSuccess) return e;
-        } else if ((e = launch_dequant(W, Wd, st)) != cudaSuccess) {
-            return e;
-        }
-        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, side_job_pairs(M, W.rows), st);
+        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, side_job_pairs(M, W.rows), r > 0,
+                              st);
     }
     return run_fused_fwd(X, M, W, XAs, B, r, Y, st);
 }
 
-// dA = X^T (sG) and dB = s (XA)^T dY on stream `st` (they share the partial buffer,
-// so they run one after the other).
+// dA = X^T (sG) and dB = s (XA)^T dY on stream `st`, sized for `sms` SMs.
 static cudaError_t adapter_grads(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, int64_t M, const NF4View &W,
                                  const __nv_bfloat16 *Gs, const __nv_bfloat16 *XA, int r, float s, float *dA,
-                                 float *dB, float *part, cudaStream_t st) {
-    int splits = 0;
-    cudaError_t e = run_skinny(true, X, M, true, Gs, W.cols, M, r, part, &splits, st);
+                                 float *dB, cudaStream_t st, int sms = 0) {
+    SkinnyOut oa;
+    oa.f32 = dA;
+    oa.s = 1.0f;
+    cudaError_t e = run_skinny(true, X, true, Gs, W.cols, M, r, oa, st, sms);
     if (e != cudaSuccess) return e;
-    QNF4_LAUNCH("k_reduce_f32", st, e = launch_pdl(k_reduce_f32, (int)reduce_grid(W.cols * r), 256, 0, st, true, part, splits, W.cols * r, 1.0f, dA));
-    if (e != cudaSuccess) return e;
-    // computed as (dY^T XA)^T with the partials written transposed
-    e = run_skinny(true, dY, M, true, XA, W.rows, M, r, part, &splits, st, true);
-    if (e != cudaSuccess) return e;
-    QNF4_LAUNCH("k_reduce_f32", st, e = launch_pdl(k_reduce_f32, (int)reduce_grid(W.rows * r), 256, 0, st, true, part, splits, W.rows * r, s, dB));
+    // computed as (dY^T XA)^T, the fp32 output written transposed
+    SkinnyOut ob;
+    ob.f32 = dB;
+    ob.f32_transposed = true;
+    ob.s = s;
+    e = run_skinny(true, dY, true, XA, W.rows, M, r, ob, st, sms);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1200,60 +1218,58 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
         if (side) {
             if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
             if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
-            if ((e = launch_dequant(W, Wd, side->s)) != cudaSuccess) return e;
+            if ((e = launch_dequant(W, Wd, side->s, kSideDequantCtas)) != cudaSuccess) return e;
             if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess) return e;
         }
     }
+    // as in the forward, the pair GEMM follows the dY*B^T reduction directly
+    if (pair && !side && (e = launch_dequant(W, Wd, st)) != cudaSuccess) return e;
     if (r > 0) {
         Gs = static_cast<__nv_bfloat16 *>(ws);
         __nv_bfloat16 *XAbuf = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + mr_bytes(M, r));
-        float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + 2 * mr_bytes(M, r));
-        int splits = 0;
         if (!XA) {
-            e = run_skinny(false, X, M, true, A, M, W.cols, r, part, &splits, st);
-            if (e != cudaSuccess) return e;
-            QNF4_LAUNCH("k_reduce_xa", st, e = launch_pdl(k_reduce_xa, (int)reduce_grid(M * r), 256, 0, st, true, part, splits, M * r, 1.0f, XAbuf, nullptr));
+            SkinnyOut ox;
+            ox.bf16 = XAbuf;
+            e = run_skinny(false, X, true, A, M, W.cols, r, ox, st);
             if (e != cudaSuccess) return e;
             XA = XAbuf;
         }
         // G = dY B^T -> sG (bf16)
-        e = run_skinny(false, dY, M, false, B, M, W.rows, r, part, &splits, st);
+        SkinnyOut og;
+        og.bf16_s = Gs;
+        og.s = s;
+        e = run_skinny(false, dY, false, B, M, W.rows, r, og, st);
         if (e != cudaSuccess) return e;
-        QNF4_LAUNCH("k_reduce_xa", st, e = launch_pdl(k_reduce_xa, (int)reduce_grid(M * r), 256, 0, st, true, part, splits, M * r, s, nullptr, Gs));
-        if (e != cudaSuccess) return e;
+        if (side && (e = cudaStreamWaitEvent(st, side->join, 0)) != cudaSuccess) return e;
     }
     if (pair) {
         // dX = dY W^ + (s G) A^T: W^ [d_out, d_in] read as the MN-major B operand
         // ([K = d_out][N = d_in]), A_lora [d_in, r] the K-major extension
-        if (side) {
-            if ((e = cudaStreamWaitEvent(st, side->join, 0)) != cudaSuccess) return e;
-        } else if ((e = launch_dequant(W, Wd, st)) != cudaSuccess) {
-            return e;
-        }
         if (r > 0) {
             // the adapter gradients need only Gs and XA: they run on the side stream
             // while the dgrad GEMM occupies the tensor cores
             if (side) {
-                float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + 2 * mr_bytes(M, r));
                 if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
-                e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, side_job_pairs(M, W.cols), st);
+                e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, side_job_pairs(M, W.cols), true,
+                                   st);
                 if (e != cudaSuccess) return e;
                 if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
-                e = adapter_grads(X, dY, M, W, Gs, XA, r, s, dA, dB, part, side->s);
+                // sized for the SMs the dgrad GEMM leaves free
+                int free_sms = num_sms() - 2 * side_job_pairs(M, W.cols);
+                if (free_sms < 2) free_sms = 2;
+                e = adapter_grads(X, dY, M, W, Gs, XA, r, s, dA, dB, side->s, free_sms);
                 if (e != cudaSuccess) return e;
                 if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess) return e;
                 return cudaStreamWaitEvent(st, side->join, 0);
             }
         }
-        e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, side_job_pairs(M, W.cols), st);
+        e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, side_job_pairs(M, W.cols), r > 0,
+                           st);
     } else {
         e = run_fused_dgrad(dY, M, W, A, Gs, r, dX, st);
     }
     if (e != cudaSuccess) return e;
-    if (r > 0) {
-        float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + 2 * mr_bytes(M, r));
-        return adapter_grads(X, dY, M, W, Gs, XA, r, s, dA, dB, part, st);
-    }
+    if (r > 0) return adapter_grads(X, dY, M, W, Gs, XA, r, s, dA, dB, st);
     return cudaGetLastError();
 }
 

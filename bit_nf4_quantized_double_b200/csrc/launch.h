@@ -16,7 +16,9 @@ struct QuantArgs {
     double *part;
 };
 cudaError_t launch_quantize_grouped(const QuantArgs *a, int count, qlora_dtype dt, cudaStream_t st);
-cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st);
+// ctas_per_sm caps the persistent grid (8 fills the SMs; fewer leave room for a kernel
+// running beside it on another stream).
+cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st, int ctas_per_sm = 8);
 cudaError_t launch_dequant_grouped(const NF4View *q, __nv_bfloat16 *const *out, int count, cudaStream_t st);
 cudaError_t launch_fmt4_quantize(const void *W, qlora_dtype dt, int64_t n, qlora_fmt4 f, uint8_t *codes,
                                  float *absmax, cudaStream_t st);
@@ -35,7 +37,7 @@ cudaError_t launch_merge_bf16(const NF4View &q, const __nv_bfloat16 *A, const __
 int gemm2sm_pairs(int max_pairs);
 cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, const __nv_bfloat16 *B, bool b_mn,
                            const __nv_bfloat16 *Be, bool be_mn, __nv_bfloat16 *C, int64_t M, int64_t N, int64_t K,
-                           int ke, int pairs, cudaStream_t st);
+                           int ke, int pairs, bool pdl, cudaStream_t st);
 
 size_t fwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r);
 

@@ -795,7 +795,8 @@ cudaError_t launch_quantize_grouped(const QuantArgs *a, int count, qlora_dtype d
 
 // One launch over up to kDeqMaxItems tensors; a persistent grid of up to eight
 // 256-thread CTAs per SM.
-static cudaError_t dequant_launch(const NF4View *q, __nv_bfloat16 *const *out, int count, cudaStream_t st) {
+static cudaError_t dequant_launch(const NF4View *q, __nv_bfloat16 *const *out, int count, int ctas_per_sm,
+                                  cudaStream_t st) {
     DeqGroup g;
     g.count = count;
     int64_t chunks = 0;
@@ -812,21 +813,21 @@ static cudaError_t dequant_launch(const NF4View *q, __nv_bfloat16 *const *out, i
     }
     g.chunks = chunks;
     int64_t grid = ceil_div(chunks, 8);                   // eight warps per CTA
-    const int64_t cap = (int64_t)num_sms() * 8;
+    const int64_t cap = (int64_t)num_sms() * ctas_per_sm;
     if (grid > cap) grid = cap;
     if (grid < count) grid = count;                       // one CTA per tensor writes its tail
     QNF4_LAUNCH("k_dequant", st, k_dequant<<<(unsigned)grid, 256, 0, st>>>(g, host_codebook()));
     return cudaGetLastError();
 }
 
-cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st) {
-    return dequant_launch(&q, &out, 1, st);
+cudaError_t launch_dequant(const NF4View &q, __nv_bfloat16 *out, cudaStream_t st, int ctas_per_sm) {
+    return dequant_launch(&q, &out, 1, ctas_per_sm, st);
 }
 
 cudaError_t launch_dequant_grouped(const NF4View *q, __nv_bfloat16 *const *out, int count, cudaStream_t st) {
     for (int i = 0; i < count; i += kDeqMaxItems) {
         const int n = count - i < kDeqMaxItems ? count - i : kDeqMaxItems;
-        cudaError_t e = dequant_launch(q + i, out + i, n, st);
+        cudaError_t e = dequant_launch(q + i, out + i, n, 8, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -94,6 +94,11 @@ __device__ __forceinline__ void fence_barrier_init() {
 }
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor core and TMA reads of shared memory).
+// Orders this thread's view of global memory (written by other grids through the generic
+// proxy) before its later TMA reads of it.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
