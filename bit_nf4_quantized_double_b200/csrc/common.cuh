@@ -85,6 +85,10 @@ int num_sms();
 // enabled, brackets it with CUDA events on its stream.
 void note_launch_begin(const char *name, cudaStream_t st, void **token);
 void note_launch_end(void *token, cudaStream_t st);
+// True while per-launch event timing is on: launches then drop programmatic dependent
+// launch, so that each kernel's events bracket its own run and not its overlap with the
+// kernel before it.
+bool profiling_launches();
 }  // namespace qnf4
 
 #define QNF4_LAUNCH(name, st, ...)                         \

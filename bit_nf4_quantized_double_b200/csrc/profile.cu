@@ -46,6 +46,8 @@ void note_launch_begin(const char *name, cudaStream_t st, void **token) {
     *token = new Token{name, a};
 }
 
+bool profiling_launches() { return g_profiling.load(std::memory_order_relaxed) != 0; }
+
 void note_launch_end(void *token, cudaStream_t st) {
     if (!token) return;
     Token *t = static_cast<Token *>(token);
