@@ -598,6 +598,7 @@ def run_components(args, peaks, peak_kind, flush):
     out["fmt4"] = run_fmt4(hbm, flush, stream)
     out["adamw"] = run_adamw(hbm, flush, stream)
     out["large_m_routes"] = run_routes(flush, stream)
+    out["mid_m"] = run_mid_m(flush, stream)
     return out
 
 
@@ -614,7 +615,7 @@ def run_routes(flush, stream):
     X, dY, A, B = inp["X"], inp["dY"], inp["A"], inp["B"]
     flops = step_flops(M, d_in, d_out, r)
     out = {"workload": "4096 x 4096 layer, M = 4096, r = 64, fwd + bwd, CUDA graph replay, L2 flushed"}
-    for name, P in (("dequant_then_pair_gemm", 512), ("fused_dequant_gemm", 2 ** 62)):
+    for name, P in (("dequant_then_pair_gemm", 512), ("fused_dequant_gemm", 2 ** 63 - 1)):
         q.lib().qlora_linear_set_pair_min_m(P)
         try:
             Y = torch.empty(M, d_out, dtype=torch.bfloat16, device="cuda")
@@ -637,6 +638,42 @@ def run_routes(flush, stream):
                          "kernels": kern}
         finally:
             q.lib().qlora_linear_set_pair_min_m(512)
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    return out
+
+
+def run_mid_m(flush, stream, M=480, r=64):
+    """Mid-sized batches (16 < M < 512) on weights with one narrow side: the default routing
+    (a direction whose fused kernel would fill fewer than half the SMs takes the pair GEMM with
+    split K) against the fused kernels everywhere."""
+    import torch
+    import bit_nf4_quantized_double_b200 as q
+    import synth_inputs as si
+    out = {"workload": f"fwd + bwd at M = {M}, r = {r}, weights 16384 x 1024 and 1024 x 16384, CUDA graph replay, "
+                       "L2 flushed"}
+    for rows, cols in ((16384, 1024), (1024, 16384)):
+        W = si.normal((rows, cols), 0.02, seed=rows + 3, device="cuda")
+        t = q.qlora_nf4_quantize(W)
+        del W
+        X = si.normal((M, cols), 1.0, seed=5, device="cuda", dtype=torch.bfloat16)
+        dY = si.normal((M, rows), 1.0, seed=6, device="cuda", dtype=torch.bfloat16)
+        A = si.normal((cols, r), 0.02, seed=7, device="cuda", dtype=torch.bfloat16)
+        B = si.normal((r, rows), 0.01, seed=8, device="cuda", dtype=torch.bfloat16)
+        flops = step_flops(M, cols, rows, r)
+        res = {}
+        for name, P in (("default", 512), ("fused_everywhere", 2 ** 63 - 1)):
+            q.lib().qlora_linear_set_pair_min_m(P)
+            try:
+                def step():
+                    Y, XA = q.qlora_linear_fwd(X, t, A, B, 2.0)
+                    q.qlora_linear_bwd(X, dY, t, A, B, 2.0, XA=XA)
+                ms = _time_graph(step, 10, flush, stream)
+                res[name] = {"ms_per_step": round(ms, 5), "TFLOP/s": round(flops / (ms / 1e3) / 1e12, 1),
+                             "kernels": _kernel_ms(KERNELS + ("k_gemm2sm_reduce",), step, 3, flush)}
+            finally:
+                q.lib().qlora_linear_set_pair_min_m(512)
+        out[f"{rows}x{cols}"] = res
+        del t
     assert q.qlora_get_device_status() == q.QLORA_OK
     return out
 
@@ -1008,7 +1045,7 @@ def run_profile_case(name, reps=3):
     elif name == "l4096fused":
         wl, L, inp = headline_inputs(0)
         t = q.qlora_nf4_quantize(inp["W"])
-        q.lib().qlora_linear_set_pair_min_m(2 ** 62)
+        q.lib().qlora_linear_set_pair_min_m(2 ** 63 - 1)
         for _ in range(reps):
             l2_flush(flush)
             Y, XA = q.qlora_linear_fwd(inp["X"], t, inp["A"], inp["B"], L.s)

@@ -19,10 +19,12 @@
 // issued by rank 0 reads both CTAs' halves, and each CTA's TMEM receives its
 // 128 accumulator rows. Per SM that is 8 KB of operand reads per K16 step, half
 // of what a one-SM 128 x 256 tile with both operands in shared memory needs.
-// Persistent: pair p takes whole tiles p, p + pairs, p + 2 pairs, ..., so that at any
+// Persistent: pair p takes work items p, p + pairs, p + 2 pairs, ..., so that at any
 // moment the pairs work on neighbouring tiles, which share the operand panels in L2.
-// Two accumulators in TMEM let the epilogue of one tile overlap the main loop of the
-// next.
+// An item is a whole tile, or, when the tiles are too few to occupy the SMs, one of
+// `splits` equal ranges of a tile's K blocks: those write fp32 partial tiles that
+// k_gemm2sm_reduce adds in split order. Two accumulators in TMEM let the epilogue of one
+// item overlap the main loop of the next.
 #include "launch.h"
 #include "tc.cuh"
 #include "tmap.h"
@@ -47,6 +49,8 @@ struct G2Params {
     int KB, KBE;       // main and extension K blocks of 64
     int ke;            // extension K extent (the extension blocks' MMAs stop at it)
     int tiles_m, tiles_n;
+    int splits;        // K ranges per tile (1: the epilogue writes C directly)
+    float *partial;    // [splits][M][N] fp32 when splits > 1
 };
 
 template <bool B_MN, bool BE_MN>
@@ -97,6 +101,7 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
 
     const int KBT = p.KB + p.KBE;
     const int ntiles = p.tiles_m * p.tiles_n;
+    const int nitems = ntiles * p.splits;           // item i: tile i % ntiles, K range i / ntiles
     const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
 
     if (warp == 0) {
@@ -104,10 +109,12 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
         if (lane == 0) {
             uint32_t st = 0, ph = 0;
             bool ok = true, ext_ready = false;
-            for (int tile = pair; tile < ntiles && ok; tile += npairs) {
+            for (int item = pair; item < nitems && ok; item += npairs) {
+                const int tile = item % ntiles, sp = item / ntiles;
+                const int kb_lo = sp * KBT / p.splits, kb_hi = (sp + 1) * KBT / p.splits;
                 const int m0 = (tile % p.tiles_m) * kTileM + (int)rank * kHalf;
                 const int n0 = (tile / p.tiles_m) * kTileN + (int)rank * kHalf;
-                for (int kb = 0; kb < KBT; ++kb) {
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (kb >= p.KB && !ext_ready) {
                         // the extension operand (s XA or s G) comes from the kernel launched just
                         // before this one, which may still run (programmatic dependent launch):
@@ -154,12 +161,14 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
             constexpr uint32_t kStageDesc = kStage >> 4;
             uint32_t st = 0, ph = 0, lt = 0;
             bool ok = true;
-            for (int tile = pair; tile < ntiles && ok; tile += npairs, ++lt) {
+            for (int item = pair; item < nitems && ok; item += npairs, ++lt) {
+                const int sp = item / ntiles;
+                const int kb_lo = sp * KBT / p.splits, kb_hi = (sp + 1) * KBT / p.splits;
                 const uint32_t acc = lt & 1u, use = lt >> 1;
                 if (!mbar_wait_cluster(tempty(acc), (use & 1u) ^ 1u, abort)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + acc * 256u;
-                for (int kb = 0; kb < KBT; ++kb) {
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!mbar_wait(full(st), ph, abort)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t ad = adesc0 + st * kStageDesc;
@@ -168,13 +177,13 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
                             mma_pair_ss(d, ad + 2u * k, bd + (B_MN ? 128u : 2u) * k, idesc_main,
-                                        (kb != 0 || k != 0) ? 1u : 0u);
+                                        (kb != kb_lo || k != 0) ? 1u : 0u);
                     } else {
                         const uint64_t bd = (BE_MN ? bm0 : bk0) + st * kStageDesc;
                         const int nk = min(4, (p.ke - (kb - p.KB) * 64 + 15) / 16);
                         for (int k = 0; k < nk; ++k)
                             mma_pair_ss(d, ad + 2u * k, bd + (BE_MN ? 128u : 2u) * k, idesc_ext,
-                                        (kb != 0 || k != 0) ? 1u : 0u);
+                                        (kb != kb_lo || k != 0) ? 1u : 0u);
                     }
                     mma_pair_commit(empty(st), 0x3);
                     if (++st == (uint32_t)kStages) { st = 0; ph ^= 1u; }
@@ -194,7 +203,8 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
         const int row = q * 32 + lane;                 // TMEM lane = tile row within this CTA
         const uint32_t tempty0 = map_to_rank(tempty(0), 0), tempty1 = map_to_rank(tempty(1), 0);
         uint32_t lt = 0;
-        for (int tile = pair; tile < ntiles; tile += npairs, ++lt) {
+        for (int item = pair; item < nitems; item += npairs, ++lt) {
+            const int tile = item % ntiles, sp = item / ntiles;
             const uint32_t acc = lt & 1u, use = lt >> 1;
             if (!mbar_wait(tfull(acc), use & 1u, abort)) break;
             tc_fence_after();
@@ -212,6 +222,22 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(acc ? tempty1 : tempty0);
+                }
+                if (p.splits > 1) {
+                    // fp32 partial of this K range: row m0 + row, columns n0 + 64 part .. + 63
+                    const int mg = m0 + row;
+                    if (mg < p.M) {
+                        float *dst = p.partial + ((int64_t)sp * p.M + mg) * p.N + n0 + part * 64;
+#pragma unroll
+                        for (int i = 0; i < 64; i += 4) {
+                            if (n0 + part * 64 + i >= p.N) break;
+                            const uint32_t *src = i < 32 ? v + i : w + (i - 32);
+                            *reinterpret_cast<float4 *>(dst + i) =
+                                make_float4(__uint_as_float(src[0]), __uint_as_float(src[1]), __uint_as_float(src[2]),
+                                            __uint_as_float(src[3]));
+                        }
+                    }
+                    continue;
                 }
                 uint8_t *stg = staging + (part & 1) * kPart;
                 if (et == 0) bulk_wait_read1();        // the store that last read this buffer is done
@@ -245,6 +271,32 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
     }
 }
 
+// C = bf16 of the sum of the splits' fp32 partials, added in split order; four consecutive
+// elements per thread, every split's load issued before the adds.
+constexpr int kMaxGemmSplits = 16;
+__global__ void __launch_bounds__(256) k_gemm2sm_reduce(const float *__restrict__ part, int splits, int64_t count,
+                                                        __nv_bfloat16 *__restrict__ C) {
+    const int64_t stride = 4 * (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < count; i += stride) {
+        float4 v[kMaxGemmSplits];
+#pragma unroll
+        for (int sp = 0; sp < kMaxGemmSplits; ++sp)
+            if (sp < splits) v[sp] = __ldcg(reinterpret_cast<const float4 *>(part + sp * count + i));
+        float4 a = v[0];
+#pragma unroll
+        for (int sp = 1; sp < kMaxGemmSplits; ++sp)
+            if (sp < splits) {
+                a.x += v[sp].x;
+                a.y += v[sp].y;
+                a.z += v[sp].z;
+                a.w += v[sp].w;
+            }
+        *reinterpret_cast<uint2 *>(C + i) = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+    }
+}
+
+int gemm2sm_max_splits() { return kMaxGemmSplits; }
+
 int gemm2sm_pairs(int max_pairs) {
     const int all = num_sms() / 2;
     return (max_pairs > 0 && max_pairs < all) ? max_pairs : all;
@@ -254,14 +306,17 @@ int gemm2sm_pairs(int max_pairs) {
 // A, Ae: K-major bf16 (row strides K and ke). B: K-major [N][K] or, with
 // b_mn, stored [K][N]. Be likewise with be_mn. ke == 0: no extension.
 // K, N, ke multiples of 8 (16-byte row strides); all pointers 16-byte aligned.
-// `pairs` CTA pairs (at most gemm2sm_pairs(0)) share the tiles. With pdl, the launch may
-// begin while the previous kernel on the stream still runs, and only the extension operands
-// Ae, Be are read after that kernel completes (it must produce nothing else this GEMM reads).
+// `pairs` CTA pairs (at most gemm2sm_pairs(0)) share the work items. With splits > 1, each
+// tile's K blocks are cut into `splits` ranges whose fp32 partials go to `partial`
+// ([splits][M][N]), and k_gemm2sm_reduce writes C. With pdl, the launch may begin while the
+// previous kernel on the stream still runs, and only the extension operands Ae, Be are read
+// after that kernel completes (it must produce nothing else this GEMM reads).
 cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, const __nv_bfloat16 *B, bool b_mn,
                            const __nv_bfloat16 *Be, bool be_mn, __nv_bfloat16 *C, int64_t M, int64_t N, int64_t K,
-                           int ke, int pairs, bool pdl, cudaStream_t st) {
+                           int ke, int pairs, int splits, float *partial, bool pdl, cudaStream_t st) {
     using namespace g2;
-    if (M < 1 || N < 1 || K < 1 || K % 8 != 0 || N % 8 != 0 || ke < 0 || ke % 8 != 0 || pairs < 1)
+    if (M < 1 || N < 1 || K < 1 || K % 8 != 0 || N % 8 != 0 || ke < 0 || ke % 8 != 0 || pairs < 1 || splits < 1 ||
+        splits > kMaxGemmSplits || (splits > 1 && !partial))
         return cudaErrorInvalidValue;
     CUtensorMap ta, tae, tb, tbe, tcm;
     bool ok = map_bf16(&ta, A, (uint64_t)K, (uint64_t)M, 64, kHalf);
@@ -285,8 +340,10 @@ cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, cons
     p.ke = ke;
     p.tiles_m = (int)ceil_div(M, kTileM);
     p.tiles_n = (int)ceil_div(N, kTileN);
-    const int ntiles = p.tiles_m * p.tiles_n;
-    if (pairs > ntiles) pairs = ntiles;            // at least one tile per pair
+    p.splits = splits;
+    p.partial = partial;
+    const int nitems = p.tiles_m * p.tiles_n * splits;
+    if (pairs > nitems) pairs = nitems;            // at least one item per pair
     cudaError_t e;
 #define QNF4_G2(BM, BEM)                                                                                  \
     e = set_smem(k_gemm2sm<BM, BEM>, kSmem);                                                            \
@@ -299,6 +356,14 @@ cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, cons
     else if (be_mn) { QNF4_G2(false, true) }
     else { QNF4_G2(false, false) }
 #undef QNF4_G2
+    if (splits > 1) {
+        const int64_t count = M * N;                   // N % 8 == 0: whole float4 groups
+        int64_t grid = ceil_div(count, (int64_t)4 * 256);
+        const int64_t cap = (int64_t)num_sms() * 8;
+        if (grid > cap) grid = cap;
+        QNF4_LAUNCH("k_gemm2sm_reduce", st,
+                    k_gemm2sm_reduce<<<(unsigned)grid, 256, 0, st>>>(partial, splits, count, C));
+    }
     return cudaGetLastError();
 }
 

@@ -880,14 +880,20 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
             const int row = m0 + rl;
             if (row >= p.Mp) continue;
             const uint32_t off = base + (uint32_t)((rl * ld + c) * 4);
-            float4 v = ld_cluster_f4(map_to_rank(off, 0));
-            for (int k = 1; k < nsplit; ++k) {
-                const float4 w = ld_cluster_f4(map_to_rank(off, (uint32_t)k));
-                v.x += w.x;
-                v.y += w.y;
-                v.z += w.z;
-                v.w += w.w;
-            }
+            // every peer's value is requested before the first add (the adds stay in rank order)
+            float4 w[kSkinnyMaxSplits];
+#pragma unroll
+            for (int k = 0; k < kSkinnyMaxSplits; ++k)
+                if (k < nsplit) w[k] = ld_cluster_f4(map_to_rank(off, (uint32_t)k));
+            float4 v = w[0];
+#pragma unroll
+            for (int k = 1; k < kSkinnyMaxSplits; ++k)
+                if (k < nsplit) {
+                    v.x += w[k].x;
+                    v.y += w[k].y;
+                    v.z += w[k].z;
+                    v.w += w[k].w;
+                }
             const int64_t o = (int64_t)row * p.Np + c;
             if (p.out) *reinterpret_cast<uint2 *>(p.out + o) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
             if (p.out_s)
@@ -1007,13 +1013,26 @@ static size_t mr_bytes(int64_t M, int r) { return align256((size_t)M * (size_t)r
 // From this many tokens on (default 512), the layer dequantises W once into bf16
 // scratch and runs the CTA-pair GEMM: the fused kernel would repeat the
 // dequantisation for every 256-token tile, and at two or more tiles that integer
-// work costs more than writing and re-reading the bf16 copy. Settable so that both
-// routes can be compared at any M (qlora_linear_set_pair_min_m).
+// work costs more than writing and re-reading the bf16 copy. From 128 tokens on, a
+// direction whose fused kernel would have fewer 128 x 256 output tiles than half the SMs
+// also takes the pair GEMM, whose K blocks then split over the idle SMs (below 128 tokens
+// the bf16 copy costs more than the fused kernel's idle SMs). Settable so that both
+// routes can be compared at any M (qlora_linear_set_pair_min_m; INT64_MAX keeps every
+// M > 16 on the fused kernels).
+constexpr int64_t kFewTilesMinM = 128;
 static std::atomic<int64_t> g_pair_min_m{512};
 // The dequantisation beside the adapter product runs two 256-thread CTAs per SM (half the
 // registers), so that the product's CTAs are scheduled next to it instead of after it.
 constexpr int kSideDequantCtas = 2;
-static bool pair_route(int64_t M) { return M >= g_pair_min_m.load(std::memory_order_relaxed); }
+// out_rows: the output dimension the fused kernel tiles by 128 (the weight rows for the
+// forward, its columns for the dgrad).
+static bool pair_route(int64_t M, int64_t out_rows) {
+    const int64_t P = g_pair_min_m.load(std::memory_order_relaxed);
+    if (M >= P) return true;
+    if (P == INT64_MAX || M < kFewTilesMinM) return false;
+    const int64_t fused_tiles = ceil_div(M, (int64_t)kTileTok) * ceil_div(out_rows, (int64_t)kTileRows);
+    return 2 * fused_tiles < num_sms();
+}
 static size_t wd_bytes(int64_t rows, int64_t cols) { return align256((size_t)rows * (size_t)cols * 2); }
 
 static size_t fwd_adapter_bytes(int64_t M, int64_t cols, int r) {
@@ -1021,21 +1040,40 @@ static size_t fwd_adapter_bytes(int64_t M, int64_t cols, int r) {
     return r == 0 ? 0 : mr_bytes(M, r);                      // s XA
 }
 
-// CTA pairs of the pair GEMM: as few pairs as give the same number of tile rounds. The
-// GEMM is bound by the power cap more than by the SM count (measured: a stream-K split of
-// the K blocks over every SM was 0.6 % slower at 4096^2 than 64 pairs of four whole tiles,
-// and its contiguous per-pair runs lost the L2 reuse of the strided tile order on the
-// 70B-like projections), and the SMs left over run the side stream's adapter gradients
-// beside the dgrad GEMM.
-static int side_job_pairs(int64_t M, int64_t N) {
+// Work plan of the pair GEMM for an [M, N] output over K inputs plus the r adapter ones.
+// With at least half as many 256 x 256 tiles as CTA pairs, whole tiles and as few pairs as
+// give the same number of tile rounds: the GEMM is bound by the power cap more than by the
+// SM count (measured: a stream-K split of the K blocks over every SM was 0.6 % slower at
+// 4096^2 than 64 pairs of four whole tiles, and its contiguous per-pair runs lost the L2
+// reuse of the strided tile order on the 70B-like projections), and the SMs left over run
+// the side stream's adapter gradients beside the dgrad GEMM. With fewer tiles, each tile's
+// K blocks are split (at least eight per range, at most gemm2sm_max_splits ranges) so that
+// the items fill the pairs, and a reduction adds the fp32 partials.
+struct PairPlan {
+    int pairs, splits;
+};
+static PairPlan pair_plan(int64_t M, int64_t N, int64_t K, int r) {
     const int64_t ntiles = ceil_div(M, 256) * ceil_div(N, 256);
     const int max_pairs = gemm2sm_pairs(0);
-    const int64_t rounds = ceil_div(ntiles, max_pairs);
-    return (int)ceil_div(ntiles, rounds);
+    const int kbt = (int)(ceil_div(K, 64) + ceil_div((int64_t)r, 64));
+    int splits = 1;
+    if (2 * ntiles <= max_pairs) {
+        splits = (int)(max_pairs / ntiles);
+        if (splits > kbt / 8) splits = kbt / 8;
+        if (splits > gemm2sm_max_splits()) splits = gemm2sm_max_splits();
+        if (splits < 1) splits = 1;
+    }
+    const int64_t items = ntiles * splits;
+    const int64_t rounds = ceil_div(items, (int64_t)max_pairs);
+    return {(int)ceil_div(items, rounds), splits};
+}
+static size_t split_bytes(const PairPlan &pp, int64_t M, int64_t N) {
+    return pp.splits > 1 ? align256((size_t)pp.splits * (size_t)M * (size_t)N * 4) : 0;
 }
 
 size_t fwd_workspace_bytes_large(int64_t M, int64_t rows, int64_t cols, int r) {
-    return fwd_adapter_bytes(M, cols, r) + (pair_route(M) ? wd_bytes(rows, cols) : 0);
+    if (!pair_route(M, rows)) return fwd_adapter_bytes(M, cols, r);
+    return fwd_adapter_bytes(M, cols, r) + wd_bytes(rows, cols) + split_bytes(pair_plan(M, rows, cols, r), M, rows);
 }
 
 static size_t bwd_adapter_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
@@ -1045,7 +1083,8 @@ static size_t bwd_adapter_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
 }
 
 size_t bwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r) {
-    return bwd_adapter_bytes(M, rows, cols, r) + (pair_route(M) ? wd_bytes(rows, cols) : 0);
+    if (!pair_route(M, cols)) return bwd_adapter_bytes(M, rows, cols, r);
+    return bwd_adapter_bytes(M, rows, cols, r) + wd_bytes(rows, cols) + split_bytes(pair_plan(M, cols, rows, r), M, cols);
 }
 
 static cudaError_t run_fused_fwd(const __nv_bfloat16 *X, int64_t M, const NF4View &W, const __nv_bfloat16 *XAs,
@@ -1139,7 +1178,7 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
                                     const __nv_bfloat16 *B, int r, float s, __nv_bfloat16 *Y,
                                     __nv_bfloat16 *XA_save, void *ws, cudaStream_t st) {
     __nv_bfloat16 *XAs = nullptr;
-    const bool pair = pair_route(M);
+    const bool pair = pair_route(M, W.rows);
     __nv_bfloat16 *Wd = pair ? reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + fwd_adapter_bytes(M, W.cols, r))
                              : nullptr;
     cudaError_t e;
@@ -1173,7 +1212,9 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
     if (pair) {
         // Y = X W^T + (s XA) B: W^ [d_out, d_in] is the K-major B operand, B_lora [r, d_out]
         // the MN-major extension
-        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, side_job_pairs(M, W.rows), r > 0,
+        const PairPlan pp = pair_plan(M, W.rows, W.cols, r);
+        float *part = reinterpret_cast<float *>(reinterpret_cast<char *>(Wd) + wd_bytes(W.rows, W.cols));
+        return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, pp.pairs, pp.splits, part, r > 0,
                               st);
     }
     return run_fused_fwd(X, M, W, XAs, B, r, Y, st);
@@ -1204,7 +1245,7 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
                               cudaStream_t st) {
     __nv_bfloat16 *Gs = nullptr;
     cudaError_t e;
-    const bool pair = pair_route(M);
+    const bool pair = pair_route(M, W.cols);
     __nv_bfloat16 *Wd = pair ? reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) +
                                                                 bwd_adapter_bytes(M, W.rows, W.cols, r))
                              : nullptr;
@@ -1245,17 +1286,19 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
     if (pair) {
         // dX = dY W^ + (s G) A^T: W^ [d_out, d_in] read as the MN-major B operand
         // ([K = d_out][N = d_in]), A_lora [d_in, r] the K-major extension
+        const PairPlan pp = pair_plan(M, W.cols, W.rows, r);
+        float *part = reinterpret_cast<float *>(reinterpret_cast<char *>(Wd) + wd_bytes(W.rows, W.cols));
         if (r > 0) {
             // the adapter gradients need only Gs and XA: they run on the side stream
             // while the dgrad GEMM occupies the tensor cores
             if (side) {
                 if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
-                e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, side_job_pairs(M, W.cols), true,
-                                   st);
+                e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, pp.pairs, pp.splits, part,
+                                   true, st);
                 if (e != cudaSuccess) return e;
                 if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
                 // sized for the SMs the dgrad GEMM leaves free
-                int free_sms = num_sms() - 2 * side_job_pairs(M, W.cols);
+                int free_sms = num_sms() - 2 * pp.pairs;
                 if (free_sms < 2) free_sms = 2;
                 e = adapter_grads(X, dY, M, W, Gs, XA, r, s, dA, dB, side->s, free_sms);
                 if (e != cudaSuccess) return e;
@@ -1263,7 +1306,7 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
                 return cudaStreamWaitEvent(st, side->join, 0);
             }
         }
-        e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, side_job_pairs(M, W.cols), r > 0,
+        e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, pp.pairs, pp.splits, part, r > 0,
                            st);
     } else {
         e = run_fused_dgrad(dY, M, W, A, Gs, r, dX, st);

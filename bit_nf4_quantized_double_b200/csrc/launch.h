@@ -35,9 +35,10 @@ cudaError_t launch_merge_bf16(const NF4View &q, const __nv_bfloat16 *A, const __
 
 // Plain bf16 GEMM on CTA pairs (tcgen05 cta_group::2), see gemm2sm.cu.
 int gemm2sm_pairs(int max_pairs);
+int gemm2sm_max_splits();
 cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, const __nv_bfloat16 *B, bool b_mn,
                            const __nv_bfloat16 *Be, bool be_mn, __nv_bfloat16 *C, int64_t M, int64_t N, int64_t K,
-                           int ke, int pairs, bool pdl, cudaStream_t st);
+                           int ke, int pairs, int splits, float *partial, bool pdl, cudaStream_t st);
 
 size_t fwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r);
 

@@ -63,8 +63,14 @@ def test_workspace_queries_positive():
     for M in (1, 16, 17, 4096):
         assert L.qlora_linear_fwd_workspace(M, 4096, 4096, 64) > 0
         assert L.qlora_linear_bwd_workspace(M, 4096, 4096, 64) > 0
-    # no adapter and a small batch: nothing to stage
-    assert L.qlora_linear_bwd_workspace(256, 4096, 4096, 0) == 0
+    # no adapter and a batch below 512 tokens whose fused kernel fills the SMs: nothing to stage
+    assert L.qlora_linear_bwd_workspace(256, 4096, 16384, 0) == 0
+    # below 512 tokens, a dgrad whose fused kernel would have only 32 output tiles takes the
+    # pair GEMM: the bf16 weight plus fp32 partials of 4 K ranges of its 16 tiles (148 SMs,
+    # the count assumed without a GPU)
+    assert L.qlora_linear_bwd_workspace(256, 4096, 4096, 0) == 4096 * 4096 * 2 + 4 * 256 * 4096 * 4
+    # under 128 tokens the fused kernels always run
+    assert L.qlora_linear_bwd_workspace(127, 4096, 4096, 0) == 0
     # from 512 tokens on, the layer keeps a bf16 copy of the dequantised weight
     assert L.qlora_linear_bwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2
     assert L.qlora_linear_fwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2

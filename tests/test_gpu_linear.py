@@ -267,11 +267,23 @@ def test_zero_adapter_equals_plain_product():
         assert m <= MAX_TOL and f <= FRO_TOL
 
 
+@pytest.mark.parametrize("M,rows,cols,r", [
+    (512, 512, 8192, 64),     # forward: 4 tiles, 16 K ranges per tile; dgrad: 64 whole tiles
+    (200, 384, 2048, 64),     # below 512 tokens: the fused kernels would use 3 and 16 CTAs
+    (4096, 256, 4096, 16),    # headline tokens, a narrow output: 16 tiles, 4 K ranges
+])
+def test_split_k_pair_route(M, rows, cols, r):
+    # few output tiles: the pair GEMM splits each tile's K blocks over the idle SMs and adds
+    # the fp32 partials in a fixed order; every element against the oracle
+    run_case(M, rows, cols, r, seed=M + rows + cols)
+
+
 @pytest.mark.parametrize("rep", [0, 1])
 def test_many_tiles_per_cta_fused_full(rep):
-    # below 512 tokens the fused dequant-GEMM kernels run; with 16384 weight rows
-    # (forward) or 16384 inputs (dgrad) every persistent CTA walks several 128 x 256
-    # tiles: compare every element, twice, so a race at tile boundaries shows
+    # below 512 tokens: the forward of the 16384-row weight and the dgrad of the
+    # 16384-input one stay on the fused kernels, where every persistent CTA walks several
+    # 128 x 256 tiles; the other two directions have 16 fused tiles and take the pair GEMM
+    # with split K. Compare every element, twice, so a race at tile boundaries shows
     M = 480
     for rows, cols in ((16384, 1024), (1024, 16384)):
         W, X, dY, A, B, s = make_problem(M, rows, cols, 64, seed=500 + rows + rep)
@@ -311,8 +323,8 @@ def test_many_tiles_per_cta_full(rep):
 
 
 @pytest.mark.parametrize("P,M,rows,cols,r", [
-    (2 ** 62, 1024, 512, 1024, 16),   # the fused dequant-GEMM at four token tiles
-    (2 ** 62, 4096, 256, 512, 64),    # ... and at the headline's 4096 tokens
+    (2 ** 63 - 1, 1024, 512, 1024, 16),   # the fused dequant-GEMM at four token tiles
+    (2 ** 63 - 1, 4096, 256, 512, 64),    # ... and at the headline's 4096 tokens
     (17, 100, 400, 320, 24),          # the dequant + CTA-pair route below one 256-token tile
     (17, 300, 272, 192, 64),
 ])
