@@ -644,21 +644,28 @@ k_merge_bf16(NF4View q, const float *__restrict__ At, const float *__restrict__ 
                                         ? dq_constant(q.scale8[n * kbs + blkk], q.scale2[(n * kbs + blkk) / kBlock2], mu)
                                         : 0.0f;
             }
-            const float *As = msm + (size_t)((step & 1) * 2) * kMergeBuf;
-            const float *Bs = As + kMergeBuf;
+            // this thread's columns of the chunk: fixed offsets from two base pointers
+            const float *Ap = msm + (size_t)((step & 1) * 2) * kMergeBuf + 4 * tk;
+            const float *Bp = msm + (size_t)((step & 1) * 2 + 1) * kMergeBuf + 8 * tn;
             const int jn = r - c * kMergeJ < kMergeJ ? r - c * kMergeJ : kMergeJ;
-#pragma unroll 2
-            for (int jj = 0; jj < jn; ++jj) {
-                const float4 a0 = *reinterpret_cast<const float4 *>(As + jj * kMergeTile + 4 * tk);
-                const float4 a1 = *reinterpret_cast<const float4 *>(As + jj * kMergeTile + 64 + 4 * tk);
-                const float4 b0 = *reinterpret_cast<const float4 *>(Bs + jj * kMergeTile + 8 * tn);
-                const float4 b1 = *reinterpret_cast<const float4 *>(Bs + jj * kMergeTile + 8 * tn + 4);
+            auto fma_step = [&](int jj) {
+                const float4 a0 = *reinterpret_cast<const float4 *>(Ap + jj * kMergeTile);
+                const float4 a1 = *reinterpret_cast<const float4 *>(Ap + jj * kMergeTile + 64);
+                const float4 b0 = *reinterpret_cast<const float4 *>(Bp + jj * kMergeTile);
+                const float4 b1 = *reinterpret_cast<const float4 *>(Bp + jj * kMergeTile + 4);
                 const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
                 const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
 #pragma unroll
                     for (int cc = 0; cc < 8; ++cc) d[i][cc] = fmaf(a[cc], b[i], d[i][cc]);
+            };
+            if (jn == kMergeJ) {
+#pragma unroll
+                for (int jj = 0; jj < kMergeJ; ++jj) fma_step(jj);
+            } else {
+#pragma unroll 1
+                for (int jj = 0; jj < jn; ++jj) fma_step(jj);
             }
             __syncthreads();   // every thread is done with this buffer before it is refilled
         }
