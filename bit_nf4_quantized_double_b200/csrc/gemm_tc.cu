@@ -737,6 +737,7 @@ struct SkinnyParams {
     int Mp, Np, BN;        // output rows, columns (r), MMA N (Np rounded up to 16)
     int kb_total, kb_per_split;
     int stages;
+    int nb;                // K blocks per stage: 2 with a K-major A read by one 3D box, else 1
     int transpose;         // the fp32 output as [Np][Mp] instead of [Mp][Np]
     float s;               // scale of out_s and out_f32
     __nv_bfloat16 *out;    // bf16 [Mp][Np] of the sum, or null
@@ -761,13 +762,15 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     uint8_t *smem = align1024(smem_raw);
-    const int S = p.stages;
+    const int S = p.stages, NB = p.nb;
     const int a_bytes = 128 * 128;
     const int b_chunks = B_MN ? (p.BN + 63) / 64 : 1;
     const int b_bytes = B_MN ? b_chunks * 8192 : p.BN * 128;
     const int b_alloc = (b_bytes + 1023) & ~1023;
+    // stage s: NB A tiles (16 KB each, consecutive K blocks) at as + s NB a_bytes, then the
+    // NB B tiles at bs + s NB b_alloc
     uint8_t *as = smem;
-    uint8_t *bs = smem + S * a_bytes;
+    uint8_t *bs = smem + S * NB * a_bytes;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t bar0 = smem_addr(bars);
     auto full = [&](int s) { return bar0 + 8u * s; };
@@ -806,22 +809,29 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
 
     if (warp == 0 && lane == 0) {
         uint32_t it = 0;
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; kb += NB, ++it) {
             const int s = it % S;
             const uint32_t ph = (it / S) & 1u;
             if (!mbar_wait(empty(s), ph ^ 1u, abort)) break;
-            mbar_arrive_expect_tx(full(s), a_bytes + b_bytes);
-            const uint32_t a = smem_addr(as + s * a_bytes), b = smem_addr(bs + s * b_alloc);
+            // a box past the split's last block (or past K, zero-filled) is loaded whole and
+            // left unused by the MMAs
+            mbar_arrive_expect_tx(full(s), NB * (a_bytes + b_bytes));
+            const uint32_t a = smem_addr(as + s * NB * a_bytes), b = smem_addr(bs + s * NB * b_alloc);
             if (A_MN) {
                 tma_load_2d(a, &tm_a, full(s), m0, kb * 64);
                 tma_load_2d(a + 8192, &tm_a, full(s), m0 + 64, kb * 64);
+            } else if (NB > 1) {
+                tma_load_3d(a, &tm_a, full(s), 0, m0, kb);     // NB K blocks of 128 rows: 128 NB-byte row runs
             } else {
                 tma_load_2d(a, &tm_a, full(s), kb * 64, m0);
             }
-            if (B_MN) {
-                for (int c = 0; c < b_chunks; ++c) tma_load_2d(b + 8192u * c, &tm_b, full(s), 64 * c, kb * 64);
-            } else {
-                tma_load_2d(b, &tm_b, full(s), kb * 64, 0);
+            for (int bi = 0; bi < NB; ++bi) {
+                const uint32_t bb = b + (uint32_t)(bi * b_alloc);
+                if (B_MN) {
+                    for (int c = 0; c < b_chunks; ++c) tma_load_2d(bb + 8192u * c, &tm_b, full(s), 64 * c, (kb + bi) * 64);
+                } else {
+                    tma_load_2d(bb, &tm_b, full(s), (kb + bi) * 64, 0);
+                }
             }
         }
         const uint32_t first = it > (uint32_t)S ? it - S : 0;
@@ -830,16 +840,20 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
         const uint32_t idesc = idesc_bf16(128, p.BN, A_MN, B_MN);
         uint32_t it = 0;
         bool ok = true;
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; kb += NB, ++it) {
             const int s = it % S;
             const uint32_t ph = (it / S) & 1u;
             if (!mbar_wait(full(s), ph, abort)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t a = smem_addr(as + s * a_bytes), b = smem_addr(bs + s * b_alloc);
-            for (int k = 0; k < 4; ++k) {
-                const uint64_t ad = A_MN ? sw128_desc(a + 2048u * k, 8192, 1024) : sw128_desc(a + 32u * k, 16, 1024);
-                const uint64_t bd = B_MN ? sw128_desc(b + 2048u * k, 8192, 1024) : sw128_desc(b + 32u * k, 16, 1024);
-                mma_ss(tmem, ad, bd, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
+            for (int bi = 0; bi < NB && kb + bi < kb1; ++bi) {
+                const uint32_t a = smem_addr(as + (s * NB + bi) * a_bytes), b = smem_addr(bs + (s * NB + bi) * b_alloc);
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t ad =
+                        A_MN ? sw128_desc(a + 2048u * k, 8192, 1024) : sw128_desc(a + 32u * k, 16, 1024);
+                    const uint64_t bd =
+                        B_MN ? sw128_desc(b + 2048u * k, 8192, 1024) : sw128_desc(b + 32u * k, 16, 1024);
+                    mma_ss(tmem, ad, bd, idesc, (kb + bi != kb0 || k != 0) ? 1u : 0u);
+                }
             }
             mma_commit(empty(s));
         }
@@ -956,9 +970,20 @@ static cudaError_t run_skinny(bool a_mn, const void *a, bool b_mn, const void *b
                               const SkinnyOut &out, cudaStream_t st, int sms = 0) {
     CUtensorMap ta, tb;
     const int BN = (int)ceil_div(r, 16) * 16;
+    // a K-major A whose rows are whole 64-element blocks is read two blocks per 3D box
+    // ([64 elements][Mp rows][Kp/64 blocks], block stride 128 bytes): 256-byte row runs
+    const int nb = (!a_mn && Kp % 64 == 0) ? 2 : 1;
     bool ok;
-    if (a_mn) ok = map_bf16(&ta, a, (uint64_t)Mp, (uint64_t)Kp, 64, 64);
-    else ok = map_bf16(&ta, a, (uint64_t)Kp, (uint64_t)Mp, 64, 128);
+    if (a_mn) {
+        ok = map_bf16(&ta, a, (uint64_t)Mp, (uint64_t)Kp, 64, 64);
+    } else if (nb > 1) {
+        const uint64_t dims[3] = {64, (uint64_t)Mp, (uint64_t)(Kp / 64)};
+        const uint64_t strides[2] = {(uint64_t)Kp * 2, 128};
+        const uint32_t box[3] = {64, 128, (uint32_t)nb};
+        ok = make_map_3d(&ta, a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    } else {
+        ok = map_bf16(&ta, a, (uint64_t)Kp, (uint64_t)Mp, 64, 128);
+    }
     if (b_mn) ok = ok && map_bf16(&tb, b, (uint64_t)r, (uint64_t)Kp, 64, 64);
     else ok = ok && map_bf16(&tb, b, (uint64_t)Kp, (uint64_t)r, 64, (uint32_t)BN);
     if (!ok) return cudaErrorInvalidValue;
@@ -975,11 +1000,14 @@ static cudaError_t run_skinny(bool a_mn, const void *a, bool b_mn, const void *b
     p.out_s = out.bf16_s;
     p.out_f32 = out.f32;
     const int b_bytes = b_mn ? (int)ceil_div(BN, 64) * 8192 : BN * 128;
-    const int stage = 128 * 128 + ((b_bytes + 1023) & ~1023);
+    const int stage = nb * (128 * 128 + ((b_bytes + 1023) & ~1023));
+    const int groups = (int)ceil_div(sp.kb_per_split, nb);      // stage loads per split
     int stages = (100 * 1024) / stage;
     if (stages > kSkinnyStages) stages = kSkinnyStages;
-    if (stages > sp.kb_per_split) stages = sp.kb_per_split < 2 ? 2 : sp.kb_per_split;
+    if (stages > groups) stages = groups < 2 ? 2 : groups;
+    if (stages < 1) stages = 1;
     p.stages = stages;
+    p.nb = nb;
     const int acc_bytes = 128 * (BN + 4) * 4;       // the staged accumulator reuses the stages
     const int smem = 1024 + (stages * stage > acc_bytes ? stages * stage : acc_bytes);
     cudaLaunchConfig_t cfg = {};
