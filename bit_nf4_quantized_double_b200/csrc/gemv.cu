@@ -323,10 +323,11 @@ __device__ __forceinline__ void x_load(const GemvGroup &grp, UnitPos p, int ks, 
 }
 
 // Y[tok][R] = sum over K chunks c in order of partial[c][R][tok] + sum_j (s XA)[tok][j] B[j][R]
-// (fused multiply-adds in increasing j), one thread per output element (R, tok), tok
-// fastest. XA = its X A chunk partials added in chunk order, staged in shared memory
-// (times s); the first CTA of a projection also saves XA as bf16. Every sum issues its
-// loads (up to eight) before the adds, so a thread waits for memory about three times.
+// (fused multiply-adds in increasing j), one thread per row R and group of up to four
+// tokens (tokens fastest), so that a B value serves up to four tokens. XA = its X A chunk
+// partials added in chunk order, staged in shared memory (times s); the first CTA of a
+// projection also saves XA as bf16. Every sum issues its loads (up to eight) before the
+// adds, so a thread waits for memory about three times.
 constexpr int kFinishThreads = 256;
 __global__ void __launch_bounds__(kFinishThreads) k_gemv_finish(const __grid_constant__ FinishGroup grp) {
     __shared__ float sx[kGemvMaxM * 256];
@@ -350,31 +351,44 @@ __global__ void __launch_bounds__(kFinishThreads) k_gemv_finish(const __grid_con
         if (blockIdx.x == it.cta0 && it.XA_save) it.XA_save[i] = __float2bfloat16_rn(v);
     }
     __syncthreads();
+    const int MQ = (M + 3) / 4;                      // token groups of four
     const int64_t e = (int64_t)(blockIdx.x - it.cta0) * kFinishThreads + threadIdx.x;
-    if (e >= (int64_t)N * M) return;
-    const int R = (int)(e / M), m = (int)(e - (int64_t)R * M);
-    float y = 0.0f;
-    for (int c0 = 0; c0 < it.nch; c0 += 8) {
-        float pv[8];
+    if (e >= (int64_t)N * MQ) return;
+    const int R = (int)(e / MQ), m0 = 4 * (int)(e - (int64_t)R * MQ);
+    const int mn = M - m0 < 4 ? M - m0 : 4;
+    float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int c0 = 0; c0 < it.nch; c0 += 4) {
+        float pv[4][4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-            pv[c] = c0 + c < it.nch ? __ldcg(it.partial + ((int64_t)(c0 + c) * N + R) * M + m) : 0.0f;
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-            if (c0 + c < it.nch) y += pv[c];
+            for (int q = 0; q < 4; ++q)
+                pv[c][q] = (c0 + c < it.nch && q < mn) ? __ldcg(it.partial + ((int64_t)(c0 + c) * N + R) * M + m0 + q)
+                                                       : 0.0f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (c0 + c < it.nch)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) y[q] += pv[c][q];
     }
     if (r > 0) {
-        float a = 0.0f;
+        float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         for (int j0 = 0; j0 < r; j0 += 8) {          // r % 8 == 0: eight B loads in flight
             float bv[8];
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) bv[jj] = __bfloat162float(it.B[(int64_t)(j0 + jj) * N + R]);
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) a = fmaf(sx[m * r + j0 + jj], bv[jj], a);
+            for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (q < mn) a[q] = fmaf(sx[(m0 + q) * r + j0 + jj], bv[jj], a[q]);
         }
-        y += a;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) y[q] += a[q];
     }
-    it.Y[(int64_t)m * N + R] = __float2bfloat16_rn(y);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        if (q < mn) it.Y[(int64_t)(m0 + q) * N + R] = __float2bfloat16_rn(y[q]);
 }
 
 // Compute warps of k_gemv (warp w < 8 RG): row group w / 8, K slice w % 8.
@@ -736,7 +750,7 @@ static cudaError_t gemv_group(int64_t M, int count, const LinearDesc *d, void *w
         fi.XA_save = d[i].r > 0 ? d[i].XA_save : nullptr;
         fi.nxa = 0;
         fi.cta0 = fc;
-        fc += (int)ceil_div(w.rows * M, (int64_t)kFinishThreads);
+        fc += (int)ceil_div(w.rows * ceil_div(M, (int64_t)4), (int64_t)kFinishThreads);
     }
     int xc = 0;
     for (int i = 0; i < count; ++i) {
