@@ -335,3 +335,39 @@ def test_routes_forced_either_way(P, M, rows, cols, r):
         run_case(M, rows, cols, r, seed=M + rows + r + 7)
     finally:
         q.lib().qlora_linear_set_pair_min_m(512)
+
+
+@pytest.mark.parametrize("M,rows,cols,r", [(512, 1024, 2048, 16), (600, 768, 1536, 0), (256, 4096, 1024, 8)])
+def test_workspace_weight_bit_exact(M, rows, cols, r):
+    # On the pair route the layer dequantises the weight into its workspace, which starts
+    # with the adapter scratch (forward: s XA, M x r bf16; backward: s G and X A), each
+    # rounded up to 256 bytes, followed by the bf16 weight: after the call that weight must
+    # equal the oracle's dequantisation bit for bit, and the layer's outputs stay within the
+    # tolerance.
+    W, X, dY, A, B, s = make_problem(M, rows, cols, r, 7100 + M + r)
+    t = q.qlora_nf4_quantize(W)
+    L = q.lib()
+    mr = ((M * r * 2 + 255) // 256) * 256 if r else 0
+    want = oracle.dequant(oracle.quantize(W.float().cpu().numpy())).reshape(rows, cols)
+    ws_f = torch.zeros(L.qlora_linear_fwd_workspace(M, rows, cols, r), dtype=torch.uint8, device="cuda")
+    Y, XA = q.qlora_linear_fwd(X, t, A, B, s, ws=ws_f)
+    ws_b = torch.zeros(L.qlora_linear_bwd_workspace(M, rows, cols, r), dtype=torch.uint8, device="cuda")
+    dX, dA, dB = q.qlora_linear_bwd(X, dY, t, A, B, s, XA=XA, ws=ws_b)
+    torch.cuda.synchronize()
+    assert q.qlora_get_device_status() == q.QLORA_OK
+    n = rows * cols * 2
+    if M >= 512:
+        got_f = ws_f[mr:mr + n].view(torch.int16).cpu().numpy().view(np.uint16).reshape(rows, cols)
+        assert np.array_equal(got_f, want), "forward workspace weight"
+    got_b = ws_b[2 * mr:2 * mr + n].view(torch.int16).cpu().numpy().view(np.uint16).reshape(rows, cols)
+    assert np.array_equal(got_b, want), "backward workspace weight"
+    Wh = oracle_weight(W)
+    Xn, dYn = f64(X), f64(dY)
+    An = f64(A) if r else np.zeros((cols, 0))
+    Bn = f64(B) if r else np.zeros((0, rows))
+    check(f64(Y), oracle.linear_fwd(Xn, Wh, An, Bn, s), "Y")
+    dXr, dAr, dBr = oracle.linear_bwd(Xn, dYn, Wh, An, Bn, s)
+    check(f64(dX), dXr, "dX")
+    if r:
+        check(f64(dA), dAr, "dA")
+        check(f64(dB), dBr, "dB")
