@@ -937,7 +937,8 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
 
 // ================================================================ host side
 // Split-K sizing: at most two CTAs per SM, all resident at once, at most
-// kSkinnyMaxSplits CTAs (one cluster) per M tile.
+// kSkinnyMaxSplits CTAs (one cluster) per M tile, and at most four when four CTAs per
+// M tile already reach three quarters of the SMs and K is at most 64 blocks.
 constexpr int kSkinnyStages = 4;
 
 struct SplitPlan { int kb_total, kb_per_split, splits; };
@@ -947,6 +948,11 @@ static SplitPlan plan_splits(int64_t Mp, int64_t Kp, int sms) {
     const int mt = (int)ceil_div(Mp, 128);
     int want = (2 * sms) / mt;
     if (want > kSkinnyMaxSplits) want = kSkinnyMaxSplits;
+    // four-CTA clusters once the tiles alone give most SMs a CTA and K is short: each tile's
+    // reduction and cluster barrier then span half as many CTAs (measured at M = 4096: 248
+    // against 253 us for the 4096^2 layer's fwd + bwd step; with K = 8192 and more, the
+    // streaming outweighs those fixed costs and two CTAs per SM stream faster)
+    if (want > 4 && 4 * mt >= (3 * sms) / 4 && sp.kb_total <= 64) want = 4;
     if (want < 1) want = 1;
     if (want > sp.kb_total) want = sp.kb_total;
     sp.kb_per_split = (int)ceil_div(sp.kb_total, want);
@@ -1049,9 +1055,15 @@ static size_t mr_bytes(int64_t M, int r) { return align256((size_t)M * (size_t)r
 // M > 16 on the fused kernels).
 constexpr int64_t kFewTilesMinM = 128;
 static std::atomic<int64_t> g_pair_min_m{512};
-// The dequantisation beside the adapter product runs two 256-thread CTAs per SM (half the
-// registers), so that the product's CTAs are scheduled next to it instead of after it.
-constexpr int kSideDequantCtas = 2;
+// CTAs per SM of the dequantisation beside an adapter product of Mp rows over Kp inputs:
+// three 256-thread CTAs when the product has at most one CTA per SM (they leave it the
+// registers for one), else two, so that the product's CTAs are scheduled next to the
+// dequantisation instead of after it (measured at 4096^2: 247.8 against 249.1 us per
+// fwd + bwd step for three against two).
+static int side_dequant_ctas(int64_t Mp, int64_t Kp) {
+    const SplitPlan sp = plan_splits(Mp, Kp, num_sms());
+    return ceil_div(Mp, (int64_t)128) * sp.splits <= num_sms() ? 3 : 2;
+}
 // out_rows: the output dimension the fused kernel tiles by 128 (the weight rows for the
 // forward, its columns for the dgrad).
 static bool pair_route(int64_t M, int64_t out_rows) {
@@ -1219,7 +1231,7 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
         if (side) {
             if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
             if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
-            if ((e = launch_dequant(W, Wd, side->s, kSideDequantCtas)) != cudaSuccess) return e;
+            if ((e = launch_dequant(W, Wd, side->s, side_dequant_ctas(M, W.cols))) != cudaSuccess) return e;
             if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess) return e;
         }
     }
@@ -1287,7 +1299,7 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
         if (side) {
             if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
             if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
-            if ((e = launch_dequant(W, Wd, side->s, kSideDequantCtas)) != cudaSuccess) return e;
+            if ((e = launch_dequant(W, Wd, side->s, side_dequant_ctas(M, W.rows))) != cudaSuccess) return e;
             if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess) return e;
         }
     }
