@@ -38,15 +38,15 @@ __device__ __forceinline__ int nf4_code(float x, const float *t) {
     return c;
 }
 
-// Code table of the quantiser's fast path. A weight's normalised value x' (see
-// k_quantize_codes) is mapped to u = sat(fl(x' / 2 + 1/2)) in [0, 1] (NaN to 0) and
-// to its bin k = z - 2^23 with z = fl(u 255 + 2^23), an integer in [0, 255]. Both
-// roundings are monotone, so each bin holds an interval of x'. Entry k holds the
-// one threshold T inside bin k (4.0 if none) and base = the number of thresholds
-// below bin k, both as floats; the code of x' is base + (x' > T). Valid when no
-// bin holds two thresholds and every threshold's neighbourhood T +- 2^-16 lies
-// inside its own bin (checked on the host), so that a threshold can sit between
-// x' and the exact quotient only if it is the threshold of x''s bin.
+// Code table of the quantiser's fast path. A weight is mapped to u in [0, 1], an
+// approximation of x / 2 + 1/2 with x its exact normalised value (see k_quantize_codes;
+// NaN to 0), and to its bin k = z - 2^23 with z = fl(u 255 + 2^23), an integer in
+// [0, 255]. The rounding is monotone, so each bin holds an interval of u. Entry k holds
+// the one threshold inside bin k in the same domain, U = fl(T / 2 + 1/2) (4.0 if none),
+// and base = the number of thresholds below bin k, both as floats; the code is
+// base + (u > U). Valid when no bin holds two thresholds and every threshold's
+// neighbourhood T +- 2^-16 lies inside its own bin (checked on the host), so that a
+// threshold can sit between u and the exact value only if it is the threshold of u's bin.
 struct CodeTable {
     float thr[256];
     float base[256];
@@ -73,7 +73,7 @@ static bool build_code_table(const Codebook &cb, CodeTable &tb) {
         int base = 0;
         for (int t = 0; t < 15; ++t) base += host_bin(cb.t[t]) < k ? 1 : 0;
         if (owner[k] >= 0 && owner[k] != base) return false;
-        tb.thr[k] = owner[k] >= 0 ? cb.t[owner[k]] : 4.0f;
+        tb.thr[k] = owner[k] >= 0 ? std::fmaf(cb.t[owner[k]], 0.5f, 0.5f) : 4.0f;
         tb.base[k] = (float)base;
     }
     return true;
@@ -180,20 +180,21 @@ __device__ __forceinline__ int quant_item(const QuantGroup &g, int64_t b, bool d
 // (integer order equals float order there; inf and NaN compare above every finite
 // value, which also flags a non-finite block).
 //
-// With BINS (default), a lane multiplies by an approximate reciprocal r of c1
-// (within 1 ulp): x' = fl(w r) lies within 3 ulp of the exact quotient
-// x = fl(w / c1), and the code is base + (x' > T) from the lane's own copy of the
-// code table (entry k of lane l at byte 256 k + 8 l: the 32 lanes never meet in one
-// bank; the address is one integer multiply-add of z's bit pattern). The per-weight
-// work stays on the FMA pipe: the compare is sat(fl(x' - T) 2^100), the codes are
-// summed into the mantissa of 2^23 (16 bits per float, joined by one byte
-// permutation), and "near" is sat(|x' - T| 2^100 - 2^79) = 0, i.e. |x' - T| <= 2^-21
-// (thresholds lie in [2^-5, 1), where 3 ulp <= 3 2^-24). Outside that band x and x'
-// are on the same side of every threshold and the code is that of x bit for bit.
-// Inside it, or where c1 is outside [2^-126, 2^125) (a reciprocal that is not a
-// normal number), the lane's 8 or 4 codes are recomputed after the batch from the
-// exact quotient and the threshold search, out of the unrolled path. Without BINS
-// every weight is divided.
+// With BINS (default), a lane takes an approximate reciprocal r of c1 (within 1 ulp)
+// and forms u = sat(fl(w (r/2) + 1/2)) with one fused multiply-add (r/2 is exact). Then
+// |u - (w/c1)/2 - 1/2| <= 2^-25 + 2^-24, and the table's U = fl(T/2 + 1/2) is within
+// 2^-25 of T/2 + 1/2, so wherever |u - U| > 2^-22 the exact value w/c1 lies on the
+// same side of T as u does of U, more than 2^-25 (half an ulp of T) away from it, and
+// so does its rounded quotient x = fl(w / c1): the code is that of x bit for bit. The
+// code is base + (u > U) from the lane's own copy of the code table (entry k of lane l
+// at byte 256 k + 8 l: the 32 lanes never meet in one bank; the address is one integer
+// multiply-add of z's bit pattern). The per-weight work stays on the FMA pipe: the
+// compare is sat(fl(u - U) 2^100), the codes are summed into the mantissa of 2^23
+// (16 bits per float, joined by one byte permutation), and the lane keeps the smallest
+// |u - U| of its weights. Where that is <= 2^-22, or where c1 is outside [2^-126, 2^125)
+// (a reciprocal that is not a normal number), the lane's 8 or 4 codes are recomputed
+// after the batch from the exact quotient and the threshold search, out of the
+// unrolled path. Without BINS every weight is divided.
 template <typename T, bool BINS>
 __global__ void __launch_bounds__(256, 3)
 k_quantize_codes(const __grid_constant__ QuantGroup grp, Codebook cb, const __grid_constant__ CodeTable tab) {
@@ -282,28 +283,27 @@ k_quantize_codes(const __grid_constant__ QuantGroup grp, Codebook cb, const __gr
             // codes of the lane's VEC elements: NBYTES bytes, byte k = hi << 4 | lo
             uint32_t packed = 0;
             if constexpr (BINS) {
-                const float rcp = mbits == 0u ? 0.0f : rcp_approx(m);
+                const float rh = mbits == 0u ? 0.0f : __fmul_rn(rcp_approx(m), 0.5f);
                 const bool odd = mbits != 0u && (mbits - 0x00800000u) >= (0x7e000000u - 0x00800000u);
                 constexpr float kNibble[4] = {16.0f, 1.0f, 4096.0f, 256.0f};   // byte = code(2i) << 4 | code(2i+1)
                 float pf[(VEC + 3) / 4];
 #pragma unroll
                 for (int h = 0; h < (VEC + 3) / 4; ++h) pf[h] = 8388608.0f;
-                float acc = 1.0f;
+                float near = 1.0f;
 #pragma unroll
                 for (int k = 0; k < VEC; ++k) {
-                    const float xa = __fmul_rn(v[k], rcp);
-                    const float u = fma_sat(xa, 0.5f, 0.5f);
+                    const float u = fma_sat(v[k], rh, 0.5f);
                     const float z = __fmaf_rn(u, 255.0f, 8388608.0f);
                     float thr, base;
                     lds_f2(__float_as_uint(z) * 256u + tab_lane, thr, base);
-                    const float d = __fsub_rn(xa, thr);
+                    const float d = __fsub_rn(u, thr);
                     const float c = __fadd_rn(base, mul_sat(d, 0x1p100f));
                     pf[k / 4] = __fmaf_rn(c, kNibble[k % 4], pf[k / 4]);
-                    acc = __fmul_rn(acc, fma_sat(fabsf(d), 0x1p100f, -0x1p79f));
+                    near = fminf(near, fabsf(d));
                 }
                 if constexpr (VEC == 8) packed = prmt(__float_as_uint(pf[0]), __float_as_uint(pf[1]), 0x5410u);
                 else packed = __float_as_uint(pf[0]) & 0xffffu;
-                redo |= (odd || acc < 1.0f) ? (1u << j) : 0u;
+                redo |= (odd || near <= 0x1p-22f) ? (1u << j) : 0u;
             } else {
 #pragma unroll
                 for (int k = 0; k < VEC; k += 2) {
