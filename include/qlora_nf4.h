@@ -290,10 +290,10 @@ qlora_status qlora_adamw_prefetch(const void *ptr, size_t bytes, int to_device, 
 
 /*
  * Test hook of the quantiser's code search (the page has no counterpart). By default a
- * weight's code is read from a 256-bin table over x' = fl(w * r), r an approximate
- * reciprocal of c1 (within 1 ulp), and the exact quotient fl(w / c1) with the full
- * threshold search decides wherever x' lies within 2^-21 of its bin's threshold (or c1
- * is outside [2^-126, 2^125)); divide_every_weight != 0 makes
+ * weight's code is read from a 256-bin table over u = sat(fl(w * r/2 + 1/2)), r an
+ * approximate reciprocal of c1 (within 1 ulp), and the exact quotient fl(w / c1) with the
+ * full threshold search decides wherever u lies within 2^-22 of its bin's threshold
+ * fl(T/2 + 1/2) (or c1 is outside [2^-126, 2^125)); divide_every_weight != 0 makes
  * every later quantisation in the process divide every weight instead. Both give the
  * same codes bit for bit; the hook lets tests compare them. Not thread-safe with
  * concurrent quantisations.

@@ -241,14 +241,16 @@ def _band_weights_bf16():
 @pytest.mark.parametrize("divide_every_weight", [0, 1])
 def test_threshold_band_both_code_searches(divide_every_weight):
     # weights whose normalised value lies within a few ulps of a decision threshold: the
-    # bin table's x' (w times an approximate 1/c1) is then inside its fallback band
-    # (|x' - T| <= 2^-21), where the exact quotient decides. Both code searches (table with fallback; a division per weight)
+    # bin table's u (about w / c1 / 2 + 1/2, from an approximate 1/c1) is then inside its
+    # fallback band (within 2^-22 of fl(T/2 + 1/2), about 2^-21 of T), where the exact
+    # quotient decides. Both code searches (table with fallback; a division per weight)
     # must match the oracle bit for bit, in fp32 and for the closest bf16 pairs.
     rng = np.random.default_rng(5)
     w32 = _band_weights_fp32(rng)
     wb, nhits, closest = _band_weights_bf16()
     assert nhits >= 10 and closest > 16
-    # the fp32 set really reaches the band: |x' - T| <= |T| 2^-21 for many of its weights
+    # the fp32 set really reaches the band: w times fl(1/c1) within |T| 2^-21 of T (inside
+    # the band, since |T| < 1) for many of its weights
     c1 = np.repeat(w32.reshape(-1, 64)[:, 0], 64)
     xa = (w32 * (np.float32(1) / c1)).astype(np.float32)
     T = oracle.midpoints().astype(np.float32)
