@@ -84,7 +84,7 @@ size_t qlora_nf4_storage_bytes(int64_t rows, int64_t cols) {
 size_t qlora_nf4_quantize_workspace(int64_t rows, int64_t cols) {
     if (rows < 1 || cols < 1) return 0;
     const int64_t n = rows * cols, nb = ceil_div(n, kBlock1), nb2 = ceil_div(nb, kBlock2);
-    return align256((size_t)nb * 4) + align256((size_t)nb2 * 8);
+    return align256((size_t)nb * 4) + align256((size_t)nb2 * 64);
 }
 
 qlora_status qlora_nf4_quantize(const void *W, qlora_dtype dt, const qlora_nf4_tensor *out,

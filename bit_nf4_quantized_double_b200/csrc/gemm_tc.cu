@@ -200,7 +200,7 @@ constexpr uint32_t kTmemD = 0, kTmemA = 256;  // A stage s at columns 256 + 32 s
 __global__ void __launch_bounds__(fwd::kThreads, 1)
 k_fused_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
             const __grid_constant__ CUtensorMap tm_xa, const __grid_constant__ CUtensorMap tm_y,
-            FusedParams p, Codebook cb) {
+            FusedParams p, const __grid_constant__ Codebook cb) {
     using namespace fwd;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[2 * (SA + SC) + 3];
@@ -470,7 +470,7 @@ constexpr uint32_t kTmemCols = 256;
 __global__ void __launch_bounds__(dg::kThreads, 1)
 k_fused_dgrad(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_codes,
               const __grid_constant__ CUtensorMap tm_alora, const __grid_constant__ CUtensorMap tm_gs,
-              const __grid_constant__ CUtensorMap tm_dx, FusedParams p, Codebook cb) {
+              const __grid_constant__ CUtensorMap tm_dx, FusedParams p, const __grid_constant__ Codebook cb) {
     using namespace dg;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[2 * (SA + SC) + 3];

@@ -21,7 +21,7 @@ constexpr int64_t kNoAllocMaxWeights = int64_t(1) << 26;                     // 
 constexpr int64_t kNoAllocMaxBlocks = kNoAllocMaxWeights / kBlock1;          // 1,048,576 absmax blocks
 constexpr int64_t kNoAllocMaxGroups = kNoAllocMaxBlocks / kBlock2;           // 4,096 second-level groups
 constexpr size_t kC1Bytes = (size_t)kNoAllocMaxBlocks * sizeof(float);       // 4 MiB, 256-byte multiple
-constexpr size_t kScratchBytes = kC1Bytes + (size_t)kNoAllocMaxGroups * sizeof(double);
+constexpr size_t kScratchBytes = kC1Bytes + (size_t)kNoAllocMaxGroups * 8 * sizeof(double);
 
 // The scratch array. In host code this name only stands for the symbol; its
 // device address is looked up below and passed to the kernels.
@@ -59,7 +59,7 @@ extern "C" qlora_status qlora_nf4_quantize_noalloc(const void *W, qlora_dtype dt
     void *scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return QLORA_ERR_CUDA;
     // The kernels write every scratch element they later read (c1 of every
-    // block, one partial per group) within this call, so the array needs no
+    // block, one partial per 32 blocks) within this call, so the array needs no
     // clearing between calls.
     float *c1 = static_cast<float *>(scratch);
     double *part = reinterpret_cast<double *>(static_cast<char *>(scratch) + kC1Bytes);

@@ -148,7 +148,7 @@ struct QuantItem {
     const void *W;
     int64_t n, nb, nb2;
     float *c1;                   // [nb] exact absmax (workspace)
-    double *part;                // [nb2] group partial sums (workspace)
+    double *part;                // [8 nb2] partial sums of the groups' 32-block eighths (workspace)
     uint8_t *codes;
     int8_t *scale8;
     float *scale2;
@@ -197,7 +197,7 @@ __device__ __forceinline__ int quant_item(const QuantGroup &g, int64_t b, bool d
 // unrolled path. Without BINS every weight is divided.
 template <typename T, bool BINS>
 __global__ void __launch_bounds__(256, 3)
-k_quantize_codes(const __grid_constant__ QuantGroup grp, Codebook cb, const __grid_constant__ CodeTable tab) {
+k_quantize_codes(const __grid_constant__ QuantGroup grp, const __grid_constant__ Codebook cb, const __grid_constant__ CodeTable tab) {
     constexpr int VEC = 16 / sizeof(T);   // elements per 16-byte lane load
     constexpr int LPB = kBlock1 / VEC;    // lanes per block
     constexpr int BPI = 32 / LPB;         // blocks per warp iteration
@@ -207,7 +207,6 @@ k_quantize_codes(const __grid_constant__ QuantGroup grp, Codebook cb, const __gr
 
     __shared__ float s_t[16];
     __shared__ float s_c1[kBlock2];
-    __shared__ double s_part[8];
     extern __shared__ __align__(16) float2 s_tab[];   // BINS: [256][32] (64 KB)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -343,32 +342,24 @@ k_quantize_codes(const __grid_constant__ QuantGroup grp, Codebook cb, const __gr
     };
     if ((group + 1) * (int64_t)(kBlock1 * kBlock2) <= n) run_group(std::true_type{});
     else run_group(std::false_type{});
-    __syncthreads();
+    __syncwarp();
 
-    // fp64 pairwise tree over the group's 256 leaves (blocks past nb are 0):
-    // node i of level l+1 = node 2i + node 2i+1 of level l.
+    // fp64 pairwise tree over the warp's 32 leaves, the group's blocks 32 w .. 32 w + 31
+    // (blocks past nb are 0): node i of level l+1 = node 2i + node 2i+1 of level l. The
+    // group's eight warp sums are leaves 8 group .. 8 group + 7 of the tree that k_offset
+    // completes, so no warp waits for another.
     double v = (double)s_c1[threadIdx.x];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const double u = __shfl_down_sync(0xffffffffu, v, o);
         if ((lane & (2 * o - 1)) == 0) v = v + u;
     }
-    if (lane == 0) s_part[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        v = (lane < 8) ? s_part[lane] : 0.0;
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
-            const double u = __shfl_down_sync(0xffffffffu, v, o);
-            if ((lane & (2 * o - 1)) == 0) v = v + u;
-        }
-        if (lane == 0) item.part[group] = v;
-    }
+    if (lane == 0) item.part[group * 8 + warp] = v;
     }
     if (__any_sync(0xffffffffu, nonfinite) && lane == 0) raise_status(QLORA_ERR_NONFINITE);
 }
 
-// Upper levels of the pairwise tree over the nb2 group partials, zero-padded
+// Upper levels of the pairwise tree over the 8 nb2 partials (32 blocks each), zero-padded
 // to a power of two (>= 1024): thread t first reduces leaves [tC, tC+C) with
 // a binary-counter stack (which forms exactly the subtree of those leaves),
 // then the 1024 subtree sums are combined level by level. mu = fl(S / nb).
@@ -377,19 +368,19 @@ k_offset(const __grid_constant__ QuantGroup grp) {
     __shared__ double s_w[32];
     const QuantItem &item = grp.it[blockIdx.x];
     const double *__restrict__ part = item.part;
-    const int64_t nb2 = item.nb2, nb = item.nb;
+    const int64_t nl = 8 * item.nb2, nb = item.nb;
     float *__restrict__ offset_out = item.offset;
     int64_t L = 1024;
-    while (L < nb2) L <<= 1;
+    while (L < nl) L <<= 1;
     const int64_t C = L / 1024;
     const int64_t i0 = (int64_t)threadIdx.x * C;
     double v = 0.0;
-    if (i0 < nb2) {
+    if (i0 < nl) {
         double stack[48];
         int level[48];
         int sp = 0;
         for (int64_t i = 0; i < C; ++i) {
-            double x = (i0 + i < nb2) ? part[i0 + i] : 0.0;
+            double x = (i0 + i < nl) ? part[i0 + i] : 0.0;
             int l = 0;
             while (sp > 0 && level[sp - 1] == l) { x = stack[--sp] + x; ++l; }
             stack[sp] = x;
@@ -485,7 +476,7 @@ __device__ __forceinline__ uint32_t dequant_pair(const float *s_q, uint32_t byte
 }
 
 __global__ void __launch_bounds__(256)
-k_dequant(const __grid_constant__ DeqGroup grp, Codebook cb) {
+k_dequant(const __grid_constant__ DeqGroup grp, const __grid_constant__ Codebook cb) {
     __shared__ float s_q[16];
     if (threadIdx.x < 16) s_q[threadIdx.x] = cb.q[threadIdx.x];
     __syncthreads();
@@ -580,7 +571,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 __global__ void __launch_bounds__(256, 2)
 k_merge_bf16(NF4View q, const float *__restrict__ At, const float *__restrict__ Bf, int64_t ldb, int r, float s,
-             Codebook cb, __nv_bfloat16 *__restrict__ out) {
+             const __grid_constant__ Codebook cb, __nv_bfloat16 *__restrict__ out) {
     extern __shared__ __align__(16) float msm[];   // [buf][At chunk | Bf chunk], each [kMergeJ][kMergeTile]
     __shared__ float s_q[16];
     __shared__ float s_ch[2 * kMergeTile];         // c^ of (row n0 + i, 64-block g of the tile) at 2 i + g

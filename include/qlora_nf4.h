@@ -91,7 +91,8 @@ typedef struct {
 size_t qlora_nf4_storage_bytes(int64_t rows, int64_t cols);
 
 /* Workspace bytes qlora_nf4_quantize needs: nb fp32 exact absmax constants and
- * nb2 fp64 partial sums of the offset, each region 256-byte aligned. */
+ * 8*nb2 fp64 partial sums of the offset (one per 32 blocks), each region 256-byte
+ * aligned. */
 size_t qlora_nf4_quantize_workspace(int64_t rows, int64_t cols);
 
 /*
