@@ -861,7 +861,15 @@ def run_l70b(args, peaks, peak_kind, flush, stream):
                                dA=it["dA"], dB=it["dB"], ws=ws_b)
 
     reps = max(3, min(args.steps, 10))
+    # SM clocks and clock-event reasons while the layer replays (seconds of tensor work
+    # right after the memory-bound components: the power cap may lower the clock here)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    clocks.mark_begin()
     ms = _time_graph(layer, reps, flush, stream)
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    clk = clocks.stop()
     kern = _kernel_ms(KERNELS, layer, 2, flush)
     assert q.qlora_get_device_status() == q.QLORA_OK
     tf = flops / (ms / 1e3) / 1e12
@@ -895,7 +903,8 @@ def run_l70b(args, peaks, peak_kind, flush, stream):
     return {"workload": "70B-like layer: q,o 8192x8192; k,v 1024x8192; gate,up 28672x8192; down 8192x28672; "
                         "r=64, alpha=128 on all seven; M=4096; fwd+bwd of each, CUDA graph replay, L2 flushed",
             "flops_per_step": flops, "ms_per_step": round(ms, 4), "TFLOP/s": round(tf, 1),
-            "frac_of_sustained_bf16": round(tf / peak, 4), "reps": reps, "kernels": kern, "cpu_baseline": cpu}
+            "frac_of_sustained_bf16": round(tf / peak, 4), "reps": reps, "clocks": clk, "kernels": kern,
+            "cpu_baseline": cpu}
 
 
 # ------------------------------------------------------------------ CPU oracle
