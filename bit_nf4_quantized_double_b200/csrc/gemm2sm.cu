@@ -51,6 +51,7 @@ struct G2Params {
     int tiles_m, tiles_n;
     int splits;        // K ranges per tile (1: the epilogue writes C directly)
     float *partial;    // [splits][M][N] fp32 when splits > 1
+    int wait_first;    // B (not only the extension) comes from the kernel launched before
 };
 
 template <bool B_MN, bool BE_MN>
@@ -109,6 +110,13 @@ k_gemm2sm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUte
         if (lane == 0) {
             uint32_t st = 0, ph = 0;
             bool ok = true, ext_ready = false;
+            if (p.wait_first) {
+                // B is written by the kernel before this one (programmatic dependent launch):
+                // only this prologue overlapped it
+                griddep_wait();
+                fence_proxy_async_global();
+                ext_ready = true;
+            }
             for (int item = pair; item < nitems && ok; item += npairs) {
                 const int tile = item % ntiles, sp = item / ntiles;
                 const int kb_lo = sp * KBT / p.splits, kb_hi = (sp + 1) * KBT / p.splits;
@@ -310,10 +318,12 @@ int gemm2sm_pairs(int max_pairs) {
 // tile's K blocks are cut into `splits` ranges whose fp32 partials go to `partial`
 // ([splits][M][N]), and k_gemm2sm_reduce writes C. With pdl, the launch may begin while the
 // previous kernel on the stream still runs, and only the extension operands Ae, Be are read
-// after that kernel completes (it must produce nothing else this GEMM reads).
+// after that kernel completes (it must produce nothing else this GEMM reads), unless
+// wait_first, when that kernel also writes B and every load waits for it.
 cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, const __nv_bfloat16 *B, bool b_mn,
                            const __nv_bfloat16 *Be, bool be_mn, __nv_bfloat16 *C, int64_t M, int64_t N, int64_t K,
-                           int ke, int pairs, int splits, float *partial, bool pdl, cudaStream_t st) {
+                           int ke, int pairs, int splits, float *partial, bool pdl, bool wait_first,
+                           cudaStream_t st) {
     using namespace g2;
     if (M < 1 || N < 1 || K < 1 || K % 8 != 0 || N % 8 != 0 || ke < 0 || ke % 8 != 0 || pairs < 1 || splits < 1 ||
         splits > kMaxGemmSplits || (splits > 1 && !partial))
@@ -342,6 +352,7 @@ cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, cons
     p.tiles_n = (int)ceil_div(N, kTileN);
     p.splits = splits;
     p.partial = partial;
+    p.wait_first = wait_first ? 1 : 0;
     const int nitems = p.tiles_m * p.tiles_n * splits;
     if (pairs > nitems) pairs = nitems;            // at least one item per pair
     cudaError_t e;

@@ -743,8 +743,16 @@ struct SkinnyParams {
     __nv_bfloat16 *out;    // bf16 [Mp][Np] of the sum, or null
     __nv_bfloat16 *out_s;  // bf16 [Mp][Np] of s times the sum, or null
     float *out_f32;        // fp32 s times the sum, or null
+    // dequantisation carried by the same CTAs (only with extra warps, see k_skinny)
+    const uint32_t *dq_codes;    // packed codes, 8 weights per word
+    const int8_t *dq_scale8;
+    const float *dq_scale2, *dq_offset;
+    uint4 *dq_out;               // bf16 weights, 8 per uint4
+    int64_t dq_words;            // whole code words (n / 8)
+    float dq_q[16];              // codebook
 };
 constexpr int kSkinnyMaxSplits = 8;    // a portable cluster
+constexpr int kPrepDeqWarps = 12;      // dequantisation warps beside a product (one CTA per SM)
 
 __device__ __forceinline__ float4 ld_cluster_f4(uint32_t caddr) {
     float4 v;
@@ -753,14 +761,60 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t caddr) {
     return v;
 }
 
-template <bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(128, 2)
-k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, SkinnyParams p) {
+// With DW > 0 the CTA has DW more warps, which dequantise one share of a weight into bf16
+// (the page's section 3: c^ = fl(fl(q8 fl(s2/127)) + mu), w^ = bf16(fl(Q[code] c^)), the
+// same roundings as the dequantisation kernel) while warps 0..3 run the product: the two
+// memory-bound passes in the same CTAs, so that their streams overlap. Used when the
+// product has at most one CTA per SM. Warp-chunks of 256 code words (2048 weights) are
+// taken grid-stride over all CTAs' extra warps; each lane expands words 32 u + lane,
+// u = 0..7, of a chunk: eight coalesced 4-byte code loads issued before any arithmetic,
+// eight coalesced 16-byte stores.
+template <int DW>
+__device__ __forceinline__ void skinny_dequant(const SkinnyParams &p, const float *s_q) {
+    const int lane = threadIdx.x & 31, dw = (threadIdx.x >> 5) - 4;
+    const int64_t cta = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
+    const int64_t nw = p.dq_words;
+    const int64_t chunks = (nw + 255) / 256;
+    const int64_t stride = (int64_t)gridDim.x * gridDim.y * DW;
+    const float mu = __ldg(p.dq_offset);
+    for (int64_t c = cta * DW + dw; c < chunks; c += stride) {
+        const int64_t w0 = c * 256;
+        uint32_t w[8];
+        int8_t q8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int64_t wi = w0 + 32 * u + lane;
+            w[u] = wi < nw ? __ldg(p.dq_codes + wi) : 0u;
+            q8[u] = wi < nw ? __ldg(p.dq_scale8 + (wi >> 3)) : (int8_t)0;
+        }
+        const float step = __fdiv_rn(__ldg(p.dq_scale2 + (w0 >> 11)), 127.0f);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int64_t wi = w0 + 32 * u + lane;
+            if (wi < nw) {
+                const float ch = __fadd_rn(__fmul_rn((float)q8[u], step), mu);
+                const uint32_t b = w[u];
+                uint4 o;
+                o.x = pack_bf16x2(__fmul_rn(s_q[(b >> 4) & 15u], ch), __fmul_rn(s_q[b & 15u], ch));
+                o.y = pack_bf16x2(__fmul_rn(s_q[(b >> 12) & 15u], ch), __fmul_rn(s_q[(b >> 8) & 15u], ch));
+                o.z = pack_bf16x2(__fmul_rn(s_q[(b >> 20) & 15u], ch), __fmul_rn(s_q[(b >> 16) & 15u], ch));
+                o.w = pack_bf16x2(__fmul_rn(s_q[(b >> 28) & 15u], ch), __fmul_rn(s_q[(b >> 24) & 15u], ch));
+                p.dq_out[wi] = o;
+            }
+        }
+    }
+}
+
+template <bool A_MN, bool B_MN, int DW>
+__global__ void __launch_bounds__(128 + 32 * DW, DW > 0 ? 1 : 2)
+k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+         const __grid_constant__ SkinnyParams p) {
     griddep_launch_dependents();                     // a following GEMM may start its main K blocks
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[2 * 8 + 2];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
+    __shared__ float s_q[16];
     uint8_t *smem = align1024(smem_raw);
     const int S = p.stages, NB = p.nb;
     const int a_bytes = 128 * 128;
@@ -791,6 +845,7 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
         tma_prefetch_desc(&tm_a);
         tma_prefetch_desc(&tm_b);
     }
+    if (DW > 0 && threadIdx.x >= 128 && threadIdx.x < 144) s_q[threadIdx.x - 128] = p.dq_q[threadIdx.x - 128];
     if (warp == 1) {
         tmem_alloc(smem_addr(&s_tmem), ncols);
         tmem_relinquish();
@@ -807,7 +862,9 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
     const int kb0 = split * p.kb_per_split;
     const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
 
-    if (warp == 0 && lane == 0) {
+    if (DW > 0 && warp >= 4) {
+        skinny_dequant<DW>(p, s_q);
+    } else if (warp == 0 && lane == 0) {
         uint32_t it = 0;
         for (int kb = kb0; kb < kb1; kb += NB, ++it) {
             const int s = it % S;
@@ -866,22 +923,25 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
     // [128 rows][BN + 4], warp w holding TMEM lanes (rows) 32w .. 32w + 31
     const int ld = p.BN + 4;
     float *acc_s = reinterpret_cast<float *>(smem);
-    if (kb1 > kb0 && mbar_wait(done, 0, abort)) {
-        tc_fence_after();
-        const int rl = warp * 32 + lane;
-        for (int c = 0; c < p.BN; c += 16) {
-            uint32_t v[16];
-            tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
-            tmem_wait_ld();
+    if (warp < 4) {
+        // TMEM lanes 0..127 belong to warps 0..3
+        if (kb1 > kb0 && mbar_wait(done, 0, abort)) {
+            tc_fence_after();
+            const int rl = warp * 32 + lane;
+            for (int c = 0; c < p.BN; c += 16) {
+                uint32_t v[16];
+                tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+                tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; i += 4)
-                *reinterpret_cast<float4 *>(acc_s + rl * ld + c + i) =
-                    make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
-                                __uint_as_float(v[i + 3]));
+                for (int i = 0; i < 16; i += 4)
+                    *reinterpret_cast<float4 *>(acc_s + rl * ld + c + i) =
+                        make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                                    __uint_as_float(v[i + 3]));
+            }
+        } else {
+            // no K blocks for this split (or an expired wait): it adds zero
+            for (int i = threadIdx.x; i < 128 * ld; i += 128) acc_s[i] = 0.0f;
         }
-    } else {
-        // no K blocks for this split (or an expired wait): it adds zero
-        for (int i = threadIdx.x; i < 128 * ld; i += blockDim.x) acc_s[i] = 0.0f;
     }
     cluster_sync();   // every CTA's accumulator is in its shared memory
     {
@@ -967,7 +1027,21 @@ struct SkinnyOut {
     float *f32 = nullptr;
     bool f32_transposed = false;
     float s = 1.0f;
+    // optional: a weight the same launch dequantises into deq_out (see skinny_takes_dequant)
+    const NF4View *deq = nullptr;
+    __nv_bfloat16 *deq_out = nullptr;
 };
+
+// Whether a product of Mp rows over Kp inputs runs one CTA on most SMs and never two, and
+// streams at least 32 K blocks, so that its CTAs can carry the dequantisation warps
+// (kPrepDeqWarps) of a weight as well with the whole GPU's memory parallelism (measured
+// at 4096^2, M = 4096: fwd + bwd 240.9 against 247.1 us; a short K leaves the pair GEMM
+// nothing to start on early, and there the two streams are kept).
+static bool skinny_takes_dequant(int64_t Mp, int64_t Kp) {
+    const SplitPlan sp = plan_splits(Mp, Kp, num_sms());
+    const int64_t ctas = ceil_div(Mp, (int64_t)128) * sp.splits;
+    return ctas <= num_sms() && 4 * ctas >= 3 * (int64_t)num_sms() && sp.kb_total >= 32;
+}
 
 // Launch one skinny product on `sms` SMs' worth of CTAs (all of them, or those a
 // concurrent GEMM leaves free). A operand: K-major [Mp rows, Kp] or MN-major [Kp rows, Mp];
@@ -1005,6 +1079,24 @@ static cudaError_t run_skinny(bool a_mn, const void *a, bool b_mn, const void *b
     p.out = out.bf16;
     p.out_s = out.bf16_s;
     p.out_f32 = out.f32;
+    const bool with_deq = out.deq != nullptr;
+    if (with_deq) {
+        if (sms > 0 || !skinny_takes_dequant(Mp, Kp)) return cudaErrorInvalidValue;
+        p.dq_codes = reinterpret_cast<const uint32_t *>(out.deq->codes);
+        p.dq_scale8 = out.deq->scale8;
+        p.dq_scale2 = out.deq->scale2;
+        p.dq_offset = out.deq->offset;
+        p.dq_out = reinterpret_cast<uint4 *>(out.deq_out);
+        p.dq_words = out.deq->rows * out.deq->cols / 8;
+        for (int i = 0; i < 16; ++i) p.dq_q[i] = host_codebook().q[i];
+    } else {
+        p.dq_codes = nullptr;
+        p.dq_scale8 = nullptr;
+        p.dq_scale2 = p.dq_offset = nullptr;
+        p.dq_out = nullptr;
+        p.dq_words = 0;
+        for (int i = 0; i < 16; ++i) p.dq_q[i] = 0.0f;
+    }
     const int b_bytes = b_mn ? (int)ceil_div(BN, 64) * 8192 : BN * 128;
     const int stage = nb * (128 * 128 + ((b_bytes + 1023) & ~1023));
     const int groups = (int)ceil_div(sp.kb_per_split, nb);      // stage loads per split
@@ -1018,7 +1110,7 @@ static cudaError_t run_skinny(bool a_mn, const void *a, bool b_mn, const void *b
     const int smem = 1024 + (stages * stage > acc_bytes ? stages * stage : acc_bytes);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)ceil_div(Mp, 128), (unsigned)sp.splits);
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3(with_deq ? 128 + 32 * kPrepDeqWarps : 128);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = st;
     cudaLaunchAttribute at[1];
@@ -1029,15 +1121,20 @@ static cudaError_t run_skinny(bool a_mn, const void *a, bool b_mn, const void *b
     cfg.attrs = at;
     cfg.numAttrs = 1;
     cudaError_t e;
-#define QNF4_SK(AM, BM)                                                      \
-    e = set_smem(k_skinny<AM, BM>, smem);                                    \
+#define QNF4_SK(AM, BM, DW)                                                  \
+    e = set_smem(k_skinny<AM, BM, DW>, smem);                                \
     if (e != cudaSuccess) return e;                                          \
-    QNF4_LAUNCH("k_skinny", st, e = cudaLaunchKernelEx(&cfg, k_skinny<AM, BM>, ta, tb, p)); \
+    QNF4_LAUNCH("k_skinny", st, e = cudaLaunchKernelEx(&cfg, k_skinny<AM, BM, DW>, ta, tb, p)); \
     if (e != cudaSuccess) return e;
-    if (a_mn && b_mn) { QNF4_SK(true, true) }
-    else if (a_mn) { QNF4_SK(true, false) }
-    else if (b_mn) { QNF4_SK(false, true) }
-    else { QNF4_SK(false, false) }
+    if (with_deq) {
+        // the products that precede a pair GEMM: X A and dY B^T (K-major A)
+        if (a_mn) return cudaErrorInvalidValue;
+        if (b_mn) { QNF4_SK(false, true, kPrepDeqWarps) }
+        else { QNF4_SK(false, false, kPrepDeqWarps) }
+    } else if (a_mn && b_mn) { QNF4_SK(true, true, 0) }
+    else if (a_mn) { QNF4_SK(true, false, 0) }
+    else if (b_mn) { QNF4_SK(false, true, 0) }
+    else { QNF4_SK(false, false, 0) }
 #undef QNF4_SK
     return cudaGetLastError();
 }
@@ -1224,8 +1321,10 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
     cudaError_t e;
     std::unique_lock<std::mutex> lock(g_side_mu, std::defer_lock);
     SideStream *side = nullptr;
-    if (pair && r > 0) {
-        // the dequantisation and X*A are independent memory-bound passes: overlap them
+    // the dequantisation and X*A are independent memory-bound passes: run them in the same
+    // CTAs when the product has at most one CTA per SM, else on two streams
+    const bool prep = pair && r > 0 && skinny_takes_dequant(M, W.cols);
+    if (pair && r > 0 && !prep) {
         lock.lock();
         side = side_stream_locked();
         if (side) {
@@ -1238,13 +1337,17 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
     // the pair GEMM follows the X*A product directly (programmatic dependent launch: its
     // main K blocks may start while the product finishes), so the dequantised weight is
     // produced before the product or joined after it
-    if (pair && !side && (e = launch_dequant(W, Wd, st)) != cudaSuccess) return e;
+    if (pair && !side && !prep && (e = launch_dequant(W, Wd, st)) != cudaSuccess) return e;
     if (r > 0) {
         XAs = static_cast<__nv_bfloat16 *>(ws);
         SkinnyOut o;
         o.bf16 = XA_save;
         o.bf16_s = XAs;
         o.s = s;
+        if (prep) {
+            o.deq = &W;
+            o.deq_out = Wd;
+        }
         e = run_skinny(false, X, true, A, M, W.cols, r, o, st);
         if (e != cudaSuccess) return e;
         if (side && (e = cudaStreamWaitEvent(st, side->join, 0)) != cudaSuccess) return e;
@@ -1255,7 +1358,7 @@ cudaError_t launch_linear_fwd_large(const __nv_bfloat16 *X, int64_t M, const NF4
         const PairPlan pp = pair_plan(M, W.rows, W.cols, r);
         float *part = reinterpret_cast<float *>(reinterpret_cast<char *>(Wd) + wd_bytes(W.rows, W.cols));
         return launch_gemm2sm(X, XAs, Wd, false, B, true, Y, M, W.rows, W.cols, r, pp.pairs, pp.splits, part, r > 0,
-                              st);
+                              prep, st);
     }
     return run_fused_fwd(X, M, W, XAs, B, r, Y, st);
 }
@@ -1291,12 +1394,13 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
                              : nullptr;
     std::unique_lock<std::mutex> lock(g_side_mu, std::defer_lock);
     SideStream *side = nullptr;
+    // the dequantisation overlaps the dY*B^T pass (in the same CTAs, or on a second
+    // stream); after the dgrad GEMM is launched, the adapter gradients run beside it
+    const bool prep = pair && r > 0 && skinny_takes_dequant(M, W.rows);
     if (pair && r > 0) {
-        // the dequantisation overlaps the dY*B^T pass; after the dgrad GEMM is
-        // launched, the adapter gradients run beside it
         lock.lock();
         side = side_stream_locked();
-        if (side) {
+        if (side && !prep) {
             if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
             if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
             if ((e = launch_dequant(W, Wd, side->s, side_dequant_ctas(M, W.rows))) != cudaSuccess) return e;
@@ -1304,7 +1408,7 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
         }
     }
     // as in the forward, the pair GEMM follows the dY*B^T reduction directly
-    if (pair && !side && (e = launch_dequant(W, Wd, st)) != cudaSuccess) return e;
+    if (pair && !side && !prep && (e = launch_dequant(W, Wd, st)) != cudaSuccess) return e;
     if (r > 0) {
         Gs = static_cast<__nv_bfloat16 *>(ws);
         __nv_bfloat16 *XAbuf = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + mr_bytes(M, r));
@@ -1319,9 +1423,13 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
         SkinnyOut og;
         og.bf16_s = Gs;
         og.s = s;
+        if (prep) {
+            og.deq = &W;
+            og.deq_out = Wd;
+        }
         e = run_skinny(false, dY, false, B, M, W.rows, r, og, st);
         if (e != cudaSuccess) return e;
-        if (side && (e = cudaStreamWaitEvent(st, side->join, 0)) != cudaSuccess) return e;
+        if (side && !prep && (e = cudaStreamWaitEvent(st, side->join, 0)) != cudaSuccess) return e;
     }
     if (pair) {
         // dX = dY W^ + (s G) A^T: W^ [d_out, d_in] read as the MN-major B operand
@@ -1334,7 +1442,7 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
             if (side) {
                 if ((e = cudaEventRecord(side->fork, st)) != cudaSuccess) return e;
                 e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, pp.pairs, pp.splits, part,
-                                   true, st);
+                                   true, prep, st);
                 if (e != cudaSuccess) return e;
                 if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
                 // sized for the SMs the dgrad GEMM leaves free
@@ -1347,7 +1455,7 @@ cudaError_t launch_linear_bwd(const __nv_bfloat16 *X, const __nv_bfloat16 *dY, i
             }
         }
         e = launch_gemm2sm(dY, Gs, Wd, true, A, false, dX, M, W.cols, W.rows, r, pp.pairs, pp.splits, part, r > 0,
-                           st);
+                           prep, st);
     } else {
         e = run_fused_dgrad(dY, M, W, A, Gs, r, dX, st);
     }

@@ -38,7 +38,8 @@ int gemm2sm_pairs(int max_pairs);
 int gemm2sm_max_splits();
 cudaError_t launch_gemm2sm(const __nv_bfloat16 *A, const __nv_bfloat16 *Ae, const __nv_bfloat16 *B, bool b_mn,
                            const __nv_bfloat16 *Be, bool be_mn, __nv_bfloat16 *C, int64_t M, int64_t N, int64_t K,
-                           int ke, int pairs, int splits, float *partial, bool pdl, cudaStream_t st);
+                           int ke, int pairs, int splits, float *partial, bool pdl, bool wait_first,
+                           cudaStream_t st);
 
 size_t fwd_workspace_bytes(int64_t M, int64_t rows, int64_t cols, int r);
 
