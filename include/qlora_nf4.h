@@ -18,17 +18,20 @@
  *   16-byte aligned unless stated otherwise. The library never allocates or
  *   frees device memory; scratch comes from a caller-provided workspace whose
  *   size the matching *_workspace() query returns.
- * - Two resources are the library's own. (1) On the first qlora_linear_fwd or
- *   qlora_linear_bwd call on a device with M >= P (512 by default, see
- *   qlora_linear_set_pair_min_m) and r > 0, it creates one non-blocking side
- *   stream and two events for that device, kept until the process exits: those
- *   calls fork the memory-bound adapter products and the dequantisation onto it
- *   and join back before they return control of `stream`. (2) A process-wide
- *   mutex is held for the host-side duration of each such fork/join sequence
- *   (the launches, not the GPU work), so host threads that issue M >= P calls
- *   concurrently are serialised while they enqueue. Calls with M < P or r = 0,
- *   the quantiser, dequantisation, merge, optimizer and grouped forward take no
- *   lock and create nothing.
+ * - Two resources are the library's own. (1) A qlora_linear_fwd or
+ *   qlora_linear_bwd call that takes the pair-GEMM route (M >= P, 512 by
+ *   default, see qlora_linear_set_pair_min_m) with r > 0 may create, on first
+ *   use on a device, one non-blocking side stream and two events for that
+ *   device, kept until the process exits: the backward forks the adapter
+ *   gradients onto it beside the dgrad GEMM, and either direction forks the
+ *   weight's dequantisation onto it when the adapter product before the GEMM
+ *   cannot carry it in its own CTAs; every fork joins back before the call
+ *   returns control of `stream`. (2) A process-wide mutex is held for the
+ *   host-side duration of each such fork/join sequence (the launches, not the
+ *   GPU work), so host threads that issue such calls concurrently are
+ *   serialised while they enqueue. Other calls (the fused route, r = 0), the
+ *   quantiser, dequantisation, merge, optimizer and the grouped small-M forward
+ *   take no lock and create nothing.
  * - bf16 tensors are passed as void pointers to IEEE bfloat16 bit patterns.
  * - The stored weight uses the nn.Linear layout [rows = d_out, cols = d_in],
  *   row-major. The W^ of the layer equation is its transpose.
