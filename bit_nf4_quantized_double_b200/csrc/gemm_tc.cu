@@ -752,7 +752,9 @@ struct SkinnyParams {
     float dq_q[16];              // codebook
 };
 constexpr int kSkinnyMaxSplits = 8;    // a portable cluster
-constexpr int kPrepDeqWarps = 12;      // dequantisation warps beside a product (one CTA per SM)
+// dequantisation warps beside a product (one CTA per SM; 20 warps x 82 registers fill the
+// register file; measured at 4096^2 fwd + bwd: 8 warps 247.6, 12 warps 242.2, 16 warps 239.3 us)
+constexpr int kPrepDeqWarps = 16;
 
 __device__ __forceinline__ float4 ld_cluster_f4(uint32_t caddr) {
     float4 v;
@@ -1035,7 +1037,7 @@ struct SkinnyOut {
 // Whether a product of Mp rows over Kp inputs runs one CTA on most SMs and never two, and
 // streams at least 32 K blocks, so that its CTAs can carry the dequantisation warps
 // (kPrepDeqWarps) of a weight as well with the whole GPU's memory parallelism (measured
-// at 4096^2, M = 4096: fwd + bwd 240.9 against 247.1 us; the 70B-like layer, whose only
+// at 4096^2, M = 4096: fwd + bwd 240.9 against 247.1 us with twelve such warps; the 70B-like layer, whose only
 // such product has K = 1024, measured 12.6 against 12.3 ms with it, so shorter products
 // keep the two streams).
 static bool skinny_takes_dequant(int64_t Mp, int64_t Kp) {
