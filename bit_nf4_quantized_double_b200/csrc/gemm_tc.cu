@@ -1037,9 +1037,9 @@ struct SkinnyOut {
 // Whether a product of Mp rows over Kp inputs runs one CTA on most SMs and never two, and
 // streams at least 32 K blocks, so that its CTAs can carry the dequantisation warps
 // (kPrepDeqWarps) of a weight as well with the whole GPU's memory parallelism (measured
-// at 4096^2, M = 4096: fwd + bwd 240.9 against 247.1 us with twelve such warps; the 70B-like layer, whose only
-// such product has K = 1024, measured 12.6 against 12.3 ms with it, so shorter products
-// keep the two streams).
+// at 4096^2, M = 4096: fwd + bwd 240.9 against 247.1 us with twelve such warps; the
+// 70B-like layer, whose only such product has K = 1024, measured 12.6 against 12.3 ms
+// with it, so shorter products keep the two streams).
 static bool skinny_takes_dequant(int64_t Mp, int64_t Kp) {
     const SplitPlan sp = plan_splits(Mp, Kp, num_sms());
     const int64_t ctas = ceil_div(Mp, (int64_t)128) * sp.splits;
