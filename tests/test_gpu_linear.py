@@ -337,13 +337,17 @@ def test_routes_forced_either_way(P, M, rows, cols, r):
         q.lib().qlora_linear_set_pair_min_m(512)
 
 
-@pytest.mark.parametrize("M,rows,cols,r", [(512, 1024, 2048, 16), (600, 768, 1536, 0), (256, 4096, 1024, 8)])
+@pytest.mark.parametrize("M,rows,cols,r", [(512, 1024, 2048, 16), (600, 768, 1536, 0), (256, 4096, 1024, 8),
+                                           (4096, 1024, 4096, 16), (4096, 2048, 1024, 16)])
 def test_workspace_weight_bit_exact(M, rows, cols, r):
     # On the pair route the layer dequantises the weight into its workspace, which starts
     # with the adapter scratch (forward: s XA, M x r bf16; backward: s G and X A), each
     # rounded up to 256 bytes, followed by the bf16 weight: after the call that weight must
     # equal the oracle's dequantisation bit for bit, and the layer's outputs stay within the
-    # tolerance.
+    # tolerance. The dequantisation runs as its own kernel on a second stream, or inside the
+    # adapter product before the GEMM when that product has one CTA on most SMs and K >= 2048:
+    # the two M = 4096 cases take that route in the forward (K = 4096) and in the backward
+    # (K = d_out = 2048).
     W, X, dY, A, B, s = make_problem(M, rows, cols, r, 7100 + M + r)
     t = q.qlora_nf4_quantize(W)
     L = q.lib()
