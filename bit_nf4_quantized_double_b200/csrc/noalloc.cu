@@ -10,7 +10,7 @@
 // allocates or frees device memory.
 //
 // Cost of that choice: every GPU that loads the library holds kScratchBytes
-// (about 4 MiB) until the process exits, whether or not the entry point is
+// (about 4.2 MiB) until the process exits, whether or not the entry point is
 // used; tensors above kNoAllocMaxWeights weights are rejected.
 #include "launch.h"
 

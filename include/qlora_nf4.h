@@ -243,7 +243,7 @@ void qlora_nf4_codebook(float out[16]);
  * scratch that qlora_nf4_quantize asks for.
  *   Computes exactly what qlora_nf4_quantize computes (bit for bit), with the
  *   same W, dt and out arguments; the scratch is a fixed array inside this
- *   library (about 4 MiB of device memory on every GPU that loads the library,
+ *   library (about 4.2 MiB of device memory on every GPU that loads the library,
  *   held until the process exits). The call allocates and frees nothing.
  *   Limit: rows * cols <= 67,108,864 (2^26) weights; larger tensors return
  *   QLORA_ERR_UNSUPPORTED_SHAPE before anything is launched.
