@@ -772,8 +772,11 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t caddr) {
 // u = 0..7, of a chunk: eight coalesced 4-byte code loads issued before any arithmetic,
 // eight coalesced 16-byte stores.
 template <int DW>
-__device__ __forceinline__ void skinny_dequant(const SkinnyParams &p, const float *s_q) {
+__device__ __forceinline__ void skinny_dequant(const SkinnyParams &p, float *s_q) {
     const int lane = threadIdx.x & 31, dw = (threadIdx.x >> 5) - 4;
+    // this warp's own copy of the codebook: the warp starts without waiting for the CTA
+    if (lane < 16) s_q[lane] = p.dq_q[lane];
+    __syncwarp();
     const int64_t cta = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
     const int64_t nw = p.dq_words;
     const int64_t chunks = (nw + 255) / 256;
@@ -816,7 +819,7 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
     __shared__ __align__(8) uint64_t bars[2 * 8 + 2];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ float s_q[16];
+    __shared__ float s_q[DW > 0 ? DW * 16 : 1];
     uint8_t *smem = align1024(smem_raw);
     const int S = p.stages, NB = p.nb;
     const int a_bytes = 128 * 128;
@@ -835,6 +838,41 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
     uint32_t ncols = 32;
     while ((int)ncols < p.BN) ncols <<= 1;
 
+    const int m0 = blockIdx.x * 128;
+    const int split = blockIdx.y;                    // also the CTA's rank in its cluster
+    const int nsplit = gridDim.y;
+    const int kb0 = split * p.kb_per_split;
+    const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+    volatile int *abort = &s_abort;
+
+    // One stage's loads (the stage is free): NB K blocks of A and B from K block kb on. A box
+    // past the split's last block (or past K, zero-filled) is loaded whole and left unused
+    // by the MMAs.
+    auto issue = [&](int kb, int s) {
+        mbar_arrive_expect_tx(full(s), NB * (a_bytes + b_bytes));
+        const uint32_t a = smem_addr(as + s * NB * a_bytes), b = smem_addr(bs + s * NB * b_alloc);
+        if (A_MN) {
+            tma_load_2d(a, &tm_a, full(s), m0, kb * 64);
+            tma_load_2d(a + 8192, &tm_a, full(s), m0 + 64, kb * 64);
+        } else if (NB > 1) {
+            tma_load_3d(a, &tm_a, full(s), 0, m0, kb);     // NB K blocks of 128 rows: 128 NB-byte row runs
+        } else {
+            tma_load_2d(a, &tm_a, full(s), kb * 64, m0);
+        }
+        for (int bi = 0; bi < NB; ++bi) {
+            const uint32_t bb = b + (uint32_t)(bi * b_alloc);
+            if (B_MN) {
+                for (int c = 0; c < b_chunks; ++c) tma_load_2d(bb + 8192u * c, &tm_b, full(s), 64 * c, (kb + bi) * 64);
+            } else {
+                tma_load_2d(bb, &tm_b, full(s), (kb + bi) * 64, 0);
+            }
+        }
+    };
+
+    // Thread 0 initialises the barriers and at once fills the S free stages (their loads need
+    // nothing else), while warp 1 allocates TMEM; the product's warps then meet at a named
+    // barrier of their own. The dequantisation warps never wait for it.
+    uint32_t issued = 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full(s), 1);
@@ -846,52 +884,28 @@ k_skinny(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUten
         fence_barrier_init();
         tma_prefetch_desc(&tm_a);
         tma_prefetch_desc(&tm_b);
+        for (int kb = kb0; kb < kb1 && (int)issued < S; kb += NB, ++issued) issue(kb, (int)issued);
     }
-    if (DW > 0 && threadIdx.x >= 128 && threadIdx.x < 144) s_q[threadIdx.x - 128] = p.dq_q[threadIdx.x - 128];
-    if (warp == 1) {
-        tmem_alloc(smem_addr(&s_tmem), ncols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = s_tmem;
-    volatile int *abort = &s_abort;
-
-    const int m0 = blockIdx.x * 128;
-    const int split = blockIdx.y;                    // also the CTA's rank in its cluster
-    const int nsplit = gridDim.y;
-    const int kb0 = split * p.kb_per_split;
-    const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
-
     if (DW > 0 && warp >= 4) {
-        skinny_dequant<DW>(p, s_q);
-    } else if (warp == 0 && lane == 0) {
-        uint32_t it = 0;
-        for (int kb = kb0; kb < kb1; kb += NB, ++it) {
+        skinny_dequant<DW>(p, s_q + (warp - 4) * 16);
+    } else {
+        if (warp == 1) {
+            tmem_alloc(smem_addr(&s_tmem), ncols);
+            tmem_relinquish();
+        }
+        tc_fence_before();
+        named_bar_sync(1, 128);
+        tc_fence_after();
+    }
+    const uint32_t tmem = s_tmem;
+
+    if (warp == 0 && lane == 0) {
+        uint32_t it = issued;
+        for (int kb = kb0 + (int)issued * NB; kb < kb1; kb += NB, ++it) {
             const int s = it % S;
             const uint32_t ph = (it / S) & 1u;
             if (!mbar_wait(empty(s), ph ^ 1u, abort)) break;
-            // a box past the split's last block (or past K, zero-filled) is loaded whole and
-            // left unused by the MMAs
-            mbar_arrive_expect_tx(full(s), NB * (a_bytes + b_bytes));
-            const uint32_t a = smem_addr(as + s * NB * a_bytes), b = smem_addr(bs + s * NB * b_alloc);
-            if (A_MN) {
-                tma_load_2d(a, &tm_a, full(s), m0, kb * 64);
-                tma_load_2d(a + 8192, &tm_a, full(s), m0 + 64, kb * 64);
-            } else if (NB > 1) {
-                tma_load_3d(a, &tm_a, full(s), 0, m0, kb);     // NB K blocks of 128 rows: 128 NB-byte row runs
-            } else {
-                tma_load_2d(a, &tm_a, full(s), kb * 64, m0);
-            }
-            for (int bi = 0; bi < NB; ++bi) {
-                const uint32_t bb = b + (uint32_t)(bi * b_alloc);
-                if (B_MN) {
-                    for (int c = 0; c < b_chunks; ++c) tma_load_2d(bb + 8192u * c, &tm_b, full(s), 64 * c, (kb + bi) * 64);
-                } else {
-                    tma_load_2d(bb, &tm_b, full(s), (kb + bi) * 64, 0);
-                }
-            }
+            issue(kb, s);
         }
         const uint32_t first = it > (uint32_t)S ? it - S : 0;
         for (uint32_t i = first; i < it; ++i) drain_wait(full(i % S), (i / S) & 1u);
