@@ -43,6 +43,7 @@ TRAFFIC_SOURCE = {"k_gemm2sm": "ncu --metrics gpu__time_duration.sum,dram__bytes
                                 "--clock-control none -k regex:k_ on bench.py --profile-case l4096 (three fwd + bwd "
                                 "steps of this workload): mean of the six k_gemm2sm launches"}
 L2_FLUSH_BYTES = 256 << 20        # 2x the 126 MB L2
+DEFAULT_PAIR_MIN_M = 128          # the library's default token count for the pair-GEMM route
 
 
 def l2_flush(buf):
@@ -615,7 +616,7 @@ def run_routes(flush, stream):
     X, dY, A, B = inp["X"], inp["dY"], inp["A"], inp["B"]
     flops = step_flops(M, d_in, d_out, r)
     out = {"workload": "4096 x 4096 layer, M = 4096, r = 64, fwd + bwd, CUDA graph replay, L2 flushed"}
-    for name, P in (("dequant_then_pair_gemm", 512), ("fused_dequant_gemm", 2 ** 63 - 1)):
+    for name, P in (("dequant_then_pair_gemm", DEFAULT_PAIR_MIN_M), ("fused_dequant_gemm", 2 ** 63 - 1)):
         q.lib().qlora_linear_set_pair_min_m(P)
         try:
             Y = torch.empty(M, d_out, dtype=torch.bfloat16, device="cuda")
@@ -637,15 +638,15 @@ def run_routes(flush, stream):
             out[name] = {"ms_per_step": round(ms, 5), "TFLOP/s": round(flops / (ms / 1e3) / 1e12, 1),
                          "kernels": kern}
         finally:
-            q.lib().qlora_linear_set_pair_min_m(512)
+            q.lib().qlora_linear_set_pair_min_m(DEFAULT_PAIR_MIN_M)
     assert q.qlora_get_device_status() == q.QLORA_OK
     return out
 
 
 def run_mid_m(flush, stream, M=480, r=64):
-    """Mid-sized batches (16 < M < 512) on weights with one narrow side: the default routing
-    (a direction whose fused kernel would fill fewer than half the SMs takes the pair GEMM with
-    split K) against the fused kernels everywhere."""
+    """Mid-sized batches on weights with one narrow side: the default routing (the pair GEMM
+    from 128 tokens on, with split K where the tiles are few) against the fused kernels
+    everywhere."""
     import torch
     import bit_nf4_quantized_double_b200 as q
     import synth_inputs as si
@@ -661,7 +662,7 @@ def run_mid_m(flush, stream, M=480, r=64):
         B = si.normal((r, rows), 0.01, seed=8, device="cuda", dtype=torch.bfloat16)
         flops = step_flops(M, cols, rows, r)
         res = {}
-        for name, P in (("default", 512), ("fused_everywhere", 2 ** 63 - 1)):
+        for name, P in (("default", DEFAULT_PAIR_MIN_M), ("fused_everywhere", 2 ** 63 - 1)):
             q.lib().qlora_linear_set_pair_min_m(P)
             try:
                 def step():
@@ -671,7 +672,7 @@ def run_mid_m(flush, stream, M=480, r=64):
                 res[name] = {"ms_per_step": round(ms, 5), "TFLOP/s": round(flops / (ms / 1e3) / 1e12, 1),
                              "kernels": _kernel_ms(KERNELS + ("k_gemm2sm_reduce",), step, 3, flush)}
             finally:
-                q.lib().qlora_linear_set_pair_min_m(512)
+                q.lib().qlora_linear_set_pair_min_m(DEFAULT_PAIR_MIN_M)
         out[f"{rows}x{cols}"] = res
         del t
     assert q.qlora_get_device_status() == q.QLORA_OK
@@ -1059,7 +1060,7 @@ def run_profile_case(name, reps=3):
             l2_flush(flush)
             Y, XA = q.qlora_linear_fwd(inp["X"], t, inp["A"], inp["B"], L.s)
             q.qlora_linear_bwd(inp["X"], inp["dY"], t, inp["A"], inp["B"], L.s, XA=XA)
-        q.lib().qlora_linear_set_pair_min_m(512)
+        q.lib().qlora_linear_set_pair_min_m(DEFAULT_PAIR_MIN_M)
     elif name == "l4096":
         wl, L, inp = headline_inputs(0)
         t = q.qlora_nf4_quantize(inp["W"])

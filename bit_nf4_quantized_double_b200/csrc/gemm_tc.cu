@@ -1158,17 +1158,19 @@ static cudaError_t run_skinny(bool a_mn, const void *a, bool b_mn, const void *b
 
 static size_t mr_bytes(int64_t M, int r) { return align256((size_t)M * (size_t)r * 2); }
 
-// From this many tokens on (default 512), the layer dequantises W once into bf16
-// scratch and runs the CTA-pair GEMM: the fused kernel would repeat the
-// dequantisation for every 256-token tile, and at two or more tiles that integer
-// work costs more than writing and re-reading the bf16 copy. From 128 tokens on, a
-// direction whose fused kernel would have fewer 128 x 256 output tiles than half the SMs
-// also takes the pair GEMM, whose K blocks then split over the idle SMs (below 128 tokens
-// the bf16 copy costs more than the fused kernel's idle SMs). Settable so that both
-// routes can be compared at any M (qlora_linear_set_pair_min_m; INT64_MAX keeps every
-// M > 16 on the fused kernels).
+// From this many tokens on (default 128), the layer dequantises W once into bf16
+// scratch and runs the CTA-pair GEMM: the fused kernel repeats the dequantisation for
+// every 256-token tile and runs at the rate of its integer work. Timed per direction at
+// M = 128 .. 480 on 4096^2, 16384 x 1024, 1024 x 16384, 11008 x 4096 and 4096 x 11008
+// weights (r = 64), the pair route was up to 30 % faster (the 16384 x 1024 forward at
+// M = 480: 40.9 against 57.5 us) and at most 1.4 us slower (the 4096^2 forward at M = 384:
+// 51.3 against 49.9 us); below 128 tokens the bf16 copy costs more than the fused kernel.
+// With a larger P, from 128 tokens on a direction whose fused kernel would have fewer
+// 128 x 256 output tiles than half the SMs still takes the pair GEMM, whose K blocks then
+// split over the idle SMs. Settable so that both routes can be compared at any M
+// (qlora_linear_set_pair_min_m; INT64_MAX keeps every M > 16 on the fused kernels).
 constexpr int64_t kFewTilesMinM = 128;
-static std::atomic<int64_t> g_pair_min_m{512};
+static std::atomic<int64_t> g_pair_min_m{128};
 // CTAs per SM of the dequantisation beside an adapter product of Mp rows over Kp inputs:
 // three 256-thread CTAs when the product has at most one CTA per SM (they leave it the
 // registers for one), else two, so that the product's CTAs are scheduled next to the

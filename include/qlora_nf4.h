@@ -19,7 +19,7 @@
  *   frees device memory; scratch comes from a caller-provided workspace whose
  *   size the matching *_workspace() query returns.
  * - Two resources are the library's own. (1) A qlora_linear_fwd or
- *   qlora_linear_bwd call that takes the pair-GEMM route (M >= P, 512 by
+ *   qlora_linear_bwd call that takes the pair-GEMM route (M >= P, 128 by
  *   default, see qlora_linear_set_pair_min_m) with r > 0 may create, on first
  *   use on a device, one non-blocking side stream and two events for that
  *   device, kept until the process exits: the backward forks the adapter
@@ -150,11 +150,12 @@ qlora_status qlora_nf4_dequant_grouped(int count, const qlora_nf4_tensor *q, voi
  * (r == 0: no adapter; A, B, XA_save ignored). M <= 16 takes the streaming GEMV
  * kernel, 16 < M < P the fused tcgen05 dequant-GEMM, and M >= P dequantises W
  * once into bf16 in the workspace (rows * cols * 2 bytes of it) and runs a
- * CTA-pair tcgen05 GEMM with the adapter term as extra K blocks; P = 512 unless
- * qlora_linear_set_pair_min_m changed it. From M = 128 on, a call whose fused kernel
- * would have fewer 128-row x 256-token output tiles than half the SMs also takes the
- * pair GEMM, with each tile's K blocks split over the idle SMs (fp32 partials in the
- * workspace, added in a fixed order).
+ * CTA-pair tcgen05 GEMM with the adapter term as extra K blocks; P = 128 unless
+ * qlora_linear_set_pair_min_m changed it. When few 256 x 256 tiles would leave most SMs
+ * idle, each tile's K blocks are split over them (fp32 partials in the workspace, added
+ * in a fixed order). With P raised above 128, a call from M = 128 on whose fused kernel
+ * would have fewer 128-row x 256-token output tiles than half the SMs still takes the
+ * pair GEMM.
  */
 size_t qlora_linear_fwd_workspace(int64_t M, int64_t rows, int64_t cols, int r);
 qlora_status qlora_linear_fwd(const void *X, int64_t M, const qlora_nf4_tensor *W,
@@ -182,7 +183,7 @@ qlora_status qlora_linear_bwd(const void *X, const void *dY, int64_t M, const ql
 /*
  * Tuning hook of the two large-M routes (the page has no counterpart): sets P, the
  * token count from which qlora_linear_fwd / qlora_linear_bwd dequantise W once and run
- * the CTA-pair GEMM instead of the fused dequant-GEMM (default 512; values below 17
+ * the CTA-pair GEMM instead of the fused dequant-GEMM (default 128; values below 17
  * are raised to 17; INT64_MAX keeps every M > 16 on the fused kernels, including the
  * few-tile calls that would otherwise take the pair GEMM). Both routes compute the same
  * layer; the workspace queries follow P, so query after setting it.

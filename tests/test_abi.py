@@ -11,6 +11,8 @@ import pytest
 import bit_nf4_quantized_double_b200 as q
 import oracle
 
+DEFAULT_PAIR_MIN_M = 128   # the library's default token count for the pair-GEMM route
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -63,14 +65,21 @@ def test_workspace_queries_positive():
     for M in (1, 16, 17, 4096):
         assert L.qlora_linear_fwd_workspace(M, 4096, 4096, 64) > 0
         assert L.qlora_linear_bwd_workspace(M, 4096, 4096, 64) > 0
-    # no adapter and a batch below 512 tokens whose fused kernel fills the SMs: nothing to stage
-    assert L.qlora_linear_bwd_workspace(256, 4096, 16384, 0) == 0
-    # below 512 tokens, a dgrad whose fused kernel would have only 32 output tiles takes the
-    # pair GEMM: the bf16 weight plus fp32 partials of 4 K ranges of its 16 tiles (148 SMs,
-    # the count assumed without a GPU)
+    # from 128 tokens on the pair GEMM runs: the bf16 weight in the workspace, here 64 whole
+    # 256 x 256 tiles (no split)
+    assert L.qlora_linear_bwd_workspace(256, 4096, 16384, 0) == 4096 * 16384 * 2
+    # ... and a dgrad with only 16 tiles splits each tile's K blocks 4 ways: the bf16 weight
+    # plus fp32 partials (148 SMs, the count assumed without a GPU)
     assert L.qlora_linear_bwd_workspace(256, 4096, 4096, 0) == 4096 * 4096 * 2 + 4 * 256 * 4096 * 4
     # under 128 tokens the fused kernels always run
     assert L.qlora_linear_bwd_workspace(127, 4096, 4096, 0) == 0
+    # with P raised to 512, a batch of 256 whose fused kernel fills the SMs stages nothing
+    L.qlora_linear_set_pair_min_m(512)
+    try:
+        assert L.qlora_linear_bwd_workspace(256, 4096, 16384, 0) == 0
+        assert L.qlora_linear_bwd_workspace(256, 4096, 4096, 0) == 4096 * 4096 * 2 + 4 * 256 * 4096 * 4
+    finally:
+        L.qlora_linear_set_pair_min_m(DEFAULT_PAIR_MIN_M)
     # from 512 tokens on, the layer keeps a bf16 copy of the dequantised weight
     assert L.qlora_linear_bwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2
     assert L.qlora_linear_fwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2

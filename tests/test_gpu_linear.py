@@ -16,6 +16,7 @@ pytestmark = pytest.mark.gpu
 
 MAX_TOL = 2e-2
 FRO_TOL = 5e-3
+DEFAULT_PAIR_MIN_M = 128   # the library's default token count for the pair-GEMM route
 
 
 def f64(t):
@@ -192,9 +193,11 @@ def test_grouped_more_than_eight(M):
         assert torch.equal(Y, Y1), i
 
 
-@pytest.mark.parametrize("M,rows,cols,r", [(3, 400, 320, 24), (200, 272, 640, 64), (1024, 512, 1024, 16)])
+@pytest.mark.parametrize("M,rows,cols,r", [(3, 400, 320, 24), (100, 272, 640, 64), (200, 272, 640, 64),
+                                           (1024, 512, 1024, 16)])
 def test_backward_recomputes_xa(M, rows, cols, r):
-    # XA = NULL: the backward recomputes X A itself (small-M, fused and CTA-pair paths)
+    # XA = NULL: the backward recomputes X A itself (small-M, fused (M = 100) and CTA-pair
+    # paths)
     W, X, dY, A, B, s = make_problem(M, rows, cols, r, seed=31 * M + rows)
     t = q.qlora_nf4_quantize(W)
     dX, dA, dB = q.qlora_linear_bwd(X, dY, t, A, B, s, XA=None)
@@ -269,7 +272,7 @@ def test_zero_adapter_equals_plain_product():
 
 @pytest.mark.parametrize("M,rows,cols,r", [
     (512, 512, 8192, 64),     # forward: 4 tiles, 16 K ranges per tile; dgrad: 64 whole tiles
-    (200, 384, 2048, 64),     # below 512 tokens: the fused kernels would use 3 and 16 CTAs
+    (200, 384, 2048, 64),     # 200 tokens: one 256-token tile, 2 and 8 output tiles
     (4096, 256, 4096, 16),    # headline tokens, a narrow output: 16 tiles, 4 K ranges
 ])
 def test_split_k_pair_route(M, rows, cols, r):
@@ -280,16 +283,21 @@ def test_split_k_pair_route(M, rows, cols, r):
 
 @pytest.mark.parametrize("rep", [0, 1])
 def test_many_tiles_per_cta_fused_full(rep):
-    # below 512 tokens: the forward of the 16384-row weight and the dgrad of the
-    # 16384-input one stay on the fused kernels, where every persistent CTA walks several
-    # 128 x 256 tiles; the other two directions have 16 fused tiles and take the pair GEMM
-    # with split K. Compare every element, twice, so a race at tile boundaries shows
+    # with the pair route raised to 512 tokens: at 480 the forward of the 16384-row weight
+    # and the dgrad of the 16384-input one stay on the fused kernels, where every persistent
+    # CTA walks several 128 x 256 tiles; the other two directions have 16 fused tiles and
+    # take the pair GEMM with split K. Compare every element, twice, so a race at tile
+    # boundaries shows
     M = 480
     for rows, cols in ((16384, 1024), (1024, 16384)):
         W, X, dY, A, B, s = make_problem(M, rows, cols, 64, seed=500 + rows + rep)
         t = q.qlora_nf4_quantize(W)
-        Y, XA = q.qlora_linear_fwd(X, t, A, B, s)
-        dX, dA, dB = q.qlora_linear_bwd(X, dY, t, A, B, s, XA=XA)
+        q.lib().qlora_linear_set_pair_min_m(512)
+        try:
+            Y, XA = q.qlora_linear_fwd(X, t, A, B, s)
+            dX, dA, dB = q.qlora_linear_bwd(X, dY, t, A, B, s, XA=XA)
+        finally:
+            q.lib().qlora_linear_set_pair_min_m(DEFAULT_PAIR_MIN_M)
         assert q.qlora_get_device_status() == q.QLORA_OK
         Wh = oracle_weight(W)
         Xn, dYn, An, Bn = f64(X), f64(dY), f64(A), f64(B)
@@ -302,7 +310,7 @@ def test_many_tiles_per_cta_fused_full(rep):
 
 @pytest.mark.parametrize("rep", [0, 1])
 def test_many_tiles_per_cta_full(rep):
-    # from 512 tokens on the CTA-pair GEMM runs; here the forward of the 8192-row
+    # at 4096 tokens the CTA-pair GEMM runs; here the forward of the 8192-row
     # weight and the dgrad of the 8192-input one give each pair about seven 256 x 256
     # tiles, so both TMEM accumulators are reused many times: compare every element,
     # twice, so a race between the epilogue and the next tile's MMAs shows
@@ -334,7 +342,7 @@ def test_routes_forced_either_way(P, M, rows, cols, r):
     try:
         run_case(M, rows, cols, r, seed=M + rows + r + 7)
     finally:
-        q.lib().qlora_linear_set_pair_min_m(512)
+        q.lib().qlora_linear_set_pair_min_m(DEFAULT_PAIR_MIN_M)
 
 
 @pytest.mark.parametrize("M,rows,cols,r", [(512, 1024, 2048, 16), (600, 768, 1536, 0), (256, 4096, 1024, 8),
