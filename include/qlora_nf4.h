@@ -200,9 +200,11 @@ void qlora_linear_set_pair_min_m(int64_t m);
  *   d      host array of `count` descriptors (1 <= count <= 64); W points to a host
  *          struct as in qlora_linear_fwd.
  *   ws     one device workspace of qlora_linear_fwd_grouped_workspace() bytes.
- * M <= 16: per group of up to eight items, two launches: X*A of every adapter, and one
- * persistent GEMV over all items' codes that adds the adapter term (s X A) B as it
- * finishes each row block (it starts early through programmatic dependent launch).
+ * M <= 16: per group of up to eight items, three launches chained by programmatic
+ * dependent launch: one persistent GEMV over all items' codes that writes fp32 sums per
+ * K chunk to the workspace; the X*A partial sums of every adapter, beside the GEMV; and
+ * a finishing kernel that adds each output's K chunks in chunk order and the adapter
+ * term (s X A) B, and rounds to bf16.
  * Larger M: the items run one after another on the single-item path, and the workspace
  * is the largest single-item requirement. Y and XA_save are bit-identical to calling
  * qlora_linear_fwd on each item: every output adds its input slices and K chunks in a
