@@ -613,11 +613,13 @@ k_merge_bf16(NF4View q, const float *__restrict__ At, const float *__restrict__ 
     int step = 0;
     for (; tile < tiles; tile += gridDim.x) {
         const int64_t n0 = (tile % tiles_n) * kMergeTile, k0 = (tile / tiles_n) * kMergeTile;
-        float d[8][8];
+        // d[i][2p], d[i][2p + 1] as one 64-bit pair dd[i][p] (low half first): two fused
+        // multiply-adds per instruction (fma.rn.f32x2, each half one IEEE fma)
+        uint64_t dd[8][4];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) d[i][c] = 0.0f;
+            for (int c = 0; c < 4; ++c) dd[i][c] = 0ull;
         for (int c = 0; c < nj; ++c, ++step) {
             // the next step's copies go out before this step's wait
             const bool more = c + 1 < nj || tile + gridDim.x < tiles;
@@ -640,16 +642,20 @@ k_merge_bf16(NF4View q, const float *__restrict__ At, const float *__restrict__ 
             const float *Bp = msm + (size_t)((step & 1) * 2 + 1) * kMergeBuf + 8 * tn;
             const int jn = r - c * kMergeJ < kMergeJ ? r - c * kMergeJ : kMergeJ;
             auto fma_step = [&](int jj) {
-                const float4 a0 = *reinterpret_cast<const float4 *>(Ap + jj * kMergeTile);
-                const float4 a1 = *reinterpret_cast<const float4 *>(Ap + jj * kMergeTile + 64);
+                const ulonglong2 a0 = *reinterpret_cast<const ulonglong2 *>(Ap + jj * kMergeTile);
+                const ulonglong2 a1 = *reinterpret_cast<const ulonglong2 *>(Ap + jj * kMergeTile + 64);
                 const float4 b0 = *reinterpret_cast<const float4 *>(Bp + jj * kMergeTile);
                 const float4 b1 = *reinterpret_cast<const float4 *>(Bp + jj * kMergeTile + 4);
-                const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                const uint64_t ap[4] = {a0.x, a0.y, a1.x, a1.y};      // inputs (2p, 2p + 1)
                 const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
+                for (int i = 0; i < 8; ++i) {
+                    uint64_t bb;
+                    asm("mov.b64 %0, {%1, %1};" : "=l"(bb) : "f"(b[i]));
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) d[i][cc] = fmaf(a[cc], b[i], d[i][cc]);
+                    for (int c = 0; c < 4; ++c)
+                        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(dd[i][c]) : "l"(ap[c]), "l"(bb));
+                }
             };
             if (jn == kMergeJ) {
 #pragma unroll
@@ -679,8 +685,9 @@ k_merge_bf16(NF4View q, const float *__restrict__ At, const float *__restrict__ 
                     const uint32_t byte = (cw >> (8 * h)) & 0xffu;
                     const float w_hi = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_q[byte >> 4], ch)));
                     const float w_lo = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_q[byte & 15u], ch)));
-                    o[h] = pack_bf16x2(__fadd_rn(w_hi, __fmul_rn(s, d[i][4 * g + 2 * h])),
-                                       __fadd_rn(w_lo, __fmul_rn(s, d[i][4 * g + 2 * h + 1])));
+                    float d0, d1;                                   // inputs 4g + 2h and 4g + 2h + 1
+                    asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(dd[i][2 * g + h]));
+                    o[h] = pack_bf16x2(__fadd_rn(w_hi, __fmul_rn(s, d0)), __fadd_rn(w_lo, __fmul_rn(s, d1)));
                 }
                 *reinterpret_cast<uint2 *>(out + e0) = make_uint2(o[0], o[1]);
             }
