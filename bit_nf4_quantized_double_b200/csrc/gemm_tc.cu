@@ -24,7 +24,9 @@
 //   k_skinny      TMA-fed tcgen05 GEMM for the rank-r products X*A, dY*B^T,
 //                 X^T*(sG), dY^T*XA, split over K across the CTAs of a thread-block
 //                 cluster that add their accumulators in a fixed order through
-//                 distributed shared memory and apply scale/layout.
+//                 distributed shared memory and apply scale/layout. Before a pair
+//                 GEMM its CTAs may also carry extra warps that dequantise the
+//                 weight into the GEMM's bf16 operand (skinny_dequant).
 // Both fused kernels keep the accumulator tile D[row, token] in TMEM and store
 // it transposed (out[token, row]) through a shared-memory staging tile and a
 // TMA store.
