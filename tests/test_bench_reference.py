@@ -30,3 +30,20 @@ def test_reference_arm_json_line():
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_step_flops_counts_every_product():
+    # the headline's work per fwd + bwd step, counted product by product: the two base GEMMs
+    # (Y = X W^T, dX = dY W^) and the six rank-r products (X A, (s XA) B, dY B^T, (s G) A^T,
+    # dA = X^T (s G), dB = (XA)^T dY), 2 m n k each
+    sys.path.insert(0, ROOT)
+    import bench
+    M, d_in, d_out, r = 4096, 4096, 4096, 64
+    products = [(M, d_out, d_in), (M, d_in, d_out),
+                (M, r, d_in), (M, d_out, r), (M, r, d_out), (M, d_in, r), (d_in, r, M), (r, d_out, M)]
+    assert bench.step_flops(M, d_in, d_out, r) == sum(2 * m * n * k for m, n, k in products) == 287762808832
+    # a non-square layer as well
+    M, d_in, d_out, r = 480, 1024, 16384, 16
+    products = [(M, d_out, d_in), (M, d_in, d_out),
+                (M, r, d_in), (M, d_out, r), (M, r, d_out), (M, d_in, r), (d_in, r, M), (r, d_out, M)]
+    assert bench.step_flops(M, d_in, d_out, r) == sum(2 * m * n * k for m, n, k in products)
