@@ -71,8 +71,11 @@ def test_workspace_queries_positive():
     # ... and a dgrad with only 16 tiles splits each tile's K blocks 4 ways: the bf16 weight
     # plus fp32 partials (148 SMs, the count assumed without a GPU)
     assert L.qlora_linear_bwd_workspace(256, 4096, 4096, 0) == 4096 * 4096 * 2 + 4 * 256 * 4096 * 4
-    # under 128 tokens the fused kernels always run
+    # under 128 tokens the fused kernels always run; from 128 on the pair route (forward too)
     assert L.qlora_linear_bwd_workspace(127, 4096, 4096, 0) == 0
+    assert L.qlora_linear_fwd_workspace(127, 11008, 4096, 0) == 0
+    assert L.qlora_linear_fwd_workspace(128, 11008, 4096, 0) >= 11008 * 4096 * 2
+    assert L.qlora_linear_bwd_workspace(128, 4096, 11008, 0) >= 4096 * 11008 * 2
     # with P raised to 512, a batch of 256 whose fused kernel fills the SMs stages nothing
     L.qlora_linear_set_pair_min_m(512)
     try:
