@@ -142,6 +142,15 @@ def test_argument_checks_run_on_host():
                               None) == q.QLORA_ERR_WORKSPACE
     assert L.qlora_linear_bwd(None, ctypes.c_void_p(fake), 0, ctypes.byref(good), None, None, 0, 1.0, None,
                               ctypes.c_void_p(fake), None, None, None, 0, None) == q.QLORA_ERR_UNSUPPORTED_SHAPE
+    # an empty batch, a row count that is not a multiple of 16, a rank above 256
+    assert L.qlora_linear_fwd(ctypes.c_void_p(fake), 0, ctypes.byref(good), None, None, 0, 1.0,
+                              ctypes.c_void_p(fake), None, None, 0, None) == q.QLORA_ERR_UNSUPPORTED_SHAPE
+    bad_rows = q._Tensor(40, 64, fake, fake, fake, fake)
+    assert L.qlora_linear_fwd(ctypes.c_void_p(fake), 4, ctypes.byref(bad_rows), None, None, 0, 1.0,
+                              ctypes.c_void_p(fake), None, None, 0, None) == q.QLORA_ERR_UNSUPPORTED_SHAPE
+    assert L.qlora_linear_fwd(ctypes.c_void_p(fake), 4, ctypes.byref(good), ctypes.c_void_p(fake),
+                              ctypes.c_void_p(fake), 264, 1.0, ctypes.c_void_p(fake), None, None, 0,
+                              None) == q.QLORA_ERR_UNSUPPORTED_SHAPE
 
 
 def test_fmt4_argument_checks_run_on_host():
