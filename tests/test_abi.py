@@ -83,7 +83,7 @@ def test_workspace_queries_positive():
         assert L.qlora_linear_bwd_workspace(256, 4096, 4096, 0) == 4096 * 4096 * 2 + 4 * 256 * 4096 * 4
     finally:
         L.qlora_linear_set_pair_min_m(DEFAULT_PAIR_MIN_M)
-    # from 512 tokens on, the layer keeps a bf16 copy of the dequantised weight
+    # at 4096 tokens the layer keeps a bf16 copy of the dequantised weight
     assert L.qlora_linear_bwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2
     assert L.qlora_linear_fwd_workspace(4096, 4096, 4096, 0) == 4096 * 4096 * 2
 
